@@ -1,0 +1,289 @@
+"""Swimba layer oracle: a plain, slow, fp64 CPU restatement of what the layer computes.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's CPU-baseline
+leg may import this module.  It shares no code with the CUDA library and imports nothing
+from it; its inputs are plain numpy arrays.
+
+Sources (all describe arXiv 2603.06938, "Swimba: Switch Mamba Model Scales State Space Models"):
+  [notes]  papernotes.org NeurIPS 2026 notes on Swimba, Method ("overall framework", its flowchart,
+           key design 1 with the two display equations, key design 2 with Theorems 3.3/3.4,
+           key design 3 with Theorem 3.5) and the efficiency table.
+  [gist]   gist.science English summary, Technical Summary section 2 "Methodology",
+           "Architecture Details" and "Theoretical Guarantees".
+Where the pages leave a step open the reading used here is stated beside the step.
+
+Notation: tokens t, batch row b, heads h (group g(h) = h // (H // G)), experts e, slots j < k.
+Shapes: X [B,T,D]; W_r [E,D]; W_dt [H,D]; b_dt [H]; A [H]; W_exp [E, H*P + 2*G*N, D].
+Everything is computed in float64.
+"""
+import numpy as np
+
+
+# ----------------------------------------------------------------------------- router
+
+def softplus(v):
+    """log(1 + e^v), evaluated without overflow."""
+    return np.logaddexp(0.0, v)
+
+
+def router_logits(X, W_r):
+    """g_t = W_r X_t: the token router R(X_t) of [notes] Method, flowchart node "token router".
+
+    Reading: a linear router without bias, temperature 1.
+    """
+    return X @ W_r.T
+
+
+def dt_proj(X, W_dt, b_dt, dt_min=1e-3, dt_max=0.1):
+    """dt_{t,h} = clamp(softplus(W_dt[h] . X_t + b_dt[h]), dt_min, dt_max).
+
+    The pages fix A as shared by all experts ([notes] key design 2; [gist] Architecture Details);
+    the step size dt that discretises it comes from one shared (non-expert) projection, so the
+    transition a_t = exp(dt_t A_h) is shared by every expert while staying input-dependent.
+    """
+    return np.clip(softplus(X @ W_dt.T + b_dt), dt_min, dt_max)
+
+
+def topk_select(g, k):
+    """Active set K_t of [notes] key design 1 ("usually top-k sparse"): the indices of the k
+    largest entries of each row of g, largest first, equal values ordered by lower expert index.
+
+    The caller passes g in the precision the decision is taken in (the kernels take it on
+    fp32 logits; pass g.astype(np.float32) for a like-for-like decision).
+    """
+    g = np.asarray(g)
+    # a stable sort of -g keeps equal values in index order, i.e. ties go to the lower index
+    order = np.argsort(-g, axis=-1, kind="stable")
+    return order[..., :k].astype(np.int64)
+
+
+def topk_weights(g, idx):
+    """pi_{t,j} = softmax(g_t) restricted to K_t and renormalised over the k winners
+    ([notes] key design 1: pi_t = softmax(g_t); renormalisation over K_t is the reading used).
+    Equal to exp(g_{K_j}) / sum_j' exp(g_{K_j'})."""
+    sel = np.take_along_axis(g, idx, axis=-1)
+    m = sel.max(axis=-1, keepdims=True)
+    ex = np.exp(sel - m)
+    return ex / ex.sum(axis=-1, keepdims=True)
+
+
+def router(X, W_r, W_dt, b_dt, k, decision_dtype=np.float32, forced_idx=None):
+    """Router stage on flattened tokens X [M, D]: returns (g, dt, topk_idx, topk_w).
+
+    forced_idx (optional [M,k]) replaces the active set on rows where it is >= 0; the tests use it
+    to replay the kernel's choice on near-tied tokens, where either choice is a correct top-k.
+    """
+    g = router_logits(X, W_r)
+    dt = dt_proj(X, W_dt, b_dt)
+    idx = topk_select(g.astype(decision_dtype), k)
+    if forced_idx is not None:
+        rows = forced_idx[:, 0] >= 0
+        idx[rows] = forced_idx[rows]
+    w = topk_weights(g, idx)
+    return g, dt, idx, w
+
+
+# ----------------------------------------------------------------------------- experts and mixing
+
+def split_streams(z, H, P, G, N):
+    """Split one expert projection z [..., H*P + 2*G*N] into the candidate streams
+    (x [...,H,P], B [...,G,N], C [...,G,N]) of [notes] key design 1.
+
+    Reading of the stream shapes: B and C are N-vectors and x a P-vector per head (the notes'
+    "B in R^{N x P}" cannot give a P-vector readout); G groups, G = H meaning every head has its own.
+    """
+    HP, GN = H * P, G * N
+    x = z[..., :HP].reshape(z.shape[:-1] + (H, P))
+    B = z[..., HP:HP + GN].reshape(z.shape[:-1] + (G, N))
+    C = z[..., HP + GN:HP + 2 * GN].reshape(z.shape[:-1] + (G, N))
+    return x, B, C
+
+
+def expert_proj(X, W_exp, idx):
+    """Candidate streams of the active experts: z[t, j] = W_exp[K_tj] X_t  ([notes] key design 1:
+    every expert applies its own linear projection to the same X_t).  X [M,D] -> z [M,k,W_e]."""
+    M, k = idx.shape
+    z = np.zeros((M, k, W_exp.shape[1]))
+    for e in range(W_exp.shape[0]):
+        rows, slots = np.nonzero(idx == e)
+        if rows.size:
+            z[rows, slots] = X[rows] @ W_exp[e].T
+    return z
+
+
+def mix(z, w, H, P, G, N):
+    """Parameter-space mixing ([notes] key design 1, first display equation; [gist] Parameter Mixing):
+      U~_t = sum_j pi_tj B_t^(j) x_t^(j)T   kept factored as (Bpi = pi B, Xs = x) per slot,
+      C~_t = sum_j pi_tj C_t^(j).
+    Returns Bpi [M,k,G,N], Xs [M,k,H,P], Ct [M,G,N] and the per-slot pi C [M,k,G,N]."""
+    x, B, C = split_streams(z, H, P, G, N)
+    Bpi = w[:, :, None, None] * B
+    Cpi = w[:, :, None, None] * C
+    return Bpi, x, Cpi.sum(axis=1), Cpi
+
+
+# ----------------------------------------------------------------------------- the single recurrence
+
+def group_of(H, G):
+    return np.arange(H) // (H // G)
+
+
+def scan_sequential(Bpi, Xs, Ct, dt, A, init=None):
+    """The single-trajectory recurrence, token by token ([notes] key design 1, second display
+    equation; [gist] "h_t = A h_{t-1} + sum pi B X"):
+        h_t = a_t h_{t-1} + sum_j Bpi_tj (x) Xs_tj,     y_t = C~_t^T h_t,     a_t = exp(dt_t A_h).
+    Reading: no dt factor on the injection (the pages' equation has none).
+
+    One batch row: Bpi [T,k,G,N], Xs [T,k,H,P], Ct [T,G,N], dt [T,H], A [H], init [H,N,P] or None.
+    Returns y [T,H,P] and the final state [H,N,P].
+    """
+    T, k, H, P = Xs.shape
+    G, N = Bpi.shape[2], Bpi.shape[3]
+    g = group_of(H, G)
+    h = np.zeros((H, N, P)) if init is None else np.array(init, dtype=np.float64)
+    y = np.zeros((T, H, P))
+    for t in range(T):
+        a = np.exp(dt[t] * A)                                           # [H]
+        U = np.einsum("jhn,jhp->hnp", Bpi[t][:, g], Xs[t])              # rank-k injection per head
+        h = a[:, None, None] * h + U
+        y[t] = np.einsum("hn,hnp->hp", Ct[t][g], h)
+    return y, h
+
+
+def scan_bruteforce(Bpi, Xs, Ct, dt, A, init=None):
+    """The same layer as one materialised semiseparable matrix product (quadratic in T):
+        y_t = sum_{s<=t} (prod_{r=s+1..t} a_r) sum_j (C~_t . Bpi_sj) Xs_sj  +  (prod_{r<=t} a_r) C~_t^T h_init.
+    Structure preservation ([notes] key design 1, Theorem 3.1): the mixed layer is one selective SSM,
+    whose input-output map is this lower-triangular matrix.  For tiny T only."""
+    T, k, H, P = Xs.shape
+    g = group_of(H, G=Bpi.shape[2])
+    dA = dt * A                                                        # [T,H]
+    y = np.zeros((T, H, P))
+    for t in range(T):
+        for s in range(t + 1):
+            decay = np.exp(dA[s + 1:t + 1].sum(axis=0))                # [H]
+            for j in range(k):
+                score = np.einsum("hn,hn->h", Ct[t][g], Bpi[s, j][g])   # C~_t . Bpi_sj
+                y[t] += (decay * score)[:, None] * Xs[s, j]
+        if init is not None:
+            decay0 = np.exp(dA[:t + 1].sum(axis=0))
+            y[t] += decay0[:, None] * np.einsum("hn,hnp->hp", Ct[t][g], init)
+    return y
+
+
+def scan_chunked(Bpi, Xs, Ct, dt, A, Q, init=None):
+    """The same recurrence solved chunk by chunk, the SSD decomposition the pages reuse
+    ([notes] overall framework: Mamba-2's chunked SSD algorithm, reused unchanged):
+      cs_t   = sum of dt*A from the chunk start to t (inclusive)
+      y_t    = sum_{s in chunk, s<=t} exp(cs_t - cs_s) sum_j (C~_t . Bpi_sj) Xs_sj      (intra-chunk)
+             + exp(cs_t) C~_t^T H_c                                                     (carried state)
+      S_c    = sum_{s in chunk} exp(cs_end - cs_s) sum_j Bpi_sj (x) Xs_sj               (chunk state)
+      H_{c+1}= exp(cs_end) H_c + S_c,   H_0 = init or 0.
+    Returns y [T,H,P], chunk-start states Hs [nc,H,N,P] (Hs[c] = H_c) and the final state."""
+    T, k, H, P = Xs.shape
+    G, N = Bpi.shape[2], Bpi.shape[3]
+    g = group_of(H, G)
+    nc = (T + Q - 1) // Q
+    Hc = np.zeros((H, N, P)) if init is None else np.array(init, dtype=np.float64)
+    Hs = np.zeros((nc, H, N, P))
+    y = np.zeros((T, H, P))
+    for c in range(nc):
+        t0, t1 = c * Q, min(T, (c + 1) * Q)
+        cs = np.cumsum(dt[t0:t1] * A, axis=0)                          # [L,H]
+        Cg = Ct[t0:t1][:, g]                                           # [L,H,N]
+        Bg = Bpi[t0:t1][:, :, g]                                       # [L,k,H,N]
+        Xc = Xs[t0:t1]                                                 # [L,k,H,P]
+        L = t1 - t0
+        Hs[c] = Hc
+        scores = np.einsum("thn,sjhn->tsjh", Cg, Bg)                   # [L,L,k,H]
+        seg = cs[:, None, :] - cs[None, :, :]                          # [L,L,H] = cs_t - cs_s
+        causal = np.tril(np.ones((L, L), dtype=bool))
+        decay = np.where(causal[:, :, None], np.exp(np.where(causal[:, :, None], seg, 0.0)), 0.0)
+        y[t0:t1] = np.einsum("tsh,tsjh,sjhp->thp", decay, scores, Xc)
+        y[t0:t1] += np.exp(cs)[:, :, None] * np.einsum("thn,hnp->thp", Cg, Hc)
+        wend = np.exp(cs[-1][None, :] - cs)                            # [L,H]
+        S = np.einsum("sh,sjhn,sjhp->hnp", wend, Bg, Xc)
+        Hc = np.exp(cs[-1])[:, None, None] * Hc + S
+    return y, Hs, Hc
+
+
+# ----------------------------------------------------------------------------- the separated contrast designs
+
+def scan_separated_k(B, Xs, Cpi, dt, A, init=None):
+    """"k scans": one trajectory per active slot j, driven by that slot's own (unscaled) injection
+    B^(K_j) x^(K_j)T, read out with pi_j C^(K_j):
+        h^(j)_t = a_t h^(j)_{t-1} + B_tj (x) Xs_tj,    y_t = sum_j (pi_tj C_tj)^T h^(j)_t.
+    This is the separated-trajectory design of [notes] key design 1 restricted to the active slots;
+    it runs k recurrences where the mixed layer runs one.  B [T,k,G,N], Cpi [T,k,G,N], init [k,H,N,P].
+    Returns y [T,H,P], the k final states [k,H,N,P] and the number of recurrences run (k)."""
+    T, k, H, P = Xs.shape
+    G, N = B.shape[2], B.shape[3]
+    g = group_of(H, G)
+    h = np.zeros((k, H, N, P)) if init is None else np.array(init, dtype=np.float64)
+    y = np.zeros((T, H, P))
+    for t in range(T):
+        a = np.exp(dt[t] * A)
+        for j in range(k):
+            h[j] = a[:, None, None] * h[j] + np.einsum("hn,hp->hnp", B[t, j][g], Xs[t, j])
+            y[t] += np.einsum("hn,hnp->hp", Cpi[t, j][g], h[j])
+    return y, h, k
+
+
+def scan_separated_dense(xE, BE, CE, pi_dense, dt, A):
+    """MoE over separated SSMs ([notes] key design 1, the O(T E C_step) design; Theorem 3.4):
+    every expert e keeps its own state h^(e), driven on every token by its own B^(e) x^(e)T, and the
+    output is y_t = sum_e pi_te C^(e)_t^T h^(e)_t (pi_te = 0 off the active set).
+    xE [T,E,H,P], BE/CE [T,E,G,N], pi_dense [T,E].  Returns y, the states [T,E,H,N,P] and E."""
+    T, E, H, P = xE.shape
+    G, N = BE.shape[2], BE.shape[3]
+    g = group_of(H, G)
+    h = np.zeros((E, H, N, P))
+    hs = np.zeros((T, E, H, N, P))
+    y = np.zeros((T, H, P))
+    for t in range(T):
+        a = np.exp(dt[t] * A)
+        for e in range(E):
+            h[e] = a[:, None, None] * h[e] + np.einsum("hn,hp->hnp", BE[t, e][g], xE[t, e])
+            y[t] += pi_dense[t, e] * np.einsum("hn,hnp->hp", CE[t, e][g], h[e])
+        hs[t] = h
+    return y, hs, E
+
+
+# ----------------------------------------------------------------------------- the layer
+
+def layer_fwd(X, W_r, W_dt, b_dt, A, W_exp, H, P, N, G, k, init=None, forced_idx=None,
+              decision_dtype=np.float32):
+    """Forward pass of one Swimba token-mixer layer ([notes] Method flowchart: router -> expert
+    projections -> parameter-space mixing -> one recurrence with the shared transition -> readout).
+
+    X [B,T,D]; init [B,H,N,P] or None; forced_idx [B,T,k] or None (see router).
+    Returns a dict: y [B,T,H,P], final [B,H,N,P] and the stage values (g, dt, idx, w, z, Bpi, Xs,
+    Ct, Cpi) flattened over tokens (row = b*T + t)."""
+    Bsz, T, D = X.shape
+    Xf = X.reshape(Bsz * T, D)
+    fidx = None if forced_idx is None else forced_idx.reshape(Bsz * T, k)
+    g, dt, idx, w = router(Xf, W_r, W_dt, b_dt, k, decision_dtype, fidx)
+    z = expert_proj(Xf, W_exp, idx)
+    Bpi, Xs, Ct, Cpi = mix(z, w, H, P, G, N)
+    y = np.zeros((Bsz, T, H, P))
+    final = np.zeros((Bsz, H, N, P))
+    for b in range(Bsz):
+        r = slice(b * T, (b + 1) * T)
+        y[b], final[b] = scan_sequential(Bpi[r], Xs[r], Ct[r], dt[r], A,
+                                         None if init is None else init[b])
+    return dict(y=y, final=final, g=g, dt=dt, idx=idx, w=w, z=z, Bpi=Bpi, Xs=Xs, Ct=Ct, Cpi=Cpi)
+
+
+def step(Xt, W_r, W_dt, b_dt, A, W_exp, H, P, N, G, k, state, forced_idx=None, decision_dtype=np.float32):
+    """One recurrent decode step per sequence: the layer applied to a single new token X_t [B,D]
+    with the cached state [B,H,N,P] (the recurrence of [notes] key design 1 advanced by one token).
+    Returns (y [B,H,P], new state [B,H,N,P], idx)."""
+    g, dt, idx, w = router(Xt, W_r, W_dt, b_dt, k, decision_dtype, forced_idx)
+    z = expert_proj(Xt, W_exp, idx)
+    Bpi, Xs, Ct, _ = mix(z, w, H, P, G, N)
+    gh = group_of(H, G)
+    a = np.exp(dt * A)                                                  # [B,H]
+    U = np.einsum("bjhn,bjhp->bhnp", Bpi[:, :, gh], Xs)
+    new = a[:, :, None, None] * state + U
+    y = np.einsum("bhn,bhnp->bhp", Ct[:, gh], new)
+    return y, new, idx
