@@ -1,0 +1,363 @@
+"""Benchmark of the Swimba layer forward on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl swimba|reference] [--workload NAME]
+
+A step is one swimba_layer_fwd (router -> dispatch -> expert projections with the fused mix ->
+chunked scan) over one batch of synthetic inputs already resident in HBM.  Default workload: the base
+layer B4 T2048 D768 H24 P64 N128 E8 k2 Q256 (bf16 weights and activations, fp32 state).  With N > 1
+(torchrun) every rank runs its own batch (weak scaling, no data-path collective; the process group only
+carries the barrier and the max-over-ranks of the timings).
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launching stream,
+with a write of 2x the L2 size between steps (outside the events) so every step reads its inputs from
+HBM.  The library's own per-stage events give the dominant kernel's duration for the roofline.
+`--impl reference` times the fp64 CPU oracle (the reference for this layer) on a bounded sample.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from parameter_space_moe_b200 import configs, inputs  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------------ work model
+
+def ssd_flops(w, T=None):
+    """Algorithmic FLOPs of the chunked solve (causal half of the intra-chunk products counted)."""
+    T = T or w.seqlen
+    Q, k, N, P = w.chunk, w.top_k, w.dstate, w.headdim
+    total = 0
+    for c in range(math.ceil(T / Q)):
+        L = min(Q, T - c * Q)
+        tri = L * (L + 1) / 2
+        total += 2 * tri * k * N + 2 * tri * k * P + 2 * N * P * k * L + 2 * L * N * P
+    return total * w.batch * w.nheads
+
+
+def work(w):
+    """Per-step algorithmic FLOPs and bytes of each stage and of the layer."""
+    M, D, E, H, k = w.M, w.d_model, w.n_experts, w.nheads, w.top_k
+    ab = 2 if w.dtype == "bf16" else 4          # activation / weight bytes
+    sb = 2 if w.dtype == "bf16" else 4          # stream bytes (fp16 or fp32)
+    used_experts = E if M * k >= 4 * E else min(E, M * k)
+    gemm_flops = 2.0 * M * k * D * w.W_e
+    streams = M * k * (2 * w.G * w.dstate + H * w.headdim) * sb
+    states = w.batch * H * w.dstate * w.headdim * 4
+    layer_bytes = (M * D * ab + used_experts * w.W_e * D * ab + (E + H) * D * ab + M * H * w.headdim * ab + states)
+    return {
+        "router": {"flops": 2.0 * M * D * (E + H), "bytes": M * D * ab + (E + H) * D * ab + M * (2 * k + H) * 4},
+        "expert_proj_mix": {"flops": gemm_flops, "bytes": M * k * D * ab + used_experts * w.W_e * D * ab + streams},
+        "ssd_scan": {"flops": ssd_flops(w), "bytes": streams + M * H * 4 + M * H * w.headdim * ab + states},
+        "layer": {"flops": 2.0 * M * D * (E + H) + gemm_flops + ssd_flops(w), "bytes": layer_bytes},
+    }
+
+
+# ------------------------------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons through NVML every ~10 ms while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                util = self.nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, util))
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        loaded = [m for m, u in self.samples if u > 0] or [m for m, _ in self.samples]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------ reference arm
+
+def cpu_oracle_sample(w, inp, budget_s=20.0, min_tokens=256):
+    """Time the fp64 oracle on the first batch rows of the workload that fit ~budget_s of CPU work."""
+    from oracle import swimba_oracle as O
+    f = inputs.to_f64
+    wt = [f(inp[k]) for k in ("W_r", "W_dt", "b_dt", "A", "W_exp")]
+    T = w.seqlen if w.seqlen <= min_tokens else min_tokens
+    t0 = time.perf_counter()
+    O.layer_fwd(f(inp["X"][:1, :T]), *wt, w.nheads, w.headdim, w.dstate, w.G, w.top_k)
+    probe = time.perf_counter() - t0
+    per_token = probe / T
+    rows = max(1, min(w.batch, int(budget_s / (per_token * w.seqlen))))
+    if per_token * w.seqlen > budget_s:
+        rows, T = 1, max(T, int(budget_s / per_token))
+    else:
+        T = w.seqlen
+    X = f(inp["X"][:rows, :T])
+    t0 = time.perf_counter()
+    O.layer_fwd(X, *wt, w.nheads, w.headdim, w.dstate, w.G, w.top_k)
+    dt = time.perf_counter() - t0
+    return rows * T / dt, f"{rows} batch row(s) x {T} tokens of {w.name} ({rows * T} tokens), fp64 oracle"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = inputs.make_inputs(w)
+    from oracle import swimba_oracle as O
+    f = inputs.to_f64
+    wt = [f(inp[k]) for k in ("W_r", "W_dt", "b_dt", "A", "W_exp")]
+    T = min(w.seqlen, 256)
+    X = f(inp["X"][:1, :T])
+    for _ in range(args.warmup):
+        O.layer_fwd(X, *wt, w.nheads, w.headdim, w.dstate, w.G, w.top_k)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.layer_fwd(X, *wt, w.nheads, w.headdim, w.dstate, w.G, w.top_k)
+        times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = args.steps * T / tot
+    sample = f"each step: 1 batch row x {T} tokens of {w.name}, fp64 oracle"
+    cores = blas_threads()
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+# ------------------------------------------------------------------------------------------ GPU arm
+
+METRIC = "Swimba layer fwd tokens/s (E=8,k=2,T=2048); % of tensor/HBM roofline"
+
+
+def config_of(w):
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.seqlen, "d_model": w.d_model, "nheads": w.nheads,
+            "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.G, "n_experts": w.n_experts, "top_k": w.top_k,
+            "chunk": w.chunk, "l2": "flushed between steps (2x L2 write outside the timed events)"}
+
+
+def run_gpu(args, w):
+    from parameter_space_moe_b200 import swimba
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    swimba.lib()
+    wr = w.with_(seed=w.seed + 1000 * rank)
+    inp = inputs.make_inputs(wr)
+    d = swimba.dims_of(w)
+    W = swimba.WeightSet(*(inp[k].to(dev) for k in ("W_r", "W_dt", "b_dt", "A", "W_exp")))
+    X = inp["X"].to(dev).reshape(w.M, w.d_model)
+    y = torch.empty(w.M, w.nheads * w.headdim, dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32,
+                    device=dev)
+    fin = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, device=dev)
+    ws = torch.empty(swimba.workspace_size(d), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        swimba.layer_fwd(d, X, W, None, y, fin, None, None, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert swimba.check_device_status() == 0
+    swimba.profile_enable(True)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_ms = {}
+    sampler = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = swimba.launch_count()
+    with sampler:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+            for name, ms in swimba.profile_read():
+                stage_ms[name] = stage_ms.get(name, 0.0) + ms
+        torch.cuda.synchronize()
+    launches = swimba.launch_count() - n0
+    if dist:
+        dist.barrier()
+    swimba.profile_enable(False)
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    assert swimba.check_device_status() == 0
+
+    # end to end through the C ABI: pinned host X in, y back to pinned host, every step
+    Xh = inp["X"].reshape(w.M, w.d_model).pin_memory()
+    yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        X.copy_(Xh, non_blocking=True); step(); yh.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    e2e_ms = 0.0
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e0.record(stream)
+        X.copy_(Xh, non_blocking=True)
+        step()
+        yh.copy_(y, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+
+    t = torch.tensor([total_ms, e2e_ms] + [stage_ms.get(n, 0.0) for n in sorted(stage_ms)], dtype=torch.float64,
+                     device=dev)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = t[0].item(), t[1].item()
+    stage_ms = {n: t[2 + i].item() for i, n in enumerate(sorted(stage_ms))}
+    if rank == 0:
+        report(args, w, world, total_ms, e2e_ms, stage_ms, launches, sampler.summary(),
+               Xh.numel() * Xh.element_size(), yh.numel() * yh.element_size(), inp)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def report(args, w, world, total_ms, e2e_ms, stage_ms, launches, clocks, h2d, d2h, inp):
+    peaks, src = load_peaks()
+    wk = work(w)
+    K = args.steps
+    tokens = w.M * world * K
+    value = tokens / (total_ms / 1e3)
+    # dominant kernel stage and its roofline
+    dom = max(stage_ms, key=stage_ms.get)
+    avg_s = stage_ms[dom] / K / 1e3
+    bound = "tensor" if dom == "expert_proj_mix" else "hbm"
+    if bound == "tensor":
+        achieved = wk[dom]["flops"] / avg_s / 1e12
+        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+        peak_note = f"bf16 dense, burst, {src}"
+    else:
+        achieved = wk[dom]["bytes"] / avg_s / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+        peak_note = f"HBM copy, {src}"
+    layer_roof_s = max(wk["layer"]["flops"] / (peaks["bf16_tflops"] * 1e12), wk["layer"]["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic", "config": config_of(w),
+        "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": None, "peak_source": peak_note,
+                     "algorithmic": wk[dom]["flops"] if bound == "tensor" else wk[dom]["bytes"]},
+        "layer_roofline": {"time_us": layer_roof_s * 1e6, "frac": layer_roof_s / (total_ms / K / 1e3),
+                           "flops": wk["layer"]["flops"], "bytes": wk["layer"]["bytes"]},
+        "stages_ms_per_step": {n: v / K for n, v in stage_ms.items()},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, sample = cpu_oracle_sample(w, inp)
+        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                               "sample": sample}
+    print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="swimba", choices=["swimba", "reference"])
+    ap.add_argument("--workload", default=configs.BASE.name, choices=sorted(configs.ALL))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = configs.ALL[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

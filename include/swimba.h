@@ -1,0 +1,174 @@
+/*
+ * swimba.h -- C ABI of libswimba.so: the forward pass of one Swimba (Switch Mamba) token-mixer layer
+ * on an NVIDIA B200 (sm_100a).
+ *
+ * The method ("Swimba: Switch Mamba Model Scales State Space Models", arXiv 2603.06938; the
+ * papernotes.org NeurIPS 2026 notes, Method, key design 1, and the gist.science Technical Summary,
+ * section 2 "Architecture Details"):
+ *   router        g_t = W_r X_t,  K_t = top-k of g_t,  pi_t = softmax over K_t (renormalised)
+ *   experts       z_t^(e) = W_exp[e] X_t, split into x^(e) (H x P), B^(e) (G x N), C^(e) (G x N)
+ *   mixing        U~_t = sum_{e in K_t} pi_te B^(e) x^(e)T,   C~_t = sum_{e in K_t} pi_te C^(e)
+ *   recurrence    h_t = a_t h_{t-1} + U~_t,  y_t = C~_t^T h_t,  a_t = exp(dt_t A_h) shared by all experts
+ *   dt            dt_t,h = clamp(softplus(W_dt[h] . X_t + b_dt[h]), 1e-3, 0.1)
+ *
+ * Conventions for every entry point
+ *  - Every pointer is caller-owned DEVICE memory unless stated; the library allocates nothing.
+ *  - Tensors are dense, row-major (last index fastest) and 16-byte aligned.
+ *  - M = batch * seqlen tokens; row m = b * seqlen + t.  W_e = H*P + 2*G*N.
+ *  - dtype (swimba_dims.dtype) is the type of X, of the three weight matrices and of y.  dt, topk_w,
+ *    b_dt, A and every SSM state are fp32.  The mixed streams (Bpi, Xs, Cpi) use the "stream dtype"
+ *    (swimba_stream_dtype): fp32 when dtype is F32, fp16 when dtype is BF16 (fp16 keeps 11 bits,
+ *    which the 2e-3 accuracy budget of bf16 outputs needs; bf16 streams would not meet it).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).  SWIMBA_OK
+ *    means "validated and launched".  Device-side conditions (a bounded wait that gave up, an
+ *    intermediate that left the fp16 range) are recorded in a sticky per-device status word and
+ *    read with swimba_check_device_status.  No C++ exception crosses this boundary.
+ *  - Invalid arguments return an error before anything is launched; unsupported shapes return
+ *    SWIMBA_ERR_UNSUPPORTED (there is no fallback path).
+ *  - Supported shapes: N, P in {16, 32, 64, 128}; chunk in {64, 128, 256}; 1 <= top_k <= min(E, 8);
+ *    E <= 64; G divides H; d_model a multiple of 64 (bf16) or 8 (fp32); every size >= 1.
+ */
+#ifndef SWIMBA_H_
+#define SWIMBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SWIMBA_OK = 0,
+  SWIMBA_ERR_INVALID_ARG = 1,  /* null or misaligned pointer, non-positive size, inconsistent dims */
+  SWIMBA_ERR_UNSUPPORTED = 2,  /* valid but outside the supported shapes listed above */
+  SWIMBA_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+  SWIMBA_ERR_WORKSPACE = 4,    /* ws is NULL or smaller than swimba_workspace_size() */
+  SWIMBA_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up (read via swimba_check_device_status) */
+  SWIMBA_ERR_RANGE = 6         /* device: a mixed-stream value did not fit the stream dtype */
+} swimba_status;
+
+typedef enum { SWIMBA_F32 = 0, SWIMBA_BF16 = 1, SWIMBA_F16 = 2 } swimba_dtype;
+
+typedef struct {
+  int32_t batch;      /* B: independent sequences */
+  int32_t seqlen;     /* T: tokens per sequence (1 for swimba_step) */
+  int32_t d_model;    /* D: width of X */
+  int32_t nheads;     /* H */
+  int32_t headdim;    /* P: width of x per head and of y per head */
+  int32_t dstate;     /* N: state dimension (width of B and C) */
+  int32_t ngroups;    /* G: heads h share the B/C of group h / (H/G); G = H gives every head its own */
+  int32_t n_experts;  /* E */
+  int32_t top_k;      /* k: active experts per token */
+  int32_t chunk;      /* Q: SSD chunk length */
+  int32_t dtype;      /* swimba_dtype of X, weights and y: SWIMBA_F32 or SWIMBA_BF16 */
+} swimba_dims;
+
+typedef struct {
+  const void* w_router;  /* [E][D] dtype: router logits g = W_r X */
+  const void* w_dt;      /* [H][D] dtype: shared dt projection */
+  const float* b_dt;     /* [H] fp32 */
+  const float* A;        /* [H] fp32, negative: a_t = exp(dt_t A_h) */
+  const void* w_exp;     /* [E][W_e][D] dtype: expert projections, rows [x: H*P | B: G*N | C: G*N] */
+} swimba_weights;
+
+/* Bytes of workspace that every entry point taking `ws` needs for these dims (0 if the dims are
+ * invalid or unsupported).  The workspace is scratch owned by the caller; its contents need no
+ * initialisation and are overwritten by each call.  Calls that share a workspace must not overlap. */
+size_t swimba_workspace_size(const swimba_dims* dims);
+
+/* Stream dtype of the mixed streams for these dims: SWIMBA_F32 or SWIMBA_F16 (-1 if invalid). */
+int swimba_stream_dtype(const swimba_dims* dims);
+
+/* Router and dt (one launch).  Paper: notes, Method, flowchart "token router R(X_t)" and key
+ * design 1 (pi_t = softmax(g_t), active set K_t).
+ *   X        [M][D] dtype
+ *   topk_idx [M][k] int32 out: expert indices, largest logit first, equal logits -> lower index
+ *   topk_w   [M][k] fp32 out: renormalised softmax weights over the k winners (sum to 1)
+ *   dt       [M][H] fp32 out: clamp(softplus(W_dt X + b_dt), 1e-3, 0.1)
+ * Logits are accumulated in fp32; the top-k decision is taken on those fp32 values. */
+swimba_status swimba_router_topk(const swimba_dims* dims, const void* X, const swimba_weights* w,
+                                 int32_t* topk_idx, float* topk_w, float* dt, void* stream);
+
+/* Expert dispatch: a stable counting sort of the M*k (token, slot) pairs by expert (the token-level
+ * routing the notes' efficiency discussion attributes Swimba's extra cost to).
+ *   topk_idx       [M][k] int32 in
+ *   expert_offsets [E+1] int32 out: pairs of expert e are perm[expert_offsets[e] .. expert_offsets[e+1])
+ *   perm           [M*k] int32 out: value m*k + j, in increasing m within each expert */
+swimba_status swimba_dispatch(const swimba_dims* dims, const int32_t* topk_idx, int32_t* expert_offsets,
+                              int32_t* perm, void* ws, size_t ws_bytes, void* stream);
+
+/* Expert projections of the active experts, unmixed (a stage probe; the fused path never writes them).
+ * Paper: notes, key design 1 ("each expert applies its own linear projection to X_t").
+ *   Z [M][k][W_e] fp32 out: Z[m][j] = W_exp[topk_idx[m][j]] X_m, accumulated in fp32. */
+swimba_status swimba_expert_proj(const swimba_dims* dims, const void* X, const swimba_weights* w,
+                                 const int32_t* topk_idx, float* Z, void* ws, size_t ws_bytes, void* stream);
+
+#define SWIMBA_MIX_UNSCALED_B 1 /* flag: write B unscaled (the separated design's injection) */
+
+/* Parameter-space mixing of unmixed projections (a stage probe of the epilogue the fused path runs).
+ * Paper: notes, key design 1, first display equation.  U~ is kept factored per slot:
+ *   Bpi [M][k][G][N] stream dtype out: pi_mj B^(j)  (B^(j) itself with SWIMBA_MIX_UNSCALED_B)
+ *   Xs  [M][k][H][P] stream dtype out: x^(j)
+ *   Cpi [M][k][G][N] stream dtype out: pi_mj C^(j)    (so C~_m = sum_j Cpi[m][j])
+ * Values outside the stream dtype's range set SWIMBA_ERR_RANGE in the device status word. */
+swimba_status swimba_mix(const swimba_dims* dims, const float* Z, const float* topk_w, int32_t flags,
+                         void* Bpi, void* Xs, void* Cpi, void* stream);
+
+/* The single shared-transition recurrence over the mixed streams, solved by chunks of `chunk` tokens.
+ * Paper: notes, key design 1, second display equation; overall framework (chunked SSD, reused as is).
+ *   Bpi, Xs, Cpi  as written by swimba_mix; dt [M][H] fp32; A [H] fp32
+ *   init_state    [B][H][N][P] fp32 or NULL (zero initial state)
+ *   y             [M][H][P] dtype out
+ *   final_state   [B][H][N][P] fp32 out, or NULL
+ *   chunk_states  [B][H][nc][N][P] fp32 out (state before each chunk, nc = ceil(T/chunk)), or NULL */
+swimba_status swimba_ssd_scan(const swimba_dims* dims, const void* Bpi, const void* Xs, const void* Cpi,
+                              const float* dt, const float* A, const float* init_state, void* y,
+                              float* final_state, float* chunk_states, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer: router -> dispatch -> expert projections with the mix fused into their epilogue
+ * -> chunked scan.  Paper: notes, Method flowchart.
+ *   X [M][D] dtype; init_state [B][H][N][P] fp32 or NULL; y [M][H][P] dtype out;
+ *   final_state [B][H][N][P] fp32 out or NULL; topk_idx_out [M][k] / topk_w_out [M][k] or NULL. */
+swimba_status swimba_layer_fwd(const swimba_dims* dims, const void* X, const swimba_weights* w,
+                               const float* init_state, void* y, float* final_state, int32_t* topk_idx_out,
+                               float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
+
+/* One recurrent decode step (dims.seqlen must be 1): each of `batch` sequences takes one token.
+ *   X [B][D] dtype; state [B][H][N][P] fp32, updated in place (h <- a h + U~); y [B][H][P] dtype out;
+ *   topk_idx_out [B][k] or NULL. */
+swimba_status swimba_step(const swimba_dims* dims, const void* X, const swimba_weights* w, float* state,
+                          void* y, int32_t* topk_idx_out, void* ws, size_t ws_bytes, void* stream);
+
+/* The separated-trajectory contrast design restricted to the active slots ("k scans"): slot j keeps
+ * its own state, driven by the unscaled injection B^(j) x^(j)T and read out with pi_j C^(j):
+ *   h^(j)_t = a_t h^(j)_{t-1} + B_tj x_tj^T,   y_t = sum_j Cpi_tj^T h^(j)_t.
+ * Paper: notes, key design 1 (separated SSMs cost O(T E C_step)) and the efficiency table.
+ *   B [M][k][G][N] (swimba_mix with SWIMBA_MIX_UNSCALED_B), Xs, Cpi, dt, A as for swimba_ssd_scan
+ *   init_states [k][B][H][N][P] fp32 or NULL; y [M][H][P] dtype out; final_states same shape or NULL. */
+swimba_status swimba_separated_scan(const swimba_dims* dims, const void* B, const void* Xs, const void* Cpi,
+                                    const float* dt, const float* A, const float* init_states, void* y,
+                                    float* final_states, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the current device's status word: SWIMBA_OK,
+ * SWIMBA_ERR_TIMEOUT or SWIMBA_ERR_RANGE (SWIMBA_ERR_CUDA if the stream reports an error).  The word
+ * is sticky: it collects every flag raised on this device since the previous check. */
+swimba_status swimba_check_device_status(void* stream);
+
+/* Profiling support.  swimba_profile_enable(1) makes every later entry-point call record a CUDA
+ * event on its stream after each kernel stage; swimba_profile_read then waits for the most recent
+ * call's events and writes up to `max` stage names (static strings) and durations in milliseconds,
+ * returning the number of stages (-1 on a CUDA error).  swimba_launch_count returns the number of
+ * kernels this library has launched in the process so far (all devices). */
+swimba_status swimba_profile_enable(int enable);
+int swimba_profile_read(const char** names, float* ms, int max);
+long long swimba_launch_count(void);
+
+/* Static, human-readable name of a status code. */
+const char* swimba_status_string(swimba_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWIMBA_H_ */

@@ -1,0 +1,138 @@
+// Shared device/host helpers of libswimba (internal; not part of the C ABI).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "swimba.h"
+
+namespace swimba {
+
+// Bits of the workspace status word.
+enum : unsigned { ST_TIMEOUT = 1u, ST_RANGE = 2u };
+
+// Largest finite fp16 value: mixed streams stored as fp16 must stay below it.
+constexpr float kF16Max = 65504.f;
+
+// Layer dimensions in the form the kernels use.
+struct Dims {
+  int Bsz, T, D, H, P, N, G, E, k, Q;
+  int M;    // Bsz * T
+  int HP;   // H * P
+  int GN;   // G * N
+  int We;   // HP + 2 * GN
+  int nc;   // chunks per sequence
+  int hpg;  // heads per group
+  int dtype;
+};
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_f32(__half v) { return __half2float(v); }
+
+template <class T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
+
+// True when v cannot be stored in T without overflow (fp16 only; fp32 streams take any value).
+template <class T>
+__device__ __forceinline__ bool out_of_range(float v) { return false; }
+template <>
+__device__ __forceinline__ bool out_of_range<__half>(float v) { return !(fabsf(v) <= kF16Max); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------------------------
+// Workspace layout (every region 256-byte aligned).  The same plan serves every entry point.
+struct WsPlan {
+  size_t status;      // unsigned status word
+  size_t topk_idx;    // int32 [M][k]
+  size_t topk_w;      // f32 [M][k]
+  size_t dt;          // f32 [M][H]
+  size_t dcounts;     // int32 [ndt][E]  per dispatch tile expert counts
+  size_t dbase;       // int32 [ndt][E]  first sorted position of each (tile, expert)
+  size_t offsets;     // int32 [E+1]
+  size_t perm;        // int32 [M*k]
+  size_t tiles;       // int32 [max_tiles][2]  GEMM row-tile schedule (expert, first sorted row)
+  size_t ntiles;      // int32 [1]
+  size_t xsorted;     // dtype [M*k][D] rows of X in sorted (expert-major) order
+  size_t bpi, xs, cpi;  // stream dtype mixed streams
+  size_t yintra;      // f32 [M][H][P]
+  size_t ysum;        // f32 [M][H][P]  separated-scan accumulator
+  size_t schunk;      // f32 [B][H][nc][N][P]  chunk-local end states
+  size_t hstart;      // f32 [B][H][nc][N][P]  state before each chunk
+  size_t cslast;      // f32 [B][H][nc]        total log-decay of each chunk
+  size_t flags;       // unsigned [B][H][nc]  chained-scan hand-off flags
+  size_t total;
+};
+
+constexpr int kDispatchTile = 1024;  // (token, slot) pairs per dispatch CTA
+constexpr int kRowTile = 128;        // GEMM row tile of the schedule
+
+inline int max_row_tiles(const Dims& d) { return ceil_div(d.M * d.k, kRowTile) + d.E; }
+inline int dispatch_tiles(const Dims& d) { return ceil_div(d.M * d.k, kDispatchTile); }
+
+size_t elem_bytes(int dtype);
+int stream_dtype_of(int dtype);
+WsPlan plan_workspace(const Dims& d);
+
+// ---------------------------------------------------------------------------------------------
+// Kernel launchers (defined in the .cu files next to their kernels).  All return cudaError_t of the
+// launch; `st` is the workspace status word.
+cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
+                          float* dt, unsigned* st, cudaStream_t s);
+cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
+                            int32_t* perm, cudaStream_t s);
+cudaError_t launch_gather_rows(const Dims& d, const void* X, const int32_t* perm, void* xsorted, cudaStream_t s);
+// mode 0: fused mix (pi-scaled B and C), 1: fused mix with unscaled B, 2: raw Z (fp32)
+cudaError_t launch_proj_simt(const Dims& d, const void* X, const void* w_exp, const int32_t* perm,
+                             const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets,
+                             const float* topk_w, int mode, void* bpi, void* xs, void* cpi, float* Z, unsigned* st,
+                             cudaStream_t s);
+// Tensor-core version (bf16 X and weights, fp16 streams): A operand is xsorted (rows in expert order).
+cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int32_t* perm,
+                           const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, const float* topk_w,
+                           int mode, void* bpi, void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s);
+cudaError_t launch_mix(const Dims& d, const float* Z, const float* topk_w, int flags, void* bpi, void* xs, void* cpi,
+                       unsigned* st, cudaStream_t s);
+// Chunked scan.  Slot ranges select which of the k per-token keys feed one trajectory and which
+// readouts form C~: the mixed scan uses all k slots in one trajectory; the separated scan runs one
+// slot per pass.
+struct ScanArgs {
+  const void* bpi; const void* xs; const void* cpi;  // streams, [M][k][...]
+  const float* dt; const float* A;
+  const float* init;  // [B][H][N][P] or null
+  void* y;            // [M][H][P] out dtype
+  bool accumulate_y;  // add into y (fp32 accumulator in yintra) instead of overwriting
+  float* final_state; // or null
+  float* hstart;      // [B][H][nc][N][P]
+  float* schunk; float* cslast;
+  float* yacc;        // [M][H][P] fp32: intra-chunk outputs
+  float* ysum;        // [M][H][P] fp32: running sum over the separated design's trajectories
+  int key_slot0;      // first slot used as a key
+  int key_slots;      // number of key slots (k for the mixed scan, 1 for a separated trajectory)
+  int read_slot0;     // first slot summed into the readout C~
+  int read_slots;     // number of readout slots
+  bool first_pass;    // separated scan: first slot initialises the fp32 accumulator
+  bool last_pass;     // separated scan: last slot converts the accumulator to y
+};
+cudaError_t launch_scan_simt(const Dims& d, const ScanArgs& a, cudaStream_t s);
+cudaError_t launch_step_update(const Dims& d, const void* bpi, const void* xs, const void* cpi, const float* dt,
+                               const float* A, float* state, void* y, cudaStream_t s);
+// Adds n to the library's launch counter (every launcher reports the kernels it issued).
+void count_launches(int n);
+
+}  // namespace swimba

@@ -1,0 +1,134 @@
+// Expert dispatch: a stable counting sort of the M*k (token, slot) pairs by expert, plus the row-tile
+// schedule of the grouped expert GEMM and the gather of X rows into expert-major order.
+//
+// Pair p = m*k + j (token m, slot j) has expert topk_idx[p].  Three launches:
+//   count    one CTA per tile of kDispatchTile consecutive pairs: per-expert counts of the tile
+//   offsets  one CTA: expert_offsets (exclusive prefix of the totals), each (tile, expert)'s first
+//            sorted position, and the GEMM schedule (expert, first row) of kRowTile-row tiles
+//   scatter  one CTA per tile: stable rank of each pair inside its tile (warp match + per-warp
+//            prefix), perm[position] = p
+// The order inside an expert is increasing p, so the permutation is deterministic.
+#include "common.cuh"
+
+namespace swimba {
+
+constexpr int kDispatchThreads = 1024;
+
+__global__ void __launch_bounds__(kDispatchThreads)
+dispatch_count_kernel(Dims d, const int32_t* __restrict__ idx, int32_t* __restrict__ counts) {
+  __shared__ int c_s[64];
+  const int tile = blockIdx.x;
+  if (threadIdx.x < 64) c_s[threadIdx.x] = 0;
+  __syncthreads();
+  const int total = d.M * d.k;
+  for (int i = threadIdx.x; i < kDispatchTile; i += blockDim.x) {
+    int p = tile * kDispatchTile + i;
+    if (p < total) atomicAdd(&c_s[idx[p]], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x < d.E) counts[tile * d.E + threadIdx.x] = c_s[threadIdx.x];
+}
+
+__global__ void __launch_bounds__(1024)
+dispatch_offsets_kernel(Dims d, int ntile, const int32_t* __restrict__ counts, int32_t* __restrict__ base,
+                        int32_t* __restrict__ offsets, int32_t* __restrict__ tiles, int32_t* __restrict__ ntiles) {
+  __shared__ int tot_s[65];
+  __shared__ int off_s[65];
+  __shared__ int toff_s[65];
+  const int e = threadIdx.x;
+  if (e < d.E) {
+    int t = 0;
+    for (int i = 0; i < ntile; ++i) t += counts[i * d.E + e];
+    tot_s[e] = t;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int o = 0, to = 0;
+    for (int x = 0; x < d.E; ++x) {
+      off_s[x] = o; toff_s[x] = to;
+      o += tot_s[x]; to += ceil_div(tot_s[x], kRowTile);
+    }
+    off_s[d.E] = o; toff_s[d.E] = to;
+    *ntiles = to;
+  }
+  __syncthreads();
+  if (e <= d.E) offsets[e] = off_s[e];
+  if (e < d.E) {
+    int o = off_s[e];
+    for (int i = 0; i < ntile; ++i) { base[i * d.E + e] = o; o += counts[i * d.E + e]; }
+  }
+  // GEMM schedule: tile r of expert e covers sorted rows [off + r*kRowTile, min(off_{e+1}, ...))
+  for (int x = 0; x < d.E; ++x) {
+    const int nt = ceil_div(tot_s[x], kRowTile);
+    for (int r = threadIdx.x; r < nt; r += blockDim.x) {
+      tiles[2 * (toff_s[x] + r) + 0] = x;
+      tiles[2 * (toff_s[x] + r) + 1] = off_s[x] + r * kRowTile;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kDispatchThreads)
+dispatch_scatter_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* __restrict__ base,
+                        int32_t* __restrict__ perm) {
+  __shared__ int wc_s[kDispatchThreads / 32][64];  // per-warp counts, turned into per-warp bases
+  const int tile = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = d.M * d.k;
+  for (int x = threadIdx.x; x < (kDispatchThreads / 32) * 64; x += blockDim.x) (&wc_s[0][0])[x] = 0;
+  __syncthreads();
+  const int p = tile * kDispatchTile + threadIdx.x;  // kDispatchTile == blockDim.x
+  const bool valid = p < total;
+  const int e = valid ? idx[p] : -1 - lane;          // distinct sentinels never match a real expert
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  if (valid && rank == 0) wc_s[warp][e] = __popc(peers);
+  __syncthreads();
+  if (threadIdx.x < d.E) {
+    int run = base[tile * d.E + threadIdx.x];
+    for (int w = 0; w < kDispatchThreads / 32; ++w) {
+      int c = wc_s[w][threadIdx.x];
+      wc_s[w][threadIdx.x] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  if (valid) perm[wc_s[warp][e] + rank] = p;
+}
+
+// X rows in sorted order: xsorted[r] = X[perm[r] / k].  One warp per row, 16-byte vectors.
+template <class T>
+__global__ void gather_rows_kernel(Dims d, const T* __restrict__ X, const int32_t* __restrict__ perm,
+                                   T* __restrict__ xs) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= d.M * d.k) return;
+  const int m = perm[warp] / d.k;
+  const int4* src = reinterpret_cast<const int4*>(X + (size_t)m * d.D);
+  int4* dst = reinterpret_cast<int4*>(xs + (size_t)warp * d.D);
+  const int nv = d.D * (int)sizeof(T) / 16;
+  for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+}
+
+cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
+                            int32_t* perm, cudaStream_t s) {
+  const int nt = dispatch_tiles(d);
+  int32_t* counts = (int32_t*)(ws + p.dcounts);
+  int32_t* base = (int32_t*)(ws + p.dbase);
+  dispatch_count_kernel<<<nt, kDispatchThreads, 0, s>>>(d, idx, counts);
+  dispatch_offsets_kernel<<<1, 1024, 0, s>>>(d, nt, counts, base, offsets, (int32_t*)(ws + p.tiles),
+                                             (int32_t*)(ws + p.ntiles));
+  dispatch_scatter_kernel<<<nt, kDispatchThreads, 0, s>>>(d, idx, base, perm);
+  count_launches(3);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const Dims& d, const void* X, const int32_t* perm, void* xsorted, cudaStream_t s) {
+  const int rows = d.M * d.k;
+  dim3 grid(ceil_div(rows, 8));
+  if (d.dtype == SWIMBA_BF16)
+    gather_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(d, (const __nv_bfloat16*)X, perm, (__nv_bfloat16*)xsorted);
+  else
+    gather_rows_kernel<float><<<grid, 256, 0, s>>>(d, (const float*)X, perm, (float*)xsorted);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace swimba

@@ -1,0 +1,263 @@
+// Grouped expert projection on the 5th-generation tensor cores, with the parameter-space mix fused into
+// the epilogue (bf16 inputs, fp32 accumulation in TMEM, fp16 streams out).
+//
+// Paper: Swimba notes, key design 1 -- every active expert e projects X_t into its candidate streams
+// (x^(e), B^(e), C^(e)) which are mixed with the router weights before the single recurrence:
+//   Xs[m][j] = x^(j),   Bpi[m][j] = pi_mj B^(j),   Cpi[m][j] = pi_mj C^(j).
+// The notes name a fused MoE operator for this input projection as the way to avoid HBM round trips of
+// router outputs and parameter slices; here the per-expert output tile never leaves the SM unmixed.
+//
+// Design (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: A = 128 gathered X rows x 64 K (16 KB), B = 256 weight rows x 64 K (32 KB)
+//               per stage, 128-byte swizzle, kStages-deep ring of mbarriers
+//   warp 1      TMEM owner and MMA issuer: 4 x tcgen05.mma M128 N256 K16 per stage into one of two
+//               256-column fp32 accumulators (double buffered: 512 TMEM columns)
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time (warp w reads TMEM lanes 32*(w%4)..), scales
+//               B and C columns by pi, converts to fp16 and stores to the destination (token, slot) row
+// Tiles: (row tile of one expert's sorted rows) x (256 output columns), handed out round-robin.
+#include "tc_common.cuh"
+
+namespace swimba {
+
+namespace {
+constexpr int BM = 128, BN = 256, BK = 64, kStages = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t kStageA = BM * BK * 2, kStageB = BN * BK * 2, kStageBytes = kStageA + kStageB;
+constexpr uint32_t kTmemCols = 2 * BN;
+constexpr uint32_t kIdesc = tc::idesc_f16(BM, BN, /*bf16=*/true);
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 256;
+
+struct TcArgs {
+  Dims d;
+  const int32_t* perm;
+  const int32_t* tiles;
+  const int32_t* ntiles;
+  const int32_t* offsets;
+  const float* topk_w;
+  int mode;  // 0 mix, 1 mix with unscaled B, 2 raw fp32 Z
+  __half* bpi;
+  __half* xs;
+  __half* cpi;
+  float* Z;
+  unsigned* st;
+};
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+// Write the 32 accumulator values of one row (columns c0 .. c0+31 of z = [x | B | C]) to their stream.
+__device__ __forceinline__ void store_chunk(const TcArgs& a, int p, float pi, int c0, const uint32_t (&r)[32],
+                                           bool& range_bad) {
+  const Dims& d = a.d;
+  if (a.mode == 2) {
+    float* dst = a.Z + (size_t)p * d.We + c0;
+    if (c0 + 32 <= d.We) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4*>(dst + i) = make_float4(u2f(r[i]), u2f(r[i + 1]), u2f(r[i + 2]), u2f(r[i + 3]));
+    } else {
+      for (int i = 0; i < 32 && c0 + i < d.We; ++i) dst[i] = u2f(r[i]);
+    }
+    return;
+  }
+  const int HP = d.HP, GN = d.GN;
+  auto stream_of = [&](int c) { return c < HP ? 0 : (c < HP + GN ? 1 : 2); };
+  const int s0 = stream_of(c0);
+  if (c0 + 32 <= d.We && stream_of(c0 + 31) == s0) {
+    __half* dst;
+    float sc;
+    if (s0 == 0) { dst = a.xs + (size_t)p * HP + c0; sc = 1.f; }
+    else if (s0 == 1) { dst = a.bpi + (size_t)p * GN + (c0 - HP); sc = a.mode == 1 ? 1.f : pi; }
+    else { dst = a.cpi + (size_t)p * GN + (c0 - HP - GN); sc = pi; }
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      uint4 v;
+      uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float f0 = sc * u2f(r[i + 2 * q]), f1 = sc * u2f(r[i + 2 * q + 1]);
+        range_bad |= !(fabsf(f0) <= kF16Max) || !(fabsf(f1) <= kF16Max);
+        __half2 h = __floats2half2_rn(f0, f1);
+        w[q] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      *reinterpret_cast<uint4*>(dst + i) = v;
+    }
+    return;
+  }
+  for (int i = 0; i < 32; ++i) {
+    const int c = c0 + i;
+    if (c >= d.We) break;
+    const int s = stream_of(c);
+    const float v = u2f(r[i]);
+    float o;
+    __half* dst;
+    if (s == 0) { o = v; dst = a.xs + (size_t)p * HP + c; }
+    else if (s == 1) { o = a.mode == 1 ? v : pi * v; dst = a.bpi + (size_t)p * GN + (c - HP); }
+    else { o = pi * v; dst = a.cpi + (size_t)p * GN + (c - HP - GN); }
+    range_bad |= !(fabsf(o) <= kF16Max);
+    *dst = __float2half_rn(o);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* full = bars;                 // [kStages]  TMA -> MMA
+  uint64_t* empty = bars + kStages;      // [kStages]  MMA -> TMA
+  uint64_t* acc_full = bars + 2 * kStages;       // [2]  MMA -> epilogue
+  uint64_t* acc_empty = bars + 2 * kStages + 2;  // [2]  epilogue -> MMA
+  uint64_t* drain = bars + 2 * kStages + 4;      // MMA completion before teardown
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Dims& d = a.d;
+  const int nct = ceil_div(d.We, BN);
+  const int nkb = d.D / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&acc_full[b], 1); tc::mbar_init(&acc_empty[b], 128); }
+    tc::mbar_init(drain, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+    tc::tma_prefetch_desc(&tmap_a);
+    tc::tma_prefetch_desc(&tmap_b);
+  }
+  if (warp == 1) { tc::tmem_alloc(tmem_slot, kTmemCols); tc::tmem_relinquish(); }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int total = *a.ntiles * nct;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    long long issued = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int rt = t / nct, ct = t % nct;
+      const int e = a.tiles[2 * rt], row0 = a.tiles[2 * rt + 1];
+      const int wrow = e * d.We + ct * BN;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+        uint8_t* sa = stage_base + stage * kStageBytes;
+        tc::mbar_arrive_expect_tx(&full[stage], kStageBytes);
+        tc::tma_load_2d(sa, &tmap_a, &full[stage], kb * BK, row0);
+        tc::tma_load_2d(sa + kStageA, &tmap_b, &full[stage], kb * BK, wrow);
+        ++issued;
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok) { *abort_flag = 1; atomicOr(a.st, ST_TIMEOUT); }
+    // make sure every copy this CTA issued has landed before the CTA can exit
+    for (long long i = 0; i < kStages && i < issued; ++i) {
+      if (--stage < 0) { stage = kStages - 1; phase ^= 1u; }
+      volatile int never = 0;
+      tc::mbar_wait(&full[stage], phase, &never);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int buf = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      if (!tc::mbar_wait(&acc_empty[buf], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+      tc::fence_after_sync();
+      const uint32_t dt = tmem + (uint32_t)(buf * BN);
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!tc::mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t sa = tc::smem_u32(stage_base + stage * kStageBytes);
+        const uint32_t sb = sa + kStageA;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          tc::mma_f16(dt, tc::sdesc_kmajor_sw128(sa + kk * 32), tc::sdesc_kmajor_sw128(sb + kk * 32), kIdesc,
+                      (kb | kk) != 0);
+        }
+        tc::mma_commit(&empty[stage]);
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      tc::mma_commit(&acc_full[buf]);
+      if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
+    }
+    if (!ok) { *abort_flag = 1; atomicOr(a.st, ST_TIMEOUT); }
+    tc::mma_commit(drain);
+    volatile int never = 0;
+    tc::mbar_wait(drain, 0, &never);
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_local = 32 * q + lane;
+    int buf = 0;
+    uint32_t acc_phase = 0;
+    bool range_bad = false;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const int rt = t / nct, ct = t % nct;
+      const int e = a.tiles[2 * rt], row0 = a.tiles[2 * rt + 1];
+      const int rg = row0 + row_local;
+      const bool valid = rg < a.offsets[e + 1];
+      const int p = valid ? a.perm[rg] : 0;
+      const float pi = (valid && a.mode != 2) ? a.topk_w[p] : 0.f;
+      if (!tc::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) {
+        *abort_flag = 1;
+        atomicOr(a.st, ST_TIMEOUT);
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tc::tmem_ld_32x32b_x32(taddr + 32 * c, r);
+        tc::tmem_ld_wait();
+        const int c0 = ct * BN + 32 * c;
+        if (valid && c0 < d.We) store_chunk(a, p, pi, c0, r, range_bad);
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(&acc_empty[buf]);
+      if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
+    }
+    if (range_bad) atomicOr(a.st, ST_RANGE);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+// Host side --------------------------------------------------------------------------------------
+cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int32_t* perm,
+                           const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, const float* topk_w,
+                           int mode, void* bpi, void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s) {
+  CUtensorMap ta, tb;
+  if (!encode_tmap_2d(&ta, xsorted, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.M * d.k, (uint64_t)d.D * 2, BK, BM))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(&tb, w_exp, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.E * d.We, (uint64_t)d.D * 2, BK, BN))
+    return cudaErrorInvalidValue;
+  TcArgs a{d, perm, tiles, ntiles, offsets, topk_w, mode, (__half*)bpi, (__half*)xs, (__half*)cpi, Z, st};
+  cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int max_tiles = max_row_tiles(d) * ceil_div(d.We, BN);
+  const int grid = max_tiles < sms ? max_tiles : sms;
+  proj_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace swimba

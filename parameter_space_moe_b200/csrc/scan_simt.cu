@@ -1,0 +1,165 @@
+// Chunked solve of the single shared-transition recurrence, CUDA-core (SIMT) version.  It serves the
+// fp32 layer and is the reference-grade scan the tensor-core scan is checked against.
+//
+// Paper: Swimba notes, key design 1 (h_t = a_t h_{t-1} + U~_t, y_t = C~_t^T h_t) solved with the
+// chunked SSD decomposition the notes' overall framework reuses.  With cs_t the running sum of
+// dt*A from the chunk start (inclusive):
+//   chunk kernel   y_intra[t] = sum_{s<=t} exp(cs_t - cs_s) sum_j (C~_t . Bpi_sj) Xs_sj
+//                  S_c        = sum_s exp(cs_end - cs_s) sum_j Bpi_sj Xs_sj^T
+//   pass kernel    H_0 = init or 0,  H_{c+1} = exp(cs_end_c) H_c + S_c     (sequential in c)
+//   output kernel  y[t] = y_intra[t] + exp(cs_t) C~_t^T H_c
+// Keys and readouts are selected by slot ranges so one code path also runs each trajectory of the
+// separated design.
+#include "common.cuh"
+
+namespace swimba {
+
+constexpr int kScanThreads = 256;
+
+// cs[i] = sum_{r<=i} dt_r A_h for the L tokens of the chunk (sequential; L <= 256).
+__device__ __forceinline__ void chunk_cumsum(const Dims& d, const float* dt, float A, int b, int h, int t0, int L,
+                                             float* cs) {
+  if (threadIdx.x == 0) {
+    float run = 0.f;
+    for (int i = 0; i < L; ++i) {
+      run += dt[(size_t)(b * d.T + t0 + i) * d.H + h] * A;
+      cs[i] = run;
+    }
+  }
+}
+
+template <class S>
+__device__ __forceinline__ void load_readout(const Dims& d, const S* cpi, int slot0, int nslots, int b, int g, int t0,
+                                             int L, float* Ct) {
+  for (int x = threadIdx.x; x < L * d.N; x += blockDim.x) {
+    const int i = x / d.N, n = x % d.N;
+    const size_t m = (size_t)b * d.T + t0 + i;
+    float v = 0.f;
+    for (int j = slot0; j < slot0 + nslots; ++j) v += to_f32(cpi[(m * d.k + j) * d.GN + (size_t)g * d.N + n]);
+    Ct[x] = v;
+  }
+}
+
+template <class S>
+__global__ void __launch_bounds__(kScanThreads)
+scan_chunk_kernel(Dims d, ScanArgs a) {
+  extern __shared__ float sm[];
+  float* cs = sm;              // [Q]
+  float* Ct = sm + d.Q;        // [Q][N]
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / d.hpg;
+  const int t0 = c * d.Q, L = min(d.Q, d.T - t0);
+  const S* bpi = (const S*)a.bpi;
+  const S* xs = (const S*)a.xs;
+  chunk_cumsum(d, a.dt, a.A[h], b, h, t0, L, cs);
+  load_readout<S>(d, (const S*)a.cpi, a.read_slot0, a.read_slots, b, g, t0, L, Ct);
+  __syncthreads();
+  if (threadIdx.x == 0) a.cslast[((size_t)b * d.H + h) * d.nc + c] = cs[L - 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // intra-chunk outputs: warp per query token, lanes over p
+  for (int i = warp; i < L; i += kScanThreads / 32) {
+    float yv[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s <= i; ++s) {
+      const float decay = expf(cs[i] - cs[s]);
+      const size_t ms = (size_t)b * d.T + t0 + s;
+      for (int j = a.key_slot0; j < a.key_slot0 + a.key_slots; ++j) {
+        const S* brow = bpi + (ms * d.k + j) * d.GN + (size_t)g * d.N;
+        float part = 0.f;
+        for (int n = lane; n < d.N; n += 32) part = fmaf(Ct[i * d.N + n], to_f32(brow[n]), part);
+        const float coef = decay * warp_sum(part);
+        const S* xrow = xs + (ms * d.k + j) * d.HP + (size_t)h * d.P;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int p = lane + 32 * q;
+          if (p < d.P) yv[q] = fmaf(coef, to_f32(xrow[p]), yv[q]);
+        }
+      }
+    }
+    const size_t mi = (size_t)b * d.T + t0 + i;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int p = lane + 32 * q;
+      if (p < d.P) a.yacc[mi * d.HP + (size_t)h * d.P + p] = yv[q];
+    }
+  }
+  // chunk end state: thread per (n, p)
+  float* Sc = a.schunk + (((size_t)b * d.H + h) * d.nc + c) * d.N * d.P;
+  const float cend = cs[L - 1];
+  for (int x = threadIdx.x; x < d.N * d.P; x += kScanThreads) {
+    const int n = x / d.P, p = x % d.P;
+    float acc = 0.f;
+    for (int s = 0; s < L; ++s) {
+      const float w = expf(cend - cs[s]);
+      const size_t ms = (size_t)b * d.T + t0 + s;
+      float u = 0.f;
+      for (int j = a.key_slot0; j < a.key_slot0 + a.key_slots; ++j)
+        u = fmaf(to_f32(bpi[(ms * d.k + j) * d.GN + (size_t)g * d.N + n]),
+                 to_f32(xs[(ms * d.k + j) * d.HP + (size_t)h * d.P + p]), u);
+      acc = fmaf(w, u, acc);
+    }
+    Sc[x] = acc;
+  }
+}
+
+__global__ void scan_pass_kernel(Dims d, ScanArgs a) {
+  const int bh = blockIdx.x;
+  const int x = blockIdx.y * blockDim.x + threadIdx.x;
+  const int NP = d.N * d.P;
+  if (x >= NP) return;
+  float hv = a.init ? a.init[(size_t)bh * NP + x] : 0.f;
+  for (int c = 0; c < d.nc; ++c) {
+    const size_t o = ((size_t)bh * d.nc + c) * NP + x;
+    a.hstart[o] = hv;
+    hv = expf(a.cslast[(size_t)bh * d.nc + c]) * hv + a.schunk[o];
+  }
+  if (a.final_state) a.final_state[(size_t)bh * NP + x] = hv;
+}
+
+template <class S, class T>
+__global__ void __launch_bounds__(kScanThreads)
+scan_out_kernel(Dims d, ScanArgs a) {
+  extern __shared__ float sm[];
+  float* cs = sm;                    // [Q]
+  float* Ct = sm + d.Q;              // [Q][N]
+  float* Hs = Ct + d.Q * d.N;        // [N][P]
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / d.hpg;
+  const int t0 = c * d.Q, L = min(d.Q, d.T - t0);
+  chunk_cumsum(d, a.dt, a.A[h], b, h, t0, L, cs);
+  load_readout<S>(d, (const S*)a.cpi, a.read_slot0, a.read_slots, b, g, t0, L, Ct);
+  const float* Hc = a.hstart + (((size_t)b * d.H + h) * d.nc + c) * d.N * d.P;
+  for (int x = threadIdx.x; x < d.N * d.P; x += kScanThreads) Hs[x] = Hc[x];
+  __syncthreads();
+  T* y = (T*)a.y;
+  for (int x = threadIdx.x; x < L * d.P; x += kScanThreads) {
+    const int i = x / d.P, p = x % d.P;
+    float acc = 0.f;
+    for (int n = 0; n < d.N; ++n) acc = fmaf(Ct[i * d.N + n], Hs[n * d.P + p], acc);
+    const size_t o = ((size_t)b * d.T + t0 + i) * d.HP + (size_t)h * d.P + p;
+    float v = a.yacc[o] + expf(cs[i]) * acc;
+    if (a.accumulate_y) {
+      // separated design: the k trajectories' outputs are summed in fp32 across the k passes
+      v += a.first_pass ? 0.f : a.ysum[o];
+      if (a.last_pass) y[o] = from_f32<T>(v);
+      else a.ysum[o] = v;
+    } else {
+      y[o] = from_f32<T>(v);
+    }
+  }
+}
+
+cudaError_t launch_scan_simt(const Dims& d, const ScanArgs& a, cudaStream_t s) {
+  dim3 grid(d.nc, d.H, d.Bsz);
+  size_t sm_chunk = sizeof(float) * ((size_t)d.Q + (size_t)d.Q * d.N);
+  size_t sm_out = sm_chunk + sizeof(float) * (size_t)d.N * d.P;
+  const bool bf = d.dtype == SWIMBA_BF16;
+  auto kc = bf ? scan_chunk_kernel<__half> : scan_chunk_kernel<float>;
+  auto ko = bf ? scan_out_kernel<__half, __nv_bfloat16> : scan_out_kernel<float, float>;
+  cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_chunk);
+  cudaFuncSetAttribute(ko, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out);
+  kc<<<grid, kScanThreads, sm_chunk, s>>>(d, a);
+  scan_pass_kernel<<<dim3(d.Bsz * d.H, ceil_div(d.N * d.P, 256)), 256, 0, s>>>(d, a);
+  ko<<<grid, kScanThreads, sm_out, s>>>(d, a);
+  count_launches(3);
+  return cudaGetLastError();
+}
+
+}  // namespace swimba

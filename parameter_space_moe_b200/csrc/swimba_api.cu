@@ -1,0 +1,388 @@
+// C ABI of libswimba: argument validation, workspace planning and the launch sequence of each entry
+// point.  Every entry point validates before launching anything and launches asynchronously on the
+// caller's stream; nothing here allocates device memory.
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace swimba {
+
+// Sticky device status word (bits ST_*), one per device; read and cleared by
+// swimba_check_device_status.  Host code only ever uses its device address (device_status()).
+__device__ unsigned g_status_word;
+
+static unsigned* device_status() {
+  static std::mutex mu;
+  static unsigned* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    addr[dev] = (unsigned*)p;
+  }
+  return addr[dev];
+}
+
+// ---------------------------------------------------------------------------------------------
+// Launch counter and optional per-stage event timing (see swimba_profile_enable).
+static std::atomic<long long> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+struct Profiler {
+  static constexpr int kMax = 16;
+  std::mutex mu;
+  bool on = false, created = false;
+  int n = 0;
+  const char* name[kMax];
+  cudaEvent_t ev[kMax + 1];
+};
+static Profiler g_prof;
+
+static void prof_begin(cudaStream_t s) {
+  if (!g_prof.on) return;
+  g_prof.n = 0;
+  cudaEventRecord(g_prof.ev[0], s);
+}
+static void prof_mark(cudaStream_t s, const char* stage) {
+  if (!g_prof.on || g_prof.n >= Profiler::kMax) return;
+  g_prof.name[g_prof.n] = stage;
+  cudaEventRecord(g_prof.ev[++g_prof.n], s);
+}
+
+size_t elem_bytes(int dtype) { return dtype == SWIMBA_F32 ? 4 : 2; }
+int stream_dtype_of(int dtype) { return dtype == SWIMBA_F32 ? SWIMBA_F32 : SWIMBA_F16; }
+
+WsPlan plan_workspace(const Dims& d) {
+  WsPlan p{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+  const size_t Mk = (size_t)d.M * d.k;
+  const size_t sb = elem_bytes(stream_dtype_of(d.dtype));
+  const size_t states = (size_t)d.Bsz * d.H * d.nc * d.N * d.P * 4;
+  p.status = take(256);
+  p.topk_idx = take(Mk * 4);
+  p.topk_w = take(Mk * 4);
+  p.dt = take((size_t)d.M * d.H * 4);
+  p.dcounts = take((size_t)dispatch_tiles(d) * d.E * 4);
+  p.dbase = take((size_t)dispatch_tiles(d) * d.E * 4);
+  p.offsets = take((size_t)(d.E + 1) * 4);
+  p.perm = take(Mk * 4);
+  p.tiles = take((size_t)max_row_tiles(d) * 8);
+  p.ntiles = take(4);
+  p.xsorted = take(Mk * d.D * elem_bytes(d.dtype));
+  p.bpi = take(Mk * d.GN * sb);
+  p.xs = take(Mk * d.HP * sb);
+  p.cpi = take(Mk * d.GN * sb);
+  p.yintra = take((size_t)d.M * d.HP * 4);
+  p.ysum = take((size_t)d.M * d.HP * 4);
+  p.schunk = take(states);
+  p.hstart = take(states);
+  p.cslast = take((size_t)d.Bsz * d.H * d.nc * 4);
+  p.flags = take((size_t)d.Bsz * d.H * d.nc * 4);
+  p.total = o;
+  return p;
+}
+
+static bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+static swimba_status make_dims(const swimba_dims* in, Dims* d) {
+  if (!in) return SWIMBA_ERR_INVALID_ARG;
+  const swimba_dims& s = *in;
+  if (s.batch < 1 || s.seqlen < 1 || s.d_model < 1 || s.nheads < 1 || s.headdim < 1 || s.dstate < 1 ||
+      s.ngroups < 1 || s.n_experts < 1 || s.top_k < 1 || s.chunk < 1)
+    return SWIMBA_ERR_INVALID_ARG;
+  if (s.dtype != SWIMBA_F32 && s.dtype != SWIMBA_BF16) return SWIMBA_ERR_INVALID_ARG;
+  if (s.top_k > s.n_experts || s.nheads % s.ngroups != 0) return SWIMBA_ERR_INVALID_ARG;
+  if (!pow2_in(s.headdim, 16, 128) || !pow2_in(s.dstate, 16, 128) || !pow2_in(s.chunk, 64, 256))
+    return SWIMBA_ERR_UNSUPPORTED;
+  if (s.top_k > 8 || s.n_experts > 64) return SWIMBA_ERR_UNSUPPORTED;
+  if (s.d_model % (s.dtype == SWIMBA_BF16 ? 64 : 8) != 0) return SWIMBA_ERR_UNSUPPORTED;
+  const long long M = (long long)s.batch * s.seqlen;
+  const long long HP = (long long)s.nheads * s.headdim, GN = (long long)s.ngroups * s.dstate;
+  if (M * s.top_k >= (1LL << 30) || HP + 2 * GN >= (1LL << 24) || M * HP >= (1LL << 40))
+    return SWIMBA_ERR_UNSUPPORTED;
+  d->Bsz = s.batch; d->T = s.seqlen; d->D = s.d_model; d->H = s.nheads; d->P = s.headdim; d->N = s.dstate;
+  d->G = s.ngroups; d->E = s.n_experts; d->k = s.top_k; d->Q = s.chunk; d->dtype = s.dtype;
+  d->M = (int)M; d->HP = (int)HP; d->GN = (int)GN; d->We = (int)(HP + 2 * GN);
+  d->nc = ceil_div(s.seqlen, s.chunk); d->hpg = s.nheads / s.ngroups;
+  return SWIMBA_OK;
+}
+
+static bool aligned(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+static bool ok_ptr(const void* p) { return p && aligned(p); }
+static bool ok_opt(const void* p) { return !p || aligned(p); }
+
+static swimba_status check_weights(const swimba_weights* w, bool need_router, bool need_exp) {
+  if (!w) return SWIMBA_ERR_INVALID_ARG;
+  if (need_router && (!ok_ptr(w->w_router) || !ok_ptr(w->w_dt) || !w->b_dt || !w->A)) return SWIMBA_ERR_INVALID_ARG;
+  if (need_exp && !ok_ptr(w->w_exp)) return SWIMBA_ERR_INVALID_ARG;
+  return SWIMBA_OK;
+}
+
+static swimba_status check_ws(const Dims& d, const void* ws, size_t bytes) {
+  if (!ws || !aligned(ws) || bytes < plan_workspace(d).total) return SWIMBA_ERR_WORKSPACE;
+  return SWIMBA_OK;
+}
+
+static swimba_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SWIMBA_OK : SWIMBA_ERR_CUDA; }
+
+#define SW_TRY(x)                                   \
+  do {                                              \
+    swimba_status s_ = (x);                         \
+    if (s_ != SWIMBA_OK) return s_;                 \
+  } while (0)
+#define SW_CUDA(x)                                  \
+  do {                                              \
+    cudaError_t e_ = (x);                           \
+    if (e_ != cudaSuccess) return SWIMBA_ERR_CUDA;  \
+  } while (0)
+
+// Expert projections of the dispatched rows (after launch_dispatch): bf16 layers gather X into expert
+// order and run the tensor-core GEMM; the fp32 layer runs the CUDA-core GEMM.
+static swimba_status run_proj(const Dims& d, const void* X, const void* w_exp, char* ws, const WsPlan& p,
+                              const float* wts, int mode, void* bpi, void* xs, void* cpi, float* Z, unsigned* st,
+                              cudaStream_t s) {
+  const int32_t* offsets = (const int32_t*)(ws + p.offsets);
+  const int32_t* perm = (const int32_t*)(ws + p.perm);
+  const int32_t* tiles = (const int32_t*)(ws + p.tiles);
+  const int32_t* ntiles = (const int32_t*)(ws + p.ntiles);
+  if (d.dtype == SWIMBA_BF16) {
+    SW_CUDA(launch_gather_rows(d, X, perm, ws + p.xsorted, s));
+    prof_mark(s, "gather");
+    SW_CUDA(launch_proj_tc(d, ws + p.xsorted, w_exp, perm, tiles, ntiles, offsets, wts, mode, bpi, xs, cpi, Z, st, s));
+  } else {
+    SW_CUDA(launch_proj_simt(d, X, w_exp, perm, tiles, ntiles, offsets, wts, mode, bpi, xs, cpi, Z, st, s));
+  }
+  prof_mark(s, "expert_proj_mix");
+  return SWIMBA_OK;
+}
+
+// Router + dispatch + projection with the fused mix, into the workspace's streams.
+static swimba_status run_front(const Dims& d, const void* X, const swimba_weights* w, char* ws, const WsPlan& p,
+                               int32_t* idx, float* wts, int mode, unsigned* st, cudaStream_t s) {
+  float* dt = (float*)(ws + p.dt);
+  SW_CUDA(launch_router(d, X, *w, idx, wts, dt, st, s));
+  prof_mark(s, "router");
+  int32_t* offsets = (int32_t*)(ws + p.offsets);
+  int32_t* perm = (int32_t*)(ws + p.perm);
+  SW_CUDA(launch_dispatch(d, idx, p, ws, offsets, perm, s));
+  prof_mark(s, "dispatch");
+  SW_TRY(run_proj(d, X, w->w_exp, ws, p, wts, mode, ws + p.bpi, ws + p.xs, ws + p.cpi, nullptr, st, s));
+  return SWIMBA_OK;
+}
+
+static ScanArgs mixed_scan_args(const Dims& d, char* ws, const WsPlan& p, const void* bpi, const void* xs,
+                                const void* cpi, const float* dt, const float* A, const float* init, void* y,
+                                float* final_state, float* chunk_states) {
+  ScanArgs a{};
+  a.bpi = bpi; a.xs = xs; a.cpi = cpi; a.dt = dt; a.A = A; a.init = init; a.y = y;
+  a.final_state = final_state;
+  a.hstart = chunk_states ? chunk_states : (float*)(ws + p.hstart);
+  a.schunk = (float*)(ws + p.schunk); a.cslast = (float*)(ws + p.cslast);
+  a.yacc = (float*)(ws + p.yintra); a.ysum = (float*)(ws + p.ysum);
+  a.key_slot0 = 0; a.key_slots = d.k; a.read_slot0 = 0; a.read_slots = d.k;
+  a.accumulate_y = false;
+  return a;
+}
+
+}  // namespace swimba
+
+using namespace swimba;
+
+extern "C" {
+
+size_t swimba_workspace_size(const swimba_dims* dims) {
+  Dims d;
+  if (make_dims(dims, &d) != SWIMBA_OK) return 0;
+  return plan_workspace(d).total;
+}
+
+int swimba_stream_dtype(const swimba_dims* dims) {
+  Dims d;
+  if (make_dims(dims, &d) != SWIMBA_OK) return -1;
+  return stream_dtype_of(d.dtype);
+}
+
+swimba_status swimba_router_topk(const swimba_dims* dims, const void* X, const swimba_weights* w,
+                                 int32_t* topk_idx, float* topk_w, float* dt, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  SW_TRY(check_weights(w, true, false));
+  if (!ok_ptr(X) || !ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_ptr(dt)) return SWIMBA_ERR_INVALID_ARG;
+  return cuda_status(launch_router(d, X, *w, topk_idx, topk_w, dt, device_status(), (cudaStream_t)stream));
+}
+
+swimba_status swimba_dispatch(const swimba_dims* dims, const int32_t* topk_idx, int32_t* expert_offsets,
+                              int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  if (!ok_ptr(topk_idx) || !ok_ptr(expert_offsets) || !ok_ptr(perm)) return SWIMBA_ERR_INVALID_ARG;
+  SW_TRY(check_ws(d, ws, ws_bytes));
+  WsPlan p = plan_workspace(d);
+  return cuda_status(launch_dispatch(d, topk_idx, p, (char*)ws, expert_offsets, perm, (cudaStream_t)stream));
+}
+
+swimba_status swimba_expert_proj(const swimba_dims* dims, const void* X, const swimba_weights* w,
+                                 const int32_t* topk_idx, float* Z, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  SW_TRY(check_weights(w, false, true));
+  if (!ok_ptr(X) || !ok_ptr(topk_idx) || !ok_ptr(Z)) return SWIMBA_ERR_INVALID_ARG;
+  SW_TRY(check_ws(d, ws, ws_bytes));
+  WsPlan p = plan_workspace(d);
+  char* b = (char*)ws;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* offsets = (int32_t*)(b + p.offsets);
+  int32_t* perm = (int32_t*)(b + p.perm);
+  SW_CUDA(launch_dispatch(d, topk_idx, p, b, offsets, perm, s));
+  return run_proj(d, X, w->w_exp, b, p, nullptr, 2, nullptr, nullptr, nullptr, Z, device_status(), s);
+}
+
+swimba_status swimba_mix(const swimba_dims* dims, const float* Z, const float* topk_w, int32_t flags, void* Bpi,
+                         void* Xs, void* Cpi, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  if (!ok_ptr(Z) || !ok_ptr(topk_w) || !ok_ptr(Bpi) || !ok_ptr(Xs) || !ok_ptr(Cpi)) return SWIMBA_ERR_INVALID_ARG;
+  if (flags & ~SWIMBA_MIX_UNSCALED_B) return SWIMBA_ERR_INVALID_ARG;
+  return cuda_status(launch_mix(d, Z, topk_w, flags, Bpi, Xs, Cpi, device_status(), (cudaStream_t)stream));
+}
+
+swimba_status swimba_ssd_scan(const swimba_dims* dims, const void* Bpi, const void* Xs, const void* Cpi,
+                              const float* dt, const float* A, const float* init_state, void* y,
+                              float* final_state, float* chunk_states, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  if (!ok_ptr(Bpi) || !ok_ptr(Xs) || !ok_ptr(Cpi) || !ok_ptr(dt) || !A || !ok_ptr(y)) return SWIMBA_ERR_INVALID_ARG;
+  if (!ok_opt(init_state) || !ok_opt(final_state) || !ok_opt(chunk_states)) return SWIMBA_ERR_INVALID_ARG;
+  SW_TRY(check_ws(d, ws, ws_bytes));
+  WsPlan p = plan_workspace(d);
+  ScanArgs a = mixed_scan_args(d, (char*)ws, p, Bpi, Xs, Cpi, dt, A, init_state, y, final_state, chunk_states);
+  cudaStream_t s = (cudaStream_t)stream;
+  prof_begin(s);
+  SW_CUDA(launch_scan_simt(d, a, s));
+  prof_mark(s, "ssd_scan");
+  return SWIMBA_OK;
+}
+
+swimba_status swimba_layer_fwd(const swimba_dims* dims, const void* X, const swimba_weights* w,
+                               const float* init_state, void* y, float* final_state, int32_t* topk_idx_out,
+                               float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  SW_TRY(check_weights(w, true, true));
+  if (!ok_ptr(X) || !ok_ptr(y) || !ok_opt(init_state) || !ok_opt(final_state) || !ok_opt(topk_idx_out) ||
+      !ok_opt(topk_w_out))
+    return SWIMBA_ERR_INVALID_ARG;
+  SW_TRY(check_ws(d, ws, ws_bytes));
+  WsPlan p = plan_workspace(d);
+  char* b = (char*)ws;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* idx = topk_idx_out ? topk_idx_out : (int32_t*)(b + p.topk_idx);
+  float* wts = topk_w_out ? topk_w_out : (float*)(b + p.topk_w);
+  prof_begin(s);
+  SW_TRY(run_front(d, X, w, b, p, idx, wts, 0, device_status(), s));
+  ScanArgs a = mixed_scan_args(d, b, p, b + p.bpi, b + p.xs, b + p.cpi, (float*)(b + p.dt), w->A, init_state, y,
+                               final_state, nullptr);
+  SW_CUDA(launch_scan_simt(d, a, s));
+  prof_mark(s, "ssd_scan");
+  return SWIMBA_OK;
+}
+
+swimba_status swimba_step(const swimba_dims* dims, const void* X, const swimba_weights* w, float* state, void* y,
+                          int32_t* topk_idx_out, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  if (d.T != 1) return SWIMBA_ERR_INVALID_ARG;
+  SW_TRY(check_weights(w, true, true));
+  if (!ok_ptr(X) || !ok_ptr(state) || !ok_ptr(y) || !ok_opt(topk_idx_out)) return SWIMBA_ERR_INVALID_ARG;
+  SW_TRY(check_ws(d, ws, ws_bytes));
+  WsPlan p = plan_workspace(d);
+  char* b = (char*)ws;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* idx = topk_idx_out ? topk_idx_out : (int32_t*)(b + p.topk_idx);
+  float* wts = (float*)(b + p.topk_w);
+  prof_begin(s);
+  SW_TRY(run_front(d, X, w, b, p, idx, wts, 0, device_status(), s));
+  SW_CUDA(launch_step_update(d, b + p.bpi, b + p.xs, b + p.cpi, (float*)(b + p.dt), w->A, state, y, s));
+  prof_mark(s, "state_update");
+  return SWIMBA_OK;
+}
+
+swimba_status swimba_separated_scan(const swimba_dims* dims, const void* B, const void* Xs, const void* Cpi,
+                                    const float* dt, const float* A, const float* init_states, void* y,
+                                    float* final_states, void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  if (!ok_ptr(B) || !ok_ptr(Xs) || !ok_ptr(Cpi) || !ok_ptr(dt) || !A || !ok_ptr(y)) return SWIMBA_ERR_INVALID_ARG;
+  if (!ok_opt(init_states) || !ok_opt(final_states)) return SWIMBA_ERR_INVALID_ARG;
+  SW_TRY(check_ws(d, ws, ws_bytes));
+  WsPlan p = plan_workspace(d);
+  char* b = (char*)ws;
+  const size_t one = (size_t)d.Bsz * d.H * d.N * d.P;
+  prof_begin((cudaStream_t)stream);
+  for (int j = 0; j < d.k; ++j) {
+    ScanArgs a = mixed_scan_args(d, b, p, B, Xs, Cpi, dt, A, init_states ? init_states + j * one : nullptr, y,
+                                 final_states ? final_states + j * one : nullptr, nullptr);
+    a.key_slot0 = j; a.key_slots = 1; a.read_slot0 = j; a.read_slots = 1;
+    a.accumulate_y = true; a.first_pass = j == 0; a.last_pass = j == d.k - 1;
+    SW_CUDA(launch_scan_simt(d, a, (cudaStream_t)stream));
+  }
+  prof_mark((cudaStream_t)stream, "separated_scan");
+  return SWIMBA_OK;
+}
+
+swimba_status swimba_check_device_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SWIMBA_ERR_CUDA;
+  unsigned* st = device_status();
+  if (!st) return SWIMBA_ERR_CUDA;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, st, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return SWIMBA_ERR_CUDA;
+  if (v && cudaMemset(st, 0, sizeof(v)) != cudaSuccess) return SWIMBA_ERR_CUDA;
+  if (v & ST_TIMEOUT) return SWIMBA_ERR_TIMEOUT;
+  if (v & ST_RANGE) return SWIMBA_ERR_RANGE;
+  return SWIMBA_OK;
+}
+
+swimba_status swimba_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  if (enable && !g_prof.created) {
+    for (int i = 0; i <= Profiler::kMax; ++i)
+      if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return SWIMBA_ERR_CUDA;
+    g_prof.created = true;
+  }
+  g_prof.on = enable != 0;
+  g_prof.n = 0;
+  return SWIMBA_OK;
+}
+
+int swimba_profile_read(const char** names, float* ms, int max) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  if (!g_prof.created) return 0;
+  const int n = g_prof.n < max ? g_prof.n : max;
+  if (n > 0 && cudaEventSynchronize(g_prof.ev[n]) != cudaSuccess) return -1;
+  for (int i = 0; i < n; ++i) {
+    if (names) names[i] = g_prof.name[i];
+    if (ms && cudaEventElapsedTime(&ms[i], g_prof.ev[i], g_prof.ev[i + 1]) != cudaSuccess) return -1;
+  }
+  return n;
+}
+
+long long swimba_launch_count(void) { return g_launches.load(); }
+
+const char* swimba_status_string(swimba_status s) {
+  switch (s) {
+    case SWIMBA_OK: return "SWIMBA_OK";
+    case SWIMBA_ERR_INVALID_ARG: return "SWIMBA_ERR_INVALID_ARG";
+    case SWIMBA_ERR_UNSUPPORTED: return "SWIMBA_ERR_UNSUPPORTED";
+    case SWIMBA_ERR_CUDA: return "SWIMBA_ERR_CUDA";
+    case SWIMBA_ERR_WORKSPACE: return "SWIMBA_ERR_WORKSPACE";
+    case SWIMBA_ERR_TIMEOUT: return "SWIMBA_ERR_TIMEOUT";
+    case SWIMBA_ERR_RANGE: return "SWIMBA_ERR_RANGE";
+  }
+  return "SWIMBA_UNKNOWN_STATUS";
+}
+
+}  // extern "C"

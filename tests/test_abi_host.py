@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every entry point that
+include/swimba.h declares, sizes workspaces, and rejects invalid or unsupported arguments before
+launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from parameter_space_moe_b200 import configs, swimba
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "swimba.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(swimba_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    try:
+        return swimba.lib()
+    except OSError:
+        import __graft_entry__
+        __graft_entry__.build()
+        return swimba.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(swimba.EXPORTS)
+
+
+def test_status_strings(L):
+    for code, name in swimba.STATUS.items():
+        assert swimba.status_string(code) == name
+
+
+def test_workspace_size_and_stream_dtype(L):
+    for w in configs.ALL.values():
+        d = swimba.dims_of(w)
+        assert swimba.workspace_size(d) > 0
+        assert swimba.stream_dtype(d) == (swimba.F16 if w.dtype == "bf16" else swimba.F32)
+    big = swimba.workspace_size(swimba.dims_of(configs.BASE))
+    small = swimba.workspace_size(swimba.dims_of(configs.BASE, seqlen=256))
+    assert big > small
+
+
+BAD_DIMS = [
+    dict(headdim=48), dict(dstate=256), dict(chunk=32), dict(chunk=512), dict(top_k=9, n_experts=16),
+    dict(n_experts=65), dict(d_model=100),
+]
+INVALID_DIMS = [dict(batch=0), dict(seqlen=-1), dict(top_k=5, n_experts=4), dict(ngroups=5), dict(dtype=7)]
+
+
+@pytest.mark.parametrize("kw", BAD_DIMS)
+def test_unsupported_shapes(L, kw):
+    base = dict(batch=1, seqlen=64, d_model=128, nheads=2, headdim=64, dstate=16, ngroups=2, n_experts=4, top_k=2,
+                chunk=64, dtype=swimba.BF16)
+    base.update(kw)
+    d = swimba.dims(**base)
+    assert swimba.workspace_size(d) == 0
+    fake = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: validation fails first
+    w = swimba.Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    rc = L.swimba_layer_fwd(ctypes.byref(d), fake, ctypes.byref(w), None, fake, None, None, None, fake, 1 << 40, None)
+    assert rc == 2
+
+
+@pytest.mark.parametrize("kw", INVALID_DIMS)
+def test_invalid_dims(L, kw):
+    base = dict(batch=1, seqlen=64, d_model=128, nheads=2, headdim=64, dstate=16, ngroups=2, n_experts=4, top_k=2,
+                chunk=64, dtype=swimba.BF16)
+    base.update(kw)
+    d = swimba.dims(**base)
+    assert swimba.workspace_size(d) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    w = swimba.Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    rc = L.swimba_router_topk(ctypes.byref(d), fake, ctypes.byref(w), fake, fake, fake, None)
+    assert rc == 1
+
+
+def test_null_misaligned_and_workspace_errors(L):
+    d = swimba.dims_of(configs.TINY_F32)
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    w = swimba.Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    need = swimba.workspace_size(d)
+    args = lambda X, ws, n: (ctypes.byref(d), X, ctypes.byref(w), None, fake, None, None, None, ws, n, None)
+    assert L.swimba_layer_fwd(*args(None, fake, need)) == 1           # null X
+    assert L.swimba_layer_fwd(*args(odd, fake, need)) == 1            # misaligned X
+    assert L.swimba_layer_fwd(*args(fake, None, need)) == 4           # no workspace
+    assert L.swimba_layer_fwd(*args(fake, fake, need - 1)) == 4       # workspace too small
+    assert L.swimba_layer_fwd(*args(fake, odd, need)) == 4            # misaligned workspace
+    wnull = swimba.Weights(1 << 20, None, 1 << 20, 1 << 20, 1 << 20)
+    assert L.swimba_layer_fwd(ctypes.byref(d), fake, ctypes.byref(wnull), None, fake, None, None, None, fake, need,
+                              None) == 1
+    assert L.swimba_layer_fwd(None, fake, ctypes.byref(w), None, fake, None, None, None, fake, need, None) == 1
+    # decode needs seqlen == 1
+    assert L.swimba_step(ctypes.byref(d), fake, ctypes.byref(w), fake, fake, None, fake, need, None) == 1
+    # mix rejects unknown flags
+    assert L.swimba_mix(ctypes.byref(d), fake, fake, 8, fake, fake, fake, None) == 1

@@ -1,0 +1,28 @@
+"""Long-sequence layer (B1 T32768 D2048 H64 E16 k2 Q256): full-size launch, sampled heads checked
+against the oracle's token-by-token recurrence over all 32768 tokens."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import swimba_oracle as O
+from parameter_space_moe_b200 import configs, inputs
+
+from .parity import check_topk, f64, oracle_heads, rel, to_np
+from .test_gpu_layer import run_layer
+
+pytestmark = pytest.mark.gpu
+
+
+def test_layer_long_sampled():
+    w = configs.LONG
+    inp = inputs.make_inputs(w)
+    y, fin, idx = run_layer(w, inp)
+    X = f64(inp["X"])
+    g = O.router_logits(X.reshape(w.M, -1), f64(inp["W_r"]))
+    fl, forced = check_topk(to_np(idx), g, w.top_k)
+    heads = [5, 40]
+    ref = oracle_heads(inp, w, X, heads, forced.reshape(1, w.seqlen, w.top_k) if fl.any() else None)
+    yg = to_np(y).reshape(1, w.seqlen, w.nheads, w.headdim)[:, :, heads]
+    print(f"long layer: flagged {int(fl.sum())}, rel err y {rel(yg, ref['y']):.3e}")
+    assert rel(yg, ref["y"]) <= 2e-3
+    assert rel(to_np(fin)[:, heads], ref["final"]) <= 2e-3

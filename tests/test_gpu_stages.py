@@ -1,0 +1,136 @@
+"""Stage-by-stage parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+Each stage runs on the GPU alone, fed with the same seeded inputs as the oracle: router (bit-exact
+top-k outside near ties), dispatch (bit-exact stable sort), expert projection, mixing and the chunked
+scan (the latter fed with the oracle's own streams rounded to the stream dtype)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import swimba_oracle as O
+from parameter_space_moe_b200 import configs, inputs, swimba
+
+from .parity import (check_topk, device_weights, f64, out_dtype, rel, stream_torch_dtype, to_np, tol_of)
+
+pytestmark = pytest.mark.gpu
+
+SMALL_BF16 = configs.BASE.with_(name="small_bf16", batch=2, seqlen=320, d_model=128, nheads=4, dstate=32,
+                                n_experts=6, top_k=3, chunk=128, seed=77)
+SMALL_G = configs.BASE.with_(name="small_groups", batch=2, seqlen=200, d_model=192, nheads=4, headdim=32,
+                             dstate=64, ngroups=2, n_experts=4, top_k=2, chunk=64, seed=78)
+STAGE_CFGS = [configs.TINY_F32, SMALL_BF16, SMALL_G, configs.BASE]
+_cache = {}
+
+
+def _setup(w):
+    if w.name in _cache:
+        return _cache[w.name]
+    inp = inputs.make_inputs(w)
+    Xf = f64(inp["X"]).reshape(w.M, w.d_model)
+    ref = O.layer_fwd(f64(inp["X"]), f64(inp["W_r"]), f64(inp["W_dt"]), f64(inp["b_dt"]), f64(inp["A"]),
+                      f64(inp["W_exp"]), w.nheads, w.headdim, w.dstate, w.G, w.top_k)
+    dev = {"X": inp["X"].cuda().reshape(w.M, w.d_model), "W": device_weights(inp)}
+    _cache[w.name] = (inp, Xf, ref, dev)
+    return _cache[w.name]
+
+
+def _ws(d):
+    return torch.empty(swimba.workspace_size(d), dtype=torch.uint8, device="cuda")
+
+
+@pytest.mark.parametrize("w", STAGE_CFGS, ids=lambda w: w.name)
+def test_router(w):
+    inp, Xf, ref, dev = _setup(w)
+    d = swimba.dims_of(w)
+    idx = torch.empty(w.M, w.top_k, dtype=torch.int32, device="cuda")
+    wts = torch.empty(w.M, w.top_k, device="cuda")
+    dt = torch.empty(w.M, w.nheads, device="cuda")
+    swimba.router_topk(d, dev["X"], dev["W"], idx, wts, dt)
+    torch.cuda.synchronize()
+    fl, forced = check_topk(to_np(idx), ref["g"], w.top_k)
+    ok = ~fl
+    np.testing.assert_allclose(to_np(wts)[ok], ref["w"][ok], rtol=2e-5, atol=1e-6)
+    np.testing.assert_allclose(to_np(wts).sum(1), 1.0, rtol=1e-6)
+    np.testing.assert_allclose(to_np(dt), ref["dt"], rtol=2e-5)
+
+
+@pytest.mark.parametrize("w", STAGE_CFGS, ids=lambda w: w.name)
+def test_dispatch_is_stable_sort(w):
+    inp, Xf, ref, dev = _setup(w)
+    d = swimba.dims_of(w)
+    idx = torch.from_numpy(ref["idx"].astype(np.int32)).cuda()
+    off = torch.empty(w.n_experts + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(w.M * w.top_k, dtype=torch.int32, device="cuda")
+    swimba.dispatch(d, idx, off, perm, _ws(d))
+    torch.cuda.synchronize()
+    flat = ref["idx"].reshape(-1)
+    np.testing.assert_array_equal(to_np(perm), np.argsort(flat, kind="stable"))
+    np.testing.assert_array_equal(to_np(off), np.concatenate([[0], np.cumsum(np.bincount(flat, minlength=w.n_experts))]))
+
+
+@pytest.mark.parametrize("w", STAGE_CFGS, ids=lambda w: w.name)
+def test_expert_proj_and_mix(w):
+    inp, Xf, ref, dev = _setup(w)
+    d = swimba.dims_of(w)
+    idx = torch.from_numpy(ref["idx"].astype(np.int32)).cuda()
+    Z = torch.empty(w.M, w.top_k, w.W_e, device="cuda")
+    ws = _ws(d)
+    swimba.expert_proj(d, dev["X"], dev["W"], idx, Z, ws)
+    torch.cuda.synchronize()
+    assert rel(to_np(Z), ref["z"]) < 1e-5
+    sdt = stream_torch_dtype(w)
+    wts = torch.from_numpy(ref["w"].astype(np.float32)).cuda()
+    Bpi = torch.empty(w.M, w.top_k, w.G, w.dstate, dtype=sdt, device="cuda")
+    Xs = torch.empty(w.M, w.top_k, w.nheads, w.headdim, dtype=sdt, device="cuda")
+    Cpi = torch.empty_like(Bpi)
+    swimba.mix(d, Z, wts, 0, Bpi, Xs, Cpi)
+    assert swimba.check_device_status() == 0
+    tol = 1e-6 if w.dtype == "f32" else 6e-4     # fp16 streams keep 11 significant bits
+    assert rel(to_np(Bpi), ref["Bpi"]) < tol
+    assert rel(to_np(Xs), ref["Xs"]) < tol
+    assert rel(to_np(Cpi), ref["Cpi"]) < tol
+    swimba.mix(d, Z, wts, swimba.MIX_UNSCALED_B, Bpi, Xs, Cpi)
+    torch.cuda.synchronize()
+    _, B, _ = O.split_streams(ref["z"], w.nheads, w.headdim, w.G, w.dstate)
+    assert rel(to_np(Bpi), B) < tol
+
+
+def _oracle_streams_on_device(w, ref):
+    sdt = stream_torch_dtype(w)
+    Bpi = torch.from_numpy(ref["Bpi"]).to(sdt)
+    Xs = torch.from_numpy(ref["Xs"]).to(sdt)
+    Cpi = torch.from_numpy(ref["Cpi"]).to(sdt)
+    dt = torch.from_numpy(ref["dt"]).float()
+    return Bpi, Xs, Cpi, dt
+
+
+@pytest.mark.parametrize("w", STAGE_CFGS, ids=lambda w: w.name)
+@pytest.mark.parametrize("with_init", [False, True])
+def test_ssd_scan(w, with_init):
+    inp, Xf, ref, dev = _setup(w)
+    if w.name == configs.BASE.name and with_init:
+        pytest.skip("covered by the small configs")
+    d = swimba.dims_of(w)
+    Bpi, Xs, Cpi, dt = _oracle_streams_on_device(w, ref)
+    A = inp["A"]
+    rng = np.random.default_rng(5)
+    init = rng.standard_normal((w.batch, w.nheads, w.dstate, w.headdim)).astype(np.float32) if with_init else None
+    y = torch.empty(w.M, w.nheads * w.headdim, dtype=out_dtype(w), device="cuda")
+    fin = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, device="cuda")
+    nc = -(-w.seqlen // w.chunk)
+    cst = torch.empty(w.batch, w.nheads, nc, w.dstate, w.headdim, device="cuda")
+    swimba.ssd_scan(d, Bpi.cuda(), Xs.cuda(), Cpi.cuda(), dt.cuda(), A.cuda(),
+                    None if init is None else torch.from_numpy(init).cuda(), y, fin, cst, _ws(d))
+    torch.cuda.synchronize()
+    # the oracle on exactly the streams the GPU read
+    Bq, Xq, Cq = (t.double().numpy() for t in (Bpi, Xs, Cpi))
+    dtq = dt.double().numpy()
+    Ct = Cq.sum(1)
+    for b in range(w.batch):
+        r = slice(b * w.seqlen, (b + 1) * w.seqlen)
+        yc, Hs, hT = O.scan_chunked(Bq[r], Xq[r], Ct[r], dtq[r], f64(A), w.chunk,
+                                    None if init is None else init[b].astype(np.float64))
+        tol = tol_of(w)
+        assert rel(to_np(y)[r].reshape(yc.shape), yc) < tol
+        assert rel(to_np(fin)[b], hT) < (1e-5 if w.dtype == "f32" else 1e-4)
+        assert rel(to_np(cst)[b].transpose(1, 0, 2, 3), Hs) < (1e-5 if w.dtype == "f32" else 1e-4)
