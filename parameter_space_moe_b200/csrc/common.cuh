@@ -75,7 +75,9 @@ struct WsPlan {
   size_t schunk;      // f32 [B][H][nc][N][P]  chunk-local end states
   size_t hstart;      // f32 [B][H][nc][N][P]  state before each chunk
   size_t cslast;      // f32 [B][H][nc]        total log-decay of each chunk
-  size_t flags;       // unsigned [B][H][nc]  chained-scan hand-off flags
+  size_t lb;          // unsigned: ticket counter (256 B) + [B*H][nsub] hand-off flags of the tensor-core scan
+  size_t lb_bytes;
+  size_t exch;        // f32 [B*H][nsub][N][P] state after each sub-chunk (tensor-core scan)
   size_t total;
 };
 
@@ -119,6 +121,7 @@ struct ScanArgs {
   bool accumulate_y;  // add into y (fp32 accumulator in yintra) instead of overwriting
   float* final_state; // or null
   float* hstart;      // [B][H][nc][N][P]
+  float* chunk_states;  // [B][H][nc][N][P] caller's buffer or null (tensor-core scan writes it directly)
   float* schunk; float* cslast;
   float* yacc;        // [M][H][P] fp32: intra-chunk outputs
   float* ysum;        // [M][H][P] fp32: running sum over the separated design's trajectories
@@ -130,6 +133,11 @@ struct ScanArgs {
   bool last_pass;     // separated scan: last slot converts the accumulator to y
 };
 cudaError_t launch_scan_simt(const Dims& d, const ScanArgs& a, cudaStream_t s);
+// Tensor-core scan (fp16 streams, N = 128, P in {64, 128}); `lb` must be zeroed before each launch.
+bool scan_tc_supported(const Dims& d);
+int scan_tc_subchunks(const Dims& d);
+cudaError_t launch_scan_tc(const Dims& d, const ScanArgs& a, unsigned* lb, float* exch, unsigned* st,
+                           cudaStream_t stream);
 cudaError_t launch_step_update(const Dims& d, const void* bpi, const void* xs, const void* cpi, const float* dt,
                                const float* A, float* state, void* y, cudaStream_t s);
 // Adds n to the library's launch counter (every launcher reports the kernels it issued).

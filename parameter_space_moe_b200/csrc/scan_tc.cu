@@ -1,0 +1,451 @@
+// Chunked solve of the single shared-transition recurrence on the tensor cores (fp16 streams, fp32
+// accumulation and state), with the inter-chunk state pass chained between CTAs.
+//
+// Paper: Swimba notes, key design 1 (h_t = a_t h_{t-1} + U~_t, y_t = C~_t^T h_t, U~_t = sum_j Bpi_tj Xs_tj^T)
+// and the overall framework's chunked SSD solve.  One CTA owns SUB = 128 consecutive tokens of one
+// (sequence, head); with cs_t the running sum of dt*A from the sub-chunk start:
+//   S_j      = C~ Bpi_j^T                        (tensor core, 128 x 128 per key slot j, in TMEM)
+//   Pm_j     = mask_{s<=t}(S_j * exp(cs_t - cs_s))   (registers -> fp16 in shared memory)
+//   Y       += Pm_j Xs_j                          (tensor core)
+//   Sc      += Bpi_j^T (exp(cs_end - cs_s) Xs_j)  (tensor core: the sub-chunk's own end state)
+//   H_out    = exp(cs_end) H_in + Sc              (fp32; H_in from the previous sub-chunk's CTA)
+//   y        = Y + exp(cs_t) C~ H_in              (tensor core, H_in split into fp16 hi + lo parts)
+// The hand-off: CTAs take tickets in launch order, ticket -> (sub-chunk = ticket / (B*H), head row =
+// ticket % (B*H)), so the CTA holding the previous sub-chunk of the same head always took its ticket
+// first and is running or done.  It publishes H_out with a release flag; the successor polls with a
+// bounded wait (on expiry it records ST_TIMEOUT, uses a zero state and still publishes its own flag).
+// Keys are the (token, slot) pairs; k slots are processed one after another through a 2-stage TMA ring.
+#include "tc_common.cuh"
+
+namespace swimba {
+
+namespace {
+constexpr int SUB = 128;
+constexpr int kThreads = 128;
+constexpr uint32_t kBlk = SUB * 128;  // one 64-wide column block of 128 swizzled 128-byte rows
+constexpr uint32_t kFlagPolls = 1u << 22;
+
+struct TcScanArgs {
+  Dims d;
+  const float* dt;
+  const float* A;
+  const float* init;
+  const __half* cpi;
+  __nv_bfloat16* y;
+  float* final_state;
+  float* chunk_states;
+  float* exch;
+  unsigned* flags;
+  unsigned* ticket;
+  unsigned* st;
+  float* ysum;
+  int nsub;
+  int key_slot0, key_slots, read_slot0, read_slots;
+  int accumulate_y, first_pass, last_pass;
+};
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
+          "r"(tc::smem_u32(dst)),
+      "l"((uint64_t)map), "r"(tc::smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <int P>
+__global__ void __launch_bounds__(kThreads, 1)
+scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_x, TcScanArgs a) {
+  constexpr int N = 128, NB = N / 64, PB = P / 64;
+  constexpr uint32_t CT_BYTES = NB * kBlk, BP_BYTES = NB * kBlk, XS_BYTES = PB * kBlk;
+  constexpr uint32_t STAGE = BP_BYTES + XS_BYTES, DX_BYTES = PB * kBlk, PM_BYTES = 2 * kBlk;
+  constexpr uint32_t TMEM_COLS = P == 64 ? 256 : 512;
+  constexpr uint32_t COL_S = 0, COL_Y = 128, COL_SC = 128 + P;
+  constexpr uint32_t ID_S = tc::idesc_f16(128, 128, false);
+  constexpr uint32_t ID_SC = tc::idesc_f16(128, P, false, true, true);
+  constexpr uint32_t ID_Y = tc::idesc_f16(128, P, false, false, true);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* CT = sm;
+  uint8_t* RING = CT + CT_BYTES;
+  uint8_t* DX = RING + 2 * STAGE;
+  uint8_t* PM = DX + DX_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(PM + PM_BYTES);  // [2]
+  uint64_t* done = full + 2;
+  float* cs_s = reinterpret_cast<float*>(full + 4);  // [SUB]
+  float* wsum = cs_s + SUB;                          // [4]
+  uint32_t* misc = reinterpret_cast<uint32_t*>(wsum + 4);  // tmem base, ticket
+
+  const Dims& d = a.d;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    tc::mbar_init(&full[0], 1);
+    tc::mbar_init(&full[1], 1);
+    tc::mbar_init(done, 1);
+    tc::fence_barrier_init();
+    misc[1] = atomicAdd(a.ticket, 1u);
+  }
+  if (warp == 0) { tc::tmem_alloc(&misc[0], TMEM_COLS); tc::tmem_relinquish(); }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = misc[0];
+  const int BH = d.Bsz * d.H;
+  const int ticket = (int)misc[1];
+  const int csub = ticket / BH, bh = ticket % BH, b = bh / d.H, h = bh % d.H, g = h / d.hpg;
+  const int t0 = csub * SUB, L = min(SUB, d.T - t0);
+  const int row0 = b * d.T + t0;
+  const int nk = a.key_slots;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  volatile int never = 0;
+  int issued = 0;
+
+  auto issue_slot = [&](int i) {
+    const int stage = i & 1, j = a.key_slot0 + i;
+    uint8_t* sb = RING + stage * STAGE;
+    tc::mbar_arrive_expect_tx(&full[stage], STAGE);
+    for (int nb = 0; nb < NB; ++nb) tma_load_3d(sb + nb * kBlk, &tm_b, &full[stage], g * N + 64 * nb, j, row0);
+    for (int pb = 0; pb < PB; ++pb)
+      tma_load_3d(sb + BP_BYTES + pb * kBlk, &tm_x, &full[stage], h * P + 64 * pb, j, row0);
+    ++issued;
+  };
+  if (tid == 0) {
+    for (int i = 0; i < nk && i < 2; ++i) issue_slot(i);
+  }
+
+  // cumulative log-decay of the sub-chunk (inclusive scan over the 128 threads)
+  float v = tid < L ? a.dt[(size_t)(row0 + tid) * d.H + h] * a.A[h] : 0.f;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float u = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) wsum[warp] = v;
+  __syncthreads();
+  for (int w = 0; w < warp; ++w) v += wsum[w];
+  cs_s[tid] = v;
+  __syncthreads();
+  const float my_cs = v, cs_end = cs_s[L - 1];
+
+  // C~ rows (sum of the readout slots) -> fp16, K-major 128-byte-swizzled
+  {
+    const bool valid = tid < L;
+    for (int nb = 0; nb < NB; ++nb) {
+      for (int c = 0; c < 8; ++c) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (valid) {
+          for (int j = a.read_slot0; j < a.read_slot0 + a.read_slots; ++j) {
+            const __half* src = a.cpi + ((size_t)(row0 + tid) * d.k + j) * d.GN + (size_t)g * N + nb * 64 + c * 8;
+            const uint4 q = *reinterpret_cast<const uint4*>(src);
+            const __half2* hq = reinterpret_cast<const __half2*>(&q);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(hq[e]);
+              acc[2 * e] += f.x;
+              acc[2 * e + 1] += f.y;
+            }
+          }
+        }
+        uint4 o;
+        o.x = pack_half2(acc[0], acc[1]); o.y = pack_half2(acc[2], acc[3]);
+        o.z = pack_half2(acc[4], acc[5]); o.w = pack_half2(acc[6], acc[7]);
+        *reinterpret_cast<uint4*>(CT + nb * kBlk + tc::sw128_chunk(tid, c)) = o;
+      }
+    }
+  }
+  tc::fence_proxy_async();
+
+  bool ok = true;
+  uint32_t done_phase = 0;
+  const float dec_end = tid < L ? expf(cs_end - my_cs) : 0.f;
+  for (int i = 0; i < nk && ok; ++i) {
+    const int stage = i & 1;
+    uint8_t* BPs = RING + stage * STAGE;
+    uint8_t* XSs = BPs + BP_BYTES;
+    ok = tc::mbar_wait(&full[stage], (uint32_t)((i >> 1) & 1), &never);
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    // values scaled by the decay to the sub-chunk end (for the end state)
+    for (int pb = 0; pb < PB; ++pb) {
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t off = pb * kBlk + tc::sw128_chunk(tid, c);
+        uint4 q = *reinterpret_cast<const uint4*>(XSs + off);
+        __half2* hq = reinterpret_cast<__half2*>(&q);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(hq[e]);
+          hq[e] = __floats2half2_rn(f.x * dec_end, f.y * dec_end);
+        }
+        *reinterpret_cast<uint4*>(DX + off) = q;
+      }
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (tid == 0) {
+      const uint32_t ct = tc::smem_u32(CT), bp = tc::smem_u32(BPs), dx = tc::smem_u32(DX);
+#pragma unroll
+      for (int kk = 0; kk < N / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
+        tc::mma_f16(tmem + COL_S, tc::sdesc_kmajor_sw128(ct + off), tc::sdesc_kmajor_sw128(bp + off), ID_S, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < SUB / 16; ++kk) {
+        tc::mma_f16(tmem + COL_SC, tc::sdesc_mnmajor_sw128(bp + kk * 2048, kBlk),
+                    tc::sdesc_mnmajor_sw128(dx + kk * 2048, kBlk), ID_SC, (i > 0) || (kk > 0));
+      }
+      tc::mma_commit(done);
+    }
+    ok = tc::mbar_wait(done, done_phase, &never);
+    done_phase ^= 1u;
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    tc::fence_after_sync();
+    // masked, decayed scores -> fp16 K-major swizzled rows of Pm
+    for (int q = 0; q < 4; ++q) {
+      uint32_t r[32];
+      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * q, r);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int s = 32 * q + 8 * c + e;
+          f[e] = (s <= tid && tid < L) ? u2f(r[8 * c + e]) * expf(my_cs - cs_s[s]) : 0.f;
+        }
+        uint4 o;
+        o.x = pack_half2(f[0], f[1]); o.y = pack_half2(f[2], f[3]);
+        o.z = pack_half2(f[4], f[5]); o.w = pack_half2(f[6], f[7]);
+        const int s0 = 32 * q + 8 * c;
+        *reinterpret_cast<uint4*>(PM + (s0 >> 6) * kBlk + tc::sw128_chunk(tid, (s0 & 63) >> 3)) = o;
+      }
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (tid == 0) {
+      const uint32_t pm = tc::smem_u32(PM), xs = tc::smem_u32(XSs);
+#pragma unroll
+      for (int kk = 0; kk < SUB / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
+        tc::mma_f16(tmem + COL_Y, tc::sdesc_kmajor_sw128(pm + off), tc::sdesc_mnmajor_sw128(xs + kk * 2048, kBlk),
+                    ID_Y, (i > 0) || (kk > 0));
+      }
+      tc::mma_commit(done);
+    }
+    ok = tc::mbar_wait(done, done_phase, &never);
+    done_phase ^= 1u;
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    if (tid == 0 && i + 2 < nk) issue_slot(i + 2);
+  }
+
+  if (ok) {
+    // ---------------------------------------------------------------- state hand-off
+    const size_t NP = (size_t)N * P;
+    if (tid == 0 && csub > 0) {
+      const unsigned* f = a.flags + (size_t)bh * a.nsub + csub - 1;
+      uint32_t n = 0;
+      while (ld_acquire(f) == 0u && n < kFlagPolls) { __nanosleep(64); ++n; }
+      if (n == kFlagPolls) atomicOr(a.st, ST_TIMEOUT);
+    }
+    __syncthreads();
+    const float* hin = csub > 0 ? a.exch + ((size_t)bh * a.nsub + csub - 1) * NP
+                                : (a.init ? a.init + (size_t)bh * NP : nullptr);
+    float* hout = a.exch + ((size_t)bh * a.nsub + csub) * NP;
+    const bool last = t0 + L == d.T;
+    const bool chunk_start = a.chunk_states && (t0 % d.Q) == 0;
+    float* cst = chunk_start ? a.chunk_states + (((size_t)b * d.H + h) * d.nc + t0 / d.Q) * NP : nullptr;
+    float* fin = (last && a.final_state) ? a.final_state + (size_t)bh * NP : nullptr;
+    const float dend = expf(cs_end);
+    uint8_t* HH = RING;                 // the ring is free now: fp16 hi and lo parts of H_in
+    uint8_t* HL = RING + PB * kBlk;
+    bool range_bad = false;
+    for (int q = 0; q < P / 32; ++q) {
+      uint32_t r[32];
+      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_SC + 32 * q, r);
+      tc::tmem_ld_wait();
+      const size_t ro = (size_t)tid * P + 32 * q;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float hp[8], hi[8], lo[8];
+#pragma unroll
+        for (int e = 0; e < 8; e += 4) {
+          float4 x = hin ? __ldcg(reinterpret_cast<const float4*>(hin + ro + 8 * c + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
+          hp[e] = x.x; hp[e + 1] = x.y; hp[e + 2] = x.z; hp[e + 3] = x.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; e += 4) {
+          float4 o = make_float4(fmaf(dend, hp[e], u2f(r[8 * c + e])), fmaf(dend, hp[e + 1], u2f(r[8 * c + e + 1])),
+                                 fmaf(dend, hp[e + 2], u2f(r[8 * c + e + 2])), fmaf(dend, hp[e + 3], u2f(r[8 * c + e + 3])));
+          __stcg(reinterpret_cast<float4*>(hout + ro + 8 * c + e), o);
+          if (fin) *reinterpret_cast<float4*>(fin + ro + 8 * c + e) = o;
+          if (cst) *reinterpret_cast<float4*>(cst + ro + 8 * c + e) =
+              make_float4(hp[e], hp[e + 1], hp[e + 2], hp[e + 3]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const __half hh = __float2half_rn(hp[e]);
+          hi[e] = __half2float(hh);
+          lo[e] = hp[e] - hi[e];
+          range_bad |= !(fabsf(hp[e]) <= kF16Max);
+        }
+        const int p0 = 32 * q + 8 * c;
+        const uint32_t off = (p0 >> 6) * kBlk + tc::sw128_chunk(tid, (p0 & 63) >> 3);
+        uint4 oh, ol;
+        oh.x = pack_half2(hi[0], hi[1]); oh.y = pack_half2(hi[2], hi[3]);
+        oh.z = pack_half2(hi[4], hi[5]); oh.w = pack_half2(hi[6], hi[7]);
+        ol.x = pack_half2(lo[0], lo[1]); ol.y = pack_half2(lo[2], lo[3]);
+        ol.z = pack_half2(lo[4], lo[5]); ol.w = pack_half2(lo[6], lo[7]);
+        *reinterpret_cast<uint4*>(HH + off) = oh;
+        *reinterpret_cast<uint4*>(HL + off) = ol;
+      }
+    }
+    if (range_bad) atomicOr(a.st, ST_RANGE);
+    __threadfence();
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (tid == 0) {
+      st_release(a.flags + (size_t)bh * a.nsub + csub, 1u);
+      const uint32_t ct = tc::smem_u32(CT), hh = tc::smem_u32(HH), hl = tc::smem_u32(HL);
+#pragma unroll
+      for (int kk = 0; kk < N / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
+        tc::mma_f16(tmem + COL_S, tc::sdesc_kmajor_sw128(ct + off), tc::sdesc_mnmajor_sw128(hh + kk * 2048, kBlk),
+                    ID_Y, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < N / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
+        tc::mma_f16(tmem + COL_S, tc::sdesc_kmajor_sw128(ct + off), tc::sdesc_mnmajor_sw128(hl + kk * 2048, kBlk),
+                    ID_Y, 1);
+      }
+      tc::mma_commit(done);
+    }
+    ok = tc::mbar_wait(done, done_phase, &never);
+    done_phase ^= 1u;
+    if (__syncthreads_and(ok)) {
+      tc::fence_after_sync();
+      // ---------------------------------------------------------------- output rows
+      const float eq = expf(my_cs);
+      const bool valid = tid < L;
+      const size_t orow = (size_t)(row0 + tid) * d.HP + (size_t)h * P;
+      for (int q = 0; q < P / 32; ++q) {
+        uint32_t ry[32], ri[32];
+        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_Y + 32 * q, ry);
+        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * q, ri);
+        tc::tmem_ld_wait();
+        if (!valid) continue;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = fmaf(eq, u2f(ri[8 * c + e]), u2f(ry[8 * c + e]));
+          const size_t o = orow + 32 * q + 8 * c;
+          if (a.accumulate_y) {
+            if (!a.first_pass) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] += a.ysum[o + e];
+            }
+            if (!a.last_pass) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) a.ysum[o + e] = f[e];
+              continue;
+            }
+          }
+          uint4 ov;
+          __nv_bfloat162 b0 = __floats2bfloat162_rn(f[0], f[1]), b1 = __floats2bfloat162_rn(f[2], f[3]);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(f[4], f[5]), b3 = __floats2bfloat162_rn(f[6], f[7]);
+          ov.x = *reinterpret_cast<uint32_t*>(&b0); ov.y = *reinterpret_cast<uint32_t*>(&b1);
+          ov.z = *reinterpret_cast<uint32_t*>(&b2); ov.w = *reinterpret_cast<uint32_t*>(&b3);
+          *reinterpret_cast<uint4*>(a.y + o) = ov;
+        }
+      }
+    }
+  }
+  if (!ok) {
+    if (tid == 0) {
+      atomicOr(a.st, ST_TIMEOUT);
+      // successors must not wait on a sub-chunk that gave up
+      st_release(a.flags + (size_t)bh * a.nsub + csub, 1u);
+    }
+  }
+  // no copy may still be landing in shared memory when the CTA exits
+  if (tid == 0) {
+    for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) tc::mbar_wait(&full[i & 1], (uint32_t)((i >> 1) & 1), &never);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+template <int P>
+size_t smem_bytes() {
+  constexpr uint32_t NB = 2, PB = P / 64;
+  return 1024 + (size_t)(NB * kBlk) + 2 * (size_t)(NB * kBlk + PB * kBlk) + PB * kBlk + 2 * kBlk + 64 +
+         SUB * 4 + 64;
+}
+
+}  // namespace
+
+bool scan_tc_supported(const Dims& d) {
+  return d.dtype == SWIMBA_BF16 && d.N == 128 && (d.P == 64 || d.P == 128);
+}
+
+int scan_tc_subchunks(const Dims& d) { return ceil_div(d.T, SUB); }
+
+// lb: zeroed by the caller (ticket counter at lb[0], flags at lb + 64); exch: [B*H][nsub][N][P] fp32.
+cudaError_t launch_scan_tc(const Dims& d, const ScanArgs& s, unsigned* lb, float* exch, unsigned* st,
+                           cudaStream_t stream) {
+  CUtensorMap tb, tx;
+  if (!encode_tmap_3d_slot(&tb, s.bpi, SWIMBA_F16, (uint64_t)d.GN, (uint64_t)d.k, (uint64_t)d.M, 64, SUB))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_3d_slot(&tx, s.xs, SWIMBA_F16, (uint64_t)d.HP, (uint64_t)d.k, (uint64_t)d.M, 64, SUB))
+    return cudaErrorInvalidValue;
+  TcScanArgs a{};
+  a.d = d; a.dt = s.dt; a.A = s.A; a.init = s.init; a.cpi = (const __half*)s.cpi; a.y = (__nv_bfloat16*)s.y;
+  a.final_state = s.final_state; a.chunk_states = s.chunk_states; a.exch = exch; a.flags = lb + 64; a.ticket = lb;
+  a.st = st; a.ysum = s.ysum; a.nsub = scan_tc_subchunks(d);
+  a.key_slot0 = s.key_slot0; a.key_slots = s.key_slots; a.read_slot0 = s.read_slot0; a.read_slots = s.read_slots;
+  a.accumulate_y = s.accumulate_y; a.first_pass = s.first_pass; a.last_pass = s.last_pass;
+  const int grid = d.Bsz * d.H * a.nsub;
+  cudaError_t e;
+  if (d.P == 64) {
+    const size_t sm = smem_bytes<64>();
+    e = cudaFuncSetAttribute(scan_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    scan_tc_kernel<64><<<grid, kThreads, sm, stream>>>(tb, tx, a);
+  } else {
+    const size_t sm = smem_bytes<128>();
+    e = cudaFuncSetAttribute(scan_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    scan_tc_kernel<128><<<grid, kThreads, sm, stream>>>(tb, tx, a);
+  }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace swimba

@@ -81,7 +81,10 @@ WsPlan plan_workspace(const Dims& d) {
   p.schunk = take(states);
   p.hstart = take(states);
   p.cslast = take((size_t)d.Bsz * d.H * d.nc * 4);
-  p.flags = take((size_t)d.Bsz * d.H * d.nc * 4);
+  const size_t nsub = (size_t)scan_tc_subchunks(d);
+  p.lb_bytes = 256 + (size_t)d.Bsz * d.H * nsub * 4;
+  p.lb = take(p.lb_bytes);
+  p.exch = take((size_t)d.Bsz * d.H * nsub * d.N * d.P * 4);
   p.total = o;
   return p;
 }
@@ -174,6 +177,18 @@ static swimba_status run_front(const Dims& d, const void* X, const swimba_weight
   return SWIMBA_OK;
 }
 
+// The chunked scan: tensor-core kernel for the shapes it covers, CUDA-core kernels otherwise (the
+// fp32 layer, N != 128, P not in {64, 128}, or per-chunk states requested at chunk 64).
+static swimba_status run_scan(const Dims& d, const ScanArgs& a, char* ws, const WsPlan& p, cudaStream_t s) {
+  if (scan_tc_supported(d) && !(a.chunk_states && d.Q < 128)) {
+    SW_CUDA(cudaMemsetAsync(ws + p.lb, 0, p.lb_bytes, s));
+    SW_CUDA(launch_scan_tc(d, a, (unsigned*)(ws + p.lb), (float*)(ws + p.exch), device_status(), s));
+  } else {
+    SW_CUDA(launch_scan_simt(d, a, s));
+  }
+  return SWIMBA_OK;
+}
+
 static ScanArgs mixed_scan_args(const Dims& d, char* ws, const WsPlan& p, const void* bpi, const void* xs,
                                 const void* cpi, const float* dt, const float* A, const float* init, void* y,
                                 float* final_state, float* chunk_states) {
@@ -181,6 +196,7 @@ static ScanArgs mixed_scan_args(const Dims& d, char* ws, const WsPlan& p, const 
   a.bpi = bpi; a.xs = xs; a.cpi = cpi; a.dt = dt; a.A = A; a.init = init; a.y = y;
   a.final_state = final_state;
   a.hstart = chunk_states ? chunk_states : (float*)(ws + p.hstart);
+  a.chunk_states = chunk_states;
   a.schunk = (float*)(ws + p.schunk); a.cslast = (float*)(ws + p.cslast);
   a.yacc = (float*)(ws + p.yintra); a.ysum = (float*)(ws + p.ysum);
   a.key_slot0 = 0; a.key_slots = d.k; a.read_slot0 = 0; a.read_slots = d.k;
@@ -262,7 +278,7 @@ swimba_status swimba_ssd_scan(const swimba_dims* dims, const void* Bpi, const vo
   ScanArgs a = mixed_scan_args(d, (char*)ws, p, Bpi, Xs, Cpi, dt, A, init_state, y, final_state, chunk_states);
   cudaStream_t s = (cudaStream_t)stream;
   prof_begin(s);
-  SW_CUDA(launch_scan_simt(d, a, s));
+  SW_TRY(run_scan(d, a, (char*)ws, p, s));
   prof_mark(s, "ssd_scan");
   return SWIMBA_OK;
 }
@@ -286,7 +302,7 @@ swimba_status swimba_layer_fwd(const swimba_dims* dims, const void* X, const swi
   SW_TRY(run_front(d, X, w, b, p, idx, wts, 0, device_status(), s));
   ScanArgs a = mixed_scan_args(d, b, p, b + p.bpi, b + p.xs, b + p.cpi, (float*)(b + p.dt), w->A, init_state, y,
                                final_state, nullptr);
-  SW_CUDA(launch_scan_simt(d, a, s));
+  SW_TRY(run_scan(d, a, b, p, s));
   prof_mark(s, "ssd_scan");
   return SWIMBA_OK;
 }
@@ -328,7 +344,7 @@ swimba_status swimba_separated_scan(const swimba_dims* dims, const void* B, cons
                                  final_states ? final_states + j * one : nullptr, nullptr);
     a.key_slot0 = j; a.key_slots = 1; a.read_slot0 = j; a.read_slots = 1;
     a.accumulate_y = true; a.first_pass = j == 0; a.last_pass = j == d.k - 1;
-    SW_CUDA(launch_scan_simt(d, a, (cudaStream_t)stream));
+    SW_TRY(run_scan(d, a, b, p, (cudaStream_t)stream));
   }
   prof_mark((cudaStream_t)stream, "separated_scan");
   return SWIMBA_OK;

@@ -120,6 +120,26 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr) {
   return d;
 }
 
+// Descriptor of an MN-major operand tile with the 128-byte swizzle: rows of 128 bytes along K (64 fp16
+// MN values per row), 8-row K groups 1024 bytes apart, and successive 64-wide MN blocks `mn_block_bytes`
+// apart.  Advancing along K by 16 rows is done by adding 2048 to `saddr`.
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr, uint32_t mn_block_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((mn_block_bytes >> 4) & 0x3FFFu) << 16;  // leading byte offset: next MN block
+  d |= (uint64_t)(1024 >> 4) << 32;                        // stride byte offset: next 8-row K group
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled block of 128-byte rows (the
+// layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B; the block starts on a 1024-byte boundary).
+__device__ __forceinline__ uint32_t sw128_chunk(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy (tensor core, TMA).
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // Instruction descriptor of tcgen05.mma.kind::f16 with fp32 accumulation.
 //   ab_bf16: operands bf16 (else fp16); a_mn / b_mn: operand is MN-major (else K-major)
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool ab_bf16, bool a_mn = false, bool b_mn = false) {
@@ -135,5 +155,9 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool ab_bf16, boo
 // box_rows} box and the 128-byte swizzle.  Returns false if the driver rejects it.
 bool encode_tmap_2d(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t rows, uint64_t pitch_bytes,
                     uint32_t box_cols, uint32_t box_rows);
+// Host: 3D map of a [rows][slots][cols] tensor (dims {cols, slots, rows}); box {box_cols, 1, box_rows}
+// selects one slot of box_rows consecutive rows.
+bool encode_tmap_3d_slot(CUtensorMap* map, const void* base, int dtype, uint64_t cols, uint64_t slots, uint64_t rows,
+                         uint32_t box_cols, uint32_t box_rows);
 
 }  // namespace swimba

@@ -18,7 +18,12 @@ SMALL_BF16 = configs.BASE.with_(name="small_bf16", batch=2, seqlen=320, d_model=
                                 n_experts=6, top_k=3, chunk=128, seed=77)
 SMALL_G = configs.BASE.with_(name="small_groups", batch=2, seqlen=200, d_model=192, nheads=4, headdim=32,
                              dstate=64, ngroups=2, n_experts=4, top_k=2, chunk=64, seed=78)
-STAGE_CFGS = [configs.TINY_F32, SMALL_BF16, SMALL_G, configs.BASE]
+# tensor-core scan shapes (N = 128): P = 128, three slots, shared groups, ragged T
+TC_P128 = configs.BASE.with_(name="tc_P128_k3_G2", batch=2, seqlen=333, d_model=128, nheads=4, headdim=128,
+                             dstate=128, ngroups=2, n_experts=5, top_k=3, chunk=128, seed=79)
+TC_Q64 = configs.BASE.with_(name="tc_Q64_ragged", batch=3, seqlen=201, d_model=128, nheads=2, n_experts=4,
+                            chunk=64, seed=80)
+STAGE_CFGS = [configs.TINY_F32, SMALL_BF16, SMALL_G, TC_P128, TC_Q64, configs.BASE]
 _cache = {}
 
 
@@ -134,3 +139,27 @@ def test_ssd_scan(w, with_init):
         assert rel(to_np(y)[r].reshape(yc.shape), yc) < tol
         assert rel(to_np(fin)[b], hT) < (1e-5 if w.dtype == "f32" else 1e-4)
         assert rel(to_np(cst)[b].transpose(1, 0, 2, 3), Hs) < (1e-5 if w.dtype == "f32" else 1e-4)
+
+
+@pytest.mark.parametrize("w", [configs.TINY_F32, TC_P128, TC_Q64], ids=lambda w: w.name)
+def test_separated_scan(w):
+    """The separated design ("k scans"): k trajectories with unscaled injections, pi-scaled readouts."""
+    inp, Xf, ref, dev = _setup(w)
+    d = swimba.dims_of(w)
+    sdt = stream_torch_dtype(w)
+    _, B, _ = O.split_streams(ref["z"], w.nheads, w.headdim, w.G, w.dstate)
+    Bq = torch.from_numpy(B).to(sdt)
+    Xq = torch.from_numpy(ref["Xs"]).to(sdt)
+    Cq = torch.from_numpy(ref["Cpi"]).to(sdt)
+    dt = torch.from_numpy(ref["dt"]).float()
+    y = torch.empty(w.M, w.nheads * w.headdim, dtype=out_dtype(w), device="cuda")
+    fin = torch.empty(w.top_k, w.batch, w.nheads, w.dstate, w.headdim, device="cuda")
+    swimba.separated_scan(d, Bq.cuda(), Xq.cuda(), Cq.cuda(), dt.cuda(), inp["A"].cuda(), None, y, fin, _ws(d))
+    assert swimba.check_device_status() == 0
+    Bd, Xd, Cd, dtd = (t.double().numpy() for t in (Bq, Xq, Cq, dt))
+    for b in range(w.batch):
+        r = slice(b * w.seqlen, (b + 1) * w.seqlen)
+        ys, hs, nrec = O.scan_separated_k(Bd[r], Xd[r], Cd[r], dtd[r], f64(inp["A"]))
+        assert nrec == w.top_k
+        assert rel(to_np(y)[r].reshape(ys.shape), ys) < tol_of(w)
+        assert rel(to_np(fin)[:, b], hs) < (1e-5 if w.dtype == "f32" else 1e-4)
