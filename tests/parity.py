@@ -17,12 +17,19 @@ from parameter_space_moe_b200 import swimba
 DELTA = 1e-4
 TOL_F32 = 1e-5      # norm-wise relative error, all-fp32 layer
 TOL_BF16 = 2e-3     # norm-wise relative error, bf16 in/out with fp32 state
+# SSM states (fp32) of bf16 layers: the tensor-core scan feeds the end-state product with the
+# decay-scaled values rounded once to fp16 (~3e-4 relative per element), so states are held to 1e-3.
+TOL_STATE_BF16 = 1e-3
 
 f64 = I.to_f64
 
 
 def tol_of(w):
     return TOL_F32 if w.dtype == "f32" else TOL_BF16
+
+
+def state_tol_of(w):
+    return TOL_F32 if w.dtype == "f32" else TOL_STATE_BF16
 
 
 def rel(a, b):

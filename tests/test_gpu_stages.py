@@ -10,7 +10,8 @@ import torch
 from oracle import swimba_oracle as O
 from parameter_space_moe_b200 import configs, inputs, swimba
 
-from .parity import (check_topk, device_weights, f64, out_dtype, rel, stream_torch_dtype, to_np, tol_of)
+from .parity import (check_topk, device_weights, f64, out_dtype, rel, state_tol_of, stream_torch_dtype, to_np,
+                     tol_of)
 
 pytestmark = pytest.mark.gpu
 
@@ -137,8 +138,8 @@ def test_ssd_scan(w, with_init):
                                     None if init is None else init[b].astype(np.float64))
         tol = tol_of(w)
         assert rel(to_np(y)[r].reshape(yc.shape), yc) < tol
-        assert rel(to_np(fin)[b], hT) < (1e-5 if w.dtype == "f32" else 1e-4)
-        assert rel(to_np(cst)[b].transpose(1, 0, 2, 3), Hs) < (1e-5 if w.dtype == "f32" else 1e-4)
+        assert rel(to_np(fin)[b], hT) < state_tol_of(w)
+        assert rel(to_np(cst)[b].transpose(1, 0, 2, 3), Hs) < state_tol_of(w)
 
 
 @pytest.mark.parametrize("w", [configs.TINY_F32, TC_P128, TC_Q64], ids=lambda w: w.name)
@@ -162,4 +163,4 @@ def test_separated_scan(w):
         ys, hs, nrec = O.scan_separated_k(Bd[r], Xd[r], Cd[r], dtd[r], f64(inp["A"]))
         assert nrec == w.top_k
         assert rel(to_np(y)[r].reshape(ys.shape), ys) < tol_of(w)
-        assert rel(to_np(fin)[:, b], hs) < (1e-5 if w.dtype == "f32" else 1e-4)
+        assert rel(to_np(fin)[:, b], hs) < state_tol_of(w)
