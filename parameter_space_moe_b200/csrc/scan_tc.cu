@@ -14,7 +14,8 @@
 // ticket % (B*H)), so the CTA holding the previous sub-chunk of the same head always took its ticket
 // first and is running or done.  It publishes H_out with a release flag; the successor polls with a
 // bounded wait (on expiry it records ST_TIMEOUT, uses a zero state and still publishes its own flag).
-// Keys are the (token, slot) pairs; k slots are processed one after another through a 2-stage TMA ring.
+// Keys are the (token, slot) pairs; the k slots are processed one after another, the next slot's keys
+// and values loaded by TMA as soon as the current slot's products no longer read them.
 #include "tc_common.cuh"
 
 namespace swimba {
@@ -69,12 +70,26 @@ __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Shared-memory plan of one CTA (byte offsets from a 1024-aligned base).  With P = 64 it is 96 KB,
+// so two CTAs share an SM and one CTA's loads overlap the other's tensor-core work.
 template <int P>
-__global__ void __launch_bounds__(kThreads, 1)
+struct ScanSmem {
+  static constexpr int N = 128, NB = N / 64, PB = P / 64;
+  static constexpr uint32_t CT = 0;               // C~ rows, K-major, NB blocks
+  static constexpr uint32_t BP = CT + NB * kBlk;  // Bpi_j (NB blocks); H_in hi/lo parts after the slot loop
+  static constexpr uint32_t XS = BP + NB * kBlk;  // Xs_j (PB blocks)
+  static constexpr uint32_t PM = XS + PB * kBlk;  // one 64-key half of Pm, or the decay-scaled Xs_j
+  static constexpr uint32_t BAR = PM + PB * kBlk; // fullB, fullX, done
+  static constexpr uint32_t CS = BAR + 64;        // cs[SUB], wsum[4], misc[2]
+  static constexpr uint32_t END = CS + SUB * 4 + 64;
+  static constexpr size_t bytes() { return 1024 + END; }
+};
+
+template <int P>
+__global__ void __launch_bounds__(kThreads, P == 64 ? 2 : 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_x, TcScanArgs a) {
-  constexpr int N = 128, NB = N / 64, PB = P / 64;
-  constexpr uint32_t CT_BYTES = NB * kBlk, BP_BYTES = NB * kBlk, XS_BYTES = PB * kBlk;
-  constexpr uint32_t STAGE = BP_BYTES + XS_BYTES, DX_BYTES = PB * kBlk, PM_BYTES = 2 * kBlk;
+  using Lay = ScanSmem<P>;
+  constexpr int N = 128, NB = Lay::NB, PB = Lay::PB;
   constexpr uint32_t TMEM_COLS = P == 64 ? 256 : 512;
   constexpr uint32_t COL_S = 0, COL_Y = 128, COL_SC = 128 + P;
   constexpr uint32_t ID_S = tc::idesc_f16(128, 128, false);
@@ -84,21 +99,22 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* CT = sm;
-  uint8_t* RING = CT + CT_BYTES;
-  uint8_t* DX = RING + 2 * STAGE;
-  uint8_t* PM = DX + DX_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(PM + PM_BYTES);  // [2]
-  uint64_t* done = full + 2;
-  float* cs_s = reinterpret_cast<float*>(full + 4);  // [SUB]
-  float* wsum = cs_s + SUB;                          // [4]
-  uint32_t* misc = reinterpret_cast<uint32_t*>(wsum + 4);  // tmem base, ticket
+  uint8_t* CT = sm + Lay::CT;
+  uint8_t* BP = sm + Lay::BP;
+  uint8_t* XS = sm + Lay::XS;
+  uint8_t* PM = sm + Lay::PM;
+  uint64_t* fullB = reinterpret_cast<uint64_t*>(sm + Lay::BAR);
+  uint64_t* fullX = fullB + 1;
+  uint64_t* done = fullB + 2;
+  float* cs_s = reinterpret_cast<float*>(sm + Lay::CS);
+  float* wsum = cs_s + SUB;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(wsum + 4);
 
   const Dims& d = a.d;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    tc::mbar_init(&full[0], 1);
-    tc::mbar_init(&full[1], 1);
+    tc::mbar_init(fullB, 1);
+    tc::mbar_init(fullX, 1);
     tc::mbar_init(done, 1);
     tc::fence_barrier_init();
     misc[1] = atomicAdd(a.ticket, 1u);
@@ -116,19 +132,59 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   const int nk = a.key_slots;
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
   volatile int never = 0;
-  int issued = 0;
+  int issuedB = 0, issuedX = 0;
 
-  auto issue_slot = [&](int i) {
-    const int stage = i & 1, j = a.key_slot0 + i;
-    uint8_t* sb = RING + stage * STAGE;
-    tc::mbar_arrive_expect_tx(&full[stage], STAGE);
-    for (int nb = 0; nb < NB; ++nb) tma_load_3d(sb + nb * kBlk, &tm_b, &full[stage], g * N + 64 * nb, j, row0);
-    for (int pb = 0; pb < PB; ++pb)
-      tma_load_3d(sb + BP_BYTES + pb * kBlk, &tm_x, &full[stage], h * P + 64 * pb, j, row0);
-    ++issued;
+  auto issue_b = [&](int i) {
+    tc::mbar_arrive_expect_tx(fullB, NB * kBlk);
+    for (int nb = 0; nb < NB; ++nb) tma_load_3d(BP + nb * kBlk, &tm_b, fullB, g * N + 64 * nb, a.key_slot0 + i, row0);
+    ++issuedB;
   };
-  if (tid == 0) {
-    for (int i = 0; i < nk && i < 2; ++i) issue_slot(i);
+  auto issue_x = [&](int i) {
+    tc::mbar_arrive_expect_tx(fullX, PB * kBlk);
+    for (int pb = 0; pb < PB; ++pb) tma_load_3d(XS + pb * kBlk, &tm_x, fullX, h * P + 64 * pb, a.key_slot0 + i, row0);
+    ++issuedX;
+  };
+  if (tid == 0) { issue_b(0); issue_x(0); }
+
+  // C~ rows: sum of the readout slots, loaded coalesced (16 lanes per 256-byte row), fp16 K-major swizzled
+  {
+    const int hl = lane >> 4, c16 = lane & 15;
+    for (int it = 0; it < 16; it += 8) {
+      float acc[8][8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
+      for (int j = a.read_slot0; j < a.read_slot0 + a.read_slots; ++j) {
+        uint4 q[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int r = 32 * warp + 2 * (it + u) + hl;
+          q[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (r < L)
+            q[u] = __ldg(reinterpret_cast<const uint4*>(a.cpi + ((size_t)(row0 + r) * d.k + j) * d.GN + (size_t)g * N +
+                                                        c16 * 8));
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const __half2* hq = reinterpret_cast<const __half2*>(&q[u]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(hq[e]);
+            acc[u][2 * e] += f.x;
+            acc[u][2 * e + 1] += f.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = 32 * warp + 2 * (it + u) + hl;
+        uint4 o;
+        o.x = pack_half2(acc[u][0], acc[u][1]); o.y = pack_half2(acc[u][2], acc[u][3]);
+        o.z = pack_half2(acc[u][4], acc[u][5]); o.w = pack_half2(acc[u][6], acc[u][7]);
+        *reinterpret_cast<uint4*>(CT + (c16 >> 3) * kBlk + tc::sw128_chunk(r, c16 & 7)) = o;
+      }
+    }
   }
 
   // cumulative log-decay of the sub-chunk (inclusive scan over the 128 threads)
@@ -139,61 +195,33 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     if (lane >= o) v += u;
   }
   if (lane == 31) wsum[warp] = v;
+  tc::fence_proxy_async();
   __syncthreads();
   for (int w = 0; w < warp; ++w) v += wsum[w];
   cs_s[tid] = v;
   __syncthreads();
   const float my_cs = v, cs_end = cs_s[L - 1];
-
-  // C~ rows (sum of the readout slots) -> fp16, K-major 128-byte-swizzled
-  {
-    const bool valid = tid < L;
-    for (int nb = 0; nb < NB; ++nb) {
-      for (int c = 0; c < 8; ++c) {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (valid) {
-          for (int j = a.read_slot0; j < a.read_slot0 + a.read_slots; ++j) {
-            const __half* src = a.cpi + ((size_t)(row0 + tid) * d.k + j) * d.GN + (size_t)g * N + nb * 64 + c * 8;
-            const uint4 q = *reinterpret_cast<const uint4*>(src);
-            const __half2* hq = reinterpret_cast<const __half2*>(&q);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __half22float2(hq[e]);
-              acc[2 * e] += f.x;
-              acc[2 * e + 1] += f.y;
-            }
-          }
-        }
-        uint4 o;
-        o.x = pack_half2(acc[0], acc[1]); o.y = pack_half2(acc[2], acc[3]);
-        o.z = pack_half2(acc[4], acc[5]); o.w = pack_half2(acc[6], acc[7]);
-        *reinterpret_cast<uint4*>(CT + nb * kBlk + tc::sw128_chunk(tid, c)) = o;
-      }
-    }
-  }
-  tc::fence_proxy_async();
+  const float dec_end = tid < L ? expf(cs_end - my_cs) : 0.f;
 
   bool ok = true;
   uint32_t done_phase = 0;
-  const float dec_end = tid < L ? expf(cs_end - my_cs) : 0.f;
   for (int i = 0; i < nk && ok; ++i) {
-    const int stage = i & 1;
-    uint8_t* BPs = RING + stage * STAGE;
-    uint8_t* XSs = BPs + BP_BYTES;
-    ok = tc::mbar_wait(&full[stage], (uint32_t)((i >> 1) & 1), &never);
+    const uint32_t par = (uint32_t)(i & 1);
+    ok = tc::mbar_wait(fullX, par, &never) && tc::mbar_wait(fullB, par, &never);
     if (!__syncthreads_and(ok)) { ok = false; break; }
-    // values scaled by the decay to the sub-chunk end (for the end state)
+    // values scaled by the decay to the sub-chunk end (for the end state), into the Pm buffer
     for (int pb = 0; pb < PB; ++pb) {
+#pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint32_t off = pb * kBlk + tc::sw128_chunk(tid, c);
-        uint4 q = *reinterpret_cast<const uint4*>(XSs + off);
+        uint4 q = *reinterpret_cast<const uint4*>(XS + off);
         __half2* hq = reinterpret_cast<__half2*>(&q);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __half22float2(hq[e]);
           hq[e] = __floats2half2_rn(f.x * dec_end, f.y * dec_end);
         }
-        *reinterpret_cast<uint4*>(DX + off) = q;
+        *reinterpret_cast<uint4*>(PM + off) = q;
       }
     }
     tc::fence_proxy_async();
@@ -201,7 +229,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     __syncthreads();
     tc::fence_after_sync();
     if (tid == 0) {
-      const uint32_t ct = tc::smem_u32(CT), bp = tc::smem_u32(BPs), dx = tc::smem_u32(DX);
+      const uint32_t ct = tc::smem_u32(CT), bp = tc::smem_u32(BP), dx = tc::smem_u32(PM);
 #pragma unroll
       for (int kk = 0; kk < N / 16; ++kk) {
         const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
@@ -218,44 +246,47 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     done_phase ^= 1u;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     tc::fence_after_sync();
-    // masked, decayed scores -> fp16 K-major swizzled rows of Pm
-    for (int q = 0; q < 4; ++q) {
-      uint32_t r[32];
-      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * q, r);
-      tc::tmem_ld_wait();
+    if (tid == 0 && i + 1 < nk) issue_b(i + 1);  // Bpi_i is no longer read
+    // masked, decayed scores, one 64-key half at a time -> fp16 K-major swizzled rows of Pm
+    for (int hk = 0; hk < 2 && ok; ++hk) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float f[8];
+      for (int q = 0; q < 2; ++q) {
+        uint32_t r[32];
+        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 64 * hk + 32 * q, r);
+        tc::tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int s = 32 * q + 8 * c + e;
-          f[e] = (s <= tid && tid < L) ? u2f(r[8 * c + e]) * expf(my_cs - cs_s[s]) : 0.f;
+        for (int c = 0; c < 4; ++c) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int s = 64 * hk + 32 * q + 8 * c + e;
+            f[e] = (s <= tid && tid < L) ? u2f(r[8 * c + e]) * expf(my_cs - cs_s[s]) : 0.f;
+          }
+          uint4 o;
+          o.x = pack_half2(f[0], f[1]); o.y = pack_half2(f[2], f[3]);
+          o.z = pack_half2(f[4], f[5]); o.w = pack_half2(f[6], f[7]);
+          *reinterpret_cast<uint4*>(PM + tc::sw128_chunk(tid, 4 * q + c)) = o;
         }
-        uint4 o;
-        o.x = pack_half2(f[0], f[1]); o.y = pack_half2(f[2], f[3]);
-        o.z = pack_half2(f[4], f[5]); o.w = pack_half2(f[6], f[7]);
-        const int s0 = 32 * q + 8 * c;
-        *reinterpret_cast<uint4*>(PM + (s0 >> 6) * kBlk + tc::sw128_chunk(tid, (s0 & 63) >> 3)) = o;
       }
-    }
-    tc::fence_proxy_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    if (tid == 0) {
-      const uint32_t pm = tc::smem_u32(PM), xs = tc::smem_u32(XSs);
+      tc::fence_proxy_async();
+      tc::fence_before_sync();
+      __syncthreads();
+      tc::fence_after_sync();
+      if (tid == 0) {
+        const uint32_t pm = tc::smem_u32(PM), xs = tc::smem_u32(XS) + hk * 8192;
 #pragma unroll
-      for (int kk = 0; kk < SUB / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
-        tc::mma_f16(tmem + COL_Y, tc::sdesc_kmajor_sw128(pm + off), tc::sdesc_mnmajor_sw128(xs + kk * 2048, kBlk),
-                    ID_Y, (i > 0) || (kk > 0));
+        for (int kk = 0; kk < 4; ++kk) {
+          tc::mma_f16(tmem + COL_Y, tc::sdesc_kmajor_sw128(pm + kk * 32), tc::sdesc_mnmajor_sw128(xs + kk * 2048, kBlk),
+                      ID_Y, (i > 0) || (hk > 0) || (kk > 0));
+        }
+        tc::mma_commit(done);
       }
-      tc::mma_commit(done);
+      ok = tc::mbar_wait(done, done_phase, &never);
+      done_phase ^= 1u;
+      if (!__syncthreads_and(ok)) { ok = false; break; }
+      tc::fence_after_sync();
     }
-    ok = tc::mbar_wait(done, done_phase, &never);
-    done_phase ^= 1u;
-    if (!__syncthreads_and(ok)) { ok = false; break; }
-    if (tid == 0 && i + 2 < nk) issue_slot(i + 2);
+    if (tid == 0 && ok && i + 1 < nk) issue_x(i + 1);  // Xs_i is no longer read
   }
 
   if (ok) {
@@ -276,47 +307,56 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     float* cst = chunk_start ? a.chunk_states + (((size_t)b * d.H + h) * d.nc + t0 / d.Q) * NP : nullptr;
     float* fin = (last && a.final_state) ? a.final_state + (size_t)bh * NP : nullptr;
     const float dend = expf(cs_end);
-    uint8_t* HH = RING;                 // the ring is free now: fp16 hi and lo parts of H_in
-    uint8_t* HL = RING + PB * kBlk;
+    uint8_t* HH = BP;  // Bpi_j and Xs_j are consumed: fp16 hi and lo parts of H_in
+    uint8_t* HL = BP + PB * kBlk;
     bool range_bad = false;
-    for (int q = 0; q < P / 32; ++q) {
-      uint32_t r[32];
-      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_SC + 32 * q, r);
-      tc::tmem_ld_wait();
-      const size_t ro = (size_t)tid * P + 32 * q;
+#pragma unroll 1
+    for (int q2 = 0; q2 < P / 64; ++q2) {
+      float4 hv[16];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float hp[8], hi[8], lo[8];
+      for (int u = 0; u < 16; ++u)
+        hv[u] = hin ? __ldcg(reinterpret_cast<const float4*>(hin + (size_t)tid * P + 64 * q2 + 4 * u))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < 8; e += 4) {
-          float4 x = hin ? __ldcg(reinterpret_cast<const float4*>(hin + ro + 8 * c + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
-          hp[e] = x.x; hp[e + 1] = x.y; hp[e + 2] = x.z; hp[e + 3] = x.w;
+      for (int q = 0; q < 2; ++q) {
+        uint32_t r[32];
+        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_SC + 64 * q2 + 32 * q, r);
+        tc::tmem_ld_wait();
+        const size_t ro = (size_t)tid * P + 64 * q2 + 32 * q;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float hp[8], hi[8], lo[8];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float4 x = hv[8 * q + 2 * c + e];
+            hp[4 * e] = x.x; hp[4 * e + 1] = x.y; hp[4 * e + 2] = x.z; hp[4 * e + 3] = x.w;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; e += 4) {
+            const float4 o = make_float4(fmaf(dend, hp[e], u2f(r[8 * c + e])), fmaf(dend, hp[e + 1], u2f(r[8 * c + e + 1])),
+                                         fmaf(dend, hp[e + 2], u2f(r[8 * c + e + 2])),
+                                         fmaf(dend, hp[e + 3], u2f(r[8 * c + e + 3])));
+            __stcg(reinterpret_cast<float4*>(hout + ro + 8 * c + e), o);
+            if (fin) *reinterpret_cast<float4*>(fin + ro + 8 * c + e) = o;
+            if (cst) *reinterpret_cast<float4*>(cst + ro + 8 * c + e) = make_float4(hp[e], hp[e + 1], hp[e + 2], hp[e + 3]);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const __half hh = __float2half_rn(hp[e]);
+            hi[e] = __half2float(hh);
+            lo[e] = hp[e] - hi[e];
+            range_bad |= !(fabsf(hp[e]) <= kF16Max);
+          }
+          const int p0 = 64 * q2 + 32 * q + 8 * c;
+          const uint32_t off = (p0 >> 6) * kBlk + tc::sw128_chunk(tid, (p0 & 63) >> 3);
+          uint4 oh, ol;
+          oh.x = pack_half2(hi[0], hi[1]); oh.y = pack_half2(hi[2], hi[3]);
+          oh.z = pack_half2(hi[4], hi[5]); oh.w = pack_half2(hi[6], hi[7]);
+          ol.x = pack_half2(lo[0], lo[1]); ol.y = pack_half2(lo[2], lo[3]);
+          ol.z = pack_half2(lo[4], lo[5]); ol.w = pack_half2(lo[6], lo[7]);
+          *reinterpret_cast<uint4*>(HH + off) = oh;
+          *reinterpret_cast<uint4*>(HL + off) = ol;
         }
-#pragma unroll
-        for (int e = 0; e < 8; e += 4) {
-          float4 o = make_float4(fmaf(dend, hp[e], u2f(r[8 * c + e])), fmaf(dend, hp[e + 1], u2f(r[8 * c + e + 1])),
-                                 fmaf(dend, hp[e + 2], u2f(r[8 * c + e + 2])), fmaf(dend, hp[e + 3], u2f(r[8 * c + e + 3])));
-          __stcg(reinterpret_cast<float4*>(hout + ro + 8 * c + e), o);
-          if (fin) *reinterpret_cast<float4*>(fin + ro + 8 * c + e) = o;
-          if (cst) *reinterpret_cast<float4*>(cst + ro + 8 * c + e) =
-              make_float4(hp[e], hp[e + 1], hp[e + 2], hp[e + 3]);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const __half hh = __float2half_rn(hp[e]);
-          hi[e] = __half2float(hh);
-          lo[e] = hp[e] - hi[e];
-          range_bad |= !(fabsf(hp[e]) <= kF16Max);
-        }
-        const int p0 = 32 * q + 8 * c;
-        const uint32_t off = (p0 >> 6) * kBlk + tc::sw128_chunk(tid, (p0 & 63) >> 3);
-        uint4 oh, ol;
-        oh.x = pack_half2(hi[0], hi[1]); oh.y = pack_half2(hi[2], hi[3]);
-        oh.z = pack_half2(hi[4], hi[5]); oh.w = pack_half2(hi[6], hi[7]);
-        ol.x = pack_half2(lo[0], lo[1]); ol.y = pack_half2(lo[2], lo[3]);
-        ol.z = pack_half2(lo[4], lo[5]); ol.w = pack_half2(lo[6], lo[7]);
-        *reinterpret_cast<uint4*>(HH + off) = oh;
-        *reinterpret_cast<uint4*>(HL + off) = ol;
       }
     }
     if (range_bad) atomicOr(a.st, ST_RANGE);
@@ -327,7 +367,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     tc::fence_after_sync();
     if (tid == 0) {
       st_release(a.flags + (size_t)bh * a.nsub + csub, 1u);
-      const uint32_t ct = tc::smem_u32(CT), hh = tc::smem_u32(HH), hl = tc::smem_u32(HL);
+      const uint32_t ct = tc::smem_u32(CT), hh = tc::smem_u32(HH), hl2 = tc::smem_u32(HL);
 #pragma unroll
       for (int kk = 0; kk < N / 16; ++kk) {
         const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
@@ -337,7 +377,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
 #pragma unroll
       for (int kk = 0; kk < N / 16; ++kk) {
         const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
-        tc::mma_f16(tmem + COL_S, tc::sdesc_kmajor_sw128(ct + off), tc::sdesc_mnmajor_sw128(hl + kk * 2048, kBlk),
+        tc::mma_f16(tmem + COL_S, tc::sdesc_kmajor_sw128(ct + off), tc::sdesc_mnmajor_sw128(hl2 + kk * 2048, kBlk),
                     ID_Y, 1);
       }
       tc::mma_commit(done);
@@ -383,16 +423,14 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
       }
     }
   }
-  if (!ok) {
-    if (tid == 0) {
-      atomicOr(a.st, ST_TIMEOUT);
-      // successors must not wait on a sub-chunk that gave up
-      st_release(a.flags + (size_t)bh * a.nsub + csub, 1u);
-    }
+  if (!ok && tid == 0) {
+    atomicOr(a.st, ST_TIMEOUT);
+    st_release(a.flags + (size_t)bh * a.nsub + csub, 1u);  // successors must not wait on a CTA that gave up
   }
   // no copy may still be landing in shared memory when the CTA exits
   if (tid == 0) {
-    for (int i = (issued > 2 ? issued - 2 : 0); i < issued; ++i) tc::mbar_wait(&full[i & 1], (uint32_t)((i >> 1) & 1), &never);
+    if (issuedB > 0) tc::mbar_wait(fullB, (uint32_t)((issuedB - 1) & 1), &never);
+    if (issuedX > 0) tc::mbar_wait(fullX, (uint32_t)((issuedX - 1) & 1), &never);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -400,13 +438,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, TMEM_COLS);
   }
-}
-
-template <int P>
-size_t smem_bytes() {
-  constexpr uint32_t NB = 2, PB = P / 64;
-  return 1024 + (size_t)(NB * kBlk) + 2 * (size_t)(NB * kBlk + PB * kBlk) + PB * kBlk + 2 * kBlk + 64 +
-         SUB * 4 + 64;
 }
 
 }  // namespace
@@ -434,12 +465,12 @@ cudaError_t launch_scan_tc(const Dims& d, const ScanArgs& s, unsigned* lb, float
   const int grid = d.Bsz * d.H * a.nsub;
   cudaError_t e;
   if (d.P == 64) {
-    const size_t sm = smem_bytes<64>();
+    const size_t sm = ScanSmem<64>::bytes();
     e = cudaFuncSetAttribute(scan_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     scan_tc_kernel<64><<<grid, kThreads, sm, stream>>>(tb, tx, a);
   } else {
-    const size_t sm = smem_bytes<128>();
+    const size_t sm = ScanSmem<128>::bytes();
     e = cudaFuncSetAttribute(scan_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     scan_tc_kernel<128><<<grid, kThreads, sm, stream>>>(tb, tx, a);
