@@ -307,8 +307,8 @@ def report(args, w, world, total_ms, e2e_ms, stage_ms, launches, clocks, h2d, d2
     K = args.steps
     tokens = w.M * world * K
     value = tokens / (total_ms / 1e3)
-    # dominant kernel stage and its roofline
-    dom = max(stage_ms, key=stage_ms.get)
+    # dominant kernel stage (among those with a work model) and its roofline
+    dom = max((n for n in stage_ms if n in wk), key=stage_ms.get)
     avg_s = stage_ms[dom] / K / 1e3
     bound = "tensor" if dom == "expert_proj_mix" else "hbm"
     if bound == "tensor":

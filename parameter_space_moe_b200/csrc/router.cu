@@ -9,7 +9,7 @@
 // The E + H dot products per token form a skinny GEMM [M x D] x [D x (E + H)].  bf16 layers run it on
 // the warp-level tensor-core path (mma.sync m16n8k16, fp32 accumulate): a CTA of 4 warps owns 64
 // tokens and streams X and the stacked [W_r; W_dt] through padded shared memory in 64-wide K chunks
-// (cp.async, double buffered).  The fp32 layer keeps a CUDA-core kernel (one warp per token, fixed xor
+// (cp.async, 4-stage pipeline).  The fp32 layer keeps a CUDA-core kernel (one warp per token, fixed xor
 // butterfly reductions).  Both finish with the same per-token top-k / softmax / dt code.
 #include "common.cuh"
 
@@ -96,6 +96,7 @@ constexpr int kMT = 64;           // tokens per CTA
 constexpr int kKC = 64;           // K chunk
 constexpr int kLd = kKC + 8;      // padded shared row (144 B: conflict-free ldmatrix)
 constexpr int kMaxNT = 16;        // up to 128 logits per token
+constexpr int kStagesR = 4;       // cp.async pipeline depth
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
   const uint32_t s = (uint32_t)__cvta_generic_to_shared(dst);
@@ -125,40 +126,43 @@ router_mma_kernel(Dims d, int RP, const __nv_bfloat16* __restrict__ X, const __n
                   const __nv_bfloat16* __restrict__ Wdt, const float* __restrict__ bdt, int32_t* __restrict__ idx_out,
                   float* __restrict__ w_out, float* __restrict__ dt_out) {
   extern __shared__ __align__(16) uint8_t rsm[];
-  __nv_bfloat16* Xs = reinterpret_cast<__nv_bfloat16*>(rsm);   // [2][kMT][kLd]
-  __nv_bfloat16* Ws = Xs + 2 * kMT * kLd;                        // [2][RP][kLd]
-  float* G = reinterpret_cast<float*>(Ws + 2 * RP * kLd);        // [kMT][RP + 1]
+  __nv_bfloat16* Xs = reinterpret_cast<__nv_bfloat16*>(rsm);   // [stages][kMT][kLd]
+  __nv_bfloat16* Ws = Xs + kStagesR * kMT * kLd;                 // [stages][RP][kLd]
+  float* G = reinterpret_cast<float*>(Ws + kStagesR * RP * kLd); // [kMT][RP + 1]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tok0 = blockIdx.x * kMT;
   const int R = d.E + d.H, NT = RP / 8, nkc = d.D / kKC;
 
   auto load = [&](int stage, int kc) {
-    const int k0 = kc * kKC;
-    __nv_bfloat16* xs = Xs + stage * kMT * kLd;
-    __nv_bfloat16* ws = Ws + stage * RP * kLd;
-    for (int i = tid; i < kMT * (kKC / 8); i += 128) {
-      const int r = i >> 3, c = i & 7;
-      const bool v = tok0 + r < d.M;
-      cp_async16(xs + r * kLd + 8 * c, X + (size_t)(v ? tok0 + r : 0) * d.D + k0 + 8 * c, v);
+    if (kc < nkc) {
+      const int k0 = kc * kKC;
+      __nv_bfloat16* xs = Xs + stage * kMT * kLd;
+      __nv_bfloat16* ws = Ws + stage * RP * kLd;
+      for (int i = tid; i < kMT * (kKC / 8); i += 128) {
+        const int r = i >> 3, c = i & 7;
+        const bool v = tok0 + r < d.M;
+        cp_async16(xs + r * kLd + 8 * c, X + (size_t)(v ? tok0 + r : 0) * d.D + k0 + 8 * c, v);
+      }
+      for (int i = tid; i < RP * (kKC / 8); i += 128) {
+        const int r = i >> 3, c = i & 7;
+        const __nv_bfloat16* src = r < d.E ? Wr + (size_t)r * d.D : Wdt + (size_t)(r < R ? r - d.E : 0) * d.D;
+        cp_async16(ws + r * kLd + 8 * c, src + k0 + 8 * c, r < R);
+      }
     }
-    for (int i = tid; i < RP * (kKC / 8); i += 128) {
-      const int r = i >> 3, c = i & 7;
-      const __nv_bfloat16* src = r < d.E ? Wr + (size_t)r * d.D : Wdt + (size_t)(r < R ? r - d.E : 0) * d.D;
-      cp_async16(ws + r * kLd + 8 * c, src + k0 + 8 * c, r < R);
-    }
-    cp_async_commit();
+    cp_async_commit();  // an empty group past the end keeps the group count uniform
   };
 
   float acc[kMaxNT][4];
 #pragma unroll
   for (int n = 0; n < kMaxNT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
 
-  load(0, 0);
+#pragma unroll
+  for (int st = 0; st < kStagesR - 1; ++st) load(st, st);
   for (int kc = 0; kc < nkc; ++kc) {
-    const int stage = kc & 1;
-    if (kc + 1 < nkc) { load(stage ^ 1, kc + 1); cp_async_wait<1>(); }
-    else cp_async_wait<0>();
+    const int stage = kc % kStagesR;
+    cp_async_wait<kStagesR - 2>();
     __syncthreads();
+    load((kc + kStagesR - 1) % kStagesR, kc + kStagesR - 1);  // refills the stage read in iteration kc - 1
     const uint32_t xb = (uint32_t)__cvta_generic_to_shared(Xs + stage * kMT * kLd);
     const uint32_t wb = (uint32_t)__cvta_generic_to_shared(Ws + stage * RP * kLd);
 #pragma unroll
@@ -176,8 +180,9 @@ router_mma_kernel(Dims d, int RP, const __nv_bfloat16* __restrict__ X, const __n
         }
       }
     }
-    __syncthreads();
   }
+  cp_async_wait<0>();
+  __syncthreads();
   // logits -> shared memory: c0,c1 at (row g, cols 2c, 2c+1), c2,c3 at (row g + 8, same cols)
   const int gr = lane >> 2, gc = 2 * (lane & 3);
 #pragma unroll
@@ -203,7 +208,7 @@ cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w,
   const int R = d.E + d.H;
   if (d.dtype == SWIMBA_BF16 && R <= 8 * kMaxNT) {
     const int RP = (R + 15) / 16 * 16;
-    const size_t smem = (size_t)2 * (kMT + RP) * kLd * 2 + (size_t)kMT * (RP + 1) * 4;
+    const size_t smem = (size_t)kStagesR * (kMT + RP) * kLd * 2 + (size_t)kMT * (RP + 1) * 4;
     cudaError_t e = cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     router_mma_kernel<<<ceil_div(d.M, kMT), 128, smem, s>>>(d, RP, (const __nv_bfloat16*)X,

@@ -22,7 +22,7 @@ namespace swimba {
 
 namespace {
 constexpr int SUB = 128;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr uint32_t kBlk = SUB * 128;  // one 64-wide column block of 128 swizzled 128-byte rows
 constexpr uint32_t kFlagPolls = 1u << 22;
 
@@ -80,16 +80,18 @@ struct ScanSmem {
   static constexpr uint32_t XS = BP + NB * kBlk;  // Xs_j (PB blocks)
   static constexpr uint32_t PM = XS + PB * kBlk;  // one 64-key half of Pm, or the decay-scaled Xs_j
   static constexpr uint32_t BAR = PM + PB * kBlk; // fullB, fullX, done
-  static constexpr uint32_t CS = BAR + 64;        // cs[SUB], wsum[4], misc[2]
-  static constexpr uint32_t END = CS + SUB * 4 + 64;
+  static constexpr uint32_t CS = BAR + 64;        // cs[SUB], fs[SUB], wsum[4], misc[2]
+  static constexpr uint32_t END = CS + 2 * SUB * 4 + 64;
   static constexpr size_t bytes() { return 1024 + END; }
 };
 
+// Thread layout: 8 warps; thread (row = tid % 128, half = tid / 128).  Warps w and w + 4 read the same
+// TMEM lane quarter (w % 4) and split the columns of each row between them.
 template <int P>
 __global__ void __launch_bounds__(kThreads, P == 64 ? 2 : 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_x, TcScanArgs a) {
   using Lay = ScanSmem<P>;
-  constexpr int N = 128, NB = Lay::NB, PB = Lay::PB;
+  constexpr int N = 128, NB = Lay::NB, PB = Lay::PB, PH = P / 2;
   constexpr uint32_t TMEM_COLS = P == 64 ? 256 : 512;
   constexpr uint32_t COL_S = 0, COL_Y = 128, COL_SC = 128 + P;
   constexpr uint32_t ID_S = tc::idesc_f16(128, 128, false);
@@ -107,11 +109,13 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   uint64_t* fullX = fullB + 1;
   uint64_t* done = fullB + 2;
   float* cs_s = reinterpret_cast<float*>(sm + Lay::CS);
-  float* wsum = cs_s + SUB;
+  float* fs_s = cs_s + SUB;
+  float* wsum = fs_s + SUB;
   uint32_t* misc = reinterpret_cast<uint32_t*>(wsum + 4);
 
   const Dims& d = a.d;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = tid & (SUB - 1), half = tid >> 7;
   if (tid == 0) {
     tc::mbar_init(fullB, 1);
     tc::mbar_init(fullX, 1);
@@ -130,7 +134,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   const int t0 = csub * SUB, L = min(SUB, d.T - t0);
   const int row0 = b * d.T + t0;
   const int nk = a.key_slots;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   volatile int never = 0;
   int issuedB = 0, issuedX = 0;
 
@@ -146,25 +150,42 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   };
   if (tid == 0) { issue_b(0); issue_x(0); }
 
-  // C~ rows: sum of the readout slots, loaded coalesced (16 lanes per 256-byte row), fp16 K-major swizzled
+  // C~ rows: sum of the readout slots, loaded coalesced (16 lanes per 256-byte row), fp16 K-major swizzled.
+  // Warp w covers rows 16w .. 16w + 15.  Two slots are added as fp16 pairs (the correctly rounded sum).
   {
     const int hl = lane >> 4, c16 = lane & 15;
-    for (int it = 0; it < 16; it += 8) {
+    uint4 q[8];
+    auto load8 = [&](int j, uint4 (&dst)[8]) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = 16 * warp + 2 * u + hl;
+        dst[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (r < L)
+          dst[u] = __ldg(reinterpret_cast<const uint4*>(a.cpi + ((size_t)(row0 + r) * d.k + j) * d.GN + (size_t)g * N +
+                                                        c16 * 8));
+      }
+    };
+    if (a.read_slots == 1 || a.read_slots == 2) {
+      load8(a.read_slot0, q);
+      if (a.read_slots == 2) {
+        uint4 q2[8];
+        load8(a.read_slot0 + 1, q2);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          __half2* x = reinterpret_cast<__half2*>(&q[u]);
+          const __half2* y = reinterpret_cast<const __half2*>(&q2[u]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[e] = __hadd2(x[e], y[e]);
+        }
+      }
+    } else {
       float acc[8][8];
 #pragma unroll
       for (int u = 0; u < 8; ++u)
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
       for (int j = a.read_slot0; j < a.read_slot0 + a.read_slots; ++j) {
-        uint4 q[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int r = 32 * warp + 2 * (it + u) + hl;
-          q[u] = make_uint4(0u, 0u, 0u, 0u);
-          if (r < L)
-            q[u] = __ldg(reinterpret_cast<const uint4*>(a.cpi + ((size_t)(row0 + r) * d.k + j) * d.GN + (size_t)g * N +
-                                                        c16 * 8));
-        }
+        load8(j, q);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const __half2* hq = reinterpret_cast<const __half2*>(&q[u]);
@@ -178,30 +199,40 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int r = 32 * warp + 2 * (it + u) + hl;
-        uint4 o;
-        o.x = pack_half2(acc[u][0], acc[u][1]); o.y = pack_half2(acc[u][2], acc[u][3]);
-        o.z = pack_half2(acc[u][4], acc[u][5]); o.w = pack_half2(acc[u][6], acc[u][7]);
-        *reinterpret_cast<uint4*>(CT + (c16 >> 3) * kBlk + tc::sw128_chunk(r, c16 & 7)) = o;
+        q[u].x = pack_half2(acc[u][0], acc[u][1]); q[u].y = pack_half2(acc[u][2], acc[u][3]);
+        q[u].z = pack_half2(acc[u][4], acc[u][5]); q[u].w = pack_half2(acc[u][6], acc[u][7]);
       }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int r = 16 * warp + 2 * u + hl;
+      *reinterpret_cast<uint4*>(CT + (c16 >> 3) * kBlk + tc::sw128_chunk(r, c16 & 7)) = q[u];
     }
   }
 
-  // cumulative log-decay of the sub-chunk (inclusive scan over the 128 threads)
-  float v = tid < L ? a.dt[(size_t)(row0 + tid) * d.H + h] * a.A[h] : 0.f;
+  // cumulative log-decay of the sub-chunk (inclusive scan over the 128 rows)
+  float v = 0.f;
+  if (half == 0) {
+    v = row < L ? a.dt[(size_t)(row0 + row) * d.H + h] * a.A[h] : 0.f;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const float u = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += u;
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    if (lane == 31) wsum[warp] = v;
   }
-  if (lane == 31) wsum[warp] = v;
   tc::fence_proxy_async();
   __syncthreads();
-  for (int w = 0; w < warp; ++w) v += wsum[w];
-  cs_s[tid] = v;
+  if (half == 0) {
+    for (int w = 0; w < warp; ++w) v += wsum[w];
+    cs_s[row] = v;
+  }
   __syncthreads();
-  const float my_cs = v, cs_end = cs_s[L - 1];
-  const float dec_end = tid < L ? expf(cs_end - my_cs) : 0.f;
+  const float my_cs = cs_s[row], cs_end = cs_s[L - 1];
+  // decay factorisation over 32-key blocks: exp(cs_t - cs_s) = exp(cs_t - cs_{32b}) * exp(cs_{32b} - cs_s)
+  if (half == 0) fs_s[row] = expf(cs_s[row & ~31] - my_cs);
+  const float dec_end = row < L ? expf(cs_end - my_cs) : 0.f;
+  __syncthreads();
 
   bool ok = true;
   uint32_t done_phase = 0;
@@ -210,10 +241,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     ok = tc::mbar_wait(fullX, par, &never) && tc::mbar_wait(fullB, par, &never);
     if (!__syncthreads_and(ok)) { ok = false; break; }
     // values scaled by the decay to the sub-chunk end (for the end state), into the Pm buffer
+#pragma unroll
     for (int pb = 0; pb < PB; ++pb) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t off = pb * kBlk + tc::sw128_chunk(tid, c);
+      for (int c = 4 * half; c < 4 * half + 4; ++c) {
+        const uint32_t off = pb * kBlk + tc::sw128_chunk(row, c);
         uint4 q = *reinterpret_cast<const uint4*>(XS + off);
         __half2* hq = reinterpret_cast<__half2*>(&q);
 #pragma unroll
@@ -247,26 +279,26 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     if (!__syncthreads_and(ok)) { ok = false; break; }
     tc::fence_after_sync();
     if (tid == 0 && i + 1 < nk) issue_b(i + 1);  // Bpi_i is no longer read
-    // masked, decayed scores, one 64-key half at a time -> fp16 K-major swizzled rows of Pm
+    // masked, decayed scores, one 64-key half at a time -> fp16 K-major swizzled rows of Pm; this thread
+    // takes the 32 keys of block 2*hk + half, whose decays share one factor exp(cs_t - cs_{32b})
     for (int hk = 0; hk < 2 && ok; ++hk) {
+      const int kb = 2 * hk + half;
+      const float et = (32 * kb <= row && row < L) ? expf(my_cs - cs_s[32 * kb]) : 0.f;
+      uint32_t r[32];
+      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * kb, r);
+      tc::tmem_ld_wait();
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t r[32];
-        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 64 * hk + 32 * q, r);
-        tc::tmem_ld_wait();
+      for (int c = 0; c < 4; ++c) {
+        float f[8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float f[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int s = 64 * hk + 32 * q + 8 * c + e;
-            f[e] = (s <= tid && tid < L) ? u2f(r[8 * c + e]) * expf(my_cs - cs_s[s]) : 0.f;
-          }
-          uint4 o;
-          o.x = pack_half2(f[0], f[1]); o.y = pack_half2(f[2], f[3]);
-          o.z = pack_half2(f[4], f[5]); o.w = pack_half2(f[6], f[7]);
-          *reinterpret_cast<uint4*>(PM + tc::sw128_chunk(tid, 4 * q + c)) = o;
+        for (int e = 0; e < 8; ++e) {
+          const int s = 32 * kb + 8 * c + e;
+          f[e] = s <= row ? u2f(r[8 * c + e]) * (et * fs_s[s]) : 0.f;
         }
+        uint4 o;
+        o.x = pack_half2(f[0], f[1]); o.y = pack_half2(f[2], f[3]);
+        o.z = pack_half2(f[4], f[5]); o.w = pack_half2(f[6], f[7]);
+        *reinterpret_cast<uint4*>(PM + tc::sw128_chunk(row, 4 * half + c)) = o;
       }
       tc::fence_proxy_async();
       tc::fence_before_sync();
@@ -295,78 +327,79 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     if (tid == 0 && csub > 0) {
       const unsigned* f = a.flags + (size_t)bh * a.nsub + csub - 1;
       uint32_t n = 0;
-      while (ld_acquire(f) == 0u && n < kFlagPolls) { __nanosleep(64); ++n; }
+      while (ld_acquire(f) == 0u && n < kFlagPolls) {
+        if (n > 64) __nanosleep(32);
+        ++n;
+      }
       if (n == kFlagPolls) atomicOr(a.st, ST_TIMEOUT);
     }
     __syncthreads();
     const float* hin = csub > 0 ? a.exch + ((size_t)bh * a.nsub + csub - 1) * NP
                                 : (a.init ? a.init + (size_t)bh * NP : nullptr);
     float* hout = a.exch + ((size_t)bh * a.nsub + csub) * NP;
+    const float dend = expf(cs_end);
+    const size_t rbase = (size_t)row * P + half * PH;
+    // this thread's half row of H_in (kept for the fp16 split below) and H_out = exp(cs_end) H_in + Sc
+    float4 hv[PH / 4];
+#pragma unroll
+    for (int u = 0; u < PH / 4; ++u)
+      hv[u] = hin ? __ldcg(reinterpret_cast<const float4*>(hin + rbase + 4 * u)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < PH / 32; ++q) {
+      uint32_t r[32];
+      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_SC + half * PH + 32 * q, r);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float4 x = hv[8 * q + u];
+        const float4 o = make_float4(fmaf(dend, x.x, u2f(r[4 * u])), fmaf(dend, x.y, u2f(r[4 * u + 1])),
+                                     fmaf(dend, x.z, u2f(r[4 * u + 2])), fmaf(dend, x.w, u2f(r[4 * u + 3])));
+        __stcg(reinterpret_cast<float4*>(hout + rbase + 32 * q + 4 * u), o);
+      }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) st_release(a.flags + (size_t)bh * a.nsub + csub, 1u);
+    // off the hand-off chain: requested states, and the fp16 hi/lo split of H_in for the readout product
     const bool last = t0 + L == d.T;
     const bool chunk_start = a.chunk_states && (t0 % d.Q) == 0;
     float* cst = chunk_start ? a.chunk_states + (((size_t)b * d.H + h) * d.nc + t0 / d.Q) * NP : nullptr;
     float* fin = (last && a.final_state) ? a.final_state + (size_t)bh * NP : nullptr;
-    const float dend = expf(cs_end);
-    uint8_t* HH = BP;  // Bpi_j and Xs_j are consumed: fp16 hi and lo parts of H_in
+    uint8_t* HH = BP;  // Bpi_j and Xs_j are consumed
     uint8_t* HL = BP + PB * kBlk;
     bool range_bad = false;
-#pragma unroll 1
-    for (int q2 = 0; q2 < P / 64; ++q2) {
-      float4 hv[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u)
-        hv[u] = hin ? __ldcg(reinterpret_cast<const float4*>(hin + (size_t)tid * P + 64 * q2 + 4 * u))
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < PH / 4; ++u) {
+      if (cst) *reinterpret_cast<float4*>(cst + rbase + 4 * u) = hv[u];
+      if (fin) *reinterpret_cast<float4*>(fin + rbase + 4 * u) = __ldcg(reinterpret_cast<const float4*>(hout + rbase + 4 * u));
+    }
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t r[32];
-        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_SC + 64 * q2 + 32 * q, r);
-        tc::tmem_ld_wait();
-        const size_t ro = (size_t)tid * P + 64 * q2 + 32 * q;
+    for (int c = 0; c < PH / 8; ++c) {
+      float hp[8], hi[8], lo[8];
+      hp[0] = hv[2 * c].x; hp[1] = hv[2 * c].y; hp[2] = hv[2 * c].z; hp[3] = hv[2 * c].w;
+      hp[4] = hv[2 * c + 1].x; hp[5] = hv[2 * c + 1].y; hp[6] = hv[2 * c + 1].z; hp[7] = hv[2 * c + 1].w;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float hp[8], hi[8], lo[8];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float4 x = hv[8 * q + 2 * c + e];
-            hp[4 * e] = x.x; hp[4 * e + 1] = x.y; hp[4 * e + 2] = x.z; hp[4 * e + 3] = x.w;
-          }
-#pragma unroll
-          for (int e = 0; e < 8; e += 4) {
-            const float4 o = make_float4(fmaf(dend, hp[e], u2f(r[8 * c + e])), fmaf(dend, hp[e + 1], u2f(r[8 * c + e + 1])),
-                                         fmaf(dend, hp[e + 2], u2f(r[8 * c + e + 2])),
-                                         fmaf(dend, hp[e + 3], u2f(r[8 * c + e + 3])));
-            __stcg(reinterpret_cast<float4*>(hout + ro + 8 * c + e), o);
-            if (fin) *reinterpret_cast<float4*>(fin + ro + 8 * c + e) = o;
-            if (cst) *reinterpret_cast<float4*>(cst + ro + 8 * c + e) = make_float4(hp[e], hp[e + 1], hp[e + 2], hp[e + 3]);
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const __half hh = __float2half_rn(hp[e]);
-            hi[e] = __half2float(hh);
-            lo[e] = hp[e] - hi[e];
-            range_bad |= !(fabsf(hp[e]) <= kF16Max);
-          }
-          const int p0 = 64 * q2 + 32 * q + 8 * c;
-          const uint32_t off = (p0 >> 6) * kBlk + tc::sw128_chunk(tid, (p0 & 63) >> 3);
-          uint4 oh, ol;
-          oh.x = pack_half2(hi[0], hi[1]); oh.y = pack_half2(hi[2], hi[3]);
-          oh.z = pack_half2(hi[4], hi[5]); oh.w = pack_half2(hi[6], hi[7]);
-          ol.x = pack_half2(lo[0], lo[1]); ol.y = pack_half2(lo[2], lo[3]);
-          ol.z = pack_half2(lo[4], lo[5]); ol.w = pack_half2(lo[6], lo[7]);
-          *reinterpret_cast<uint4*>(HH + off) = oh;
-          *reinterpret_cast<uint4*>(HL + off) = ol;
-        }
+      for (int e = 0; e < 8; ++e) {
+        hi[e] = __half2float(__float2half_rn(hp[e]));
+        lo[e] = hp[e] - hi[e];
+        range_bad |= !(fabsf(hp[e]) <= kF16Max);
       }
+      const int p0 = half * PH + 8 * c;
+      const uint32_t off = (p0 >> 6) * kBlk + tc::sw128_chunk(row, (p0 & 63) >> 3);
+      uint4 oh, ol;
+      oh.x = pack_half2(hi[0], hi[1]); oh.y = pack_half2(hi[2], hi[3]);
+      oh.z = pack_half2(hi[4], hi[5]); oh.w = pack_half2(hi[6], hi[7]);
+      ol.x = pack_half2(lo[0], lo[1]); ol.y = pack_half2(lo[2], lo[3]);
+      ol.z = pack_half2(lo[4], lo[5]); ol.w = pack_half2(lo[6], lo[7]);
+      *reinterpret_cast<uint4*>(HH + off) = oh;
+      *reinterpret_cast<uint4*>(HL + off) = ol;
     }
     if (range_bad) atomicOr(a.st, ST_RANGE);
-    __threadfence();
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     if (tid == 0) {
-      st_release(a.flags + (size_t)bh * a.nsub + csub, 1u);
       const uint32_t ct = tc::smem_u32(CT), hh = tc::smem_u32(HH), hl2 = tc::smem_u32(HL);
 #pragma unroll
       for (int kk = 0; kk < N / 16; ++kk) {
@@ -386,14 +419,15 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     done_phase ^= 1u;
     if (__syncthreads_and(ok)) {
       tc::fence_after_sync();
-      // ---------------------------------------------------------------- output rows
+      // ---------------------------------------------------------------- output rows (this thread's half)
       const float eq = expf(my_cs);
-      const bool valid = tid < L;
-      const size_t orow = (size_t)(row0 + tid) * d.HP + (size_t)h * P;
-      for (int q = 0; q < P / 32; ++q) {
+      const bool valid = row < L;
+      const size_t orow = (size_t)(row0 + row) * d.HP + (size_t)h * P + half * PH;
+#pragma unroll
+      for (int q = 0; q < PH / 32; ++q) {
         uint32_t ry[32], ri[32];
-        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_Y + 32 * q, ry);
-        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * q, ri);
+        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_Y + half * PH + 32 * q, ry);
+        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + half * PH + 32 * q, ri);
         tc::tmem_ld_wait();
         if (!valid) continue;
 #pragma unroll
