@@ -98,6 +98,19 @@ swimba_status swimba_router_topk(const swimba_dims* dims, const void* X, const s
 swimba_status swimba_dispatch(const swimba_dims* dims, const int32_t* topk_idx, int32_t* expert_offsets,
                               int32_t* perm, void* ws, size_t ws_bytes, void* stream);
 
+/* Expert dispatch that allocates nothing and takes no workspace.  The paper has no counterpart: this entry
+ * point is for callers that cannot give the library scratch memory -- plugin-style hosts whose interface
+ * hands an operator only its inputs and outputs, and runtimes that plan all device memory at start-up and
+ * refuse allocations afterwards.  Same arguments (minus the workspace) and the same results as
+ * swimba_dispatch.  Its scratch is one fixed 1 MiB array inside the library, held on every device that
+ * loads the library until the process exits; a shape that needs more (about 0.56 * M * k bytes with 64
+ * experts, 0.125 * M * k with 8) returns SWIMBA_ERR_WORKSPACE before launching anything.  The first call on
+ * a device looks up the array's device address with that device current; make that first call before
+ * any stream capture.  All calls share the array and it keeps the last call's contents (nothing in it
+ * needs clearing: each call writes every word it reads); calls whose work overlaps on the GPU race. */
+swimba_status swimba_dispatch_noalloc(const swimba_dims* dims, const int32_t* topk_idx, int32_t* expert_offsets,
+                                      int32_t* perm, void* stream);
+
 /* Expert projections of the active experts, unmixed (a stage probe; the fused path never writes them).
  * Paper: notes, key design 1 ("each expert applies its own linear projection to X_t").
  *   Z [M][k][W_e] fp32 out: Z[m][j] = W_exp[topk_idx[m][j]] X_m, accumulated in fp32. */

@@ -20,7 +20,7 @@ STATUS = {0: "SWIMBA_OK", 1: "SWIMBA_ERR_INVALID_ARG", 2: "SWIMBA_ERR_UNSUPPORTE
 EXPORTS = ("swimba_workspace_size", "swimba_stream_dtype", "swimba_router_topk", "swimba_dispatch",
            "swimba_expert_proj", "swimba_mix", "swimba_ssd_scan", "swimba_layer_fwd", "swimba_step",
            "swimba_separated_scan", "swimba_check_device_status", "swimba_status_string",
-           "swimba_profile_enable", "swimba_profile_read", "swimba_launch_count")
+           "swimba_profile_enable", "swimba_profile_read", "swimba_launch_count", "swimba_dispatch_noalloc")
 
 
 class SwimbaError(RuntimeError):
@@ -60,6 +60,7 @@ def lib():
         sig = {
             "swimba_router_topk": [P(Dims), vp, P(Weights), vp, vp, vp, vp],
             "swimba_dispatch": [P(Dims), vp, vp, vp, vp, sz, vp],
+            "swimba_dispatch_noalloc": [P(Dims), vp, vp, vp, vp],
             "swimba_expert_proj": [P(Dims), vp, P(Weights), vp, vp, vp, sz, vp],
             "swimba_mix": [P(Dims), vp, vp, i32, vp, vp, vp, vp],
             "swimba_ssd_scan": [P(Dims), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -130,6 +131,13 @@ def router_topk(d, X, W, topk_idx, topk_w, dt, stream=None):
 def dispatch(d, topk_idx, expert_offsets, perm, ws, stream=None):
     _check("swimba_dispatch", lib().swimba_dispatch(ctypes.byref(d), _p(topk_idx), _p(expert_offsets), _p(perm),
                                                      _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def dispatch_noalloc(d, topk_idx, expert_offsets, perm, stream=None):
+    """swimba_dispatch without a workspace (scratch in a fixed array inside the library); for callers
+    that cannot allocate device memory."""
+    _check("swimba_dispatch_noalloc", lib().swimba_dispatch_noalloc(ctypes.byref(d), _p(topk_idx),
+                                                                     _p(expert_offsets), _p(perm), _stream(stream)))
 
 
 def expert_proj(d, X, W, topk_idx, Z, ws, stream=None):
