@@ -75,6 +75,22 @@ def work(w):
     }
 
 
+def decode_work(w):
+    """Per-step algorithmic FLOPs and bytes of the recurrent decode step (one token per sequence)."""
+    B, D, E, H, k, N, P = w.batch, w.d_model, w.n_experts, w.nheads, w.top_k, w.dstate, w.headdim
+    used = min(E, B * k)
+    weights = used * w.W_e * D * 2
+    streams = B * k * (2 * w.G * N + H * P) * 2
+    state = 2 * B * H * N * P * 4
+    return {
+        "router": {"flops": 2.0 * B * D * (E + H), "bytes": B * D * 2 + (E + H) * D * 2},
+        "expert_proj_mix": {"flops": 2.0 * B * k * D * w.W_e, "bytes": weights + streams + B * k * D * 2},
+        "state_update": {"flops": 2.0 * B * H * N * P * (k + 1), "bytes": state + streams + B * H * P * 2},
+        "layer": {"flops": 2.0 * B * k * D * w.W_e + 2.0 * B * D * (E + H),
+                  "bytes": weights + state + B * D * 2 + B * H * P * 2},
+    }
+
+
 # ------------------------------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -208,6 +224,103 @@ def config_of(w):
             "chunk": w.chunk, "l2": "flushed between steps (2x L2 write outside the timed events)"}
 
 
+class LayerSession:
+    """Forward-pass workloads: one step = swimba_layer_fwd over B x T tokens."""
+
+    def __init__(self, w, dev, inp, swimba):
+        self.w, self.sw = w, swimba
+        self.d = swimba.dims_of(w)
+        self.W = swimba.WeightSet(*(inp[k].to(dev) for k in ("W_r", "W_dt", "b_dt", "A", "W_exp")))
+        self.X = inp["X"].to(dev).reshape(w.M, w.d_model)
+        odt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.y = torch.empty(w.M, w.nheads * w.headdim, dtype=odt, device=dev)
+        self.fin = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, device=dev)
+        self.ws = torch.empty(swimba.workspace_size(self.d), dtype=torch.uint8, device=dev)
+        self.Xh = inp["X"].reshape(w.M, w.d_model).pin_memory()
+        self.yh = torch.empty(self.y.shape, dtype=odt).pin_memory()
+        self.tokens = w.M
+        self.metric = METRIC
+        self.work = work(w)
+
+    def step(self):
+        self.sw.layer_fwd(self.d, self.X, self.W, None, self.y, self.fin, None, None, self.ws)
+
+    def h2d(self):
+        self.X.copy_(self.Xh, non_blocking=True)
+
+    def d2h(self):
+        self.yh.copy_(self.y, non_blocking=True)
+
+    def extras(self, stream, steps):
+        """Separated-trajectory variant ("k scans") on this layer's streams, timed alone."""
+        w, sw = self.w, self.sw
+        sdt = torch.float16 if w.dtype == "bf16" else torch.float32
+        dev = self.X.device
+        idx = torch.empty(w.M, w.top_k, dtype=torch.int32, device=dev)
+        wts = torch.empty(w.M, w.top_k, device=dev)
+        dt = torch.empty(w.M, w.nheads, device=dev)
+        sw.router_topk(self.d, self.X, self.W, idx, wts, dt)
+        Z = torch.empty(w.M, w.top_k, w.W_e, device=dev)
+        sw.expert_proj(self.d, self.X, self.W, idx, Z, self.ws)
+        B = torch.empty(w.M, w.top_k, w.G, w.dstate, dtype=sdt, device=dev)
+        Xs = torch.empty(w.M, w.top_k, w.nheads, w.headdim, dtype=sdt, device=dev)
+        C = torch.empty_like(B)
+        sw.mix(self.d, Z, wts, sw.MIX_UNSCALED_B, B, Xs, C)
+        del Z
+        A = self.W.tensors[3]
+        ys = torch.empty_like(self.y)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(3):
+            sw.separated_scan(self.d, B, Xs, C, dt, A, None, ys, None, self.ws)
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(steps):
+            e0.record(stream)
+            sw.separated_scan(self.d, B, Xs, C, dt, A, None, ys, None, self.ws)
+            e1.record(stream)
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        return {"separated_scan_ms": tot / steps, "separated_trajectories": w.top_k, "mixed_trajectories": 1}
+
+
+class DecodeSession:
+    """Recurrent decode: one step = swimba_step, one new token for each of `batch` sequences, on a state
+    built by a prefill of `prefill` tokens through swimba_layer_fwd."""
+
+    def __init__(self, w, dev, inp, swimba):
+        self.w, self.sw = w, swimba
+        self.W = swimba.WeightSet(*(inp[k].to(dev) for k in ("W_r", "W_dt", "b_dt", "A", "W_exp")))
+        dp = swimba.dims_of(w, seqlen=w.prefill)
+        Mp = w.batch * w.prefill
+        self.state = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, device=dev)
+        wsp = torch.empty(swimba.workspace_size(dp), dtype=torch.uint8, device=dev)
+        yp = torch.empty(Mp, w.nheads * w.headdim, dtype=torch.bfloat16, device=dev)
+        swimba.layer_fwd(dp, inp["X"].to(dev).reshape(Mp, w.d_model), self.W, None, yp, self.state, None, None, wsp)
+        torch.cuda.synchronize()
+        del wsp, yp
+        self.d = swimba.dims_of(w, seqlen=1)
+        self.X = inp["X_step"].to(dev)
+        self.y = torch.empty(w.batch, w.nheads * w.headdim, dtype=torch.bfloat16, device=dev)
+        self.ws = torch.empty(swimba.workspace_size(self.d), dtype=torch.uint8, device=dev)
+        self.Xh = inp["X_step"].pin_memory()
+        self.yh = torch.empty(self.y.shape, dtype=self.y.dtype).pin_memory()
+        self.tokens = w.batch
+        self.metric = "Swimba decode step tokens/s (256 seqs, H64 N128 P64 E16 k2); % of HBM roofline"
+        self.work = decode_work(w)
+
+    def step(self):
+        self.sw.step(self.d, self.X, self.W, self.state, self.y, None, self.ws)
+
+    def h2d(self):
+        self.X.copy_(self.Xh, non_blocking=True)
+
+    def d2h(self):
+        self.yh.copy_(self.y, non_blocking=True)
+
+    def extras(self, stream, steps):
+        return {}
+
+
 def run_gpu(args, w):
     from parameter_space_moe_b200 import swimba
     rank = int(os.environ.get("RANK", "0"))
@@ -226,22 +339,13 @@ def run_gpu(args, w):
     swimba.lib()
     wr = w.with_(seed=w.seed + 1000 * rank)
     inp = inputs.make_inputs(wr)
-    d = swimba.dims_of(w)
-    W = swimba.WeightSet(*(inp[k].to(dev) for k in ("W_r", "W_dt", "b_dt", "A", "W_exp")))
-    X = inp["X"].to(dev).reshape(w.M, w.d_model)
-    y = torch.empty(w.M, w.nheads * w.headdim, dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32,
-                    device=dev)
-    fin = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, device=dev)
-    ws = torch.empty(swimba.workspace_size(d), dtype=torch.uint8, device=dev)
+    sess = (DecodeSession if w.prefill else LayerSession)(w, dev, inp, swimba)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        swimba.layer_fwd(d, X, W, None, y, fin, None, None, ws)
-
     for _ in range(args.warmup):
-        step()
+        sess.step()
     torch.cuda.synchronize()
     assert swimba.check_device_status() == 0
     swimba.profile_enable(True)
@@ -257,7 +361,7 @@ def run_gpu(args, w):
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
             starts[i].record(stream)
-            step()
+            sess.step()
             ends[i].record(stream)
             for name, ms in swimba.profile_read():
                 stage_ms[name] = stage_ms.get(name, 0.0) + ms
@@ -269,23 +373,22 @@ def run_gpu(args, w):
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     assert swimba.check_device_status() == 0
 
-    # end to end through the C ABI: pinned host X in, y back to pinned host, every step
-    Xh = inp["X"].reshape(w.M, w.d_model).pin_memory()
-    yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    # end to end through the C ABI: pinned host input in, output back to pinned host, every step
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(2):
-        X.copy_(Xh, non_blocking=True); step(); yh.copy_(y, non_blocking=True)
+        sess.h2d(); sess.step(); sess.d2h()
     torch.cuda.synchronize()
     e2e_ms = 0.0
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         e0.record(stream)
-        X.copy_(Xh, non_blocking=True)
-        step()
-        yh.copy_(y, non_blocking=True)
+        sess.h2d()
+        sess.step()
+        sess.d2h()
         e1.record(stream)
         e1.synchronize()
         e2e_ms += e0.elapsed_time(e1)
+    extras = sess.extras(stream, args.steps) if args.separated else {}
 
     t = torch.tensor([total_ms, e2e_ms] + [stage_ms.get(n, 0.0) for n in sorted(stage_ms)], dtype=torch.float64,
                      device=dev)
@@ -294,40 +397,41 @@ def run_gpu(args, w):
     total_ms, e2e_ms = t[0].item(), t[1].item()
     stage_ms = {n: t[2 + i].item() for i, n in enumerate(sorted(stage_ms))}
     if rank == 0:
-        report(args, w, world, total_ms, e2e_ms, stage_ms, launches, sampler.summary(),
-               Xh.numel() * Xh.element_size(), yh.numel() * yh.element_size(), inp)
+        report(args, w, sess, world, total_ms, e2e_ms, stage_ms, launches, sampler.summary(),
+               sess.Xh.numel() * sess.Xh.element_size(), sess.yh.numel() * sess.yh.element_size(), inp, extras)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
 
 
-def report(args, w, world, total_ms, e2e_ms, stage_ms, launches, clocks, h2d, d2h, inp):
+def stage_roofline(model, secs, peaks):
+    """Bound (tensor or hbm), achieved, peak and unit of one stage from its work model and duration."""
+    t_tensor = model["flops"] / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = model["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        return "tensor", model["flops"] / secs / 1e12, peaks["bf16_tflops"], "TFLOP/s", model["flops"]
+    return "hbm", model["bytes"] / secs / 1e9, peaks["hbm_gbs"], "GB/s", model["bytes"]
+
+
+def report(args, w, sess, world, total_ms, e2e_ms, stage_ms, launches, clocks, h2d, d2h, inp, extras):
     peaks, src = load_peaks()
-    wk = work(w)
+    wk = sess.work
     K = args.steps
-    tokens = w.M * world * K
+    tokens = sess.tokens * world * K
     value = tokens / (total_ms / 1e3)
     # dominant kernel stage (among those with a work model) and its roofline
     dom = max((n for n in stage_ms if n in wk), key=stage_ms.get)
     avg_s = stage_ms[dom] / K / 1e3
-    bound = "tensor" if dom == "expert_proj_mix" else "hbm"
-    if bound == "tensor":
-        achieved = wk[dom]["flops"] / avg_s / 1e12
-        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
-        peak_note = f"bf16 dense, burst, {src}"
-    else:
-        achieved = wk[dom]["bytes"] / avg_s / 1e9
-        peak, unit = peaks["hbm_gbs"], "GB/s"
-        peak_note = f"HBM copy, {src}"
-    layer_roof_s = max(wk["layer"]["flops"] / (peaks["bf16_tflops"] * 1e12), wk["layer"]["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    bound, achieved, peak, unit, alg = stage_roofline(wk[dom], avg_s, peaks)
+    peak_note = (f"bf16 dense, burst, {src}" if bound == "tensor" else f"HBM copy, {src}")
+    roof_s = max(wk["layer"]["flops"] / (peaks["bf16_tflops"] * 1e12), wk["layer"]["bytes"] / (peaks["hbm_gbs"] * 1e9))
     out = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "metric": sess.metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic", "config": config_of(w),
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": None, "peak_source": peak_note,
-                     "algorithmic": wk[dom]["flops"] if bound == "tensor" else wk[dom]["bytes"]},
-        "layer_roofline": {"time_us": layer_roof_s * 1e6, "frac": layer_roof_s / (total_ms / K / 1e3),
+                     "frac": achieved / peak, "traffic": None, "peak_source": peak_note, "algorithmic": alg},
+        "layer_roofline": {"time_us": roof_s * 1e6, "frac": roof_s / (total_ms / K / 1e3),
                            "flops": wk["layer"]["flops"], "bytes": wk["layer"]["bytes"]},
         "stages_ms_per_step": {n: v / K for n, v in stage_ms.items()},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -335,7 +439,8 @@ def report(args, w, world, total_ms, e2e_ms, stage_ms, launches, clocks, h2d, d2
         "gpu_launches": launches,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    out.update(extras)
+    if world == 1 and not args.no_cpu_baseline and not w.prefill:
         v, sample = cpu_oracle_sample(w, inp)
         out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                                "sample": sample}
@@ -350,6 +455,8 @@ def main():
     ap.add_argument("--impl", default="swimba", choices=["swimba", "reference"])
     ap.add_argument("--workload", default=configs.BASE.name, choices=sorted(configs.ALL))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--separated", action="store_true",
+                    help="also time the separated-trajectory scan (k scans) on the layer's streams")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = configs.ALL[args.workload]
