@@ -94,10 +94,15 @@ WsPlan plan_workspace(const Dims& d);
 // ---------------------------------------------------------------------------------------------
 // Kernel launchers (defined in the .cu files next to their kernels).  All return cudaError_t of the
 // launch; `st` is the workspace status word.
+// counts (nullable): [dispatch tile][E] table, zeroed by the caller, that the router increments for the
+// (token, slot) pairs it routes (dispatch tile = pair index / kDispatchTile).
 cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
-                          float* dt, unsigned* st, cudaStream_t s);
+                          float* dt, int32_t* counts, cudaStream_t s);
 cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
                             int32_t* perm, cudaStream_t s);
+// The layer's one-launch dispatch over counts the router produced (see launch_router).
+cudaError_t launch_dispatch_fused(const Dims& d, const int32_t* idx, const int32_t* counts, const WsPlan& p, char* ws,
+                                  int32_t* offsets, int32_t* perm, cudaStream_t s);
 cudaError_t launch_gather_rows(const Dims& d, const void* X, const int32_t* perm, void* xsorted, cudaStream_t s);
 // mode 0: fused mix (pi-scaled B and C), 1: fused mix with unscaled B, 2: raw Z (fp32)
 cudaError_t launch_proj_simt(const Dims& d, const void* X, const void* w_exp, const int32_t* perm,

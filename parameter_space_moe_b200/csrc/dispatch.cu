@@ -94,17 +94,98 @@ dispatch_scatter_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* 
   if (valid) perm[wc_s[warp][e] + rank] = p;
 }
 
-// X rows in sorted order: xsorted[r] = X[perm[r] / k].  One warp per row, 16-byte vectors.
+// The layer's dispatch in one launch: per-tile counts arrive from the router (integer atomics into a
+// zeroed [tile][E] table), so each CTA derives the global expert offsets and its tile's bases itself
+// (sums over at most M*k/1024 tiles), CTA 0 publishes expert_offsets and the GEMM row-tile schedule, and
+// every CTA scatters its pairs with the same stable ranking as dispatch_scatter_kernel.
+__global__ void __launch_bounds__(kDispatchThreads)
+dispatch_fused_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
+                      int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ tiles,
+                      int32_t* __restrict__ ntiles) {
+  __shared__ int wc_s[kDispatchThreads / 32][64];
+  __shared__ int tot_s[64], pre_s[64], off_s[65], toff_s[65];
+  const int tile = blockIdx.x, ntile = gridDim.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = d.M * d.k;
+  if (threadIdx.x < d.E) {
+    const int e = threadIdx.x;
+    int t = 0, pre = 0;
+    for (int i = 0; i < ntile; ++i) {
+      const int c = counts[i * d.E + e];
+      t += c;
+      if (i < tile) pre += c;
+    }
+    tot_s[e] = t;
+    pre_s[e] = pre;
+  }
+  for (int x = threadIdx.x; x < (kDispatchThreads / 32) * 64; x += blockDim.x) (&wc_s[0][0])[x] = 0;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int o = 0, to = 0;
+    for (int e = 0; e < d.E; ++e) {
+      off_s[e] = o; toff_s[e] = to;
+      o += tot_s[e]; to += ceil_div(tot_s[e], kRowTile);
+    }
+    off_s[d.E] = o; toff_s[d.E] = to;
+    if (tile == 0) *ntiles = to;
+  }
+  __syncthreads();
+  if (tile == 0) {
+    if (threadIdx.x <= d.E) offsets[threadIdx.x] = off_s[threadIdx.x];
+    for (int e = 0; e < d.E; ++e) {
+      const int nt = ceil_div(tot_s[e], kRowTile);
+      for (int r = threadIdx.x; r < nt; r += blockDim.x) {
+        tiles[2 * (toff_s[e] + r) + 0] = e;
+        tiles[2 * (toff_s[e] + r) + 1] = off_s[e] + r * kRowTile;
+      }
+    }
+  }
+  const int p = tile * kDispatchTile + threadIdx.x;
+  const bool valid = p < total;
+  const int e = valid ? idx[p] : -1 - lane;
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  if (valid && rank == 0) wc_s[warp][e] = __popc(peers);
+  __syncthreads();
+  if (threadIdx.x < d.E) {
+    int run = off_s[threadIdx.x] + pre_s[threadIdx.x];
+    for (int w = 0; w < kDispatchThreads / 32; ++w) {
+      const int c = wc_s[w][threadIdx.x];
+      wc_s[w][threadIdx.x] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  if (valid) perm[wc_s[warp][e] + rank] = p;
+}
+
+// X rows in sorted order: xsorted[r] = X[perm[r] / k].  The copy is flat over 16-byte chunks; each
+// thread moves kGatherUnroll chunks a stride apart with all loads issued before the stores.
+constexpr int kGatherUnroll = 4;
 template <class T>
-__global__ void gather_rows_kernel(Dims d, const T* __restrict__ X, const int32_t* __restrict__ perm,
-                                   T* __restrict__ xs) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= d.M * d.k) return;
-  const int m = perm[warp] / d.k;
-  const int4* src = reinterpret_cast<const int4*>(X + (size_t)m * d.D);
-  int4* dst = reinterpret_cast<int4*>(xs + (size_t)warp * d.D);
-  const int nv = d.D * (int)sizeof(T) / 16;
-  for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(Dims d, const T* __restrict__ X, const int32_t* __restrict__ perm, T* __restrict__ xs) {
+  const int cpr = d.D * (int)sizeof(T) / 16;  // chunks per row
+  const long long total = (long long)d.M * d.k * cpr;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  long long i0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i0 < total; i0 += stride * kGatherUnroll) {
+    int4 v[kGatherUnroll];
+    long long dst[kGatherUnroll];
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      const long long i = i0 + u * stride;
+      dst[u] = -1;
+      if (i < total) {
+        const int r = (int)(i / cpr), c = (int)(i % cpr);
+        const int m = __ldg(perm + r) / d.k;
+        v[u] = __ldg(reinterpret_cast<const int4*>(X + (size_t)m * d.D) + c);
+        dst[u] = i;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u)
+      if (dst[u] >= 0) reinterpret_cast<int4*>(xs)[dst[u]] = v[u];
+  }
 }
 
 cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
@@ -120,9 +201,19 @@ cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, 
   return cudaGetLastError();
 }
 
+cudaError_t launch_dispatch_fused(const Dims& d, const int32_t* idx, const int32_t* counts, const WsPlan& p, char* ws,
+                                  int32_t* offsets, int32_t* perm, cudaStream_t s) {
+  dispatch_fused_kernel<<<dispatch_tiles(d), kDispatchThreads, 0, s>>>(d, idx, counts, offsets, perm,
+                                                                        (int32_t*)(ws + p.tiles),
+                                                                        (int32_t*)(ws + p.ntiles));
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gather_rows(const Dims& d, const void* X, const int32_t* perm, void* xsorted, cudaStream_t s) {
-  const int rows = d.M * d.k;
-  dim3 grid(ceil_div(rows, 8));
+  const long long chunks = (long long)d.M * d.k * (d.D * (long long)elem_bytes(d.dtype) / 16);
+  const long long want = (chunks + 256LL * kGatherUnroll - 1) / (256LL * kGatherUnroll);
+  const int grid = (int)(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
   if (d.dtype == SWIMBA_BF16)
     gather_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(d, (const __nv_bfloat16*)X, perm, (__nv_bfloat16*)xsorted);
   else

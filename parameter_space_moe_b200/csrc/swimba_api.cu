@@ -67,6 +67,9 @@ WsPlan plan_workspace(const Dims& d) {
   p.topk_w = take(Mk * 4);
   p.dt = take((size_t)d.M * d.H * 4);
   p.dcounts = take((size_t)dispatch_tiles(d) * d.E * 4);
+  const size_t nsub = (size_t)scan_tc_subchunks(d);
+  p.lb_bytes = 256 + (size_t)d.Bsz * d.H * nsub * 4;
+  p.lb = take(p.lb_bytes);  // directly after dcounts: run_front clears both with one memset
   p.dbase = take((size_t)dispatch_tiles(d) * d.E * 4);
   p.offsets = take((size_t)(d.E + 1) * 4);
   p.perm = take(Mk * 4);
@@ -81,9 +84,6 @@ WsPlan plan_workspace(const Dims& d) {
   p.schunk = take(states);
   p.hstart = take(states);
   p.cslast = take((size_t)d.Bsz * d.H * d.nc * 4);
-  const size_t nsub = (size_t)scan_tc_subchunks(d);
-  p.lb_bytes = 256 + (size_t)d.Bsz * d.H * nsub * 4;
-  p.lb = take(p.lb_bytes);
   p.exch = take((size_t)d.Bsz * d.H * nsub * d.N * d.P * 4);
   p.total = o;
   return p;
@@ -167,11 +167,14 @@ static swimba_status run_proj(const Dims& d, const void* X, const void* w_exp, c
 static swimba_status run_front(const Dims& d, const void* X, const swimba_weights* w, char* ws, const WsPlan& p,
                                int32_t* idx, float* wts, int mode, unsigned* st, cudaStream_t s) {
   float* dt = (float*)(ws + p.dt);
-  SW_CUDA(launch_router(d, X, *w, idx, wts, dt, st, s));
+  // one memset clears the router's per-tile counts and the scan's hand-off flags (adjacent regions)
+  SW_CUDA(cudaMemsetAsync(ws + p.dcounts, 0, p.lb + p.lb_bytes - p.dcounts, s));
+  int32_t* counts = (int32_t*)(ws + p.dcounts);
+  SW_CUDA(launch_router(d, X, *w, idx, wts, dt, counts, s));
   prof_mark(s, "router");
   int32_t* offsets = (int32_t*)(ws + p.offsets);
   int32_t* perm = (int32_t*)(ws + p.perm);
-  SW_CUDA(launch_dispatch(d, idx, p, ws, offsets, perm, s));
+  SW_CUDA(launch_dispatch_fused(d, idx, counts, p, ws, offsets, perm, s));
   prof_mark(s, "dispatch");
   SW_TRY(run_proj(d, X, w->w_exp, ws, p, wts, mode, ws + p.bpi, ws + p.xs, ws + p.cpi, nullptr, st, s));
   return SWIMBA_OK;
@@ -179,9 +182,10 @@ static swimba_status run_front(const Dims& d, const void* X, const swimba_weight
 
 // The chunked scan: tensor-core kernel for the shapes it covers, CUDA-core kernels otherwise (the
 // fp32 layer, N != 128, P not in {64, 128}, or per-chunk states requested at chunk 64).
-static swimba_status run_scan(const Dims& d, const ScanArgs& a, char* ws, const WsPlan& p, cudaStream_t s) {
+static swimba_status run_scan(const Dims& d, const ScanArgs& a, char* ws, const WsPlan& p, cudaStream_t s,
+                              bool lb_clear = false) {
   if (scan_tc_supported(d) && !(a.chunk_states && d.Q < 128)) {
-    SW_CUDA(cudaMemsetAsync(ws + p.lb, 0, p.lb_bytes, s));
+    if (!lb_clear) SW_CUDA(cudaMemsetAsync(ws + p.lb, 0, p.lb_bytes, s));
     SW_CUDA(launch_scan_tc(d, a, (unsigned*)(ws + p.lb), (float*)(ws + p.exch), device_status(), s));
   } else {
     SW_CUDA(launch_scan_simt(d, a, s));
@@ -228,7 +232,7 @@ swimba_status swimba_router_topk(const swimba_dims* dims, const void* X, const s
   SW_TRY(make_dims(dims, &d));
   SW_TRY(check_weights(w, true, false));
   if (!ok_ptr(X) || !ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_ptr(dt)) return SWIMBA_ERR_INVALID_ARG;
-  return cuda_status(launch_router(d, X, *w, topk_idx, topk_w, dt, device_status(), (cudaStream_t)stream));
+  return cuda_status(launch_router(d, X, *w, topk_idx, topk_w, dt, nullptr, (cudaStream_t)stream));
 }
 
 swimba_status swimba_dispatch(const swimba_dims* dims, const int32_t* topk_idx, int32_t* expert_offsets,
@@ -302,7 +306,7 @@ swimba_status swimba_layer_fwd(const swimba_dims* dims, const void* X, const swi
   SW_TRY(run_front(d, X, w, b, p, idx, wts, 0, device_status(), s));
   ScanArgs a = mixed_scan_args(d, b, p, b + p.bpi, b + p.xs, b + p.cpi, (float*)(b + p.dt), w->A, init_state, y,
                                final_state, nullptr);
-  SW_TRY(run_scan(d, a, b, p, s));
+  SW_TRY(run_scan(d, a, b, p, s, /*lb_clear=*/true));  // run_front already cleared the hand-off flags
   prof_mark(s, "ssd_scan");
   return SWIMBA_OK;
 }
