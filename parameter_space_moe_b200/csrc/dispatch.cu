@@ -158,34 +158,17 @@ dispatch_fused_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* __
   if (valid) perm[wc_s[warp][e] + rank] = p;
 }
 
-// X rows in sorted order: xsorted[r] = X[perm[r] / k].  The copy is flat over 16-byte chunks; each
-// thread moves kGatherUnroll chunks a stride apart with all loads issued before the stores.
-constexpr int kGatherUnroll = 4;
+// X rows in sorted order: xsorted[r] = X[perm[r] / k].  One warp per row, 16-byte vectors.
 template <class T>
-__global__ void __launch_bounds__(256)
-gather_rows_kernel(Dims d, const T* __restrict__ X, const int32_t* __restrict__ perm, T* __restrict__ xs) {
-  const int cpr = d.D * (int)sizeof(T) / 16;  // chunks per row
-  const long long total = (long long)d.M * d.k * cpr;
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  long long i0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  for (; i0 < total; i0 += stride * kGatherUnroll) {
-    int4 v[kGatherUnroll];
-    long long dst[kGatherUnroll];
-#pragma unroll
-    for (int u = 0; u < kGatherUnroll; ++u) {
-      const long long i = i0 + u * stride;
-      dst[u] = -1;
-      if (i < total) {
-        const int r = (int)(i / cpr), c = (int)(i % cpr);
-        const int m = __ldg(perm + r) / d.k;
-        v[u] = __ldg(reinterpret_cast<const int4*>(X + (size_t)m * d.D) + c);
-        dst[u] = i;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kGatherUnroll; ++u)
-      if (dst[u] >= 0) reinterpret_cast<int4*>(xs)[dst[u]] = v[u];
-  }
+__global__ void gather_rows_kernel(Dims d, const T* __restrict__ X, const int32_t* __restrict__ perm,
+                                   T* __restrict__ xs) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= d.M * d.k) return;
+  const int m = perm[warp] / d.k;
+  const int4* src = reinterpret_cast<const int4*>(X + (size_t)m * d.D);
+  int4* dst = reinterpret_cast<int4*>(xs + (size_t)warp * d.D);
+  const int nv = d.D * (int)sizeof(T) / 16;
+  for (int i = lane; i < nv; i += 32) dst[i] = src[i];
 }
 
 cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
@@ -211,9 +194,8 @@ cudaError_t launch_dispatch_fused(const Dims& d, const int32_t* idx, const int32
 }
 
 cudaError_t launch_gather_rows(const Dims& d, const void* X, const int32_t* perm, void* xsorted, cudaStream_t s) {
-  const long long chunks = (long long)d.M * d.k * (d.D * (long long)elem_bytes(d.dtype) / 16);
-  const long long want = (chunks + 256LL * kGatherUnroll - 1) / (256LL * kGatherUnroll);
-  const int grid = (int)(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
+  const int rows = d.M * d.k;
+  dim3 grid(ceil_div(rows, 8));
   if (d.dtype == SWIMBA_BF16)
     gather_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(d, (const __nv_bfloat16*)X, perm, (__nv_bfloat16*)xsorted);
   else

@@ -7,9 +7,10 @@
 //   pi_t,j = exp(g_{K_j} - g_{K_0}) / sum_j' exp(g_{K_j'} - g_{K_0})
 //   dt_t,h = clamp(softplus(W_dt[h] . X_t + b_dt[h]), 1e-3, 0.1)
 // The E + H dot products per token form a skinny GEMM [M x D] x [D x (E + H)].  bf16 layers run it on
-// the warp-level tensor-core path (mma.sync m16n8k16, fp32 accumulate), 16 tokens per CTA with the K
-// reduction split over 8 warps.  The fp32 layer keeps a CUDA-core kernel (one warp per token, fixed xor
-// butterfly reductions).
+// the warp-level tensor-core path (mma.sync m16n8k16, fp32 accumulate): a CTA of 4 warps owns 64
+// tokens and streams X and the stacked [W_r; W_dt] through padded shared memory in 64-wide K chunks
+// (cp.async, 4-stage pipeline); then threads over (token, head) finish dt and one thread per token takes
+// the top-k.  The fp32 layer keeps a CUDA-core kernel (one warp per token, fixed xor butterfly reductions).
 #include "common.cuh"
 
 namespace swimba {
@@ -92,15 +93,26 @@ router_simt_kernel(Dims d, const T* __restrict__ X, const T* __restrict__ Wr, co
 }
 
 // ------------------------------------------------------------------------------------------ mma.sync
-// A CTA owns one m16 tile of tokens; its 8 warps split the K = D reduction into 8 contiguous ranges and
-// load their mma.sync fragments straight from global memory (X rows and the stacked [W_r; W_dt] rows are
-// read 16 bytes per row per k-step by 4 lanes, so sectors are fully used); the partial logits are summed
-// across warps in shared memory in a fixed order; then one thread per token takes the top-k and threads
-// over (token, head) finish dt.
-constexpr int kTokTile = 16;
-constexpr int kRWarps = 8;
-constexpr int kMaxNT = 16;  // up to 128 logits per token
+constexpr int kMT = 64;           // tokens per CTA
+constexpr int kKC = 64;           // K chunk
+constexpr int kLd = kKC + 8;      // padded shared row (144 B: conflict-free ldmatrix)
+constexpr int kMaxNT = 16;        // up to 128 logits per token
+constexpr int kStagesR = 4;       // cp.async pipeline depth
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(dst);
+  const int n = valid ? 16 : 0;  // zero-fill when invalid
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -110,77 +122,93 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t ldg32(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const unsigned*>(p)); }
-
-__global__ void __launch_bounds__(kRWarps * 32, 1)
+__global__ void __launch_bounds__(128)
 router_mma_kernel(Dims d, int RP, const __nv_bfloat16* __restrict__ X, const __nv_bfloat16* __restrict__ Wr,
                   const __nv_bfloat16* __restrict__ Wdt, const float* __restrict__ bdt, int32_t* __restrict__ idx_out,
                   float* __restrict__ w_out, float* __restrict__ dt_out, int32_t* __restrict__ counts) {
-  extern __shared__ __align__(16) float part[];  // [kRWarps][kTokTile][RP + 1] partial logits, then sums
+  extern __shared__ __align__(16) uint8_t rsm[];
+  __nv_bfloat16* Xs = reinterpret_cast<__nv_bfloat16*>(rsm);   // [stages][kMT][kLd]
+  __nv_bfloat16* Ws = Xs + kStagesR * kMT * kLd;                 // [stages][RP][kLd]
+  float* G = reinterpret_cast<float*>(Ws + kStagesR * RP * kLd); // [kMT][RP + 1]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tok0 = blockIdx.x * kTokTile;
-  const int R = d.E + d.H, NT = RP / 8;
-  const int g = lane >> 2, c2 = 2 * (lane & 3);
-  // this warp's range of 16-wide k-steps
-  const int steps = d.D / 16, per = (steps + kRWarps - 1) / kRWarps;
-  const int s0 = warp * per, s1 = min(steps, s0 + per);
-  const int r0 = min(tok0 + g, d.M - 1), r1 = min(tok0 + g + 8, d.M - 1);  // clamped rows (masked at the end)
-  const __nv_bfloat16* xa = X + (size_t)r0 * d.D + c2;
-  const __nv_bfloat16* xb = X + (size_t)r1 * d.D + c2;
-  const __nv_bfloat16* wrow[kMaxNT];
-#pragma unroll
-  for (int n = 0; n < kMaxNT; ++n) {
-    const int r = min(8 * n + g, R - 1);
-    wrow[n] = (r < d.E ? Wr + (size_t)r * d.D : Wdt + (size_t)(r - d.E) * d.D) + c2;
-  }
+  const int tok0 = blockIdx.x * kMT;
+  const int R = d.E + d.H, NT = RP / 8, nkc = d.D / kKC;
+
+  auto load = [&](int stage, int kc) {
+    if (kc < nkc) {
+      const int k0 = kc * kKC;
+      __nv_bfloat16* xs = Xs + stage * kMT * kLd;
+      __nv_bfloat16* ws = Ws + stage * RP * kLd;
+      for (int i = tid; i < kMT * (kKC / 8); i += 128) {
+        const int r = i >> 3, c = i & 7;
+        const bool v = tok0 + r < d.M;
+        cp_async16(xs + r * kLd + 8 * c, X + (size_t)(v ? tok0 + r : 0) * d.D + k0 + 8 * c, v);
+      }
+      for (int i = tid; i < RP * (kKC / 8); i += 128) {
+        const int r = i >> 3, c = i & 7;
+        const __nv_bfloat16* src = r < d.E ? Wr + (size_t)r * d.D : Wdt + (size_t)(r < R ? r - d.E : 0) * d.D;
+        cp_async16(ws + r * kLd + 8 * c, src + k0 + 8 * c, r < R);
+      }
+    }
+    cp_async_commit();  // an empty group past the end keeps the group count uniform
+  };
+
   float acc[kMaxNT][4];
 #pragma unroll
   for (int n = 0; n < kMaxNT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-#pragma unroll 4
-  for (int st = s0; st < s1; ++st) {
-    const int k0 = 16 * st;
-    const uint32_t a0 = ldg32(xa + k0), a1 = ldg32(xb + k0), a2 = ldg32(xa + k0 + 8), a3 = ldg32(xb + k0 + 8);
+
 #pragma unroll
-    for (int n = 0; n < kMaxNT; ++n) {
-      if (n < NT) {
-        const uint32_t b0 = ldg32(wrow[n] + k0), b1 = ldg32(wrow[n] + k0 + 8);
-        mma_bf16_16816(acc[n], a0, a1, a2, a3, b0, b1);
+  for (int st = 0; st < kStagesR - 1; ++st) load(st, st);
+  for (int kc = 0; kc < nkc; ++kc) {
+    const int stage = kc % kStagesR;
+    cp_async_wait<kStagesR - 2>();
+    __syncthreads();
+    load((kc + kStagesR - 1) % kStagesR, kc + kStagesR - 1);  // refills the stage read in iteration kc - 1
+    const uint32_t xb = (uint32_t)__cvta_generic_to_shared(Xs + stage * kMT * kLd);
+    const uint32_t wb = (uint32_t)__cvta_generic_to_shared(Ws + stage * RP * kLd);
+#pragma unroll
+    for (int ks = 0; ks < kKC / 16; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4(xb + (uint32_t)(((16 * warp + (lane & 15)) * kLd + 16 * ks + (lane >> 4) * 8) * 2), a0, a1, a2, a3);
+#pragma unroll
+      for (int np = 0; np < kMaxNT / 2; ++np) {
+        if (2 * np < NT) {
+          uint32_t b0, b1, b2, b3;
+          const int n = 16 * np + (lane & 7) + 8 * (lane >> 4);
+          ldmatrix_x4(wb + (uint32_t)((n * kLd + 16 * ks + ((lane >> 3) & 1) * 8) * 2), b0, b1, b2, b3);
+          mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+        }
       }
     }
   }
-  // partials: c0,c1 at (row g, cols 2c, 2c+1), c2,c3 at (row g + 8, same cols)
-  float* mine = part + (size_t)warp * kTokTile * (RP + 1);
+  cp_async_wait<0>();
+  __syncthreads();
+  // logits -> shared memory: c0,c1 at (row g, cols 2c, 2c+1), c2,c3 at (row g + 8, same cols)
+  const int gr = lane >> 2, gc = 2 * (lane & 3);
 #pragma unroll
   for (int n = 0; n < kMaxNT; ++n) {
     if (n < NT) {
-      float* p0 = mine + g * (RP + 1) + 8 * n + c2;
-      float* p1 = p0 + 8 * (RP + 1);
-      p0[0] = acc[n][0]; p0[1] = acc[n][1];
-      p1[0] = acc[n][2]; p1[1] = acc[n][3];
+      float* r0 = G + (16 * warp + gr) * (RP + 1) + 8 * n + gc;
+      float* r1 = r0 + 8 * (RP + 1);
+      r0[0] = acc[n][0]; r0[1] = acc[n][1];
+      r1[0] = acc[n][2]; r1[1] = acc[n][3];
     }
   }
   __syncthreads();
-  // fixed-order sum over the warps' partials into slot 0
-  for (int i = tid; i < kTokTile * RP; i += kRWarps * 32) {
-    const int t = i / RP, r = i % RP;
-    float v = 0.f;
-    for (int w = 0; w < kRWarps; ++w) v += part[(size_t)w * kTokTile * (RP + 1) + t * (RP + 1) + r];
-    part[t * (RP + 1) + r] = v;
-  }
-  __syncthreads();
-  // dt for every (token, head)
-  for (int i = tid; i < kTokTile * d.H; i += kRWarps * 32) {
+  // dt for every (token, head), then the top-k with one thread per token: k passes over the E logits,
+  // strict '>' so equal values keep the lower index
+  for (int i = tid; i < kMT * d.H; i += 128) {
     const int t = i / d.H, h = i % d.H, m = tok0 + t;
     if (m < d.M) {
-      const float v = part[t * (RP + 1) + d.E + h] + bdt[h];
+      const float v = G[t * (RP + 1) + d.E + h] + bdt[h];
       const float sp = v > 20.f ? v : log1pf(expf(v));
       dt_out[(size_t)m * d.H + h] = fminf(fmaxf(sp, 1e-3f), 0.1f);
     }
   }
-  // top-k, one thread per token: k passes over the E logits, strict '>' so equal values keep the lower index
-  if (tid < kTokTile && tok0 + tid < d.M) {
+  if (tid < kMT && tok0 + tid < d.M) {
     const int m = tok0 + tid;
-    const float* gl = part + tid * (RP + 1);
+    const float* gl = G + tid * (RP + 1);
     unsigned long long taken = 0ull;
     float gsel[8];
     int isel[8];
@@ -210,14 +238,14 @@ cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w,
                           float* dt, int32_t* counts, cudaStream_t s) {
   const int R = d.E + d.H;
   if (d.dtype == SWIMBA_BF16 && R <= 8 * kMaxNT) {
-    const int RP = (R + 7) / 8 * 8;
-    const size_t smem = (size_t)kRWarps * kTokTile * (RP + 1) * 4;
+    const int RP = (R + 15) / 16 * 16;
+    const size_t smem = (size_t)kStagesR * (kMT + RP) * kLd * 2 + (size_t)kMT * (RP + 1) * 4;
     cudaError_t e = cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    router_mma_kernel<<<ceil_div(d.M, kTokTile), kRWarps * 32, smem, s>>>(d, RP, (const __nv_bfloat16*)X,
-                                                                         (const __nv_bfloat16*)w.w_router,
-                                                                         (const __nv_bfloat16*)w.w_dt, w.b_dt, idx,
-                                                                         wts, dt, counts);
+    router_mma_kernel<<<ceil_div(d.M, kMT), 128, smem, s>>>(d, RP, (const __nv_bfloat16*)X,
+                                                             (const __nv_bfloat16*)w.w_router,
+                                                             (const __nv_bfloat16*)w.w_dt, w.b_dt, idx, wts, dt,
+                                                             counts);
   } else {
     const size_t smem = sizeof(float) * (size_t)kRouterWarps * (d.D + R);
     if (d.dtype == SWIMBA_BF16) {
