@@ -7,35 +7,31 @@
 // The notes name a fused MoE operator for this input projection as the way to avoid HBM round trips of
 // router outputs and parameter slices; here the per-expert output tile never leaves the SM unmixed.
 //
-// Design (one persistent CTA per SM, 10 warps, 256 x 256 output tile):
-//   warp 0      TMA producer: A = 2 x (128 gathered X rows x 64 K), B = 256 weight rows x 64 K per stage
-//               (64 KB), 128-byte swizzle, 3-stage ring of mbarriers
-//   warp 1      TMEM owner and MMA issuer: per 16-wide K step two tcgen05.mma M128 N256, one per M half,
-//               into the two 256-column fp32 accumulators (all 512 TMEM columns)
-//   warps 2..9  epilogue: warp w drains TMEM lane quarter w % 4 of M half (w - 2) / 4, 32 columns at a
-//               time; scales B and C columns by pi, converts to fp16, stores each row to its (token, slot)
-// The 256-row tile halves the weight-tile traffic per FLOP of a 128-row tile (the operands stream from L2
-// at a rate the tensor core would otherwise outrun).  With one accumulator set the MMA issuer waits for
-// the epilogue between tiles; 8 epilogue warps keep that gap short.  A tile whose expert segment ends in
-// its first half skips the second half's MMAs and stores.
-// The row-tile schedule (expert, first row) is derived on the device from expert_offsets.
+// Design (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: A = 128 gathered X rows x 64 K (16 KB), B = 256 weight rows x 64 K (32 KB)
+//               per stage, 128-byte swizzle, kStages-deep ring of mbarriers
+//   warp 1      TMEM owner and MMA issuer: 4 x tcgen05.mma M128 N256 K16 per stage into one of two
+//               256-column fp32 accumulators (double buffered: 512 TMEM columns)
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time (warp w reads TMEM lanes 32*(w%4)..), scales
+//               B and C columns by pi, converts to fp16 and stores to the destination (token, slot) row
+// Tiles: (row tile of one expert's sorted rows) x (256 output columns), handed out round-robin.
 #include "tc_common.cuh"
 
 namespace swimba {
 
 namespace {
-constexpr int BM = 256, BN = 256, BK = 64, kStages = 3;
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr uint32_t kHalfA = 128 * BK * 2, kStageA = 2 * kHalfA, kStageB = BN * BK * 2;
-constexpr uint32_t kStageBytes = kStageA + kStageB;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kIdesc = tc::idesc_f16(128, BN, /*bf16=*/true);
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 1024;
+constexpr int BM = 128, BN = 256, BK = 64, kStages = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t kStageA = BM * BK * 2, kStageB = BN * BK * 2, kStageBytes = kStageA + kStageB;
+constexpr uint32_t kTmemCols = 2 * BN;
+constexpr uint32_t kIdesc = tc::idesc_f16(BM, BN, /*bf16=*/true);
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 256;
 
 struct TcArgs {
   Dims d;
   const int32_t* perm;
+  const int32_t* tiles;
+  const int32_t* ntiles;
   const int32_t* offsets;
   const float* topk_w;
   int mode;  // 0 mix, 1 mix with unscaled B, 2 raw fp32 Z
@@ -102,16 +98,6 @@ __device__ __forceinline__ void store_chunk(const TcArgs& a, int p, float pi, in
   }
 }
 
-// Row tile rt -> (expert, first sorted row, rows in the tile); schedule prefix sums live in shared memory.
-__device__ __forceinline__ void row_tile(const int* tpre, const int* off, int E, int rt, int& e, int& row0,
-                                         int& rows) {
-  int x = 0;
-  while (x + 1 < E && tpre[x + 1] <= rt) ++x;
-  e = x;
-  row0 = off[x] + (rt - tpre[x]) * BM;
-  rows = min(BM, off[x + 1] - row0);
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
 proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -121,13 +107,11 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
   uint64_t* full = bars;                 // [kStages]  TMA -> MMA
   uint64_t* empty = bars + kStages;      // [kStages]  MMA -> TMA
-  uint64_t* acc_full = bars + 2 * kStages;       // MMA -> epilogue
-  uint64_t* acc_empty = bars + 2 * kStages + 1;  // epilogue -> MMA
-  uint64_t* drain = bars + 2 * kStages + 2;      // MMA completion before teardown
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 3);
+  uint64_t* acc_full = bars + 2 * kStages;       // [2]  MMA -> epilogue
+  uint64_t* acc_empty = bars + 2 * kStages + 2;  // [2]  epilogue -> MMA
+  uint64_t* drain = bars + 2 * kStages + 4;      // MMA completion before teardown
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* off_s = reinterpret_cast<int*>(tmem_slot + 2);  // [E + 1]
-  int* tpre_s = off_s + 65;                            // [E + 1] row-tile prefix
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Dims& d = a.d;
@@ -136,26 +120,19 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
-    tc::mbar_init(acc_full, 1);
-    tc::mbar_init(acc_empty, 32 * kEpiWarps);
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&acc_full[b], 1); tc::mbar_init(&acc_empty[b], 128); }
     tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tmap_a);
     tc::tma_prefetch_desc(&tmap_b);
-    int t = 0;
-    for (int e = 0; e <= d.E; ++e) {
-      off_s[e] = a.offsets[e];
-      tpre_s[e] = t;
-      if (e < d.E) t += ceil_div(a.offsets[e + 1] - a.offsets[e], BM);
-    }
   }
   if (warp == 1) { tc::tmem_alloc(tmem_slot, kTmemCols); tc::tmem_relinquish(); }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int total = tpre_s[d.E] * nct;
+  const int total = *a.ntiles * nct;
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -165,15 +142,13 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const int rt = t / nct, ct = t % nct;
-      int e, row0, rows;
-      row_tile(tpre_s, off_s, d.E, rt, e, row0, rows);
+      const int e = a.tiles[2 * rt], row0 = a.tiles[2 * rt + 1];
       const int wrow = e * d.We + ct * BN;
       for (int kb = 0; kb < nkb; ++kb) {
         if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
         uint8_t* sa = stage_base + stage * kStageBytes;
         tc::mbar_arrive_expect_tx(&full[stage], kStageBytes);
         tc::tma_load_2d(sa, &tmap_a, &full[stage], kb * BK, row0);
-        tc::tma_load_2d(sa + kHalfA, &tmap_a, &full[stage], kb * BK, row0 + 128);
         tc::tma_load_2d(sa + kStageA, &tmap_b, &full[stage], kb * BK, wrow);
         ++issued;
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -190,14 +165,13 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     // ---------------------------------------------------------------- MMA issuer
     int stage = 0;
     uint32_t phase = 0;
+    int buf = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      int e, row0, rows;
-      row_tile(tpre_s, off_s, d.E, t / nct, e, row0, rows);
-      const bool two = rows > 128;
-      if (!tc::mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+      if (!tc::mbar_wait(&acc_empty[buf], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
+      const uint32_t dt = tmem + (uint32_t)(buf * BN);
       for (int kb = 0; kb < nkb; ++kb) {
         if (!tc::mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
@@ -205,16 +179,15 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         const uint32_t sb = sa + kStageA;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t bdesc = tc::sdesc_kmajor_sw128(sb + kk * 32);
-          tc::mma_f16(tmem, tc::sdesc_kmajor_sw128(sa + kk * 32), bdesc, kIdesc, (kb | kk) != 0);
-          if (two) tc::mma_f16(tmem + BN, tc::sdesc_kmajor_sw128(sa + kHalfA + kk * 32), bdesc, kIdesc, (kb | kk) != 0);
+          tc::mma_f16(dt, tc::sdesc_kmajor_sw128(sa + kk * 32), tc::sdesc_kmajor_sw128(sb + kk * 32), kIdesc,
+                      (kb | kk) != 0);
         }
         tc::mma_commit(&empty[stage]);
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
-      tc::mma_commit(acc_full);
-      acc_phase ^= 1u;
+      tc::mma_commit(&acc_full[buf]);
+      if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
     }
     if (!ok) { *abort_flag = 1; atomicOr(a.st, ST_TIMEOUT); }
     tc::mma_commit(drain);
@@ -222,39 +195,36 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     tc::mbar_wait(drain, 0, &never);
   } else if (warp >= 2) {
     // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;                 // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;       // M half this warp drains
-    const int row_local = 128 * half + 32 * q + lane;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_local = 32 * q + lane;
+    int buf = 0;
     uint32_t acc_phase = 0;
     bool range_bad = false;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const int rt = t / nct, ct = t % nct;
-      int e, row0, rows;
-      row_tile(tpre_s, off_s, d.E, rt, e, row0, rows);
-      const bool active = half == 0 || rows > 128;
-      const bool valid = row_local < rows;
-      const int p = valid ? a.perm[row0 + row_local] : 0;
+      const int e = a.tiles[2 * rt], row0 = a.tiles[2 * rt + 1];
+      const int rg = row0 + row_local;
+      const bool valid = rg < a.offsets[e + 1];
+      const int p = valid ? a.perm[rg] : 0;
       const float pi = (valid && a.mode != 2) ? a.topk_w[p] : 0.f;
-      if (!tc::mbar_wait(acc_full, acc_phase, abort_flag)) {
+      if (!tc::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) {
         *abort_flag = 1;
         atomicOr(a.st, ST_TIMEOUT);
         break;
       }
       tc::fence_after_sync();
-      if (active) {
-        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(half * BN);
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          tc::tmem_ld_32x32b_x32(taddr + 32 * c, r);
-          tc::tmem_ld_wait();
-          const int c0 = ct * BN + 32 * c;
-          if (valid && c0 < d.We) store_chunk(a, p, pi, c0, r, range_bad);
-        }
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tc::tmem_ld_32x32b_x32(taddr + 32 * c, r);
+        tc::tmem_ld_wait();
+        const int c0 = ct * BN + 32 * c;
+        if (valid && c0 < d.We) store_chunk(a, p, pi, c0, r, range_bad);
       }
       tc::fence_before_sync();
-      tc::mbar_arrive(acc_empty);
-      acc_phase ^= 1u;
+      tc::mbar_arrive(&acc_empty[buf]);
+      if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
     }
     if (range_bad) atomicOr(a.st, ST_RANGE);
   }
@@ -272,20 +242,18 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
 cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int32_t* perm,
                            const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, const float* topk_w,
                            int mode, void* bpi, void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s) {
-  (void)tiles;
-  (void)ntiles;
   CUtensorMap ta, tb;
-  if (!encode_tmap_2d(&ta, xsorted, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.M * d.k, (uint64_t)d.D * 2, BK, 128))
+  if (!encode_tmap_2d(&ta, xsorted, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.M * d.k, (uint64_t)d.D * 2, BK, BM))
     return cudaErrorInvalidValue;
   if (!encode_tmap_2d(&tb, w_exp, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.E * d.We, (uint64_t)d.D * 2, BK, BN))
     return cudaErrorInvalidValue;
-  TcArgs a{d, perm, offsets, topk_w, mode, (__half*)bpi, (__half*)xs, (__half*)cpi, Z, st};
+  TcArgs a{d, perm, tiles, ntiles, offsets, topk_w, mode, (__half*)bpi, (__half*)xs, (__half*)cpi, Z, st};
   cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int max_tiles = (ceil_div(d.M * d.k, BM) + d.E) * ceil_div(d.We, BN);
+  const int max_tiles = max_row_tiles(d) * ceil_div(d.We, BN);
   const int grid = max_tiles < sms ? max_tiles : sms;
   proj_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, a);
   count_launches(1);
