@@ -108,6 +108,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   uint64_t* fullB = reinterpret_cast<uint64_t*>(sm + Lay::BAR);
   uint64_t* fullX = fullB + 1;
   uint64_t* done = fullB + 2;
+  uint64_t* hbar = fullB + 3;  // bulk copy of H_in into the Bpi region
   float* cs_s = reinterpret_cast<float*>(sm + Lay::CS);
   float* fs_s = cs_s + SUB;
   float* wsum = fs_s + SUB;
@@ -120,6 +121,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     tc::mbar_init(fullB, 1);
     tc::mbar_init(fullX, 1);
     tc::mbar_init(done, 1);
+    tc::mbar_init(hbar, 1);
     tc::fence_barrier_init();
     misc[1] = atomicAdd(a.ticket, 1u);
   }
@@ -149,6 +151,30 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     ++issuedX;
   };
   if (tid == 0) { issue_b(0); issue_x(0); }
+  // H_in of this sub-chunk is the previous sub-chunk's H_out.  With P = 64 it fits the Bpi region once the
+  // last slot's key products are done, so thread 0 fetches it with one bulk copy as soon as the
+  // predecessor's flag is up, while the other threads still work on the last slot.
+  constexpr bool kEarlyFetch = P == 64;
+  const size_t NPs = (size_t)N * P;
+  const float* hprev = csub > 0 ? a.exch + ((size_t)bh * a.nsub + csub - 1) * NPs : nullptr;
+  const unsigned* pflag = csub > 0 ? a.flags + (size_t)bh * a.nsub + csub - 1 : nullptr;
+  bool h_issued = false;
+  auto try_fetch_hin = [&](bool block) {  // thread 0 only
+    if (!kEarlyFetch || h_issued || csub == 0) return;
+    uint32_t n = 0;
+    while (ld_acquire(pflag) == 0u) {
+      if (!block) return;
+      if (++n >= kFlagPolls) { atomicOr(a.st, ST_TIMEOUT); break; }
+      if (n > 64) __nanosleep(32);
+    }
+    tc::fence_proxy_async_global();
+    tc::mbar_arrive_expect_tx(hbar, (uint32_t)(NPs * 4));
+    tc::bulk_load(BP, hprev, (uint32_t)(NPs * 4), hbar);
+    h_issued = true;
+  };
+
+  // this row's dt is loaded first so its latency overlaps the readout loads below
+  const float dt_row = (half == 0 && row < L) ? a.dt[(size_t)(row0 + row) * d.H + h] : 0.f;
 
   // C~ rows: sum of the readout slots, loaded coalesced (16 lanes per 256-byte row), fp16 K-major swizzled.
   // Warp w covers rows 16w .. 16w + 15.  Two slots are added as fp16 pairs (the correctly rounded sum).
@@ -213,7 +239,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   // cumulative log-decay of the sub-chunk (inclusive scan over the 128 rows)
   float v = 0.f;
   if (half == 0) {
-    v = row < L ? a.dt[(size_t)(row0 + row) * d.H + h] * a.A[h] : 0.f;
+    v = dt_row * a.A[h];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const float u = __shfl_up_sync(0xffffffffu, v, o);
@@ -279,6 +305,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     if (!__syncthreads_and(ok)) { ok = false; break; }
     tc::fence_after_sync();
     if (tid == 0 && i + 1 < nk) issue_b(i + 1);  // Bpi_i is no longer read
+    if (tid == 0 && i + 1 == nk) try_fetch_hin(false);  // the Bpi region is free for good
     // masked, decayed scores, one 64-key half at a time -> fp16 K-major swizzled rows of Pm; this thread
     // takes the 32 keys of block 2*hk + half, whose decays share one factor exp(cs_t - cs_{32b})
     for (int hk = 0; hk < 2 && ok; ++hk) {
@@ -317,24 +344,32 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
       done_phase ^= 1u;
       if (!__syncthreads_and(ok)) { ok = false; break; }
       tc::fence_after_sync();
+      if (tid == 0 && i + 1 == nk) try_fetch_hin(false);
     }
     if (tid == 0 && ok && i + 1 < nk) issue_x(i + 1);  // Xs_i is no longer read
   }
 
   if (ok) {
     // ---------------------------------------------------------------- state hand-off
-    const size_t NP = (size_t)N * P;
+    const size_t NP = NPs;
     if (tid == 0 && csub > 0) {
-      const unsigned* f = a.flags + (size_t)bh * a.nsub + csub - 1;
-      uint32_t n = 0;
-      while (ld_acquire(f) == 0u && n < kFlagPolls) {
-        if (n > 64) __nanosleep(32);
-        ++n;
+      if (kEarlyFetch) {
+        try_fetch_hin(true);
+      } else {
+        uint32_t n = 0;
+        while (ld_acquire(pflag) == 0u && n < kFlagPolls) {
+          if (n > 64) __nanosleep(32);
+          ++n;
+        }
+        if (n == kFlagPolls) atomicOr(a.st, ST_TIMEOUT);
       }
-      if (n == kFlagPolls) atomicOr(a.st, ST_TIMEOUT);
     }
-    __syncthreads();
-    const float* hin = csub > 0 ? a.exch + ((size_t)bh * a.nsub + csub - 1) * NP
+    bool hok = true;
+    if (kEarlyFetch && csub > 0) hok = tc::mbar_wait(hbar, 0, &never);
+    hok = __syncthreads_and(hok);
+    if (!hok && tid == 0) atomicOr(a.st, ST_TIMEOUT);  // continues with a zero state; the result is flagged
+    const bool hin_shared = kEarlyFetch && csub > 0;
+    const float* hin = csub > 0 ? (hin_shared ? (hok ? reinterpret_cast<const float*>(BP) : nullptr) : hprev)
                                 : (a.init ? a.init + (size_t)bh * NP : nullptr);
     float* hout = a.exch + ((size_t)bh * a.nsub + csub) * NP;
     const float dend = expf(cs_end);
@@ -343,7 +378,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     float4 hv[PH / 4];
 #pragma unroll
     for (int u = 0; u < PH / 4; ++u)
-      hv[u] = hin ? __ldcg(reinterpret_cast<const float4*>(hin + rbase + 4 * u)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      hv[u] = !hin ? make_float4(0.f, 0.f, 0.f, 0.f)
+                   : (hin_shared ? *reinterpret_cast<const float4*>(hin + rbase + 4 * u)
+                                 : __ldcg(reinterpret_cast<const float4*>(hin + rbase + 4 * u)));
 #pragma unroll
     for (int q = 0; q < PH / 32; ++q) {
       uint32_t r[32];
@@ -357,7 +394,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
         __stcg(reinterpret_cast<float4*>(hout + rbase + 32 * q + 4 * u), o);
       }
     }
-    __threadfence();
+    // every thread's H_out stores are ordered before the barrier; thread 0's release store at device scope
+    // is cumulative over them, so a consumer that acquires the flag sees the whole state
     __syncthreads();
     if (tid == 0) st_release(a.flags + (size_t)bh * a.nsub + csub, 1u);
     // off the hand-off chain: requested states, and the fp16 hi/lo split of H_in for the readout product
@@ -465,6 +503,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   if (tid == 0) {
     if (issuedB > 0) tc::mbar_wait(fullB, (uint32_t)((issuedB - 1) & 1), &never);
     if (issuedX > 0) tc::mbar_wait(fullX, (uint32_t)((issuedX - 1) & 1), &never);
+    if (h_issued) tc::mbar_wait(hbar, 0, &never);
   }
   tc::fence_before_sync();
   __syncthreads();
