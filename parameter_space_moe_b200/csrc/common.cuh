@@ -66,6 +66,7 @@ struct WsPlan {
   size_t dbase;       // int32 [ndt][E]  first sorted position of each (tile, expert)
   size_t offsets;     // int32 [E+1]
   size_t perm;        // int32 [M*k]
+  size_t rowmeta;     // int2 [M*k]: per sorted row (pair index, router weight bits) for the GEMM epilogue
   size_t tiles;       // int32 [max_tiles][2]  GEMM row-tile schedule (expert, first sorted row)
   size_t ntiles;      // int32 [1]
   size_t xsorted;     // dtype [M*k][D] rows of X in sorted (expert-major) order
@@ -98,11 +99,12 @@ WsPlan plan_workspace(const Dims& d);
 // (token, slot) pairs it routes (dispatch tile = pair index / kDispatchTile).
 cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
                           float* dt, int32_t* counts, cudaStream_t s);
+// rowmeta (nullable): per sorted row, (pair index p, router weight of p as float bits; 0 without topk_w)
 cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
-                            int32_t* perm, cudaStream_t s);
+                            int32_t* perm, int2* rowmeta, const float* topk_w, cudaStream_t s);
 // The layer's one-launch dispatch over counts the router produced (see launch_router).
 cudaError_t launch_dispatch_fused(const Dims& d, const int32_t* idx, const int32_t* counts, const WsPlan& p, char* ws,
-                                  int32_t* offsets, int32_t* perm, cudaStream_t s);
+                                  int32_t* offsets, int32_t* perm, const float* topk_w, cudaStream_t s);
 cudaError_t launch_gather_rows(const Dims& d, const void* X, const int32_t* perm, void* xsorted, cudaStream_t s);
 // mode 0: fused mix (pi-scaled B and C), 1: fused mix with unscaled B, 2: raw Z (fp32)
 cudaError_t launch_proj_simt(const Dims& d, const void* X, const void* w_exp, const int32_t* perm,
@@ -110,9 +112,9 @@ cudaError_t launch_proj_simt(const Dims& d, const void* X, const void* w_exp, co
                              const float* topk_w, int mode, void* bpi, void* xs, void* cpi, float* Z, unsigned* st,
                              cudaStream_t s);
 // Tensor-core version (bf16 X and weights, fp16 streams): A operand is xsorted (rows in expert order).
-cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int32_t* perm,
-                           const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, const float* topk_w,
-                           int mode, void* bpi, void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s);
+cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int2* rowmeta,
+                           const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, int mode, void* bpi,
+                           void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s);
 cudaError_t launch_mix(const Dims& d, const float* Z, const float* topk_w, int flags, void* bpi, void* xs, void* cpi,
                        unsigned* st, cudaStream_t s);
 // Chunked scan.  Slot ranges select which of the k per-token keys feed one trajectory and which

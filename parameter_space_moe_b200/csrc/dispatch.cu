@@ -69,7 +69,7 @@ dispatch_offsets_kernel(Dims d, int ntile, const int32_t* __restrict__ counts, i
 
 __global__ void __launch_bounds__(kDispatchThreads)
 dispatch_scatter_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* __restrict__ base,
-                        int32_t* __restrict__ perm) {
+                        int32_t* __restrict__ perm, int2* __restrict__ rowmeta, const float* __restrict__ topk_w) {
   __shared__ int wc_s[kDispatchThreads / 32][64];  // per-warp counts, turned into per-warp bases
   const int tile = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = d.M * d.k;
@@ -91,7 +91,11 @@ dispatch_scatter_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* 
     }
   }
   __syncthreads();
-  if (valid) perm[wc_s[warp][e] + rank] = p;
+  if (valid) {
+    const int pos = wc_s[warp][e] + rank;
+    perm[pos] = p;
+    if (rowmeta) rowmeta[pos] = make_int2(p, topk_w ? __float_as_int(topk_w[p]) : 0);
+  }
 }
 
 // The layer's dispatch in one launch: per-tile counts arrive from the router (integer atomics into a
@@ -101,7 +105,7 @@ dispatch_scatter_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* 
 __global__ void __launch_bounds__(kDispatchThreads)
 dispatch_fused_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* __restrict__ counts,
                       int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ tiles,
-                      int32_t* __restrict__ ntiles) {
+                      int32_t* __restrict__ ntiles, int2* __restrict__ rowmeta, const float* __restrict__ topk_w) {
   __shared__ int wc_s[kDispatchThreads / 32][64];
   __shared__ int tot_s[64], pre_s[64], off_s[65], toff_s[65];
   const int tile = blockIdx.x, ntile = gridDim.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -155,7 +159,11 @@ dispatch_fused_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* __
     }
   }
   __syncthreads();
-  if (valid) perm[wc_s[warp][e] + rank] = p;
+  if (valid) {
+    const int pos = wc_s[warp][e] + rank;
+    perm[pos] = p;
+    rowmeta[pos] = make_int2(p, __float_as_int(topk_w[p]));
+  }
 }
 
 // X rows in sorted order: xsorted[r] = X[perm[r] / k].  One warp per row, 16-byte vectors.
@@ -172,23 +180,24 @@ __global__ void gather_rows_kernel(Dims d, const T* __restrict__ X, const int32_
 }
 
 cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
-                            int32_t* perm, cudaStream_t s) {
+                            int32_t* perm, int2* rowmeta, const float* topk_w, cudaStream_t s) {
   const int nt = dispatch_tiles(d);
   int32_t* counts = (int32_t*)(ws + p.dcounts);
   int32_t* base = (int32_t*)(ws + p.dbase);
   dispatch_count_kernel<<<nt, kDispatchThreads, 0, s>>>(d, idx, counts);
   dispatch_offsets_kernel<<<1, 1024, 0, s>>>(d, nt, counts, base, offsets, (int32_t*)(ws + p.tiles),
                                              (int32_t*)(ws + p.ntiles));
-  dispatch_scatter_kernel<<<nt, kDispatchThreads, 0, s>>>(d, idx, base, perm);
+  dispatch_scatter_kernel<<<nt, kDispatchThreads, 0, s>>>(d, idx, base, perm, rowmeta, topk_w);
   count_launches(3);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dispatch_fused(const Dims& d, const int32_t* idx, const int32_t* counts, const WsPlan& p, char* ws,
-                                  int32_t* offsets, int32_t* perm, cudaStream_t s) {
+                                  int32_t* offsets, int32_t* perm, const float* topk_w, cudaStream_t s) {
   dispatch_fused_kernel<<<dispatch_tiles(d), kDispatchThreads, 0, s>>>(d, idx, counts, offsets, perm,
                                                                         (int32_t*)(ws + p.tiles),
-                                                                        (int32_t*)(ws + p.ntiles));
+                                                                        (int32_t*)(ws + p.ntiles),
+                                                                        (int2*)(ws + p.rowmeta), topk_w);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -77,7 +77,8 @@ extern "C" swimba_status swimba_dispatch_noalloc(const swimba_dims* dims, const 
   if (!scratch_plan(d, &p)) return SWIMBA_ERR_WORKSPACE;  // needs more than the fixed 1 MiB scratch
   char* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return SWIMBA_ERR_CUDA;
-  return launch_dispatch(d, topk_idx, p, scratch, expert_offsets, perm, (cudaStream_t)stream) == cudaSuccess
+  return launch_dispatch(d, topk_idx, p, scratch, expert_offsets, perm, nullptr, nullptr, (cudaStream_t)stream) ==
+                 cudaSuccess
              ? SWIMBA_OK
              : SWIMBA_ERR_CUDA;
 }

@@ -7,13 +7,16 @@
 // The notes name a fused MoE operator for this input projection as the way to avoid HBM round trips of
 // router outputs and parameter slices; here the per-expert output tile never leaves the SM unmixed.
 //
-// Design (one persistent CTA per SM, 6 warps):
+// Design (one persistent CTA per SM, 10 warps):
 //   warp 0      TMA producer: A = 128 gathered X rows x 64 K (16 KB), B = 256 weight rows x 64 K (32 KB)
 //               per stage, 128-byte swizzle, kStages-deep ring of mbarriers
 //   warp 1      TMEM owner and MMA issuer: 4 x tcgen05.mma M128 N256 K16 per stage into one of two
 //               256-column fp32 accumulators (double buffered: 512 TMEM columns)
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time (warp w reads TMEM lanes 32*(w%4)..), scales
-//               B and C columns by pi, converts to fp16 and stores to the destination (token, slot) row
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4).. and one 128-column half of the tile,
+//               32 columns at a time; scales B and C columns by pi, converts to fp16 and stores to the
+//               destination (token, slot) row.  Each row's (pair, pi) comes from the dispatch's per-row
+//               metadata in one load issued before the accumulator wait; the next tile's schedule entry
+//               is prefetched while the current tile drains.
 // Tiles: (row tile of one expert's sorted rows) x (256 output columns), handed out round-robin.
 #include "tc_common.cuh"
 
@@ -21,19 +24,21 @@ namespace swimba {
 
 namespace {
 constexpr int BM = 128, BN = 256, BK = 64, kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kStageA = BM * BK * 2, kStageB = BN * BK * 2, kStageBytes = kStageA + kStageB;
 constexpr uint32_t kTmemCols = 2 * BN;
 constexpr uint32_t kIdesc = tc::idesc_f16(BM, BN, /*bf16=*/true);
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 256;
+constexpr int kStageRow = 80;                             // 64 B of fp16 + 16 B pad (conflict-free)
+constexpr uint32_t kEpiStage = 32 * kStageRow;            // one warp's 32 rows x 32 columns
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 1024 + (size_t)kEpiWarps * kEpiStage;
 
 struct TcArgs {
   Dims d;
-  const int32_t* perm;
+  const int2* rowmeta;  // per sorted row: (pair index, router weight bits)
   const int32_t* tiles;
   const int32_t* ntiles;
   const int32_t* offsets;
-  const float* topk_w;
   int mode;  // 0 mix, 1 mix with unscaled B, 2 raw fp32 Z
   __half* bpi;
   __half* xs;
@@ -98,6 +103,49 @@ __device__ __forceinline__ void store_chunk(const TcArgs& a, int p, float pi, in
   }
 }
 
+// Destination of the 32-column group starting at column c0 of z when it lies in one stream (else null),
+// and the scale its values take.
+__device__ __forceinline__ __half* group_dst(const TcArgs& a, int p, float pi, int c0, float& sc) {
+  const Dims& d = a.d;
+  const int HP = d.HP, GN = d.GN;
+  if (c0 + 32 > d.We) return nullptr;
+  if (c0 + 32 <= HP) { sc = 1.f; return a.xs + (size_t)p * HP + c0; }
+  if (c0 >= HP && c0 + 32 <= HP + GN) { sc = a.mode == 1 ? 1.f : pi; return a.bpi + (size_t)p * GN + (c0 - HP); }
+  if (c0 >= HP + GN) { sc = pi; return a.cpi + (size_t)p * GN + (c0 - HP - GN); }
+  return nullptr;
+}
+
+// One warp stores 32 columns of its 32 rows: each thread converts its row's values to fp16 into the warp's
+// staging rows, then every store instruction writes 8 whole 64-byte row segments.
+__device__ __forceinline__ void store_group32(const TcArgs& a, uint8_t* stage, int lane, bool valid, int p, float pi,
+                                              int c0, const uint32_t (&r)[32], bool& range_bad) {
+  float sc = 0.f;
+  __half* dst = valid ? group_dst(a, p, pi, c0, sc) : nullptr;
+  uint8_t* my = stage + lane * kStageRow;
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    uint4 v;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float f0 = sc * u2f(r[i + 2 * q]), f1 = sc * u2f(r[i + 2 * q + 1]);
+      range_bad |= dst && (!(fabsf(f0) <= kF16Max) || !(fabsf(f1) <= kF16Max));
+      __half2 h = __floats2half2_rn(f0, f1);
+      w[q] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(my + 2 * i) = v;
+  }
+  __syncwarp();
+  const unsigned long long dptr = reinterpret_cast<unsigned long long>(dst);
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int row = 8 * it + (lane >> 2), chunk = lane & 3;
+    const unsigned long long rd = __shfl_sync(0xffffffffu, dptr, row);
+    if (rd) *reinterpret_cast<uint4*>(rd + 16 * chunk) = *reinterpret_cast<const uint4*>(stage + row * kStageRow + 16 * chunk);
+  }
+  __syncwarp();
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -112,6 +160,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
   uint64_t* drain = bars + 2 * kStages + 4;      // MMA completion before teardown
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* off_s = reinterpret_cast<int*>(tmem_slot + 2);  // [E + 1] expert offsets
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Dims& d = a.d;
@@ -120,7 +169,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { tc::mbar_init(&acc_full[b], 1); tc::mbar_init(&acc_empty[b], 128); }
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&acc_full[b], 1); tc::mbar_init(&acc_empty[b], 32 * kEpiWarps); }
     tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -128,6 +177,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     tc::tma_prefetch_desc(&tmap_b);
   }
   if (warp == 1) { tc::tmem_alloc(tmem_slot, kTmemCols); tc::tmem_relinquish(); }
+  for (int e = threadIdx.x; e <= d.E; e += blockDim.x) off_s[e] = a.offsets[e];
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -195,32 +245,42 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     tc::mbar_wait(drain, 0, &never);
   } else if (warp >= 2) {
     // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int ch = (warp - 2) >> 2;      // which 128-column half of the tile
     const int row_local = 32 * q + lane;
+    uint8_t* epi_stage = smem + kStages * kStageBytes + 1024 + (warp - 2) * kEpiStage;
     int buf = 0;
     uint32_t acc_phase = 0;
     bool range_bad = false;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const int rt = t / nct, ct = t % nct;
-      const int e = a.tiles[2 * rt], row0 = a.tiles[2 * rt + 1];
-      const int rg = row0 + row_local;
-      const bool valid = rg < a.offsets[e + 1];
-      const int p = valid ? a.perm[rg] : 0;
-      const float pi = (valid && a.mode != 2) ? a.topk_w[p] : 0.f;
+    int t = blockIdx.x;
+    int2 tinfo = t < total ? *reinterpret_cast<const int2*>(a.tiles + 2 * (t / nct)) : make_int2(0, 0);
+    for (; t < total; t += gridDim.x) {
+      const int ct = t % nct;
+      const int e = tinfo.x, row0 = tinfo.y;
+      const bool valid = row0 + row_local < off_s[e + 1];
+      const int2 meta = valid ? a.rowmeta[row0 + row_local] : make_int2(0, 0);
+      const int tn = t + gridDim.x;
+      if (tn < total) tinfo = *reinterpret_cast<const int2*>(a.tiles + 2 * (tn / nct));
       if (!tc::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) {
         *abort_flag = 1;
         atomicOr(a.st, ST_TIMEOUT);
         break;
       }
       tc::fence_after_sync();
-      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + ch * (BN / 2));
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < BN / 64; ++c) {
         uint32_t r[32];
         tc::tmem_ld_32x32b_x32(taddr + 32 * c, r);
         tc::tmem_ld_wait();
-        const int c0 = ct * BN + 32 * c;
-        if (valid && c0 < d.We) store_chunk(a, p, pi, c0, r, range_bad);
+        const int c0 = ct * BN + ch * (BN / 2) + 32 * c;
+        const float pi = __int_as_float(meta.y);
+        float sc_probe;
+        // fast path: the warp's 32-column group lies in one fp16 stream for every valid row
+        const bool fast = a.mode != 2 && c0 + 32 <= d.We &&
+                          __all_sync(0xffffffffu, !valid || group_dst(a, meta.x, pi, c0, sc_probe) != nullptr);
+        if (fast) store_group32(a, epi_stage, lane, valid, meta.x, pi, c0, r, range_bad);
+        else if (valid && c0 < d.We) store_chunk(a, meta.x, pi, c0, r, range_bad);
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&acc_empty[buf]);
@@ -239,15 +299,15 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
 }  // namespace
 
 // Host side --------------------------------------------------------------------------------------
-cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int32_t* perm,
-                           const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, const float* topk_w,
-                           int mode, void* bpi, void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s) {
+cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int2* rowmeta,
+                           const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, int mode, void* bpi,
+                           void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s) {
   CUtensorMap ta, tb;
   if (!encode_tmap_2d(&ta, xsorted, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.M * d.k, (uint64_t)d.D * 2, BK, BM))
     return cudaErrorInvalidValue;
   if (!encode_tmap_2d(&tb, w_exp, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.E * d.We, (uint64_t)d.D * 2, BK, BN))
     return cudaErrorInvalidValue;
-  TcArgs a{d, perm, tiles, ntiles, offsets, topk_w, mode, (__half*)bpi, (__half*)xs, (__half*)cpi, Z, st};
+  TcArgs a{d, rowmeta, tiles, ntiles, offsets, mode, (__half*)bpi, (__half*)xs, (__half*)cpi, Z, st};
   cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   int sms = 148;

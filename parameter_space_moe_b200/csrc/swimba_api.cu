@@ -73,6 +73,7 @@ WsPlan plan_workspace(const Dims& d) {
   p.dbase = take((size_t)dispatch_tiles(d) * d.E * 4);
   p.offsets = take((size_t)(d.E + 1) * 4);
   p.perm = take(Mk * 4);
+  p.rowmeta = take(Mk * 8);
   p.tiles = take((size_t)max_row_tiles(d) * 8);
   p.ntiles = take(4);
   p.xsorted = take(Mk * d.D * elem_bytes(d.dtype));
@@ -155,7 +156,8 @@ static swimba_status run_proj(const Dims& d, const void* X, const void* w_exp, c
   if (d.dtype == SWIMBA_BF16) {
     SW_CUDA(launch_gather_rows(d, X, perm, ws + p.xsorted, s));
     prof_mark(s, "gather");
-    SW_CUDA(launch_proj_tc(d, ws + p.xsorted, w_exp, perm, tiles, ntiles, offsets, wts, mode, bpi, xs, cpi, Z, st, s));
+    SW_CUDA(launch_proj_tc(d, ws + p.xsorted, w_exp, (const int2*)(ws + p.rowmeta), tiles, ntiles, offsets, mode, bpi,
+                           xs, cpi, Z, st, s));
   } else {
     SW_CUDA(launch_proj_simt(d, X, w_exp, perm, tiles, ntiles, offsets, wts, mode, bpi, xs, cpi, Z, st, s));
   }
@@ -174,7 +176,7 @@ static swimba_status run_front(const Dims& d, const void* X, const swimba_weight
   prof_mark(s, "router");
   int32_t* offsets = (int32_t*)(ws + p.offsets);
   int32_t* perm = (int32_t*)(ws + p.perm);
-  SW_CUDA(launch_dispatch_fused(d, idx, counts, p, ws, offsets, perm, s));
+  SW_CUDA(launch_dispatch_fused(d, idx, counts, p, ws, offsets, perm, wts, s));
   prof_mark(s, "dispatch");
   SW_TRY(run_proj(d, X, w->w_exp, ws, p, wts, mode, ws + p.bpi, ws + p.xs, ws + p.cpi, nullptr, st, s));
   return SWIMBA_OK;
@@ -242,7 +244,8 @@ swimba_status swimba_dispatch(const swimba_dims* dims, const int32_t* topk_idx, 
   if (!ok_ptr(topk_idx) || !ok_ptr(expert_offsets) || !ok_ptr(perm)) return SWIMBA_ERR_INVALID_ARG;
   SW_TRY(check_ws(d, ws, ws_bytes));
   WsPlan p = plan_workspace(d);
-  return cuda_status(launch_dispatch(d, topk_idx, p, (char*)ws, expert_offsets, perm, (cudaStream_t)stream));
+  return cuda_status(
+      launch_dispatch(d, topk_idx, p, (char*)ws, expert_offsets, perm, nullptr, nullptr, (cudaStream_t)stream));
 }
 
 swimba_status swimba_expert_proj(const swimba_dims* dims, const void* X, const swimba_weights* w,
@@ -257,7 +260,7 @@ swimba_status swimba_expert_proj(const swimba_dims* dims, const void* X, const s
   cudaStream_t s = (cudaStream_t)stream;
   int32_t* offsets = (int32_t*)(b + p.offsets);
   int32_t* perm = (int32_t*)(b + p.perm);
-  SW_CUDA(launch_dispatch(d, topk_idx, p, b, offsets, perm, s));
+  SW_CUDA(launch_dispatch(d, topk_idx, p, b, offsets, perm, (int2*)(b + p.rowmeta), nullptr, s));
   return run_proj(d, X, w->w_exp, b, p, nullptr, 2, nullptr, nullptr, nullptr, Z, device_status(), s);
 }
 
