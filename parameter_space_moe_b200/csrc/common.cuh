@@ -98,7 +98,11 @@ WsPlan plan_workspace(const Dims& d);
 // counts (nullable): [dispatch tile][E] table, zeroed by the caller, that the router increments for the
 // (token, slot) pairs it routes (dispatch tile = pair index / kDispatchTile).
 cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
-                          float* dt, int32_t* counts, cudaStream_t s);
+                          float* dt, int32_t* counts, unsigned* st, cudaStream_t s);
+// The tensor-core (tcgen05) router that launch_router prefers where it applies.
+bool router_tc_supported(const Dims& d);
+cudaError_t launch_router_tc(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
+                             float* dt, int32_t* counts, unsigned* st, cudaStream_t s);
 // rowmeta (nullable): per sorted row, (pair index p, router weight of p as float bits; 0 without topk_w)
 cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
                             int32_t* perm, int2* rowmeta, const float* topk_w, cudaStream_t s);
@@ -149,5 +153,9 @@ cudaError_t launch_step_update(const Dims& d, const void* bpi, const void* xs, c
                                const float* A, float* state, void* y, cudaStream_t s);
 // Adds n to the library's launch counter (every launcher reports the kernels it issued).
 void count_launches(int n);
+// Raises a kernel's dynamic shared-memory limit on the current device to at least `bytes`; the driver is
+// asked only when a larger limit than any earlier one is needed (the call costs microseconds of host time
+// that would otherwise sit in front of every launch).
+cudaError_t set_max_dynamic_smem(const void* kernel, size_t bytes);
 
 }  // namespace swimba

@@ -308,7 +308,7 @@ cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp
   if (!encode_tmap_2d(&tb, w_exp, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.E * d.We, (uint64_t)d.D * 2, BK, BN))
     return cudaErrorInvalidValue;
   TcArgs a{d, rowmeta, tiles, ntiles, offsets, mode, (__half*)bpi, (__half*)xs, (__half*)cpi, Z, st};
-  cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  cudaError_t e = set_max_dynamic_smem((const void*)proj_tc_kernel, kSmemBytes);
   if (e != cudaSuccess) return e;
   int sms = 148;
   int dev = 0;

@@ -16,7 +16,6 @@
 namespace swimba {
 
 namespace {
-constexpr int kMaxE = 64;
 
 // Top-k, renormalised weights and dt for one token; logits g[0..E) and pre-activations g[E..E+H) in
 // (shared) memory, called by a whole warp.
@@ -235,12 +234,16 @@ router_mma_kernel(Dims d, int RP, const __nv_bfloat16* __restrict__ X, const __n
 }  // namespace
 
 cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
-                          float* dt, int32_t* counts, cudaStream_t s) {
+                          float* dt, int32_t* counts, unsigned* st, cudaStream_t s) {
   const int R = d.E + d.H;
+  if (st && router_tc_supported(d)) {
+    const cudaError_t e = launch_router_tc(d, X, w, idx, wts, dt, counts, st, s);
+    if (e != cudaErrorNotSupported) return e;
+  }
   if (d.dtype == SWIMBA_BF16 && R <= 8 * kMaxNT) {
     const int RP = (R + 15) / 16 * 16;
     const size_t smem = (size_t)kStagesR * (kMT + RP) * kLd * 2 + (size_t)kMT * (RP + 1) * 4;
-    cudaError_t e = cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem((const void*)router_mma_kernel, smem);
     if (e != cudaSuccess) return e;
     router_mma_kernel<<<ceil_div(d.M, kMT), 128, smem, s>>>(d, RP, (const __nv_bfloat16*)X,
                                                              (const __nv_bfloat16*)w.w_router,
@@ -250,14 +253,14 @@ cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w,
     const size_t smem = sizeof(float) * (size_t)kRouterWarps * (d.D + R);
     if (d.dtype == SWIMBA_BF16) {
       auto k = router_simt_kernel<__nv_bfloat16>;
-      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaError_t e = set_max_dynamic_smem((const void*)k, smem);
       if (e != cudaSuccess) return e;
       k<<<ceil_div(d.M, kRouterWarps), kRouterWarps * 32, smem, s>>>(
           d, (const __nv_bfloat16*)X, (const __nv_bfloat16*)w.w_router, (const __nv_bfloat16*)w.w_dt, w.b_dt, idx,
           wts, dt, counts);
     } else {
       auto k = router_simt_kernel<float>;
-      cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaError_t e = set_max_dynamic_smem((const void*)k, smem);
       if (e != cudaSuccess) return e;
       k<<<ceil_div(d.M, kRouterWarps), kRouterWarps * 32, smem, s>>>(d, (const float*)X, (const float*)w.w_router,
                                                                       (const float*)w.w_dt, w.b_dt, idx, wts, dt,

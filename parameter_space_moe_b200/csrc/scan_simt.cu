@@ -153,8 +153,8 @@ cudaError_t launch_scan_simt(const Dims& d, const ScanArgs& a, cudaStream_t s) {
   const bool bf = d.dtype == SWIMBA_BF16;
   auto kc = bf ? scan_chunk_kernel<__half> : scan_chunk_kernel<float>;
   auto ko = bf ? scan_out_kernel<__half, __nv_bfloat16> : scan_out_kernel<float, float>;
-  cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_chunk);
-  cudaFuncSetAttribute(ko, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out);
+  set_max_dynamic_smem((const void*)kc, sm_chunk);
+  set_max_dynamic_smem((const void*)ko, sm_out);
   kc<<<grid, kScanThreads, sm_chunk, s>>>(d, a);
   scan_pass_kernel<<<dim3(d.Bsz * d.H, ceil_div(d.N * d.P, 256)), 256, 0, s>>>(d, a);
   ko<<<grid, kScanThreads, sm_out, s>>>(d, a);

@@ -5,8 +5,8 @@
 // and the overall framework's chunked SSD solve.  One CTA owns SUB = 128 consecutive tokens of one
 // (sequence, head); with cs_t the running sum of dt*A from the sub-chunk start:
 //   S_j      = C~ Bpi_j^T                        (tensor core, 128 x 128 per key slot j, in TMEM)
-//   Pm_j     = mask_{s<=t}(S_j * exp(cs_t - cs_s))   (registers -> fp16 in shared memory)
-//   Y       += Pm_j Xs_j                          (tensor core)
+//   Pm_j     = mask_{s<=t}(S_j * exp(cs_t - cs_s))   (registers -> fp16 pairs back into TMEM over S_j)
+//   Y       += Pm_j Xs_j                          (tensor core, Pm_j read from TMEM)
 //   Sc      += Bpi_j^T (exp(cs_end - cs_s) Xs_j)  (tensor core: the sub-chunk's own end state)
 //   H_out    = exp(cs_end) H_in + Sc              (fp32; H_in from the previous sub-chunk's CTA)
 //   y        = Y + exp(cs_t) C~ H_in              (tensor core, H_in split into fp16 hi + lo parts)
@@ -78,7 +78,7 @@ struct ScanSmem {
   static constexpr uint32_t CT = 0;               // C~ rows, K-major, NB blocks
   static constexpr uint32_t BP = CT + NB * kBlk;  // Bpi_j (NB blocks); H_in hi/lo parts after the slot loop
   static constexpr uint32_t XS = BP + NB * kBlk;  // Xs_j (PB blocks)
-  static constexpr uint32_t PM = XS + PB * kBlk;  // one 64-key half of Pm, or the decay-scaled Xs_j
+  static constexpr uint32_t PM = XS + PB * kBlk;  // the decay-scaled Xs_j
   static constexpr uint32_t BAR = PM + PB * kBlk; // fullB, fullX, done
   static constexpr uint32_t CS = BAR + 64;        // cs[SUB], fs[SUB], wsum[4], misc[2]
   static constexpr uint32_t END = CS + 2 * SUB * 4 + 64;
@@ -306,46 +306,50 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     tc::fence_after_sync();
     if (tid == 0 && i + 1 < nk) issue_b(i + 1);  // Bpi_i is no longer read
     if (tid == 0 && i + 1 == nk) try_fetch_hin(false);  // the Bpi region is free for good
-    // masked, decayed scores, one 64-key half at a time -> fp16 K-major swizzled rows of Pm; this thread
-    // takes the 32 keys of block 2*hk + half, whose decays share one factor exp(cs_t - cs_{32b})
-    for (int hk = 0; hk < 2 && ok; ++hk) {
-      const int kb = 2 * hk + half;
-      const float et = (32 * kb <= row && row < L) ? expf(my_cs - cs_s[32 * kb]) : 0.f;
-      uint32_t r[32];
-      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * kb, r);
+    // masked, decayed scores of this thread's two 32-key blocks kb = half and half + 2 (their decays share
+    // one factor exp(cs_t - cs_{32b}) per block), packed to fp16 pairs and stored back into TMEM over the
+    // first 64 columns of S, where the next product takes them as its A operand
+    {
+      uint32_t r0[32], r1[32];
+      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * half, r0);
+      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * (half + 2), r1);
       tc::tmem_ld_wait();
+      uint32_t p0[16], p1[16];
+      auto pack = [&](const uint32_t (&r)[32], int kb, uint32_t (&pk)[16]) {
+        const float et = (32 * kb <= row && row < L) ? expf(my_cs - cs_s[32 * kb]) : 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int s = 32 * kb + 8 * c + e;
-          f[e] = s <= row ? u2f(r[8 * c + e]) * (et * fs_s[s]) : 0.f;
+        for (int e = 0; e < 16; ++e) {
+          const int s0 = 32 * kb + 2 * e;
+          const float f0 = s0 <= row ? u2f(r[2 * e]) * (et * fs_s[s0]) : 0.f;
+          const float f1 = s0 + 1 <= row ? u2f(r[2 * e + 1]) * (et * fs_s[s0 + 1]) : 0.f;
+          pk[e] = pack_half2(f0, f1);
         }
-        uint4 o;
-        o.x = pack_half2(f[0], f[1]); o.y = pack_half2(f[2], f[3]);
-        o.z = pack_half2(f[4], f[5]); o.w = pack_half2(f[6], f[7]);
-        *reinterpret_cast<uint4*>(PM + tc::sw128_chunk(row, 4 * half + c)) = o;
-      }
-      tc::fence_proxy_async();
+      };
+      pack(r0, half, p0);
+      pack(r1, half + 2, p1);
       tc::fence_before_sync();
-      __syncthreads();
+      __syncthreads();  // every row's scores are read before any packed store lands on them
       tc::fence_after_sync();
-      if (tid == 0) {
-        const uint32_t pm = tc::smem_u32(PM), xs = tc::smem_u32(XS) + hk * 8192;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          tc::mma_f16(tmem + COL_Y, tc::sdesc_kmajor_sw128(pm + kk * 32), tc::sdesc_mnmajor_sw128(xs + kk * 2048, kBlk),
-                      ID_Y, (i > 0) || (hk > 0) || (kk > 0));
-        }
-        tc::mma_commit(done);
-      }
-      ok = tc::mbar_wait(done, done_phase, &never);
-      done_phase ^= 1u;
-      if (!__syncthreads_and(ok)) { ok = false; break; }
-      tc::fence_after_sync();
-      if (tid == 0 && i + 1 == nk) try_fetch_hin(false);
+      tc::tmem_st_32x32b_x16(tmem + lane_base + COL_S + 16 * half, p0);
+      tc::tmem_st_32x32b_x16(tmem + lane_base + COL_S + 16 * (half + 2), p1);
+      tc::tmem_st_wait();
     }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (tid == 0) {
+      const uint32_t xs = tc::smem_u32(XS);
+#pragma unroll
+      for (int kk = 0; kk < SUB / 16; ++kk)
+        tc::mma_f16_tmem_a(tmem + COL_Y, tmem + COL_S + 8 * kk, tc::sdesc_mnmajor_sw128(xs + kk * 2048, kBlk), ID_Y,
+                           (i > 0) || (kk > 0));
+      tc::mma_commit(done);
+    }
+    ok = tc::mbar_wait(done, done_phase, &never);
+    done_phase ^= 1u;
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    tc::fence_after_sync();
+    if (tid == 0 && i + 1 == nk) try_fetch_hin(false);
     if (tid == 0 && ok && i + 1 < nk) issue_x(i + 1);  // Xs_i is no longer read
   }
 
@@ -539,12 +543,12 @@ cudaError_t launch_scan_tc(const Dims& d, const ScanArgs& s, unsigned* lb, float
   cudaError_t e;
   if (d.P == 64) {
     const size_t sm = ScanSmem<64>::bytes();
-    e = cudaFuncSetAttribute(scan_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    e = set_max_dynamic_smem((const void*)scan_tc_kernel<64>, sm);
     if (e != cudaSuccess) return e;
     scan_tc_kernel<64><<<grid, kThreads, sm, stream>>>(tb, tx, a);
   } else {
     const size_t sm = ScanSmem<128>::bytes();
-    e = cudaFuncSetAttribute(scan_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    e = set_max_dynamic_smem((const void*)scan_tc_kernel<128>, sm);
     if (e != cudaSuccess) return e;
     scan_tc_kernel<128><<<grid, kThreads, sm, stream>>>(tb, tx, a);
   }

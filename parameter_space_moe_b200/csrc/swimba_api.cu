@@ -2,6 +2,7 @@
 // point.  Every entry point validates before launching anything and launches asynchronously on the
 // caller's stream; nothing here allocates device memory.
 #include <atomic>
+#include <map>
 #include <mutex>
 
 #include "common.cuh"
@@ -30,6 +31,20 @@ static unsigned* device_status() {
 // Launch counter and optional per-stage event timing (see swimba_profile_enable).
 static std::atomic<long long> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+cudaError_t set_max_dynamic_smem(const void* kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, size_t> granted;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  size_t& g = granted[{dev, kernel}];
+  if (bytes <= g) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) g = bytes;
+  return e;
+}
 
 struct Profiler {
   static constexpr int kMax = 16;
@@ -172,7 +187,7 @@ static swimba_status run_front(const Dims& d, const void* X, const swimba_weight
   // one memset clears the router's per-tile counts and the scan's hand-off flags (adjacent regions)
   SW_CUDA(cudaMemsetAsync(ws + p.dcounts, 0, p.lb + p.lb_bytes - p.dcounts, s));
   int32_t* counts = (int32_t*)(ws + p.dcounts);
-  SW_CUDA(launch_router(d, X, *w, idx, wts, dt, counts, s));
+  SW_CUDA(launch_router(d, X, *w, idx, wts, dt, counts, st, s));
   prof_mark(s, "router");
   int32_t* offsets = (int32_t*)(ws + p.offsets);
   int32_t* perm = (int32_t*)(ws + p.perm);
@@ -234,7 +249,9 @@ swimba_status swimba_router_topk(const swimba_dims* dims, const void* X, const s
   SW_TRY(make_dims(dims, &d));
   SW_TRY(check_weights(w, true, false));
   if (!ok_ptr(X) || !ok_ptr(topk_idx) || !ok_ptr(topk_w) || !ok_ptr(dt)) return SWIMBA_ERR_INVALID_ARG;
-  return cuda_status(launch_router(d, X, *w, topk_idx, topk_w, dt, nullptr, (cudaStream_t)stream));
+  unsigned* st = device_status();
+  if (!st) return SWIMBA_ERR_CUDA;
+  return cuda_status(launch_router(d, X, *w, topk_idx, topk_w, dt, nullptr, st, (cudaStream_t)stream));
 }
 
 swimba_status swimba_dispatch(const swimba_dims* dims, const int32_t* topk_idx, int32_t* expert_offsets,

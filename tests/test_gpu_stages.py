@@ -44,6 +44,44 @@ def _ws(d):
     return torch.empty(swimba.workspace_size(d), dtype=torch.uint8, device="cuda")
 
 
+# Router shapes at the edges of the tensor-core router: one partial 128-token tile, E = 64 with k = 8,
+# the widest logit row it takes (ceil8(E) + H = 128 columns), one column past it (the CUDA-core router
+# takes over), an odd number of 64-wide K blocks (no K split) and a K split over 4 CTAs on a ragged tail.
+ROUTER_EDGES = [
+    configs.BASE.with_(name="r_one_partial_tile", batch=1, seqlen=50, d_model=256, nheads=8, n_experts=64,
+                       top_k=8, seed=81),
+    configs.BASE.with_(name="r_row128", batch=3, seqlen=300, d_model=512, nheads=64, n_experts=64, top_k=4,
+                       seed=82),
+    configs.BASE.with_(name="r_row129_fallback", batch=3, seqlen=300, d_model=512, nheads=66, n_experts=63,
+                       top_k=2, seed=83),
+    configs.BASE.with_(name="r_odd_kblocks", batch=2, seqlen=777, d_model=320, nheads=12, n_experts=12, top_k=3,
+                       seed=84),
+    configs.BASE.with_(name="r_ksplit4_ragged", batch=5, seqlen=1001, d_model=1024, nheads=16, n_experts=32,
+                       top_k=2, seed=85),
+]
+
+
+@pytest.mark.parametrize("w", ROUTER_EDGES, ids=lambda w: w.name)
+def test_router_edges(w):
+    inp = inputs.make_inputs(w)
+    g, dt_ref, _, _ = O.router(f64(inp["X"]).reshape(w.M, w.d_model), f64(inp["W_r"]), f64(inp["W_dt"]),
+                               f64(inp["b_dt"]), w.top_k)
+    d = swimba.dims_of(w)
+    W = device_weights(inp)
+    X = inp["X"].cuda().reshape(w.M, w.d_model)
+    idx = torch.empty(w.M, w.top_k, dtype=torch.int32, device="cuda")
+    wts = torch.empty(w.M, w.top_k, device="cuda")
+    dt = torch.empty(w.M, w.nheads, device="cuda")
+    swimba.router_topk(d, X, W, idx, wts, dt)
+    torch.cuda.synchronize()
+    assert swimba.check_device_status() == 0
+    fl, forced = check_topk(to_np(idx), g, w.top_k)
+    _, _, _, w_ref = O.router(f64(inp["X"]).reshape(w.M, w.d_model), f64(inp["W_r"]), f64(inp["W_dt"]),
+                              f64(inp["b_dt"]), w.top_k, forced_idx=forced)
+    np.testing.assert_allclose(to_np(wts), w_ref, rtol=2e-5, atol=1e-6)
+    np.testing.assert_allclose(to_np(dt), dt_ref, rtol=2e-5)
+
+
 @pytest.mark.parametrize("w", STAGE_CFGS, ids=lambda w: w.name)
 def test_router(w):
     inp, Xf, ref, dev = _setup(w)
