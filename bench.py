@@ -412,12 +412,32 @@ def run_gpu(args, w):
         dist.destroy_process_group()
 
 
-def stage_roofline(model, secs, peaks):
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, bytes per launch) of a stage's kernel from one
+# ncu capture of the current kernel build, with the summary it comes from; a stage/workload not listed
+# reports null.  An entry is removed whenever its kernel changes.
+PROFILED_TRAFFIC = {
+    ("base_B4_T2048_D768_H24_E8_k2", "expert_proj_mix"): (327.0e6, "profiles/proj_tc_base_B4_T2048_D768_H24_E8_k2.md"),
+    ("base_B4_T2048_D768_H24_E8_k2", "ssd_scan"): (303.3e6, "profiles/scan_tc_base_B4_T2048_D768_H24_E8_k2.md"),
+    ("base_B4_T2048_D768_H24_E8_k2", "router"): (12.7e6, "profiles/router_tc_base_B4_T2048_D768_H24_E8_k2.md"),
+}
+
+
+def tensor_peak(peaks, clocks):
+    """The bf16 GEMM peak that applies: the sustained figure when the timed region ran under the power
+    cap (sw_power_cap seen, or the median SM clock well below its maximum), else the burst figure."""
+    capped = "sw_power_cap" in clocks.get("reasons", []) or (
+        clocks.get("sm_mhz") and clocks.get("sm_max_mhz") and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
+    if capped:
+        return peaks["bf16_tflops_sustained"], "sustained"
+    return peaks["bf16_tflops"], "burst"
+
+
+def stage_roofline(model, secs, peaks, tpeak):
     """Bound (tensor or hbm), achieved, peak and unit of one stage from its work model and duration."""
-    t_tensor = model["flops"] / (peaks["bf16_tflops"] * 1e12)
+    t_tensor = model["flops"] / (tpeak * 1e12)
     t_hbm = model["bytes"] / (peaks["hbm_gbs"] * 1e9)
     if t_tensor >= t_hbm:
-        return "tensor", model["flops"] / secs / 1e12, peaks["bf16_tflops"], "TFLOP/s", model["flops"]
+        return "tensor", model["flops"] / secs / 1e12, tpeak, "TFLOP/s", model["flops"]
     return "hbm", model["bytes"] / secs / 1e9, peaks["hbm_gbs"], "GB/s", model["bytes"]
 
 
@@ -430,15 +450,19 @@ def report(args, w, sess, world, total_ms, e2e_ms, stage_ms, launches, clocks, h
     # dominant kernel stage (among those with a work model) and its roofline
     dom = max((n for n in stage_ms if n in wk), key=stage_ms.get)
     avg_s = stage_ms[dom] / K / 1e3
-    bound, achieved, peak, unit, alg = stage_roofline(wk[dom], avg_s, peaks)
-    peak_note = (f"bf16 dense, burst, {src}" if bound == "tensor" else f"HBM copy, {src}")
-    roof_s = max(wk["layer"]["flops"] / (peaks["bf16_tflops"] * 1e12), wk["layer"]["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    tpeak, tkind = tensor_peak(peaks, clocks)
+    traffic = PROFILED_TRAFFIC.get((w.name, dom))
+    bound, achieved, peak, unit, alg = stage_roofline(wk[dom], avg_s, peaks, tpeak)
+    peak_note = (f"bf16 dense, {tkind}, {src}" if bound == "tensor" else f"HBM copy, {src}")
+    roof_s = max(wk["layer"]["flops"] / (tpeak * 1e12), wk["layer"]["bytes"] / (peaks["hbm_gbs"] * 1e9))
     out = {
         "metric": sess.metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic", "config": config_of(w),
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": None, "peak_source": peak_note, "algorithmic": alg},
+                     "frac": achieved / peak, "traffic": traffic[0] if traffic else None,
+                     "traffic_source": traffic[1] if traffic else None, "peak_source": peak_note,
+                     "algorithmic": alg},
         "layer_roofline": {"time_us": roof_s * 1e6, "frac": roof_s / (total_ms / K / 1e3),
                            "flops": wk["layer"]["flops"], "bytes": wk["layer"]["bytes"]},
         "stages_ms_per_step": {n: v / K for n, v in stage_ms.items()},

@@ -296,6 +296,193 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// CTA-pair variant: a cluster of 2 CTAs computes one 256-row x 256-column tile with tcgen05.mma
+// cta_group::2 (M256 N256 K16).  Each CTA loads 128 gathered X rows and 128 of the 256 weight rows per
+// 64-wide K slice (32 KB per stage instead of 48 KB for half the FLOPs of a 128 x 256 tile per CTA), so a
+// stage's copies keep pace with the tensor pipe.  The even CTA's producer arms its full barrier for both
+// CTAs' bytes; the odd CTA's copies complete on that barrier.  The even CTA's warp 1 issues the MMAs and
+// its commits arrive on both CTAs' barriers (stage free, accumulator ready); both CTAs drain their own
+// 128 accumulator rows with the same epilogue as above and tell the even CTA's MMA warp when a buffer is
+// free.  Tiles: 256 consecutive sorted rows of one expert (rows past the expert's end are computed and
+// dropped) x 256 output columns; the pair-tile schedule is derived from the expert offsets in the kernel.
+constexpr int kPairStages = 6;
+constexpr uint32_t kPairStageA = 128 * BK * 2, kPairStageB = 128 * BK * 2;
+constexpr uint32_t kPairStageBytes = kPairStageA + kPairStageB;
+constexpr uint32_t kPairIdesc = tc::idesc_f16(256, BN, /*bf16=*/true);
+constexpr size_t kPairSmemBytes = 1024 + (size_t)kPairStages * kPairStageBytes + 1024 + (size_t)kEpiWarps * kEpiStage;
+constexpr int kPairRows = 256;
+
+// Pair tile rt -> (expert, first sorted row), from pt_s[e] = number of 256-row tiles of experts < e.
+__device__ __forceinline__ int2 pair_tile(const int* off_s, const int* pt_s, int E, int rt) {
+  int e = 0;
+  while (e + 1 < E && pt_s[e + 1] <= rt) ++e;
+  return make_int2(e, off_s[e] + (rt - pt_s[e]) * kPairRows);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPairStages * kPairStageBytes);
+  uint64_t* full = bars;                               // [kPairStages] copies of both CTAs -> MMA (even CTA)
+  uint64_t* empty = bars + kPairStages;                // [kPairStages] MMA -> this CTA's producer
+  uint64_t* acc_full = bars + 2 * kPairStages;         // [2] MMA -> this CTA's epilogue
+  uint64_t* acc_empty = bars + 2 * kPairStages + 2;    // [2] both epilogues -> MMA (even CTA)
+  uint64_t* drain = bars + 2 * kPairStages + 4;        // all MMAs complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kPairStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* off_s = reinterpret_cast<int*>(tmem_slot + 2);  // [E + 1] expert offsets
+  int* pt_s = off_s + 65;                               // [E + 1] pair-tile prefix
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = tc::cluster_ctarank();
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  const Dims& d = a.d;
+  const int nct = ceil_div(d.We, BN);
+  const int nkb = d.D / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&acc_full[b], 1); tc::mbar_init(&acc_empty[b], 2 * kEpiWarps); }
+    tc::mbar_init(drain, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+    tc::tma_prefetch_desc(&tmap_a);
+    tc::tma_prefetch_desc(&tmap_b);
+  }
+  if (warp == 1) { tc::tmem_alloc_pair(tmem_slot, kTmemCols); tc::tmem_relinquish_pair(); }
+  for (int e = threadIdx.x; e <= d.E; e += blockDim.x) off_s[e] = a.offsets[e];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int e = 0; e < d.E; ++e) { pt_s[e] = acc; acc += ceil_div(off_s[e + 1] - off_s[e], kPairRows); }
+    pt_s[d.E] = acc;
+  }
+  tc::fence_before_sync();
+  tc::cluster_sync();  // both CTAs' barriers are initialised before any copy or commit can reach them
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int total = pt_s[d.E] * nct;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    long long issued = 0;
+    bool ok = true;
+    const uint32_t full0 = tc::map_shared(tc::smem_u32(full), 0u);  // the even CTA's full barriers
+    for (int t = cid; t < total && ok; t += ncl) {
+      const int rt = t / nct, ct = t % nct;
+      const int2 tl = pair_tile(off_s, pt_s, d.E, rt);
+      const int arow = tl.y + 128 * (int)rank;
+      const int wrow = tl.x * d.We + ct * BN + 128 * (int)rank;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+        uint8_t* sa = stage_base + stage * kPairStageBytes;
+        if (rank == 0) tc::mbar_arrive_expect_tx(&full[stage], 2 * kPairStageBytes);
+        const uint32_t fb = full0 + 8u * (uint32_t)stage;
+        tc::tma_load_2d_pair(sa, &tmap_a, fb, kb * BK, arow);
+        tc::tma_load_2d_pair(sa + kPairStageA, &tmap_b, fb, kb * BK, wrow);
+        ++issued;
+        if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok) { *abort_flag = 1; atomicOr(a.st, ST_TIMEOUT); }
+    // every copy this CTA issued has been consumed by an MMA (its stage was released) or is waited for here
+    for (long long i = 0; i < kPairStages && i < issued; ++i) {
+      if (--stage < 0) { stage = kPairStages - 1; phase ^= 1u; }
+      volatile int never = 0;
+      tc::mbar_wait(&empty[stage], phase, &never);
+    }
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ---------------------------------------------------------------- MMA issuer (even CTA)
+    int stage = 0;
+    uint32_t phase = 0;
+    int buf = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int t = cid; t < total && ok; t += ncl) {
+      if (!tc::mbar_wait(&acc_empty[buf], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+      tc::fence_after_sync();
+      const uint32_t dt = tmem + (uint32_t)(buf * BN);
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!tc::mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t sa = tc::smem_u32(stage_base + stage * kPairStageBytes);
+        const uint32_t sb = sa + kPairStageA;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          tc::mma_f16_pair(dt, tc::sdesc_kmajor_sw128(sa + kk * 32), tc::sdesc_kmajor_sw128(sb + kk * 32), kPairIdesc,
+                           (kb | kk) != 0);
+        }
+        tc::mma_commit_pair(&empty[stage], 0x3);
+        if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      tc::mma_commit_pair(&acc_full[buf], 0x3);
+      if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
+    }
+    if (!ok) { *abort_flag = 1; atomicOr(a.st, ST_TIMEOUT); }
+    tc::mma_commit_pair(drain, 0x3);
+    volatile int never = 0;
+    tc::mbar_wait(drain, 0, &never);
+  } else if (warp == 1 && lane == 0) {
+    // odd CTA: its TMEM and shared memory are in use until the even CTA's last MMA has completed
+    volatile int never = 0;
+    tc::mbar_wait(drain, 0, &never);
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int ch = (warp - 2) >> 2;
+    const int row_local = 128 * (int)rank + 32 * q + lane;  // row inside the 256-row pair tile
+    uint8_t* epi_stage = smem + kPairStages * kPairStageBytes + 1024 + (warp - 2) * kEpiStage;
+    const uint32_t acc_empty0 = tc::map_shared(tc::smem_u32(acc_empty), 0u);
+    int buf = 0;
+    uint32_t acc_phase = 0;
+    bool range_bad = false;
+    for (int t = cid; t < total; t += ncl) {
+      const int rt = t / nct, ct = t % nct;
+      const int2 tl = pair_tile(off_s, pt_s, d.E, rt);
+      const bool valid = tl.y + row_local < off_s[tl.x + 1];
+      const int2 meta = valid ? a.rowmeta[tl.y + row_local] : make_int2(0, 0);
+      if (!tc::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) {
+        *abort_flag = 1;
+        atomicOr(a.st, ST_TIMEOUT);
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + ch * (BN / 2));
+#pragma unroll 1
+      for (int c = 0; c < BN / 64; ++c) {
+        uint32_t r[32];
+        tc::tmem_ld_32x32b_x32(taddr + 32 * c, r);
+        tc::tmem_ld_wait();
+        const int c0 = ct * BN + ch * (BN / 2) + 32 * c;
+        const float pi = __int_as_float(meta.y);
+        float sc_probe;
+        const bool fast = a.mode != 2 && c0 + 32 <= d.We &&
+                          __all_sync(0xffffffffu, !valid || group_dst(a, meta.x, pi, c0, sc_probe) != nullptr);
+        if (fast) store_group32(a, epi_stage, lane, valid, meta.x, pi, c0, r, range_bad);
+        else if (valid && c0 < d.We) store_chunk(a, meta.x, pi, c0, r, range_bad);
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive_cluster(acc_empty0 + 8u * (uint32_t)buf);
+      if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
+    }
+    if (range_bad) atomicOr(a.st, ST_RANGE);
+  }
+  tc::fence_before_sync();
+  tc::cluster_sync();  // no CTA leaves while the other may still signal its barriers or read its operands
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
 }  // namespace
 
 // Host side --------------------------------------------------------------------------------------
@@ -308,11 +495,49 @@ cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp
   if (!encode_tmap_2d(&tb, w_exp, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.E * d.We, (uint64_t)d.D * 2, BK, BN))
     return cudaErrorInvalidValue;
   TcArgs a{d, rowmeta, tiles, ntiles, offsets, mode, (__half*)bpi, (__half*)xs, (__half*)cpi, Z, st};
-  cudaError_t e = set_max_dynamic_smem((const void*)proj_tc_kernel, kSmemBytes);
-  if (e != cudaSuccess) return e;
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t e;
+  // CTA pairs when experts average at least 3072 rows: each expert's last pair tile is partly past its
+  // rows, and below that the 256-row tiles waste more tensor time than the pairs save
+  if ((long long)d.M * d.k >= 3072LL * d.E) {
+    // CTA pairs: A boxes of 128 rows (the pair's two halves), B boxes of 128 weight rows
+    CUtensorMap tb2;
+    if (!encode_tmap_2d(&tb2, w_exp, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.E * d.We, (uint64_t)d.D * 2, BK, 128))
+      return cudaErrorInvalidValue;
+    e = set_max_dynamic_smem((const void*)proj_tc_pair_kernel, kPairSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: as many pairs as can be resident at once (at most one per tile)
+    static int resident = 0;
+    if (resident == 0) {
+      cfg.gridDim = dim3((unsigned)sms);
+      int n = 0;
+      resident = cudaOccupancyMaxActiveClusters(&n, proj_tc_pair_kernel, &cfg) == cudaSuccess && n > 0 ? n : sms / 2;
+    }
+    const int max_pairs = (ceil_div(d.M * d.k, kPairRows) + d.E) * ceil_div(d.We, BN);
+    const int pairs = resident < max_pairs ? resident : max_pairs;
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    e = cudaLaunchKernelEx(&cfg, proj_tc_pair_kernel, ta, tb2, a);
+    if (e == cudaSuccess) {
+      count_launches(1);
+      return cudaGetLastError();
+    }
+    (void)cudaGetLastError();  // pairs could not be launched: the one-CTA kernel below does the work
+  }
+  e = set_max_dynamic_smem((const void*)proj_tc_kernel, kSmemBytes);
+  if (e != cudaSuccess) return e;
   const int max_tiles = max_row_tiles(d) * ceil_div(d.We, BN);
   const int grid = max_tiles < sms ? max_tiles : sms;
   proj_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, a);

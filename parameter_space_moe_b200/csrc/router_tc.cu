@@ -59,28 +59,10 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
         "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// Address of the same shared-memory location in cluster CTA `rank`.
-__device__ __forceinline__ uint32_t map_shared(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
 __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t e) {
   asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(e)
                : "memory");
 }
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 __global__ void __launch_bounds__(128)
 router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wr,
@@ -99,7 +81,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const uint32_t rank = C > 1 ? cluster_ctarank() : 0u;
+  const uint32_t rank = C > 1 ? tc::cluster_ctarank() : 0u;
   const int tile = blockIdx.x / C;
   const int tok0 = tile * RBM;
   const int R = RBM / C;                    // token rows this CTA finishes
@@ -123,7 +105,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   const uint32_t tmem = *tslot;
   // every CTA of the cluster has started (its shared memory exists) once this barrier phase completes;
   // waited for just before the first store into another CTA's shared memory
-  if (C > 1) cluster_arrive_relaxed();
+  if (C > 1) tc::cluster_arrive_relaxed();
 
   bool ok = true;
   if (tid == 0) {  // producer + MMA issuer; the rest of warp 0 waits at the __syncwarp below, not on `done`
@@ -171,11 +153,11 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   ok = tc::mbar_wait(done, 0, &never) && ok;
   ok = __syncthreads_and(ok);
   tc::fence_after_sync();
-  if (C > 1) cluster_wait();
+  if (C > 1) tc::cluster_wait();
   {
     // this thread's token row (TMEM lane tid) of partial logits -> row (tid % R) of source slot `rank` in
     // the finishing CTA (tid / R)
-    const uint32_t dst = map_shared(tc::smem_u32(G) + ((rank * R + (tid % R)) * L.gs) * 4u, (uint32_t)(tid / R));
+    const uint32_t dst = tc::map_shared(tc::smem_u32(G) + ((rank * R + (tid % R)) * L.gs) * 4u, (uint32_t)(tid / R));
     if (ok) {
       for (int c = 0; c < RP; c += 16) {
         uint32_t r[16];
@@ -187,7 +169,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     }
   }
   tc::fence_before_sync();
-  if (C > 1) cluster_sync(); else __syncthreads();
+  if (C > 1) tc::cluster_sync(); else __syncthreads();
   if (warp == 0) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, tcols);
