@@ -79,7 +79,7 @@ struct ScanSmem {
   static constexpr uint32_t BP = CT + NB * kBlk;  // Bpi_j (NB blocks); H_in hi/lo parts after the slot loop
   static constexpr uint32_t XS = BP + NB * kBlk;  // Xs_j (PB blocks)
   static constexpr uint32_t PM = XS + PB * kBlk;  // the decay-scaled Xs_j
-  static constexpr uint32_t BAR = PM + PB * kBlk; // fullB, fullX, done
+  static constexpr uint32_t BAR = PM + PB * kBlk; // fullB, fullX, done, hbar, fullC
   static constexpr uint32_t CS = BAR + 64;        // cs[SUB], fs[SUB], wsum[4], misc[2]
   static constexpr uint32_t END = CS + 2 * SUB * 4 + 64;
   static constexpr size_t bytes() { return 1024 + END; }
@@ -89,7 +89,8 @@ struct ScanSmem {
 // TMEM lane quarter (w % 4) and split the columns of each row between them.
 template <int P>
 __global__ void __launch_bounds__(kThreads, P == 64 ? 2 : 1)
-scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_x, TcScanArgs a) {
+scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_x,
+               const __grid_constant__ CUtensorMap tm_c, TcScanArgs a) {
   using Lay = ScanSmem<P>;
   constexpr int N = 128, NB = Lay::NB, PB = Lay::PB, PH = P / 2;
   constexpr uint32_t TMEM_COLS = P == 64 ? 256 : 512;
@@ -109,6 +110,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   uint64_t* fullX = fullB + 1;
   uint64_t* done = fullB + 2;
   uint64_t* hbar = fullB + 3;  // bulk copy of H_in into the Bpi region
+  uint64_t* fullC = fullB + 4;  // first read slot of C~ into CT
   float* cs_s = reinterpret_cast<float*>(sm + Lay::CS);
   float* fs_s = cs_s + SUB;
   float* wsum = fs_s + SUB;
@@ -122,6 +124,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     tc::mbar_init(fullX, 1);
     tc::mbar_init(done, 1);
     tc::mbar_init(hbar, 1);
+    tc::mbar_init(fullC, 1);
     tc::fence_barrier_init();
     misc[1] = atomicAdd(a.ticket, 1u);
   }
@@ -150,7 +153,12 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     for (int pb = 0; pb < PB; ++pb) tma_load_3d(XS + pb * kBlk, &tm_x, fullX, h * P + 64 * pb, a.key_slot0 + i, row0);
     ++issuedX;
   };
-  if (tid == 0) { issue_b(0); issue_x(0); }
+  if (tid == 0) {
+    issue_b(0);
+    issue_x(0);
+    tc::mbar_arrive_expect_tx(fullC, NB * kBlk);
+    for (int nb = 0; nb < NB; ++nb) tma_load_3d(CT + nb * kBlk, &tm_c, fullC, g * N + 64 * nb, a.read_slot0, row0);
+  }
   // H_in of this sub-chunk is the previous sub-chunk's H_out.  With P = 64 it fits the Bpi region once the
   // last slot's key products are done, so thread 0 fetches it with one bulk copy as soon as the
   // predecessor's flag is up, while the other threads still work on the last slot.
@@ -176,65 +184,77 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   // this row's dt is loaded first so its latency overlaps the readout loads below
   const float dt_row = (half == 0 && row < L) ? a.dt[(size_t)(row0 + row) * d.H + h] : 0.f;
 
-  // C~ rows: sum of the readout slots, loaded coalesced (16 lanes per 256-byte row), fp16 K-major swizzled.
-  // Warp w covers rows 16w .. 16w + 15.  Two slots are added as fp16 pairs (the correctly rounded sum).
-  {
-    const int hl = lane >> 4, c16 = lane & 15;
-    uint4 q[8];
-    auto load8 = [&](int j, uint4 (&dst)[8]) {
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int r = 16 * warp + 2 * u + hl;
-        dst[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (r < L)
-          dst[u] = __ldg(reinterpret_cast<const uint4*>(a.cpi + ((size_t)(row0 + r) * d.k + j) * d.GN + (size_t)g * N +
-                                                        c16 * 8));
-      }
-    };
-    if (a.read_slots == 1 || a.read_slots == 2) {
-      load8(a.read_slot0, q);
-      if (a.read_slots == 2) {
-        uint4 q2[8];
-        load8(a.read_slot0 + 1, q2);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          __half2* x = reinterpret_cast<__half2*>(&q[u]);
-          const __half2* y = reinterpret_cast<const __half2*>(&q2[u]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) x[e] = __hadd2(x[e], y[e]);
-        }
-      }
-    } else {
-      float acc[8][8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
-      for (int j = a.read_slot0; j < a.read_slot0 + a.read_slots; ++j) {
-        load8(j, q);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const __half2* hq = reinterpret_cast<const __half2*>(&q[u]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(hq[e]);
-            acc[u][2 * e] += f.x;
-            acc[u][2 * e + 1] += f.y;
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        q[u].x = pack_half2(acc[u][0], acc[u][1]); q[u].y = pack_half2(acc[u][2], acc[u][3]);
-        q[u].z = pack_half2(acc[u][4], acc[u][5]); q[u].w = pack_half2(acc[u][6], acc[u][7]);
-      }
-    }
+  // C~ rows = sum of the readout slots.  The first slot comes by TMA into CT (issued above with slot 0's
+  // keys and values); the others are loaded coalesced (16 lanes per 256-byte row, warp w covers rows
+  // 16w .. 16w + 15) and added to CT in shared memory: two slots as one fp16 pair add (the correctly
+  // rounded sum), after slot 0's decay-scaled values so that the loads' latency overlaps that work; more
+  // slots in fp32, rounded once.
+  const int hl = lane >> 4, c16 = lane & 15;
+  auto ct_chunk = [&](int u) { const int r = 16 * warp + 2 * u + hl; return CT + (c16 >> 3) * kBlk + tc::sw128_chunk(r, c16 & 7); };
+  auto load8 = [&](int j, uint4 (&dst)[8]) {
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int r = 16 * warp + 2 * u + hl;
-      *reinterpret_cast<uint4*>(CT + (c16 >> 3) * kBlk + tc::sw128_chunk(r, c16 & 7)) = q[u];
+      dst[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (r < L)
+        dst[u] = __ldg(reinterpret_cast<const uint4*>(a.cpi + ((size_t)(row0 + r) * d.k + j) * d.GN + (size_t)g * N +
+                                                      c16 * 8));
+    }
+  };
+  uint4 cq[8];  // the second read slot (two read slots)
+  bool c_ok = true;
+  if (a.read_slots == 2) {
+    load8(a.read_slot0 + 1, cq);
+  } else if (a.read_slots >= 3) {
+    float acc[8][8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[u][e] = 0.f;
+    for (int j = a.read_slot0 + 1; j < a.read_slot0 + a.read_slots; ++j) {
+      load8(j, cq);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const __half2* hq = reinterpret_cast<const __half2*>(&cq[u]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(hq[e]);
+          acc[u][2 * e] += f.x;
+          acc[u][2 * e + 1] += f.y;
+        }
+      }
+    }
+    c_ok = tc::mbar_wait(fullC, 0, &never);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      uint4* dst = reinterpret_cast<uint4*>(ct_chunk(u));
+      uint4 v = *dst;
+      __half2* hv2 = reinterpret_cast<__half2*>(&v);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(hv2[e]);
+        hv2[e] = __floats2half2_rn(f.x + acc[u][2 * e], f.y + acc[u][2 * e + 1]);
+      }
+      *dst = v;
     }
   }
+  // C~ complete in CT (called by every thread before the first product that reads CT)
+  auto finish_ct = [&]() {
+    if (a.read_slots >= 3) return;
+    c_ok = tc::mbar_wait(fullC, 0, &never) && c_ok;
+    if (a.read_slots == 2) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        uint4* dst = reinterpret_cast<uint4*>(ct_chunk(u));
+        uint4 v = *dst;
+        __half2* x = reinterpret_cast<__half2*>(&v);
+        const __half2* y = reinterpret_cast<const __half2*>(&cq[u]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = __hadd2(x[e], y[e]);
+        *dst = v;
+      }
+    }
+  };
 
   // cumulative log-decay of the sub-chunk (inclusive scan over the 128 rows)
   float v = 0.f;
@@ -286,17 +306,31 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    const uint32_t ct = tc::smem_u32(CT), bp = tc::smem_u32(BP), dx = tc::smem_u32(PM);
     if (tid == 0) {
-      const uint32_t ct = tc::smem_u32(CT), bp = tc::smem_u32(BP), dx = tc::smem_u32(PM);
-#pragma unroll
-      for (int kk = 0; kk < N / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
-        tc::mma_f16(tmem + COL_S, tc::sdesc_kmajor_sw128(ct + off), tc::sdesc_kmajor_sw128(bp + off), ID_S, kk > 0);
-      }
 #pragma unroll
       for (int kk = 0; kk < SUB / 16; ++kk) {
         tc::mma_f16(tmem + COL_SC, tc::sdesc_mnmajor_sw128(bp + kk * 2048, kBlk),
                     tc::sdesc_mnmajor_sw128(dx + kk * 2048, kBlk), ID_SC, (i > 0) || (kk > 0));
+      }
+    }
+    if (i == 0) {  // the end-state product runs while C~ is completed
+      finish_ct();
+      tc::fence_proxy_async();
+      if (!__syncthreads_and(c_ok)) {
+        ok = false;
+        if (tid == 0) {  // the end-state product is in flight: let it finish before TMEM is freed
+          tc::mma_commit(done);
+          tc::mbar_wait(done, done_phase, &never);
+        }
+        break;
+      }
+    }
+    if (tid == 0) {
+#pragma unroll
+      for (int kk = 0; kk < N / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kBlk + (kk & 3) * 32;
+        tc::mma_f16(tmem + COL_S, tc::sdesc_kmajor_sw128(ct + off), tc::sdesc_kmajor_sw128(bp + off), ID_S, kk > 0);
       }
       tc::mma_commit(done);
     }
@@ -379,12 +413,16 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     const float dend = expf(cs_end);
     const size_t rbase = (size_t)row * P + half * PH;
     // this thread's half row of H_in (kept for the fp16 split below) and H_out = exp(cs_end) H_in + Sc
+    // exchanged states are stored thread-major (float4 U of thread tid at (U * kThreads + tid) * 4) so the
+    // stores coalesce and the reads from shared memory are conflict-free; the initial state is [N][P]
+    auto xidx = [&](int U) { return ((size_t)U * kThreads + tid) * 4; };
+    const bool hin_canon = csub == 0;
     float4 hv[PH / 4];
 #pragma unroll
     for (int u = 0; u < PH / 4; ++u)
       hv[u] = !hin ? make_float4(0.f, 0.f, 0.f, 0.f)
-                   : (hin_shared ? *reinterpret_cast<const float4*>(hin + rbase + 4 * u)
-                                 : __ldcg(reinterpret_cast<const float4*>(hin + rbase + 4 * u)));
+                   : (hin_shared ? *reinterpret_cast<const float4*>(hin + xidx(u))
+                                 : __ldcg(reinterpret_cast<const float4*>(hin + (hin_canon ? rbase + 4 * u : xidx(u)))));
 #pragma unroll
     for (int q = 0; q < PH / 32; ++q) {
       uint32_t r[32];
@@ -395,7 +433,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
         const float4 x = hv[8 * q + u];
         const float4 o = make_float4(fmaf(dend, x.x, u2f(r[4 * u])), fmaf(dend, x.y, u2f(r[4 * u + 1])),
                                      fmaf(dend, x.z, u2f(r[4 * u + 2])), fmaf(dend, x.w, u2f(r[4 * u + 3])));
-        __stcg(reinterpret_cast<float4*>(hout + rbase + 32 * q + 4 * u), o);
+        __stcg(reinterpret_cast<float4*>(hout + xidx(8 * q + u)), o);
       }
     }
     // every thread's H_out stores are ordered before the barrier; thread 0's release store at device scope
@@ -413,7 +451,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
 #pragma unroll
     for (int u = 0; u < PH / 4; ++u) {
       if (cst) *reinterpret_cast<float4*>(cst + rbase + 4 * u) = hv[u];
-      if (fin) *reinterpret_cast<float4*>(fin + rbase + 4 * u) = __ldcg(reinterpret_cast<const float4*>(hout + rbase + 4 * u));
+      if (fin) *reinterpret_cast<float4*>(fin + rbase + 4 * u) = __ldcg(reinterpret_cast<const float4*>(hout + xidx(u)));
     }
 #pragma unroll
     for (int c = 0; c < PH / 8; ++c) {
@@ -508,6 +546,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     if (issuedB > 0) tc::mbar_wait(fullB, (uint32_t)((issuedB - 1) & 1), &never);
     if (issuedX > 0) tc::mbar_wait(fullX, (uint32_t)((issuedX - 1) & 1), &never);
     if (h_issued) tc::mbar_wait(hbar, 0, &never);
+    tc::mbar_wait(fullC, 0, &never);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -525,13 +564,17 @@ bool scan_tc_supported(const Dims& d) {
 
 int scan_tc_subchunks(const Dims& d) { return ceil_div(d.T, SUB); }
 
-// lb: zeroed by the caller (ticket counter at lb[0], flags at lb + 64); exch: [B*H][nsub][N][P] fp32.
+// lb: zeroed by the caller (ticket counter at lb[0], flags at lb + 64); exch: [B*H][nsub] states of N*P
+// fp32, each stored thread-major (see the hand-off).
 cudaError_t launch_scan_tc(const Dims& d, const ScanArgs& s, unsigned* lb, float* exch, unsigned* st,
                            cudaStream_t stream) {
   CUtensorMap tb, tx;
   if (!encode_tmap_3d_slot(&tb, s.bpi, SWIMBA_F16, (uint64_t)d.GN, (uint64_t)d.k, (uint64_t)d.M, 64, SUB))
     return cudaErrorInvalidValue;
   if (!encode_tmap_3d_slot(&tx, s.xs, SWIMBA_F16, (uint64_t)d.HP, (uint64_t)d.k, (uint64_t)d.M, 64, SUB))
+    return cudaErrorInvalidValue;
+  CUtensorMap tc3;
+  if (!encode_tmap_3d_slot(&tc3, s.cpi, SWIMBA_F16, (uint64_t)d.GN, (uint64_t)d.k, (uint64_t)d.M, 64, SUB))
     return cudaErrorInvalidValue;
   TcScanArgs a{};
   a.d = d; a.dt = s.dt; a.A = s.A; a.init = s.init; a.cpi = (const __half*)s.cpi; a.y = (__nv_bfloat16*)s.y;
@@ -545,12 +588,12 @@ cudaError_t launch_scan_tc(const Dims& d, const ScanArgs& s, unsigned* lb, float
     const size_t sm = ScanSmem<64>::bytes();
     e = set_max_dynamic_smem((const void*)scan_tc_kernel<64>, sm);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<64><<<grid, kThreads, sm, stream>>>(tb, tx, a);
+    scan_tc_kernel<64><<<grid, kThreads, sm, stream>>>(tb, tx, tc3, a);
   } else {
     const size_t sm = ScanSmem<128>::bytes();
     e = set_max_dynamic_smem((const void*)scan_tc_kernel<128>, sm);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<128><<<grid, kThreads, sm, stream>>>(tb, tx, a);
+    scan_tc_kernel<128><<<grid, kThreads, sm, stream>>>(tb, tx, tc3, a);
   }
   count_launches(1);
   return cudaGetLastError();
