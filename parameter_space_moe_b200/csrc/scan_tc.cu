@@ -66,6 +66,12 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -77,8 +83,8 @@ struct ScanSmem {
   static constexpr int N = 128, NB = N / 64, PB = P / 64;
   static constexpr uint32_t CT = 0;               // C~ rows, K-major, NB blocks
   static constexpr uint32_t BP = CT + NB * kBlk;  // Bpi_j (NB blocks); H_in hi/lo parts after the slot loop
-  static constexpr uint32_t XS = BP + NB * kBlk;  // Xs_j (PB blocks)
-  static constexpr uint32_t PM = XS + PB * kBlk;  // the decay-scaled Xs_j
+  static constexpr uint32_t XS = BP + NB * kBlk;  // Xs_j of even slots / decay-scaled Xs_j of odd slots
+  static constexpr uint32_t PM = XS + PB * kBlk;  // the other way round
   static constexpr uint32_t BAR = PM + PB * kBlk; // fullB, fullX, done, hbar, fullC
   static constexpr uint32_t CS = BAR + 64;        // cs[SUB], fs[SUB], wsum[4], misc[2]
   static constexpr uint32_t END = CS + 2 * SUB * 4 + 64;
@@ -150,7 +156,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   };
   auto issue_x = [&](int i) {
     tc::mbar_arrive_expect_tx(fullX, PB * kBlk);
-    for (int pb = 0; pb < PB; ++pb) tma_load_3d(XS + pb * kBlk, &tm_x, fullX, h * P + 64 * pb, a.key_slot0 + i, row0);
+    uint8_t* dst = (i & 1) ? PM : XS;
+    for (int pb = 0; pb < PB; ++pb) tma_load_3d(dst + pb * kBlk, &tm_x, fullX, h * P + 64 * pb, a.key_slot0 + i, row0);
     ++issuedX;
   };
   if (tid == 0) {
@@ -167,18 +174,32 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   const float* hprev = csub > 0 ? a.exch + ((size_t)bh * a.nsub + csub - 1) * NPs : nullptr;
   const unsigned* pflag = csub > 0 ? a.flags + (size_t)bh * a.nsub + csub - 1 : nullptr;
   bool h_issued = false;
-  auto try_fetch_hin = [&](bool block) {  // thread 0 only
-    if (!kEarlyFetch || h_issued || csub == 0) return;
-    uint32_t n = 0;
-    while (ld_acquire(pflag) == 0u) {
-      if (!block) return;
-      if (++n >= kFlagPolls) { atomicOr(a.st, ST_TIMEOUT); break; }
-      if (n > 64) __nanosleep(32);
-    }
+  unsigned fpeek = 0u;  // thread 0: a relaxed read of the predecessor's flag, looked at one phase later
+  auto fetch_hin = [&]() {
     tc::fence_proxy_async_global();
     tc::mbar_arrive_expect_tx(hbar, (uint32_t)(NPs * 4));
     tc::bulk_load(BP, hprev, (uint32_t)(NPs * 4), hbar);
     h_issued = true;
+  };
+  // during the last slot (thread 0 only): read the flag without waiting for the value, and one phase later
+  // fetch H_in if it was up (the relaxed read that saw the release store plus fence.acq_rel is the acquire)
+  auto peek_hin = [&]() {
+    if (!kEarlyFetch || h_issued || csub == 0) return;
+    if (fpeek) {
+      fence_acq_rel_gpu();
+      fetch_hin();
+    } else {
+      fpeek = ld_relaxed(pflag);
+    }
+  };
+  auto wait_fetch_hin = [&]() {  // thread 0 only, at the hand-off
+    if (!kEarlyFetch || h_issued || csub == 0) return;
+    uint32_t n = 0;
+    while (ld_acquire(pflag) == 0u) {
+      if (++n >= kFlagPolls) { atomicOr(a.st, ST_TIMEOUT); break; }
+      if (n > 64) __nanosleep(32);
+    }
+    fetch_hin();
   };
 
   // this row's dt is loaded first so its latency overlaps the readout loads below
@@ -282,50 +303,66 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
 
   bool ok = true;
   uint32_t done_phase = 0;
-  for (int i = 0; i < nk && ok; ++i) {
+  const uint32_t ct = tc::smem_u32(CT), bp = tc::smem_u32(BP);
+  // slot i's values sit in one of the two value buffers and its decay-scaled copy goes to the other, so
+  // slot i + 1's values can be loaded into this copy's buffer once the end-state product has read it
+  auto value_buf = [&](int i) { return (i & 1) ? PM : XS; };
+  auto scaled_buf = [&](int i) { return (i & 1) ? XS : PM; };
+  // wait for slot i's keys and values, scale the values by the decay to the sub-chunk end and issue the
+  // end-state product Sc += Bpi_i^T (decay_end * Xs_i)
+  auto begin_slot = [&](int i) -> bool {
     const uint32_t par = (uint32_t)(i & 1);
-    ok = tc::mbar_wait(fullX, par, &never) && tc::mbar_wait(fullB, par, &never);
-    if (!__syncthreads_and(ok)) { ok = false; break; }
-    // values scaled by the decay to the sub-chunk end (for the end state), into the Pm buffer
+    bool w = tc::mbar_wait(fullX, par, &never) && tc::mbar_wait(fullB, par, &never);
+    if (!__syncthreads_and(w)) return false;
+    uint8_t* XV = value_buf(i);
+    uint8_t* DXV = scaled_buf(i);
+    if (tid == 0 && i + 1 == nk) peek_hin();
 #pragma unroll
     for (int pb = 0; pb < PB; ++pb) {
 #pragma unroll
       for (int c = 4 * half; c < 4 * half + 4; ++c) {
         const uint32_t off = pb * kBlk + tc::sw128_chunk(row, c);
-        uint4 q = *reinterpret_cast<const uint4*>(XS + off);
+        uint4 q = *reinterpret_cast<const uint4*>(XV + off);
         __half2* hq = reinterpret_cast<__half2*>(&q);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __half22float2(hq[e]);
           hq[e] = __floats2half2_rn(f.x * dec_end, f.y * dec_end);
         }
-        *reinterpret_cast<uint4*>(PM + off) = q;
+        *reinterpret_cast<uint4*>(DXV + off) = q;
       }
     }
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t ct = tc::smem_u32(CT), bp = tc::smem_u32(BP), dx = tc::smem_u32(PM);
     if (tid == 0) {
+      const uint32_t dx = tc::smem_u32(DXV);
 #pragma unroll
       for (int kk = 0; kk < SUB / 16; ++kk) {
         tc::mma_f16(tmem + COL_SC, tc::sdesc_mnmajor_sw128(bp + kk * 2048, kBlk),
                     tc::sdesc_mnmajor_sw128(dx + kk * 2048, kBlk), ID_SC, (i > 0) || (kk > 0));
       }
     }
-    if (i == 0) {  // the end-state product runs while C~ is completed
-      finish_ct();
-      tc::fence_proxy_async();
-      if (!__syncthreads_and(c_ok)) {
-        ok = false;
-        if (tid == 0) {  // the end-state product is in flight: let it finish before TMEM is freed
-          tc::mma_commit(done);
-          tc::mbar_wait(done, done_phase, &never);
-        }
-        break;
+    return true;
+  };
+  // slot 0's end-state product runs while C~ is completed (outside the loop, so the registers holding the
+  // second read slot are free in it)
+  ok = begin_slot(0);
+  if (ok) {
+    finish_ct();
+    tc::fence_proxy_async();
+    if (!__syncthreads_and(c_ok)) {
+      ok = false;
+      if (tid == 0) {  // the end-state product is in flight: let it finish before TMEM is freed
+        tc::mma_commit(done);
+        tc::mbar_wait(done, done_phase, &never);
       }
     }
+  }
+  for (int i = 0; i < nk && ok; ++i) {
+    if (i > 0 && !begin_slot(i)) { ok = false; break; }
+    uint8_t* XV = value_buf(i);
     if (tid == 0) {
 #pragma unroll
       for (int kk = 0; kk < N / 16; ++kk) {
@@ -338,53 +375,55 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     done_phase ^= 1u;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     tc::fence_after_sync();
-    if (tid == 0 && i + 1 < nk) issue_b(i + 1);  // Bpi_i is no longer read
-    if (tid == 0 && i + 1 == nk) try_fetch_hin(false);  // the Bpi region is free for good
-    // masked, decayed scores of this thread's two 32-key blocks kb = half and half + 2 (their decays share
-    // one factor exp(cs_t - cs_{32b}) per block), packed to fp16 pairs and stored back into TMEM over the
-    // first 64 columns of S, where the next product takes them as its A operand
+    if (tid == 0 && i + 1 < nk) {  // Bpi_i and the decay-scaled Xs_i are no longer read
+      issue_b(i + 1);
+      issue_x(i + 1);
+    }
+    if (tid == 0 && i + 1 == nk) peek_hin();  // the Bpi region is free for good
+    // masked, decayed scores of this thread's 64 keys (32-key blocks kb = 2 half and 2 half + 1, whose decays
+    // share one factor exp(cs_t - cs_{32b}) per block), packed to fp16 pairs and stored back into TMEM over
+    // the first 32 of the same 64 S columns (no other thread reads those), where the next product takes
+    // them as its A operand
     {
-      uint32_t r0[32], r1[32];
-      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * half, r0);
-      tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * (half + 2), r1);
-      tc::tmem_ld_wait();
-      uint32_t p0[16], p1[16];
-      auto pack = [&](const uint32_t (&r)[32], int kb, uint32_t (&pk)[16]) {
+      uint32_t pk0[16], pk1[16];
+      auto pack = [&](int kb, uint32_t (&pk)[16]) {
+        uint32_t r[32];
+        tc::tmem_ld_32x32b_x32(tmem + lane_base + COL_S + 32 * kb, r);
         const float et = (32 * kb <= row && row < L) ? expf(my_cs - cs_s[32 * kb]) : 0.f;
+        float fs[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) fs[e] = et * fs_s[32 * kb + e];
+        tc::tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int s0 = 32 * kb + 2 * e;
-          const float f0 = s0 <= row ? u2f(r[2 * e]) * (et * fs_s[s0]) : 0.f;
-          const float f1 = s0 + 1 <= row ? u2f(r[2 * e + 1]) * (et * fs_s[s0 + 1]) : 0.f;
+          const float f0 = s0 <= row ? u2f(r[2 * e]) * fs[2 * e] : 0.f;
+          const float f1 = s0 + 1 <= row ? u2f(r[2 * e + 1]) * fs[2 * e + 1] : 0.f;
           pk[e] = pack_half2(f0, f1);
         }
       };
-      pack(r0, half, p0);
-      pack(r1, half + 2, p1);
-      tc::fence_before_sync();
-      __syncthreads();  // every row's scores are read before any packed store lands on them
-      tc::fence_after_sync();
-      tc::tmem_st_32x32b_x16(tmem + lane_base + COL_S + 16 * half, p0);
-      tc::tmem_st_32x32b_x16(tmem + lane_base + COL_S + 16 * (half + 2), p1);
+      pack(2 * half, pk0);
+      pack(2 * half + 1, pk1);
+      tc::tmem_st_32x32b_x16(tmem + lane_base + COL_S + 64 * half, pk0);
+      tc::tmem_st_32x32b_x16(tmem + lane_base + COL_S + 64 * half + 16, pk1);
       tc::tmem_st_wait();
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     if (tid == 0) {
-      const uint32_t xs = tc::smem_u32(XS);
+      const uint32_t xs = tc::smem_u32(XV);
 #pragma unroll
       for (int kk = 0; kk < SUB / 16; ++kk)
-        tc::mma_f16_tmem_a(tmem + COL_Y, tmem + COL_S + 8 * kk, tc::sdesc_mnmajor_sw128(xs + kk * 2048, kBlk), ID_Y,
-                           (i > 0) || (kk > 0));
+        tc::mma_f16_tmem_a(tmem + COL_Y, tmem + COL_S + 8 * kk + (kk >= 4 ? 32 : 0),
+                           tc::sdesc_mnmajor_sw128(xs + kk * 2048, kBlk), ID_Y, (i > 0) || (kk > 0));
       tc::mma_commit(done);
     }
     ok = tc::mbar_wait(done, done_phase, &never);
     done_phase ^= 1u;
     if (!__syncthreads_and(ok)) { ok = false; break; }
     tc::fence_after_sync();
-    if (tid == 0 && i + 1 == nk) try_fetch_hin(false);
-    if (tid == 0 && ok && i + 1 < nk) issue_x(i + 1);  // Xs_i is no longer read
+    if (tid == 0 && i + 1 == nk) peek_hin();
   }
 
   if (ok) {
@@ -392,7 +431,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     const size_t NP = NPs;
     if (tid == 0 && csub > 0) {
       if (kEarlyFetch) {
-        try_fetch_hin(true);
+        wait_fetch_hin();
       } else {
         uint32_t n = 0;
         while (ld_acquire(pflag) == 0u && n < kFlagPolls) {
