@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "swimba.h"
 
 namespace swimba {
@@ -153,6 +155,39 @@ cudaError_t launch_step_update(const Dims& d, const void* bpi, const void* xs, c
                                const float* A, float* state, void* y, cudaStream_t s);
 // Adds n to the library's launch counter (every launcher reports the kernels it issued).
 void count_launches(int n);
+
+// Programmatic dependent launch.  A kernel launched with launch_dependent() may be scheduled while the
+// previous kernel in the stream is still finishing (once that kernel's CTAs have all signalled
+// griddep_launch_dependents() or exited); it runs its prologue and calls griddep_wait() before it touches
+// anything the previous kernels wrote.  Without the launch attribute griddep_wait() returns at once.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 // Raises a kernel's dynamic shared-memory limit on the current device to at least `bytes`; the driver is
 // asked only when a larger limit than any earlier one is needed (the call costs microseconds of host time
 // that would otherwise sit in front of every launch).

@@ -110,6 +110,8 @@ dispatch_fused_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* __
   __shared__ int tot_s[64], pre_s[64], off_s[65], toff_s[65];
   const int tile = blockIdx.x, ntile = gridDim.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = d.M * d.k;
+  griddep_launch_dependents();
+  griddep_wait();  // the router's counts, indices and weights
   if (threadIdx.x < d.E) {
     const int e = threadIdx.x;
     int t = 0, pre = 0;
@@ -171,6 +173,8 @@ template <class T>
 __global__ void gather_rows_kernel(Dims d, const T* __restrict__ X, const int32_t* __restrict__ perm,
                                    T* __restrict__ xs) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  griddep_launch_dependents();
+  griddep_wait();  // the dispatch's permutation
   if (warp >= d.M * d.k) return;
   const int m = perm[warp] / d.k;
   const int4* src = reinterpret_cast<const int4*>(X + (size_t)m * d.D);
@@ -194,23 +198,25 @@ cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, 
 
 cudaError_t launch_dispatch_fused(const Dims& d, const int32_t* idx, const int32_t* counts, const WsPlan& p, char* ws,
                                   int32_t* offsets, int32_t* perm, const float* topk_w, cudaStream_t s) {
-  dispatch_fused_kernel<<<dispatch_tiles(d), kDispatchThreads, 0, s>>>(d, idx, counts, offsets, perm,
-                                                                        (int32_t*)(ws + p.tiles),
-                                                                        (int32_t*)(ws + p.ntiles),
-                                                                        (int2*)(ws + p.rowmeta), topk_w);
+  const cudaError_t e = launch_dependent(dispatch_fused_kernel, dim3(dispatch_tiles(d)), dim3(kDispatchThreads), 0, s,
+                                         1, d, idx, counts, offsets, perm, (int32_t*)(ws + p.tiles),
+                                         (int32_t*)(ws + p.ntiles), (int2*)(ws + p.rowmeta), topk_w);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows(const Dims& d, const void* X, const int32_t* perm, void* xsorted, cudaStream_t s) {
   const int rows = d.M * d.k;
   dim3 grid(ceil_div(rows, 8));
+  cudaError_t e;
   if (d.dtype == SWIMBA_BF16)
-    gather_rows_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(d, (const __nv_bfloat16*)X, perm, (__nv_bfloat16*)xsorted);
+    e = launch_dependent(gather_rows_kernel<__nv_bfloat16>, grid, dim3(256), 0, s, 1, d, (const __nv_bfloat16*)X, perm,
+                         (__nv_bfloat16*)xsorted);
   else
-    gather_rows_kernel<float><<<grid, 256, 0, s>>>(d, (const float*)X, perm, (float*)xsorted);
+    e = launch_dependent(gather_rows_kernel<float>, grid, dim3(256), 0, s, 1, d, (const float*)X, perm,
+                         (float*)xsorted);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace swimba

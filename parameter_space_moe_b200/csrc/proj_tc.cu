@@ -176,7 +176,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     tc::tma_prefetch_desc(&tmap_a);
     tc::tma_prefetch_desc(&tmap_b);
   }
+  griddep_launch_dependents();
   if (warp == 1) { tc::tmem_alloc(tmem_slot, kTmemCols); tc::tmem_relinquish(); }
+  griddep_wait();  // the dispatch's offsets and schedule, the gathered rows
   for (int e = threadIdx.x; e <= d.E; e += blockDim.x) off_s[e] = a.offsets[e];
   tc::fence_before_sync();
   __syncthreads();
@@ -353,7 +355,9 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     tc::tma_prefetch_desc(&tmap_a);
     tc::tma_prefetch_desc(&tmap_b);
   }
+  griddep_launch_dependents();
   if (warp == 1) { tc::tmem_alloc_pair(tmem_slot, kTmemCols); tc::tmem_relinquish_pair(); }
+  griddep_wait();  // the dispatch's offsets, the gathered rows
   for (int e = threadIdx.x; e <= d.E; e += blockDim.x) off_s[e] = a.offsets[e];
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -508,28 +512,28 @@ cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp
       return cudaErrorInvalidValue;
     e = set_max_dynamic_smem((const void*)proj_tc_pair_kernel, kPairSmemBytes);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kPairSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     // persistent: as many pairs as can be resident at once (at most one per tile)
     static int resident = 0;
     if (resident == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kPairSmemBytes;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
       cfg.gridDim = dim3((unsigned)sms);
       int n = 0;
       resident = cudaOccupancyMaxActiveClusters(&n, proj_tc_pair_kernel, &cfg) == cudaSuccess && n > 0 ? n : sms / 2;
     }
     const int max_pairs = (ceil_div(d.M * d.k, kPairRows) + d.E) * ceil_div(d.We, BN);
     const int pairs = resident < max_pairs ? resident : max_pairs;
-    cfg.gridDim = dim3((unsigned)(2 * pairs));
-    e = cudaLaunchKernelEx(&cfg, proj_tc_pair_kernel, ta, tb2, a);
+    e = launch_dependent(proj_tc_pair_kernel, dim3((unsigned)(2 * pairs)), dim3(kThreads), kPairSmemBytes, s, 2, ta, tb2,
+                         a);
     if (e == cudaSuccess) {
       count_launches(1);
       return cudaGetLastError();
@@ -540,9 +544,9 @@ cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp
   if (e != cudaSuccess) return e;
   const int max_tiles = max_row_tiles(d) * ceil_div(d.We, BN);
   const int grid = max_tiles < sms ? max_tiles : sms;
-  proj_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, a);
+  e = launch_dependent(proj_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, s, 1, ta, tb, a);
   count_launches(1);
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace swimba

@@ -81,6 +81,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
+  griddep_launch_dependents();  // the dispatch may start its prologue; it waits for this grid to finish
   const uint32_t rank = C > 1 ? tc::cluster_ctarank() : 0u;
   const int tile = blockIdx.x / C;
   const int tok0 = tile * RBM;

@@ -149,6 +149,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   volatile int never = 0;
   int issuedB = 0, issuedX = 0;
 
+  griddep_wait();  // the streams of the expert projection, dt of the router
   auto issue_b = [&](int i) {
     tc::mbar_arrive_expect_tx(fullB, NB * kBlk);
     for (int nb = 0; nb < NB; ++nb) tma_load_3d(BP + nb * kBlk, &tm_b, fullB, g * N + 64 * nb, a.key_slot0 + i, row0);
@@ -627,12 +628,14 @@ cudaError_t launch_scan_tc(const Dims& d, const ScanArgs& s, unsigned* lb, float
     const size_t sm = ScanSmem<64>::bytes();
     e = set_max_dynamic_smem((const void*)scan_tc_kernel<64>, sm);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<64><<<grid, kThreads, sm, stream>>>(tb, tx, tc3, a);
+    e = launch_dependent(scan_tc_kernel<64>, dim3(grid), dim3(kThreads), sm, stream, 1, tb, tx, tc3, a);
+    if (e != cudaSuccess) return e;
   } else {
     const size_t sm = ScanSmem<128>::bytes();
     e = set_max_dynamic_smem((const void*)scan_tc_kernel<128>, sm);
     if (e != cudaSuccess) return e;
-    scan_tc_kernel<128><<<grid, kThreads, sm, stream>>>(tb, tx, tc3, a);
+    e = launch_dependent(scan_tc_kernel<128>, dim3(grid), dim3(kThreads), sm, stream, 1, tb, tx, tc3, a);
+    if (e != cudaSuccess) return e;
   }
   count_launches(1);
   return cudaGetLastError();
