@@ -7,13 +7,13 @@
 // The notes name a fused MoE operator for this input projection as the way to avoid HBM round trips of
 // router outputs and parameter slices; here the per-expert output tile never leaves the SM unmixed.
 //
-// Design (one persistent CTA per SM, 10 warps):
+// Design (one persistent CTA per SM, 14 warps):
 //   warp 0      TMA producer: A = 128 gathered X rows x 64 K (16 KB), B = 256 weight rows x 64 K (32 KB)
 //               per stage, 128-byte swizzle, kStages-deep ring of mbarriers
 //   warp 1      TMEM owner and MMA issuer: 4 x tcgen05.mma M128 N256 K16 per stage into one of two
 //               256-column fp32 accumulators (double buffered: 512 TMEM columns)
-//   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4).. and one 128-column half of the tile,
-//               32 columns at a time; scales B and C columns by pi, converts to fp16 and stores to the
+//   warps 2..13 epilogue: warp w reads TMEM lanes 32*(w%4).. and one column part of the tile (96, 96 or
+//               64 columns), 32 columns at a time; scales B and C columns by pi, converts to fp16 and stores to the
 //               destination (token, slot) row.  Each row's (pair, pi) comes from the dispatch's per-row
 //               metadata in one load issued before the accumulator wait; the next tile's schedule entry
 //               is prefetched while the current tile drains.
@@ -24,7 +24,10 @@ namespace swimba {
 
 namespace {
 constexpr int BM = 128, BN = 256, BK = 64, kStages = 4;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 12;                             // 3 per TMEM lane quarter
+constexpr int kEpiParts = kEpiWarps / 4;                  // column parts of a tile
+constexpr int kChunks = BN / 32;                          // 32-column chunks of a tile row
+constexpr int kChunksPerPart = (kChunks + kEpiParts - 1) / kEpiParts;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kStageA = BM * BK * 2, kStageB = BN * BK * 2, kStageBytes = kStageA + kStageB;
 constexpr uint32_t kTmemCols = 2 * BN;
@@ -146,6 +149,31 @@ __device__ __forceinline__ void store_group32(const TcArgs& a, uint8_t* stage, i
   __syncwarp();
 }
 
+// One epilogue warp drains its 32 accumulator rows x nch 32-column chunks (starting at output column col0)
+// of a tile: the TMEM load of the next chunk is in flight while the current one is converted and stored.
+__device__ __forceinline__ void drain_tile(const TcArgs& a, uint32_t taddr, int col0, int nch, bool valid, int2 meta,
+                                           uint8_t* stage, int lane, bool& range_bad) {
+  const Dims& d = a.d;
+  const float pi = __int_as_float(meta.y);
+  uint32_t ra[32], rb[32];
+  tc::tmem_ld_32x32b_x32(taddr, ra);
+#pragma unroll
+  for (int c = 0; c < kChunksPerPart; ++c) {
+    if (c >= nch) break;
+    uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+    uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+    tc::tmem_ld_wait(cur);
+    if (c + 1 < nch) tc::tmem_ld_32x32b_x32(taddr + 32 * (c + 1), nxt);
+    const int c0 = col0 + 32 * c;
+    float sc_probe;
+    // fast path: the warp's 32-column group lies in one fp16 stream for every valid row
+    const bool fast = a.mode != 2 && c0 + 32 <= d.We &&
+                      __all_sync(0xffffffffu, !valid || group_dst(a, meta.x, pi, c0, sc_probe) != nullptr);
+    if (fast) store_group32(a, stage, lane, valid, meta.x, pi, c0, cur, range_bad);
+    else if (valid && c0 < d.We) store_chunk(a, meta.x, pi, c0, cur, range_bad);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -248,7 +276,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
   } else if (warp >= 2) {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;              // TMEM lane quarter this warp may access
-    const int ch = (warp - 2) >> 2;      // which 128-column half of the tile
+    const int part = (warp - 2) >> 2;    // which column part of the tile (chunks part*3 .. , 3 / 3 / 2)
+    const int ch0 = part * kChunksPerPart, nch = min(kChunksPerPart, kChunks - ch0);
     const int row_local = 32 * q + lane;
     uint8_t* epi_stage = smem + kStages * kStageBytes + 1024 + (warp - 2) * kEpiStage;
     int buf = 0;
@@ -269,21 +298,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         break;
       }
       tc::fence_after_sync();
-      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + ch * (BN / 2));
-#pragma unroll 1
-      for (int c = 0; c < BN / 64; ++c) {
-        uint32_t r[32];
-        tc::tmem_ld_32x32b_x32(taddr + 32 * c, r);
-        tc::tmem_ld_wait();
-        const int c0 = ct * BN + ch * (BN / 2) + 32 * c;
-        const float pi = __int_as_float(meta.y);
-        float sc_probe;
-        // fast path: the warp's 32-column group lies in one fp16 stream for every valid row
-        const bool fast = a.mode != 2 && c0 + 32 <= d.We &&
-                          __all_sync(0xffffffffu, !valid || group_dst(a, meta.x, pi, c0, sc_probe) != nullptr);
-        if (fast) store_group32(a, epi_stage, lane, valid, meta.x, pi, c0, r, range_bad);
-        else if (valid && c0 < d.We) store_chunk(a, meta.x, pi, c0, r, range_bad);
-      }
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 32 * ch0);
+      drain_tile(a, taddr, ct * BN + 32 * ch0, nch, valid, meta, epi_stage, lane, range_bad);
       tc::fence_before_sync();
       tc::mbar_arrive(&acc_empty[buf]);
       if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
@@ -440,7 +456,8 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
   } else if (warp >= 2) {
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
-    const int ch = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;
+    const int ch0 = part * kChunksPerPart, nch = min(kChunksPerPart, kChunks - ch0);
     const int row_local = 128 * (int)rank + 32 * q + lane;  // row inside the 256-row pair tile
     uint8_t* epi_stage = smem + kPairStages * kPairStageBytes + 1024 + (warp - 2) * kEpiStage;
     const uint32_t acc_empty0 = tc::map_shared(tc::smem_u32(acc_empty), 0u);
@@ -458,20 +475,8 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         break;
       }
       tc::fence_after_sync();
-      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + ch * (BN / 2));
-#pragma unroll 1
-      for (int c = 0; c < BN / 64; ++c) {
-        uint32_t r[32];
-        tc::tmem_ld_32x32b_x32(taddr + 32 * c, r);
-        tc::tmem_ld_wait();
-        const int c0 = ct * BN + ch * (BN / 2) + 32 * c;
-        const float pi = __int_as_float(meta.y);
-        float sc_probe;
-        const bool fast = a.mode != 2 && c0 + 32 <= d.We &&
-                          __all_sync(0xffffffffu, !valid || group_dst(a, meta.x, pi, c0, sc_probe) != nullptr);
-        if (fast) store_group32(a, epi_stage, lane, valid, meta.x, pi, c0, r, range_bad);
-        else if (valid && c0 < d.We) store_chunk(a, meta.x, pi, c0, r, range_bad);
-      }
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 32 * ch0);
+      drain_tile(a, taddr, ct * BN + 32 * ch0, nch, valid, meta, epi_stage, lane, range_bad);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive_cluster(acc_empty0 + 8u * (uint32_t)buf);
