@@ -108,6 +108,10 @@ cudaError_t launch_router_tc(const Dims& d, const void* X, const swimba_weights&
 // rowmeta (nullable): per sorted row, (pair index p, router weight of p as float bits; 0 without topk_w)
 cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
                             int32_t* perm, int2* rowmeta, const float* topk_w, cudaStream_t s);
+// bf16 layers: the same dispatch with the gather of X rows into expert-major order (xsorted) fused in.
+cudaError_t launch_dispatch_gather(const Dims& d, const int32_t* idx, const int32_t* counts, const WsPlan& p, char* ws,
+                                   int32_t* offsets, int32_t* perm, const float* topk_w, const void* X,
+                                   cudaStream_t s);
 // The layer's one-launch dispatch over counts the router produced (see launch_router).
 cudaError_t launch_dispatch_fused(const Dims& d, const int32_t* idx, const int32_t* counts, const WsPlan& p, char* ws,
                                   int32_t* offsets, int32_t* perm, const float* topk_w, cudaStream_t s);

@@ -163,14 +163,16 @@ static swimba_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SWIM
 // order and run the tensor-core GEMM; the fp32 layer runs the CUDA-core GEMM.
 static swimba_status run_proj(const Dims& d, const void* X, const void* w_exp, char* ws, const WsPlan& p,
                               const float* wts, int mode, void* bpi, void* xs, void* cpi, float* Z, unsigned* st,
-                              cudaStream_t s) {
+                              cudaStream_t s, bool gathered = false) {
   const int32_t* offsets = (const int32_t*)(ws + p.offsets);
   const int32_t* perm = (const int32_t*)(ws + p.perm);
   const int32_t* tiles = (const int32_t*)(ws + p.tiles);
   const int32_t* ntiles = (const int32_t*)(ws + p.ntiles);
   if (d.dtype == SWIMBA_BF16) {
-    SW_CUDA(launch_gather_rows(d, X, perm, ws + p.xsorted, s));
-    prof_mark(s, "gather");
+    if (!gathered) {
+      SW_CUDA(launch_gather_rows(d, X, perm, ws + p.xsorted, s));
+      prof_mark(s, "gather");
+    }
     SW_CUDA(launch_proj_tc(d, ws + p.xsorted, w_exp, (const int2*)(ws + p.rowmeta), tiles, ntiles, offsets, mode, bpi,
                            xs, cpi, Z, st, s));
   } else {
@@ -191,9 +193,15 @@ static swimba_status run_front(const Dims& d, const void* X, const swimba_weight
   prof_mark(s, "router");
   int32_t* offsets = (int32_t*)(ws + p.offsets);
   int32_t* perm = (int32_t*)(ws + p.perm);
-  SW_CUDA(launch_dispatch_fused(d, idx, counts, p, ws, offsets, perm, wts, s));
-  prof_mark(s, "dispatch");
-  SW_TRY(run_proj(d, X, w->w_exp, ws, p, wts, mode, ws + p.bpi, ws + p.xs, ws + p.cpi, nullptr, st, s));
+  const bool fused_gather = d.dtype == SWIMBA_BF16;
+  if (fused_gather) {
+    SW_CUDA(launch_dispatch_gather(d, idx, counts, p, ws, offsets, perm, wts, X, s));
+    prof_mark(s, "dispatch_gather");
+  } else {
+    SW_CUDA(launch_dispatch_fused(d, idx, counts, p, ws, offsets, perm, wts, s));
+    prof_mark(s, "dispatch");
+  }
+  SW_TRY(run_proj(d, X, w->w_exp, ws, p, wts, mode, ws + p.bpi, ws + p.xs, ws + p.cpi, nullptr, st, s, fused_gather));
   return SWIMBA_OK;
 }
 
