@@ -412,14 +412,18 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
+    // With P = 64 the last slot's Y product runs under the state hand-off that follows (which touches only
+    // the Bpi region, TMEM's end-state columns and global memory); the readout product's commit covers it.
+    const bool defer = P == 64 && i + 1 == nk;
     if (tid == 0) {
       const uint32_t xs = tc::smem_u32(XV);
 #pragma unroll
       for (int kk = 0; kk < SUB / 16; ++kk)
         tc::mma_f16_tmem_a(tmem + COL_Y, tmem + COL_S + 8 * kk + (kk >= 4 ? 32 : 0),
                            tc::sdesc_mnmajor_sw128(xs + kk * 2048, kBlk), ID_Y, (i > 0) || (kk > 0));
-      tc::mma_commit(done);
+      if (!defer) tc::mma_commit(done);
     }
+    if (defer) break;
     ok = tc::mbar_wait(done, done_phase, &never);
     done_phase ^= 1u;
     if (!__syncthreads_and(ok)) { ok = false; break; }
