@@ -246,11 +246,11 @@ class LayerSession:
     def step(self):
         self.sw.layer_fwd(self.d, self.X, self.W, None, self.y, self.fin, None, None, self.ws)
 
-    def h2d(self):
-        self.X.copy_(self.Xh, non_blocking=True)
-
-    def d2h(self):
-        self.yh.copy_(self.y, non_blocking=True)
+    def e2e_step(self):
+        """Host X in, host y out through swimba_layer_fwd_host (copies of one group of sequences overlap
+        the compute of another)."""
+        self.sw.layer_fwd_host(self.d, self.Xh, self.W, None, self.yh, self.fin, self.X, self.y, self.ws,
+                               chunks=min(self.w.batch, 4))
 
     def extras(self, stream, steps):
         """Separated-trajectory variant ("k scans") on this layer's streams, timed alone."""
@@ -312,10 +312,10 @@ class DecodeSession:
     def step(self):
         self.sw.step(self.d, self.X, self.W, self.state, self.y, None, self.ws)
 
-    def h2d(self):
+    def e2e_step(self):
+        """Host X in, host y out: copy, swimba_step, copy back (one step is too small to split)."""
         self.X.copy_(self.Xh, non_blocking=True)
-
-    def d2h(self):
+        self.step()
         self.yh.copy_(self.y, non_blocking=True)
 
     def extras(self, stream, steps):
@@ -384,15 +384,13 @@ def run_gpu(args, w):
     # end to end through the C ABI: pinned host input in, output back to pinned host, every step
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(2):
-        sess.h2d(); sess.step(); sess.d2h()
+        sess.e2e_step()
     torch.cuda.synchronize()
     e2e_ms = 0.0
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         e0.record(stream)
-        sess.h2d()
-        sess.step()
-        sess.d2h()
+        sess.e2e_step()
         e1.record(stream)
         e1.synchronize()
         e2e_ms += e0.elapsed_time(e1)

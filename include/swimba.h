@@ -147,6 +147,22 @@ swimba_status swimba_layer_fwd(const swimba_dims* dims, const void* X, const swi
                                const float* init_state, void* y, float* final_state, int32_t* topk_idx_out,
                                float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
 
+/* The whole layer for inputs and outputs in host memory (no counterpart in the paper; a serving
+ * convenience).  The batch is split into `chunks` groups of consecutive sequences; group c's X rows are
+ * copied host -> device, its layer forward runs on `stream`, and its y rows are copied device -> host,
+ * the three kinds of work for different groups overlapping on library-owned copy streams (created once
+ * per device) with events between them.  `stream` waits for the last copy before any later work on it.
+ *   X_host [M][D] dtype, pinned host memory; y_host [M][H][P] dtype, pinned host memory, out
+ *   X_dev, y_dev: device staging buffers of the same sizes (caller-owned)
+ *   init_state / final_state: device [B][H][N][P] fp32 or NULL, as for swimba_layer_fwd
+ *   ws: workspace sized for the full dims; chunks in [1, 16], clamped to the batch
+ * Returns SWIMBA_ERR_INVALID_ARG for null or misaligned pointers; the result is complete once `stream`
+ * reaches the point after this call (synchronise `stream` before reading y_host).  The copy streams are
+ * shared by all calls on a device: calls that may overlap in time must come from one host thread. */
+swimba_status swimba_layer_fwd_host(const swimba_dims* dims, const void* X_host, const swimba_weights* w,
+                                    const float* init_state, void* y_host, float* final_state, void* X_dev,
+                                    void* y_dev, void* ws, size_t ws_bytes, int chunks, void* stream);
+
 /* One recurrent decode step (dims.seqlen must be 1): each of `batch` sequences takes one token.
  *   X [B][D] dtype; state [B][H][N][P] fp32, updated in place (h <- a h + U~); y [B][H][P] dtype out;
  *   topk_idx_out [B][k] or NULL. */

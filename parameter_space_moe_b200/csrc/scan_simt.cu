@@ -58,6 +58,7 @@ scan_chunk_kernel(Dims d, ScanArgs a) {
   // intra-chunk outputs: warp per query token, lanes over p
   for (int i = warp; i < L; i += kScanThreads / 32) {
     float yv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
     for (int s = 0; s <= i; ++s) {
       const float decay = expf(cs[i] - cs[s]);
       const size_t ms = (size_t)b * d.T + t0 + s;
@@ -87,6 +88,7 @@ scan_chunk_kernel(Dims d, ScanArgs a) {
   for (int x = threadIdx.x; x < d.N * d.P; x += kScanThreads) {
     const int n = x / d.P, p = x % d.P;
     float acc = 0.f;
+#pragma unroll 8
     for (int s = 0; s < L; ++s) {
       const float w = expf(cend - cs[s]);
       const size_t ms = (size_t)b * d.T + t0 + s;
@@ -132,6 +134,7 @@ scan_out_kernel(Dims d, ScanArgs a) {
   for (int x = threadIdx.x; x < L * d.P; x += kScanThreads) {
     const int i = x / d.P, p = x % d.P;
     float acc = 0.f;
+#pragma unroll 8
     for (int n = 0; n < d.N; ++n) acc = fmaf(Ct[i * d.N + n], Hs[n * d.P + p], acc);
     const size_t o = ((size_t)b * d.T + t0 + i) * d.HP + (size_t)h * d.P + p;
     float v = a.yacc[o] + expf(cs[i]) * acc;

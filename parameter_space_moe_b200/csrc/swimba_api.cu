@@ -339,6 +339,78 @@ swimba_status swimba_layer_fwd(const swimba_dims* dims, const void* X, const swi
   return SWIMBA_OK;
 }
 
+// Copy streams and events of swimba_layer_fwd_host, created once per device.
+namespace {
+constexpr int kMaxHostChunks = 16;
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, in[kMaxHostChunks] = {}, out[kMaxHostChunks] = {}, done = nullptr;
+  bool ready = false;
+};
+cudaError_t host_pipe(HostPipe** out) {
+  static std::mutex mu;
+  static HostPipe pipes[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  HostPipe& q = pipes[dev];
+  if (!q.ready) {
+    if ((e = cudaStreamCreateWithFlags(&q.h2d, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithFlags(&q.d2h, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&q.start, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&q.done, cudaEventDisableTiming)) != cudaSuccess) return e;
+    for (int c = 0; c < kMaxHostChunks; ++c) {
+      if ((e = cudaEventCreateWithFlags(&q.in[c], cudaEventDisableTiming)) != cudaSuccess) return e;
+      if ((e = cudaEventCreateWithFlags(&q.out[c], cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
+    q.ready = true;
+  }
+  *out = &q;
+  return cudaSuccess;
+}
+}  // namespace
+
+swimba_status swimba_layer_fwd_host(const swimba_dims* dims, const void* X_host, const swimba_weights* w,
+                                    const float* init_state, void* y_host, float* final_state, void* X_dev,
+                                    void* y_dev, void* ws, size_t ws_bytes, int chunks, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  if (!X_host || !y_host || !ok_ptr(X_dev) || !ok_ptr(y_dev) || chunks < 1) return SWIMBA_ERR_INVALID_ARG;
+  SW_TRY(check_ws(d, ws, ws_bytes));
+  HostPipe* q = nullptr;
+  SW_CUDA(host_pipe(&q));
+  cudaStream_t s = (cudaStream_t)stream;
+  const int nch = chunks < d.Bsz ? (chunks < kMaxHostChunks ? chunks : kMaxHostChunks) : d.Bsz;
+  const size_t xrow = (size_t)d.D * elem_bytes(d.dtype), yrow = (size_t)d.HP * elem_bytes(d.dtype);
+  const size_t state = (size_t)d.H * d.N * d.P;
+  // the copies start after the work already queued on `stream`
+  SW_CUDA(cudaEventRecord(q->start, s));
+  SW_CUDA(cudaStreamWaitEvent(q->h2d, q->start, 0));
+  SW_CUDA(cudaStreamWaitEvent(q->d2h, q->start, 0));
+  for (int c = 0; c < nch; ++c) {
+    const int b0 = (int)((long long)d.Bsz * c / nch), b1 = (int)((long long)d.Bsz * (c + 1) / nch);
+    const size_t r0 = (size_t)b0 * d.T, rows = (size_t)(b1 - b0) * d.T;
+    SW_CUDA(cudaMemcpyAsync((char*)X_dev + r0 * xrow, (const char*)X_host + r0 * xrow, rows * xrow,
+                            cudaMemcpyHostToDevice, q->h2d));
+    SW_CUDA(cudaEventRecord(q->in[c], q->h2d));
+    SW_CUDA(cudaStreamWaitEvent(s, q->in[c], 0));
+    swimba_dims dc = *dims;
+    dc.batch = b1 - b0;
+    SW_TRY(swimba_layer_fwd(&dc, (const char*)X_dev + r0 * xrow, w, init_state ? init_state + (size_t)b0 * state : nullptr,
+                            (char*)y_dev + r0 * yrow, final_state ? final_state + (size_t)b0 * state : nullptr,
+                            nullptr, nullptr, ws, ws_bytes, stream));
+    SW_CUDA(cudaEventRecord(q->out[c], s));
+    SW_CUDA(cudaStreamWaitEvent(q->d2h, q->out[c], 0));
+    SW_CUDA(cudaMemcpyAsync((char*)y_host + r0 * yrow, (const char*)y_dev + r0 * yrow, rows * yrow,
+                            cudaMemcpyDeviceToHost, q->d2h));
+  }
+  SW_CUDA(cudaEventRecord(q->done, q->d2h));
+  SW_CUDA(cudaStreamWaitEvent(s, q->done, 0));
+  return SWIMBA_OK;
+}
+
 swimba_status swimba_step(const swimba_dims* dims, const void* X, const swimba_weights* w, float* state, void* y,
                           int32_t* topk_idx_out, void* ws, size_t ws_bytes, void* stream) {
   Dims d;

@@ -20,7 +20,8 @@ STATUS = {0: "SWIMBA_OK", 1: "SWIMBA_ERR_INVALID_ARG", 2: "SWIMBA_ERR_UNSUPPORTE
 EXPORTS = ("swimba_workspace_size", "swimba_stream_dtype", "swimba_router_topk", "swimba_dispatch",
            "swimba_expert_proj", "swimba_mix", "swimba_ssd_scan", "swimba_layer_fwd", "swimba_step",
            "swimba_separated_scan", "swimba_check_device_status", "swimba_status_string",
-           "swimba_profile_enable", "swimba_profile_read", "swimba_launch_count", "swimba_dispatch_noalloc")
+           "swimba_profile_enable", "swimba_profile_read", "swimba_launch_count", "swimba_dispatch_noalloc",
+           "swimba_layer_fwd_host")
 
 
 class SwimbaError(RuntimeError):
@@ -65,6 +66,7 @@ def lib():
             "swimba_mix": [P(Dims), vp, vp, i32, vp, vp, vp, vp],
             "swimba_ssd_scan": [P(Dims), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_layer_fwd": [P(Dims), vp, P(Weights), vp, vp, vp, vp, vp, vp, sz, vp],
+            "swimba_layer_fwd_host": [P(Dims), vp, P(Weights), vp, vp, vp, vp, vp, vp, sz, i32, vp],
             "swimba_step": [P(Dims), vp, P(Weights), vp, vp, vp, vp, sz, vp],
             "swimba_separated_scan": [P(Dims), vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_check_device_status": [vp],
@@ -161,6 +163,13 @@ def layer_fwd(d, X, W, init_state, y, final_state, topk_idx_out, topk_w_out, ws,
     _check("swimba_layer_fwd", lib().swimba_layer_fwd(ctypes.byref(d), _p(X), ctypes.byref(W.c), _p(init_state),
                                                        _p(y), _p(final_state), _p(topk_idx_out), _p(topk_w_out),
                                                        _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def layer_fwd_host(d, X_host, W, init_state, y_host, final_state, X_dev, y_dev, ws, chunks=4, stream=None):
+    """X_host / y_host: pinned CPU tensors; X_dev / y_dev: device staging tensors of the same shapes."""
+    _check("swimba_layer_fwd_host", lib().swimba_layer_fwd_host(
+        ctypes.byref(d), _p(X_host), ctypes.byref(W.c), _p(init_state), _p(y_host), _p(final_state), _p(X_dev),
+        _p(y_dev), _p(ws), ws.numel() * ws.element_size(), int(chunks), _stream(stream)))
 
 
 def step(d, X, W, state, y, topk_idx_out, ws, stream=None):

@@ -133,6 +133,28 @@ def test_determinism():
         assert torch.equal(u, v)
 
 
+@pytest.mark.parametrize("chunks", [1, 2, 3, 5])
+def test_host_pipeline_matches_device_call(chunks):
+    """swimba_layer_fwd_host (host X in, host y out, per-group copies overlapping compute) gives exactly the
+    device-resident call's y and final states: every row's arithmetic is independent of the grouping."""
+    w = configs.BASE.with_(batch=5, seqlen=300, d_model=256, nheads=4, seed=35)
+    inp = inputs.make_inputs(w)
+    y, fin, _ = run_layer(w, inp)
+    d = swimba.dims_of(w)
+    W = device_weights(inp)
+    Xh = inp["X"].reshape(w.M, -1).contiguous().pin_memory()
+    yh = torch.empty(w.M, w.nheads * w.headdim, dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty(w.M, w.d_model, dtype=torch.bfloat16, device="cuda")
+    yd = torch.empty_like(yh, device="cuda")
+    fh = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, device="cuda")
+    ws = torch.empty(swimba.workspace_size(d), dtype=torch.uint8, device="cuda")
+    swimba.layer_fwd_host(d, Xh, W, None, yh, fh, Xd, yd, ws, chunks=chunks)
+    torch.cuda.synchronize()
+    assert swimba.check_device_status() == 0
+    assert torch.equal(yh, y.cpu())
+    assert torch.equal(fh, fin)
+
+
 def test_range_flag_on_fp16_overflow():
     """Inputs whose projections exceed the fp16 stream range raise SWIMBA_ERR_RANGE (no fault)."""
     w = configs.BASE.with_(batch=1, seqlen=64, d_model=128, nheads=2, seed=34)
