@@ -249,8 +249,7 @@ class LayerSession:
     def e2e_step(self):
         """Host X in, host y out through swimba_layer_fwd_host (copies of one group of sequences overlap
         the compute of another)."""
-        self.sw.layer_fwd_host(self.d, self.Xh, self.W, None, self.yh, self.fin, self.X, self.y, self.ws,
-                               chunks=min(self.w.batch, 4))
+        self.sw.layer_fwd_host(self.d, self.Xh, self.W, None, self.yh, self.fin, self.X, self.y, self.ws, chunks=4)
 
     def extras(self, stream, steps):
         """Separated-trajectory variant ("k scans") on this layer's streams, timed alone."""

@@ -382,25 +382,44 @@ swimba_status swimba_layer_fwd_host(const swimba_dims* dims, const void* X_host,
   HostPipe* q = nullptr;
   SW_CUDA(host_pipe(&q));
   cudaStream_t s = (cudaStream_t)stream;
-  const int nch = chunks < d.Bsz ? (chunks < kMaxHostChunks ? chunks : kMaxHostChunks) : d.Bsz;
+  const int want = chunks < kMaxHostChunks ? chunks : kMaxHostChunks;
   const size_t xrow = (size_t)d.D * elem_bytes(d.dtype), yrow = (size_t)d.HP * elem_bytes(d.dtype);
   const size_t state = (size_t)d.H * d.N * d.P;
+  // A single sequence is split along time instead, into segments of whole 128-token sub-chunks chained
+  // through final_state (segment c starts from segment c - 1's final state), when final_state is given.
+  const int max_seg = ceil_div(d.T, 128);
+  const bool by_time = d.Bsz == 1 && want > 1 && final_state != nullptr && max_seg > 1;
+  const int nch = by_time ? (want < max_seg ? want : max_seg) : (want < d.Bsz ? want : d.Bsz);
   // the copies start after the work already queued on `stream`
   SW_CUDA(cudaEventRecord(q->start, s));
   SW_CUDA(cudaStreamWaitEvent(q->h2d, q->start, 0));
   SW_CUDA(cudaStreamWaitEvent(q->d2h, q->start, 0));
   for (int c = 0; c < nch; ++c) {
-    const int b0 = (int)((long long)d.Bsz * c / nch), b1 = (int)((long long)d.Bsz * (c + 1) / nch);
-    const size_t r0 = (size_t)b0 * d.T, rows = (size_t)(b1 - b0) * d.T;
+    swimba_dims dc = *dims;
+    size_t r0, rows;
+    const float* init_c;
+    float* fin_c;
+    if (by_time) {  // sub-chunk-aligned time segments of the one sequence
+      const int s0 = (int)((long long)max_seg * c / nch) * 128, s1 = c + 1 == nch ? d.T : (int)((long long)max_seg * (c + 1) / nch) * 128;
+      r0 = (size_t)s0;
+      rows = (size_t)(s1 - s0);
+      dc.seqlen = s1 - s0;
+      init_c = c == 0 ? init_state : final_state;
+      fin_c = final_state;
+    } else {  // groups of whole sequences
+      const int b0 = (int)((long long)d.Bsz * c / nch), b1 = (int)((long long)d.Bsz * (c + 1) / nch);
+      r0 = (size_t)b0 * d.T;
+      rows = (size_t)(b1 - b0) * d.T;
+      dc.batch = b1 - b0;
+      init_c = init_state ? init_state + (size_t)b0 * state : nullptr;
+      fin_c = final_state ? final_state + (size_t)b0 * state : nullptr;
+    }
     SW_CUDA(cudaMemcpyAsync((char*)X_dev + r0 * xrow, (const char*)X_host + r0 * xrow, rows * xrow,
                             cudaMemcpyHostToDevice, q->h2d));
     SW_CUDA(cudaEventRecord(q->in[c], q->h2d));
     SW_CUDA(cudaStreamWaitEvent(s, q->in[c], 0));
-    swimba_dims dc = *dims;
-    dc.batch = b1 - b0;
-    SW_TRY(swimba_layer_fwd(&dc, (const char*)X_dev + r0 * xrow, w, init_state ? init_state + (size_t)b0 * state : nullptr,
-                            (char*)y_dev + r0 * yrow, final_state ? final_state + (size_t)b0 * state : nullptr,
-                            nullptr, nullptr, ws, ws_bytes, stream));
+    SW_TRY(swimba_layer_fwd(&dc, (const char*)X_dev + r0 * xrow, w, init_c, (char*)y_dev + r0 * yrow, fin_c, nullptr,
+                            nullptr, ws, ws_bytes, stream));
     SW_CUDA(cudaEventRecord(q->out[c], s));
     SW_CUDA(cudaStreamWaitEvent(q->d2h, q->out[c], 0));
     SW_CUDA(cudaMemcpyAsync((char*)y_host + r0 * yrow, (const char*)y_dev + r0 * yrow, rows * yrow,

@@ -155,6 +155,29 @@ def test_host_pipeline_matches_device_call(chunks):
     assert torch.equal(fh, fin)
 
 
+@pytest.mark.parametrize("chunks", [2, 4])
+def test_host_pipeline_time_segments(chunks):
+    """One sequence is split into sub-chunk-aligned time segments chained through the final state; the
+    result is the one-call result bit for bit (the decays restart at every 128-token sub-chunk and the
+    state passes through fp32 unchanged)."""
+    w = configs.BASE.with_(batch=1, seqlen=1000, d_model=256, nheads=4, seed=36)
+    inp = inputs.make_inputs(w)
+    y, fin, _ = run_layer(w, inp)
+    d = swimba.dims_of(w)
+    W = device_weights(inp)
+    Xh = inp["X"].reshape(w.M, -1).contiguous().pin_memory()
+    yh = torch.empty(w.M, w.nheads * w.headdim, dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty(w.M, w.d_model, dtype=torch.bfloat16, device="cuda")
+    yd = torch.empty_like(yh, device="cuda")
+    fh = torch.empty(w.batch, w.nheads, w.dstate, w.headdim, device="cuda")
+    ws = torch.empty(swimba.workspace_size(d), dtype=torch.uint8, device="cuda")
+    swimba.layer_fwd_host(d, Xh, W, None, yh, fh, Xd, yd, ws, chunks=chunks)
+    torch.cuda.synchronize()
+    assert swimba.check_device_status() == 0
+    assert torch.equal(yh, y.cpu())
+    assert torch.equal(fh, fin)
+
+
 def test_range_flag_on_fp16_overflow():
     """Inputs whose projections exceed the fp16 stream range raise SWIMBA_ERR_RANGE (no fault)."""
     w = configs.BASE.with_(batch=1, seqlen=64, d_model=128, nheads=2, seed=34)
