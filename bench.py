@@ -184,8 +184,8 @@ def blas_threads():
 
 
 def run_reference(args, w):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    rank, _, _ = rank_env()
+    if rank != 0:  # under torchrun only rank 0 times the oracle; the others exit without work
         return
     inp = inputs.make_inputs(w)
     from oracle import swimba_oracle as O
@@ -321,11 +321,33 @@ class DecodeSession:
         return {}
 
 
+def rank_env():
+    """(rank, world size, local rank) from the torchrun environment (1 process when absent)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_workload(w, rank):
+    """Weak scaling: every rank runs the same shapes on its own batch (its own input seed)."""
+    return w.with_(seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of a list of floats over all ranks (the job's time is its slowest rank's)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(tokens_per_rank, world, steps, total_ms):
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (total_ms / 1e3)
+
+
 def run_gpu(args, w):
     from parameter_space_moe_b200 import swimba
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     dist = None
     if world > 1:
         import datetime
@@ -337,7 +359,7 @@ def run_gpu(args, w):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     swimba.lib()
-    wr = w.with_(seed=w.seed + 1000 * rank)
+    wr = rank_workload(w, rank)
     inp = inputs.make_inputs(wr)
     sess = (DecodeSession if w.prefill else LayerSession)(w, dev, inp, swimba)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -395,12 +417,9 @@ def run_gpu(args, w):
         e2e_ms += e0.elapsed_time(e1)
     extras = sess.extras(stream, args.steps) if args.separated else {}
 
-    t = torch.tensor([total_ms, e2e_ms] + [stage_ms.get(n, 0.0) for n in sorted(stage_ms)], dtype=torch.float64,
-                     device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = t[0].item(), t[1].item()
-    stage_ms = {n: t[2 + i].item() for i, n in enumerate(sorted(stage_ms))}
+    t = max_over_ranks([total_ms, e2e_ms] + [stage_ms.get(n, 0.0) for n in sorted(stage_ms)], dist, dev)
+    total_ms, e2e_ms = t[0], t[1]
+    stage_ms = {n: t[2 + i] for i, n in enumerate(sorted(stage_ms))}
     if rank == 0:
         report(args, w, sess, world, total_ms, e2e_ms, stage_ms, launches, sampler.summary(),
                sess.Xh.numel() * sess.Xh.element_size(), sess.yh.numel() * sess.yh.element_size(), inp, extras)
@@ -443,7 +462,7 @@ def report(args, w, sess, world, total_ms, e2e_ms, stage_ms, launches, clocks, h
     wk = sess.work
     K = args.steps
     tokens = sess.tokens * world * K
-    value = tokens / (total_ms / 1e3)
+    value = job_throughput(sess.tokens, world, K, total_ms)
     # dominant kernel stage (among those with a work model) and its roofline
     dom = max((n for n in stage_ms if n in wk), key=stage_ms.get)
     avg_s = stage_ms[dom] / K / 1e3
