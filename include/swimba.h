@@ -139,6 +139,17 @@ swimba_status swimba_ssd_scan(const swimba_dims* dims, const void* Bpi, const vo
                               const float* dt, const float* A, const float* init_state, void* y,
                               float* final_state, float* chunk_states, void* ws, size_t ws_bytes, void* stream);
 
+/* Test hook for failure detection (no counterpart in the paper): runs the tensor-core scan as if the
+ * first sub-chunk of every (sequence, head) had been lost -- the work counter starts past those
+ * sub-chunks, so nothing ever publishes their end states.  Their successors' bounded waits run out
+ * (about a second), record SWIMBA_ERR_TIMEOUT in the status word and continue from a zero state; the
+ * later sub-chunks complete normally.  No fault, no hang: swimba_check_device_status() then returns
+ * SWIMBA_ERR_TIMEOUT and the context stays usable.  Arguments as swimba_ssd_scan (no states); needs a
+ * shape the tensor-core scan covers and seqlen > 128 (else SWIMBA_ERR_UNSUPPORTED). */
+swimba_status swimba_debug_scan_lost_first_chunk(const swimba_dims* dims, const void* Bpi, const void* Xs,
+                                                 const void* Cpi, const float* dt, const float* A, void* y,
+                                                 void* ws, size_t ws_bytes, void* stream);
+
 /* The whole layer: router -> dispatch -> expert projections with the mix fused into their epilogue
  * -> chunked scan.  Paper: notes, Method flowchart.
  *   X [M][D] dtype; init_state [B][H][N][P] fp32 or NULL; y [M][H][P] dtype out;

@@ -141,6 +141,15 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
   const uint32_t tmem = misc[0];
   const int BH = d.Bsz * d.H;
   const int ticket = (int)misc[1];
+  if (ticket >= BH * a.nsub) {  // no sub-chunk left for this CTA (the counter started past zero)
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+      tc::fence_after_sync();
+      tc::tmem_dealloc(misc[0], TMEM_COLS);
+    }
+    return;
+  }
   const int csub = ticket / BH, bh = ticket % BH, b = bh / d.H, h = bh % d.H, g = h / d.hpg;
   const int t0 = csub * SUB, L = min(SUB, d.T - t0);
   const int row0 = b * d.T + t0;

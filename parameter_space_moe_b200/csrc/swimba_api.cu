@@ -315,6 +315,34 @@ swimba_status swimba_ssd_scan(const swimba_dims* dims, const void* Bpi, const vo
   return SWIMBA_OK;
 }
 
+namespace {
+__global__ void set_u32_kernel(unsigned* p, unsigned v) { *p = v; }
+cudaError_t launch_fill_u32(unsigned* p, unsigned v, cudaStream_t s) {
+  set_u32_kernel<<<1, 1, 0, s>>>(p, v);
+  count_launches(1);
+  return cudaGetLastError();
+}
+}  // namespace
+
+swimba_status swimba_debug_scan_lost_first_chunk(const swimba_dims* dims, const void* Bpi, const void* Xs,
+                                                 const void* Cpi, const float* dt, const float* A, void* y,
+                                                 void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  if (!scan_tc_supported(d) || d.T <= 128) return SWIMBA_ERR_UNSUPPORTED;
+  if (!ok_ptr(Bpi) || !ok_ptr(Xs) || !ok_ptr(Cpi) || !ok_ptr(dt) || !A || !ok_ptr(y)) return SWIMBA_ERR_INVALID_ARG;
+  SW_TRY(check_ws(d, ws, ws_bytes));
+  WsPlan p = plan_workspace(d);
+  char* b = (char*)ws;
+  ScanArgs a = mixed_scan_args(d, b, p, Bpi, Xs, Cpi, dt, A, nullptr, y, nullptr, nullptr);
+  cudaStream_t s = (cudaStream_t)stream;
+  // flags zeroed, ticket counter past every head's first sub-chunk: nothing ever publishes those flags
+  SW_CUDA(cudaMemsetAsync(b + p.lb, 0, p.lb_bytes, s));
+  SW_CUDA(launch_fill_u32((unsigned*)(b + p.lb), (unsigned)(d.Bsz * d.H), s));
+  SW_CUDA(launch_scan_tc(d, a, (unsigned*)(b + p.lb), (float*)(b + p.exch), device_status(), s));
+  return SWIMBA_OK;
+}
+
 swimba_status swimba_layer_fwd(const swimba_dims* dims, const void* X, const swimba_weights* w,
                                const float* init_state, void* y, float* final_state, int32_t* topk_idx_out,
                                float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {

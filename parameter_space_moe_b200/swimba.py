@@ -21,7 +21,7 @@ EXPORTS = ("swimba_workspace_size", "swimba_stream_dtype", "swimba_router_topk",
            "swimba_expert_proj", "swimba_mix", "swimba_ssd_scan", "swimba_layer_fwd", "swimba_step",
            "swimba_separated_scan", "swimba_check_device_status", "swimba_status_string",
            "swimba_profile_enable", "swimba_profile_read", "swimba_launch_count", "swimba_dispatch_noalloc",
-           "swimba_layer_fwd_host")
+           "swimba_layer_fwd_host", "swimba_debug_scan_lost_first_chunk")
 
 
 class SwimbaError(RuntimeError):
@@ -67,6 +67,7 @@ def lib():
             "swimba_ssd_scan": [P(Dims), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_layer_fwd": [P(Dims), vp, P(Weights), vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_layer_fwd_host": [P(Dims), vp, P(Weights), vp, vp, vp, vp, vp, vp, sz, i32, vp],
+            "swimba_debug_scan_lost_first_chunk": [P(Dims), vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_step": [P(Dims), vp, P(Weights), vp, vp, vp, vp, sz, vp],
             "swimba_separated_scan": [P(Dims), vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_check_device_status": [vp],
@@ -183,6 +184,12 @@ def separated_scan(d, B, Xs, Cpi, dt, A, init_states, y, final_states, ws, strea
                                                                  _p(A), _p(init_states), _p(y), _p(final_states),
                                                                  _p(ws), ws.numel() * ws.element_size(),
                                                                  _stream(stream)))
+
+
+def debug_scan_lost_first_chunk(d, Bpi, Xs, Cpi, dt, A, y, ws, stream=None):
+    _check("swimba_debug_scan_lost_first_chunk", lib().swimba_debug_scan_lost_first_chunk(
+        ctypes.byref(d), _p(Bpi), _p(Xs), _p(Cpi), _p(dt), _p(A), _p(y), _p(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
 
 
 def check_device_status(stream=None):

@@ -205,3 +205,30 @@ def test_separated_scan(w):
         assert nrec == w.top_k
         assert rel(to_np(y)[r].reshape(ys.shape), ys) < tol_of(w)
         assert rel(to_np(fin)[:, b], hs) < state_tol_of(w)
+
+
+def test_scan_lost_predecessor_times_out_without_fault():
+    """Failure detection: the first sub-chunk of every head is made to go missing, so the successors'
+    flag waits can never succeed.  They give up after their bounded wait, the status word reports
+    SWIMBA_ERR_TIMEOUT (no fault, no hang), and the context stays usable: the normal scan that follows
+    is correct."""
+    import time
+    w = configs.BASE.with_(name="lost_chunk", batch=1, seqlen=512, d_model=128, nheads=2, seed=87)
+    inp, Xf, ref, dev = _setup(w)
+    d = swimba.dims_of(w)
+    Bpi, Xs, Cpi, dt = (t.cuda() for t in _oracle_streams_on_device(w, ref))
+    A = inp["A"].cuda()
+    y = torch.empty(w.M, w.nheads * w.headdim, dtype=out_dtype(w), device="cuda")
+    ws = _ws(d)
+    assert swimba.check_device_status() == 0
+    t0 = time.time()
+    swimba.debug_scan_lost_first_chunk(d, Bpi, Xs, Cpi, dt, A, y, ws)
+    assert swimba.check_device_status() == 5          # SWIMBA_ERR_TIMEOUT, read and cleared
+    assert time.time() - t0 < 30.0
+    assert swimba.check_device_status() == 0
+    swimba.ssd_scan(d, Bpi, Xs, Cpi, dt, A, None, y, None, None, ws)
+    torch.cuda.synchronize()
+    assert swimba.check_device_status() == 0
+    Bq, Xq, Cq = (t.double().cpu().numpy() for t in (Bpi, Xs, Cpi))
+    yc, _, _ = O.scan_chunked(Bq, Xq, Cq.sum(1), dt.double().cpu().numpy(), f64(inp["A"]), w.chunk, None)
+    assert rel(to_np(y).reshape(yc.shape), yc) < tol_of(w)
