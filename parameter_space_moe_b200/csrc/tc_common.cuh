@@ -51,7 +51,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ------------------------------------------------------------------------------------------ TMA
-// 2D tiled bulk copy global -> shared (no multicast), completion counted on `bar` in bytes.
+// 2D tiled bulk copy global -> this CTA's shared memory, completion counted on `bar` in bytes.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
@@ -209,7 +209,7 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask
       : "memory");
 }
 // 2D tiled copy into this CTA's shared memory whose completion (bytes) is counted on an mbarrier that may
-// sit in the peer CTA of the pair (shared::cluster address).  No multicast.
+// sit in the peer CTA of the pair (shared::cluster address); the data lands in this CTA only.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster_addr, int c0,
                                                  int c1) {
   asm volatile(
