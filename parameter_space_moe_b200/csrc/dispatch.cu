@@ -1,12 +1,16 @@
 // Expert dispatch: a stable counting sort of the M*k (token, slot) pairs by expert, plus the row-tile
 // schedule of the grouped expert GEMM and the gather of X rows into expert-major order.
 //
-// Pair p = m*k + j (token m, slot j) has expert topk_idx[p].  Three launches:
+// Pair p = m*k + j (token m, slot j) has expert topk_idx[p].  Standalone dispatch (swimba_dispatch,
+// swimba_expert_proj), three launches:
 //   count    one CTA per tile of kDispatchTile consecutive pairs: per-expert counts of the tile
 //   offsets  one CTA: expert_offsets (exclusive prefix of the totals), each (tile, expert)'s first
 //            sorted position, and the GEMM schedule (expert, first row) of kRowTile-row tiles
 //   scatter  one CTA per tile: stable rank of each pair inside its tile (warp match + per-warp
 //            prefix), perm[position] = p
+// Inside the layer the router already produced the per-tile counts, so one launch does the rest:
+// dispatch_fused_kernel (fp32 layers, followed by no gather) or dispatch_gather_kernel (bf16 layers,
+// which also copies the X rows into expert order for the tensor-core GEMM).
 // The order inside an expert is increasing p, so the permutation is deterministic.
 #include "common.cuh"
 

@@ -7,10 +7,11 @@
 //   pi_t,j = exp(g_{K_j} - g_{K_0}) / sum_j' exp(g_{K_j'} - g_{K_0})
 //   dt_t,h = clamp(softplus(W_dt[h] . X_t + b_dt[h]), 1e-3, 0.1)
 // The E + H dot products per token form a skinny GEMM [M x D] x [D x (E + H)].  bf16 layers run it on
-// the warp-level tensor-core path (mma.sync m16n8k16, fp32 accumulate): a CTA of 4 warps owns 64
-// tokens and streams X and the stacked [W_r; W_dt] through padded shared memory in 64-wide K chunks
-// (cp.async, 4-stage pipeline); then threads over (token, head) finish dt and one thread per token takes
-// the top-k.  The fp32 layer keeps a CUDA-core kernel (one warp per token, fixed xor butterfly reductions).
+// the tcgen05 kernel in router_tc.cu where its logit row fits; otherwise on the warp-level tensor-core
+// path here (mma.sync m16n8k16, fp32 accumulate): a CTA of 4 warps owns 64 tokens and streams X and the
+// stacked [W_r; W_dt] through padded shared memory in 64-wide K chunks (cp.async, 4-stage pipeline);
+// then threads over (token, head) finish dt and one thread per token takes the top-k.  The fp32 layer
+// keeps a CUDA-core kernel (one warp per token, fixed xor butterfly reductions).
 #include "common.cuh"
 
 namespace swimba {
