@@ -104,3 +104,25 @@ def test_null_misaligned_and_workspace_errors(L):
     assert L.swimba_step(ctypes.byref(d), fake, ctypes.byref(w), fake, fake, None, fake, need, None) == 1
     # mix rejects unknown flags
     assert L.swimba_mix(ctypes.byref(d), fake, fake, 8, fake, fake, fake, None) == 1
+
+
+def test_host_pipeline_and_debug_hook_validation(L):
+    """swimba_layer_fwd_host and the failure-detection hook reject bad arguments before any CUDA call."""
+    d = swimba.dims_of(configs.BASE.with_(batch=2, seqlen=512, d_model=128, nheads=2))
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    w = swimba.Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    need = swimba.workspace_size(d)
+    host = lambda Xh, yh, Xd, yd, chunks, ws=fake, n=need: L.swimba_layer_fwd_host(
+        ctypes.byref(d), Xh, ctypes.byref(w), None, yh, None, Xd, yd, ws, n, chunks, None)
+    assert host(None, fake, fake, fake, 2) == 1        # no host input
+    assert host(fake, None, fake, fake, 2) == 1        # no host output
+    assert host(fake, fake, odd, fake, 2) == 1         # misaligned device staging
+    assert host(fake, fake, fake, None, 2) == 1        # no device staging for y
+    assert host(fake, fake, fake, fake, 0) == 1        # at least one group
+    assert host(fake, fake, fake, fake, 2, n=need - 1) == 4   # workspace too small
+    hook = lambda dims, Bpi=fake: L.swimba_debug_scan_lost_first_chunk(
+        ctypes.byref(dims), Bpi, fake, fake, fake, fake, fake, fake, swimba.workspace_size(dims), None)
+    assert hook(swimba.dims_of(configs.TINY_F32)) == 2                      # not a tensor-core scan shape
+    assert hook(swimba.dims_of(configs.BASE.with_(batch=1, seqlen=128))) == 2   # one sub-chunk: nothing to lose
+    assert hook(d, Bpi=None) == 1
