@@ -1,0 +1,173 @@
+"""The pins are strong enough: each plausible mistake, planted in the oracle (on the CPU, by replacing one
+of its functions for the duration of a test), makes at least one pin of tests/test_oracle_pins.py fail.
+
+Mistakes planted: no renormalisation over the winners, ties broken toward the higher expert index, the
+dt clamp dropped, every slot projected with its first slot's expert, B and C swapped in the stream
+split, C~ summed without the router weights, the injection added before the decay, the decay's sign
+flipped, the chunked form's causal mask shifted by one, and the chunk-state decay taken from the chunk
+start instead of its end."""
+import numpy as np
+import pytest
+
+from oracle import swimba_oracle as O
+
+from . import test_oracle_pins as pins
+
+
+def _topk_weights_not_renormalised(g, idx):
+    sel = np.take_along_axis(g, idx, axis=-1)
+    m = g.max(axis=-1, keepdims=True)
+    return np.exp(sel - m) / np.exp(g - m).sum(axis=-1, keepdims=True)
+
+
+def _topk_select_ties_high(g, k):
+    g = np.asarray(g)
+    rev = g[..., ::-1]
+    order = np.argsort(-rev, axis=-1, kind="stable")
+    return (g.shape[-1] - 1 - order[..., :k]).astype(np.int64)
+
+
+def _dt_unclamped(X, W_dt, b_dt, dt_min=1e-3, dt_max=0.1):
+    return O.softplus(X @ W_dt.T + b_dt)
+
+
+def _expert_proj_first_slot(X, W_exp, idx):
+    M, k = idx.shape
+    z = np.zeros((M, k, W_exp.shape[1]))
+    for m in range(M):
+        for j in range(k):
+            z[m, j] = W_exp[idx[m, 0]] @ X[m]
+    return z
+
+
+def _split_swapped(z, H, P, G, N):
+    x, B, C = ORIG["split_streams"](z, H, P, G, N)
+    return x, C, B
+
+
+def _mix_unweighted_c(z, w, H, P, G, N):
+    x, B, C = O.split_streams(z, H, P, G, N)
+    Bpi = w[:, :, None, None] * B
+    Cpi = w[:, :, None, None] * C
+    return Bpi, x, C.sum(axis=1), Cpi
+
+
+def _scan_inject_then_decay(Bpi, Xs, Ct, dt, A, init=None):
+    T, k, H, P = Xs.shape
+    G, N = Bpi.shape[2], Bpi.shape[3]
+    g = O.group_of(H, G)
+    h = np.zeros((H, N, P)) if init is None else np.array(init, dtype=np.float64)
+    y = np.zeros((T, H, P))
+    for t in range(T):
+        a = np.exp(dt[t] * A)
+        U = np.einsum("jhn,jhp->hnp", Bpi[t][:, g], Xs[t])
+        h = a[:, None, None] * (h + U)
+        y[t] = np.einsum("hn,hnp->hp", Ct[t][g], h)
+    return y, h
+
+
+def _scan_decay_sign(Bpi, Xs, Ct, dt, A, init=None):
+    return ORIG["scan_sequential"](Bpi, Xs, Ct, dt, -A, init)
+
+
+def _chunked_strict_mask(Bpi, Xs, Ct, dt, A, Q, init=None):
+    # the intra-chunk sum over s < t instead of s <= t
+    T, k, H, P = Xs.shape
+    G, N = Bpi.shape[2], Bpi.shape[3]
+    g = O.group_of(H, G)
+    nc = (T + Q - 1) // Q
+    Hc = np.zeros((H, N, P)) if init is None else np.array(init, dtype=np.float64)
+    Hs = np.zeros((nc, H, N, P))
+    y = np.zeros((T, H, P))
+    for c in range(nc):
+        t0, t1 = c * Q, min(T, (c + 1) * Q)
+        cs = np.cumsum(dt[t0:t1] * A, axis=0)
+        Cg, Bg, Xc = Ct[t0:t1][:, g], Bpi[t0:t1][:, :, g], Xs[t0:t1]
+        L = t1 - t0
+        Hs[c] = Hc
+        scores = np.einsum("thn,sjhn->tsjh", Cg, Bg)
+        seg = cs[:, None, :] - cs[None, :, :]
+        causal = np.tril(np.ones((L, L), dtype=bool), k=-1)
+        decay = np.where(causal[:, :, None], np.exp(np.where(causal[:, :, None], seg, 0.0)), 0.0)
+        y[t0:t1] = np.einsum("tsh,tsjh,sjhp->thp", decay, scores, Xc)
+        y[t0:t1] += np.exp(cs)[:, :, None] * np.einsum("thn,hnp->thp", Cg, Hc)
+        wend = np.exp(cs[-1][None, :] - cs)
+        Hc = np.exp(cs[-1])[:, None, None] * Hc + np.einsum("sh,sjhn,sjhp->hnp", wend, Bg, Xc)
+    return y, Hs, Hc
+
+
+def _chunked_state_decay_from_start(Bpi, Xs, Ct, dt, A, Q, init=None):
+    # the chunk state weighted by exp(cs_s) (decay from the chunk start) instead of exp(cs_end - cs_s)
+    T, k, H, P = Xs.shape
+    G, N = Bpi.shape[2], Bpi.shape[3]
+    g = O.group_of(H, G)
+    nc = (T + Q - 1) // Q
+    Hc = np.zeros((H, N, P)) if init is None else np.array(init, dtype=np.float64)
+    Hs = np.zeros((nc, H, N, P))
+    y = np.zeros((T, H, P))
+    for c in range(nc):
+        t0, t1 = c * Q, min(T, (c + 1) * Q)
+        cs = np.cumsum(dt[t0:t1] * A, axis=0)
+        Cg, Bg, Xc = Ct[t0:t1][:, g], Bpi[t0:t1][:, :, g], Xs[t0:t1]
+        L = t1 - t0
+        Hs[c] = Hc
+        scores = np.einsum("thn,sjhn->tsjh", Cg, Bg)
+        seg = cs[:, None, :] - cs[None, :, :]
+        causal = np.tril(np.ones((L, L), dtype=bool))
+        decay = np.where(causal[:, :, None], np.exp(np.where(causal[:, :, None], seg, 0.0)), 0.0)
+        y[t0:t1] = np.einsum("tsh,tsjh,sjhp->thp", decay, scores, Xc)
+        y[t0:t1] += np.exp(cs)[:, :, None] * np.einsum("thn,hnp->thp", Cg, Hc)
+        wstart = np.exp(cs)
+        Hc = np.exp(cs[-1])[:, None, None] * Hc + np.einsum("sh,sjhn,sjhp->hnp", wstart, Bg, Xc)
+    return y, Hs, Hc
+
+
+ORIG = {name: getattr(O, name) for name in
+        ("topk_weights", "topk_select", "dt_proj", "expert_proj", "split_streams", "mix", "scan_sequential",
+         "scan_chunked")}
+
+# every pin, called with the parameters its decorator gives
+ALL_PINS = [
+    pins.test_topk_matches_bruteforce_sort_with_ties, pins.test_topk_is_a_maximal_set,
+    pins.test_topk_weights_are_renormalised_softmax, pins.test_thm35_sigmoid_worked_example,
+    pins.test_dt_recipe_and_clamp, pins.test_expert_proj_matches_elementwise_dot_products,
+    pins.test_split_streams_layout, pins.test_group_map, pins.test_polynomial_degree_three_single_expert,
+    pins.test_single_expert_reduces_to_plain_ssm_streams, pins.test_identical_experts_equal_unrouted_ssm,
+    pins.test_geometric_closed_form_one_injection, lambda: pins.test_sequential_equals_bruteforce_semiseparable(2),
+    pins.test_groups_equal_replicated_heads, lambda: pins.test_chunked_equals_sequential(70, 16),
+    pins.test_thm33_bibo_bound, pins.test_thm34_static_routing_equivalence_and_counts,
+    pins.test_thm34_dynamic_routing_bound, pins.test_layer_fwd_state_handoff, pins.test_steps_equal_layer_fwd,
+    pins.test_forced_routing_replays_given_indices,
+]
+
+MUTATIONS = {
+    "weights_not_renormalised": ("topk_weights", _topk_weights_not_renormalised),
+    "ties_to_higher_index": ("topk_select", _topk_select_ties_high),
+    "dt_clamp_dropped": ("dt_proj", _dt_unclamped),
+    "slots_use_first_expert": ("expert_proj", _expert_proj_first_slot),
+    "B_and_C_swapped": ("split_streams", _split_swapped),
+    "C_tilde_without_weights": ("mix", _mix_unweighted_c),
+    "inject_before_decay": ("scan_sequential", _scan_inject_then_decay),
+    "decay_sign_flipped": ("scan_sequential", _scan_decay_sign),
+    "causal_mask_shifted": ("scan_chunked", _chunked_strict_mask),
+    "chunk_state_decay_from_start": ("scan_chunked", _chunked_state_decay_from_start),
+}
+
+
+def test_unmutated_oracle_passes_every_pin():
+    for pin in ALL_PINS:
+        pin()
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(O, attr, fn)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin()
+        except Exception as e:  # an assertion, or an error a wrong shape or value leads to
+            caught.append(getattr(pin, "__name__", "pin"))
+    assert caught, f"no pin caught the planted mistake {name}"
