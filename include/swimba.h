@@ -12,7 +12,8 @@
  *   dt            dt_t,h = clamp(softplus(W_dt[h] . X_t + b_dt[h]), 1e-3, 0.1)
  *
  * Conventions for every entry point
- *  - Every pointer is caller-owned DEVICE memory unless stated; the library allocates nothing.
+ *  - Every pointer is caller-owned DEVICE memory unless stated; the library allocates no device memory
+ *    (swimba_layer_fwd_host creates two copy streams and a few events once per device).
  *  - Tensors are dense, row-major (last index fastest) and 16-byte aligned.
  *  - M = batch * seqlen tokens; row m = b * seqlen + t.  W_e = H*P + 2*G*N.
  *  - dtype (swimba_dims.dtype) is the type of X, of the three weight matrices and of y.  dt, topk_w,
