@@ -128,14 +128,21 @@ def group_of(H, G):
     return np.arange(H) // (H // G)
 
 
-def scan_sequential(Bpi, Xs, Ct, dt, A, init=None):
+def _count_update(stats):
+    """Counts one state update of one trajectory (all heads at once) when a stats dict is passed."""
+    if stats is not None:
+        stats["updates"] = stats.get("updates", 0) + 1
+
+
+def scan_sequential(Bpi, Xs, Ct, dt, A, init=None, stats=None):
     """The single-trajectory recurrence, token by token ([notes] key design 1, second display
     equation; [gist] "h_t = A h_{t-1} + sum pi B X"):
         h_t = a_t h_{t-1} + sum_j Bpi_tj (x) Xs_tj,     y_t = C~_t^T h_t,     a_t = exp(dt_t A_h).
     Reading: no dt factor on the injection (the pages' equation has none).
 
     One batch row: Bpi [T,k,G,N], Xs [T,k,H,P], Ct [T,G,N], dt [T,H], A [H], init [H,N,P] or None.
-    Returns y [T,H,P] and the final state [H,N,P].
+    Returns y [T,H,P] and the final state [H,N,P].  stats (optional dict): "updates" is increased by one
+    for every state update, so a T-token call adds T (one trajectory).
     """
     T, k, H, P = Xs.shape
     G, N = Bpi.shape[2], Bpi.shape[3]
@@ -146,6 +153,7 @@ def scan_sequential(Bpi, Xs, Ct, dt, A, init=None):
         a = np.exp(dt[t] * A)                                           # [H]
         U = np.einsum("jhn,jhp->hnp", Bpi[t][:, g], Xs[t])              # rank-k injection per head
         h = a[:, None, None] * h + U
+        _count_update(stats)
         y[t] = np.einsum("hn,hnp->hp", Ct[t][g], h)
     return y, h
 
@@ -215,38 +223,44 @@ def scan_separated_k(B, Xs, Cpi, dt, A, init=None):
         h^(j)_t = a_t h^(j)_{t-1} + B_tj (x) Xs_tj,    y_t = sum_j (pi_tj C_tj)^T h^(j)_t.
     This is the separated-trajectory design of [notes] key design 1 restricted to the active slots;
     it runs k recurrences where the mixed layer runs one.  B [T,k,G,N], Cpi [T,k,G,N], init [k,H,N,P].
-    Returns y [T,H,P], the k final states [k,H,N,P] and the number of recurrences run (k)."""
+    Returns y [T,H,P], the k final states [k,H,N,P] and the number of trajectories it ran, counted as
+    state updates per token."""
     T, k, H, P = Xs.shape
     G, N = B.shape[2], B.shape[3]
     g = group_of(H, G)
     h = np.zeros((k, H, N, P)) if init is None else np.array(init, dtype=np.float64)
     y = np.zeros((T, H, P))
+    stats = {}
     for t in range(T):
         a = np.exp(dt[t] * A)
         for j in range(k):
             h[j] = a[:, None, None] * h[j] + np.einsum("hn,hp->hnp", B[t, j][g], Xs[t, j])
+            _count_update(stats)
             y[t] += np.einsum("hn,hnp->hp", Cpi[t, j][g], h[j])
-    return y, h, k
+    return y, h, stats.get("updates", 0) // max(T, 1)
 
 
 def scan_separated_dense(xE, BE, CE, pi_dense, dt, A):
     """MoE over separated SSMs ([notes] key design 1, the O(T E C_step) design; Theorem 3.4):
     every expert e keeps its own state h^(e), driven on every token by its own B^(e) x^(e)T, and the
     output is y_t = sum_e pi_te C^(e)_t^T h^(e)_t (pi_te = 0 off the active set).
-    xE [T,E,H,P], BE/CE [T,E,G,N], pi_dense [T,E].  Returns y, the states [T,E,H,N,P] and E."""
+    xE [T,E,H,P], BE/CE [T,E,G,N], pi_dense [T,E].  Returns y, the states [T,E,H,N,P] and the number
+    of trajectories it ran, counted as state updates per token."""
     T, E, H, P = xE.shape
     G, N = BE.shape[2], BE.shape[3]
     g = group_of(H, G)
     h = np.zeros((E, H, N, P))
     hs = np.zeros((T, E, H, N, P))
     y = np.zeros((T, H, P))
+    stats = {}
     for t in range(T):
         a = np.exp(dt[t] * A)
         for e in range(E):
             h[e] = a[:, None, None] * h[e] + np.einsum("hn,hp->hnp", BE[t, e][g], xE[t, e])
+            _count_update(stats)
             y[t] += pi_dense[t, e] * np.einsum("hn,hnp->hp", CE[t, e][g], h[e])
         hs[t] = h
-    return y, hs, E
+    return y, hs, stats.get("updates", 0) // max(T, 1)
 
 
 # ----------------------------------------------------------------------------- the layer

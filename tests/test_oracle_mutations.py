@@ -4,8 +4,8 @@ of its functions for the duration of a test), makes at least one pin of tests/te
 Mistakes planted: no renormalisation over the winners, ties broken toward the higher expert index, the
 dt clamp dropped, every slot projected with its first slot's expert, B and C swapped in the stream
 split, C~ summed without the router weights, the injection added before the decay, the decay's sign
-flipped, the chunked form's causal mask shifted by one, and the chunk-state decay taken from the chunk
-start instead of its end."""
+flipped, the chunked form's causal mask shifted by one, the chunk-state decay taken from the chunk
+start instead of its end, and the separated-E design advancing only the active experts."""
 import numpy as np
 import pytest
 
@@ -52,7 +52,7 @@ def _mix_unweighted_c(z, w, H, P, G, N):
     return Bpi, x, C.sum(axis=1), Cpi
 
 
-def _scan_inject_then_decay(Bpi, Xs, Ct, dt, A, init=None):
+def _scan_inject_then_decay(Bpi, Xs, Ct, dt, A, init=None, stats=None):
     T, k, H, P = Xs.shape
     G, N = Bpi.shape[2], Bpi.shape[3]
     g = O.group_of(H, G)
@@ -62,12 +62,35 @@ def _scan_inject_then_decay(Bpi, Xs, Ct, dt, A, init=None):
         a = np.exp(dt[t] * A)
         U = np.einsum("jhn,jhp->hnp", Bpi[t][:, g], Xs[t])
         h = a[:, None, None] * (h + U)
+        O._count_update(stats)
         y[t] = np.einsum("hn,hnp->hp", Ct[t][g], h)
     return y, h
 
 
-def _scan_decay_sign(Bpi, Xs, Ct, dt, A, init=None):
-    return ORIG["scan_sequential"](Bpi, Xs, Ct, dt, -A, init)
+def _scan_decay_sign(Bpi, Xs, Ct, dt, A, init=None, stats=None):
+    return ORIG["scan_sequential"](Bpi, Xs, Ct, dt, -A, init, stats)
+
+
+def _dense_skips_inactive_experts(xE, BE, CE, pi_dense, dt, A):
+    # the separated-E design advancing only the experts active on a token (k trajectories, not E); its
+    # output is unchanged under static routing, so only the trajectory count can catch it
+    T, E, H, P = xE.shape
+    G, N = BE.shape[2], BE.shape[3]
+    g = O.group_of(H, G)
+    h = np.zeros((E, H, N, P))
+    hs = np.zeros((T, E, H, N, P))
+    y = np.zeros((T, H, P))
+    stats = {}
+    for t in range(T):
+        a = np.exp(dt[t] * A)
+        for e in range(E):
+            if pi_dense[t, e] == 0:
+                continue
+            h[e] = a[:, None, None] * h[e] + np.einsum("hn,hp->hnp", BE[t, e][g], xE[t, e])
+            O._count_update(stats)
+            y[t] += pi_dense[t, e] * np.einsum("hn,hnp->hp", CE[t, e][g], h[e])
+        hs[t] = h
+    return y, hs, stats.get("updates", 0) // max(T, 1)
 
 
 def _chunked_strict_mask(Bpi, Xs, Ct, dt, A, Q, init=None):
@@ -124,7 +147,7 @@ def _chunked_state_decay_from_start(Bpi, Xs, Ct, dt, A, Q, init=None):
 
 ORIG = {name: getattr(O, name) for name in
         ("topk_weights", "topk_select", "dt_proj", "expert_proj", "split_streams", "mix", "scan_sequential",
-         "scan_chunked")}
+         "scan_chunked", "scan_separated_dense")}
 
 # every pin, called with the parameters its decorator gives
 ALL_PINS = [
@@ -151,6 +174,7 @@ MUTATIONS = {
     "decay_sign_flipped": ("scan_sequential", _scan_decay_sign),
     "causal_mask_shifted": ("scan_chunked", _chunked_strict_mask),
     "chunk_state_decay_from_start": ("scan_chunked", _chunked_state_decay_from_start),
+    "dense_skips_inactive_experts": ("scan_separated_dense", _dense_skips_inactive_experts),
 }
 
 

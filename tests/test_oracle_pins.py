@@ -295,7 +295,8 @@ def test_thm34_static_routing_equivalence_and_counts():
     Bk, Xk, Ck = BE[:, K], xE[:, K], CE[:, K]
     Bpi = pi[None, :, None, None] * Bk
     Cpi = pi[None, :, None, None] * Ck
-    y_mix, _ = O.scan_sequential(Bpi, Xk, Cpi.sum(1), dt, A)
+    mixed_stats = {}
+    y_mix, _ = O.scan_sequential(Bpi, Xk, Cpi.sum(1), dt, A, stats=mixed_stats)
     y_sepk, _, nk = O.scan_separated_k(Bk, Xk, Cpi, dt, A)
     # separated-E keeps all E experts running but reads out only the active ones: with the inactive
     # experts' contribution weighted 0 it matches as well
@@ -304,11 +305,17 @@ def test_thm34_static_routing_equivalence_and_counts():
     rows = [l.split() for l in open(os.path.join(GOLD, "efficiency_table_trajectories.txt"))
             if not l.startswith("#")]
     counts = {r[0]: int(r[3]) for r in rows}
-    assert counts["mixed"] == 1
+    # the counts are state updates the oracle actually performed, divided by T
+    assert mixed_stats["updates"] == T * counts["mixed"]
     _, _, n1 = O.scan_separated_k(Bk[:, :1], Xk[:, :1], Cpi[:, :1], dt, A)
     assert n1 == counts["separated_k"]
     _, _, n4 = O.scan_separated_dense(xE, BE, CE, pi_dense, dt, A)
     assert n4 == counts["separated_E"] == E and nk == k
+    # the mixed layer's count does not grow with k (one trajectory whatever the number of slots)
+    s1, s2 = {}, {}
+    O.scan_sequential(Bpi[:, :1], Xk[:, :1], Cpi[:, :1].sum(1), dt, A, stats=s1)
+    O.scan_sequential(Bpi, Xk, Cpi.sum(1), dt, A, stats=s2)
+    assert s1["updates"] == s2["updates"] == T
 
 
 def test_thm34_dynamic_routing_bound():
