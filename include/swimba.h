@@ -28,6 +28,12 @@
  *    SWIMBA_ERR_UNSUPPORTED (there is no fallback path).
  *  - Supported shapes: N, P in {16, 32, 64, 128}; chunk in {64, 128, 256}; 1 <= top_k <= min(E, 8);
  *    E <= 64; G divides H; d_model a multiple of 64 (bf16) or 8 (fp32); every size >= 1.
+ *  - Supported values (bf16 layers): every mixed-stream value (x, pi*B, pi*C) and every carried state
+ *    element must stay within the fp16 range (|v| <= 65504); a value outside it is recorded as
+ *    SWIMBA_ERR_RANGE and the layer's outputs are then not valid.  There is no wider-range path.
+ *  - Chunk length: `chunk` fixes where chunk_states are reported.  The tensor-core scan (bf16, N = 128,
+ *    P in {64, 128}) always solves in 128-token sub-chunks, which gives the same result up to rounding
+ *    for every chunk; the CUDA-core scan (fp32 layers and the other shapes) solves in `chunk`-token chunks.
  */
 #ifndef SWIMBA_H_
 #define SWIMBA_H_
@@ -46,7 +52,8 @@ typedef enum {
   SWIMBA_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
   SWIMBA_ERR_WORKSPACE = 4,    /* ws is NULL or smaller than swimba_workspace_size() */
   SWIMBA_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up (read via swimba_check_device_status) */
-  SWIMBA_ERR_RANGE = 6         /* device: a mixed-stream value did not fit the stream dtype */
+  SWIMBA_ERR_RANGE = 6,        /* device: a mixed-stream value did not fit the stream dtype */
+  SWIMBA_ERR_INDEX = 7         /* device: a caller-given expert index lay outside [0, E) */
 } swimba_status;
 
 typedef enum { SWIMBA_F32 = 0, SWIMBA_BF16 = 1, SWIMBA_F16 = 2 } swimba_dtype;
@@ -93,17 +100,19 @@ swimba_status swimba_router_topk(const swimba_dims* dims, const void* X, const s
 
 /* Expert dispatch: a stable counting sort of the M*k (token, slot) pairs by expert (the token-level
  * routing the notes' efficiency discussion attributes Swimba's extra cost to).
- *   topk_idx       [M][k] int32 in
+ *   topk_idx       [M][k] int32 in, every value in [0, E)
  *   expert_offsets [E+1] int32 out: pairs of expert e are perm[expert_offsets[e] .. expert_offsets[e+1])
- *   perm           [M*k] int32 out: value m*k + j, in increasing m within each expert */
+ *   perm           [M*k] int32 out: value m*k + j, in increasing m within each expert
+ * A pair whose index lies outside [0, E) is left out of the sort (expert_offsets[E] then counts only the
+ * valid pairs and perm's tail is not written) and SWIMBA_ERR_INDEX is recorded in the status word. */
 swimba_status swimba_dispatch(const swimba_dims* dims, const int32_t* topk_idx, int32_t* expert_offsets,
                               int32_t* perm, void* ws, size_t ws_bytes, void* stream);
 
 /* Expert dispatch that allocates nothing and takes no workspace.  The paper has no counterpart: this entry
  * point is for callers that cannot give the library scratch memory -- plugin-style hosts whose interface
  * hands an operator only its inputs and outputs, and runtimes that plan all device memory at start-up and
- * refuse allocations afterwards.  Same arguments (minus the workspace) and the same results as
- * swimba_dispatch.  Its scratch is one fixed 1 MiB array inside the library, held on every device that
+ * refuse allocations afterwards.  Same arguments (minus the workspace; topk_idx values in [0, E)), the
+ * same status codes and the same results as swimba_dispatch.  Its scratch is one fixed 1 MiB array inside the library, held on every device that
  * loads the library until the process exits; a shape that needs more (about 0.56 * M * k bytes with 64
  * experts, 0.125 * M * k with 8) returns SWIMBA_ERR_WORKSPACE before launching anything.  The first call on
  * a device looks up the array's device address with that device current; make that first call before
@@ -178,6 +187,8 @@ swimba_status swimba_layer_fwd_host(const swimba_dims* dims, const void* X_host,
                                     void* y_dev, void* ws, size_t ws_bytes, int chunks, void* stream);
 
 /* One recurrent decode step (dims.seqlen must be 1): each of `batch` sequences takes one token.
+ * Paper: notes, key design 1, second display equation advanced by a single token (h_t = a_t h_{t-1} +
+ * U~_t, y_t = C~_t^T h_t with the cached h_{t-1}); router, experts and mixing as in swimba_layer_fwd.
  *   X [B][D] dtype; state [B][H][N][P] fp32, updated in place (h <- a h + U~); y [B][H][P] dtype out;
  *   topk_idx_out [B][k] or NULL. */
 swimba_status swimba_step(const swimba_dims* dims, const void* X, const swimba_weights* w, float* state,
@@ -194,8 +205,10 @@ swimba_status swimba_separated_scan(const swimba_dims* dims, const void* B, cons
                                     float* final_states, void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, then reads and clears the current device's status word: SWIMBA_OK,
- * SWIMBA_ERR_TIMEOUT or SWIMBA_ERR_RANGE (SWIMBA_ERR_CUDA if the stream reports an error).  The word
- * is sticky: it collects every flag raised on this device since the previous check. */
+ * SWIMBA_ERR_TIMEOUT, SWIMBA_ERR_RANGE or SWIMBA_ERR_INDEX, in that order of precedence (SWIMBA_ERR_CUDA
+ * if the stream reports an error).  The word is sticky: it collects every flag raised on this device
+ * since the previous check.  Its device address is looked up once per device; a device reset between
+ * calls into the library is not supported. */
 swimba_status swimba_check_device_status(void* stream);
 
 /* Profiling support.  swimba_profile_enable(1) makes every later entry-point call record a CUDA

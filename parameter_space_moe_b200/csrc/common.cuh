@@ -11,8 +11,8 @@
 
 namespace swimba {
 
-// Bits of the workspace status word.
-enum : unsigned { ST_TIMEOUT = 1u, ST_RANGE = 2u };
+// Bits of the device status word.
+enum : unsigned { ST_TIMEOUT = 1u, ST_RANGE = 2u, ST_INDEX = 4u };
 
 // Largest finite fp16 value: mixed streams stored as fp16 must stay below it.
 constexpr float kF16Max = 65504.f;
@@ -93,6 +93,10 @@ inline int dispatch_tiles(const Dims& d) { return ceil_div(d.M * d.k, kDispatchT
 size_t elem_bytes(int dtype);
 int stream_dtype_of(int dtype);
 WsPlan plan_workspace(const Dims& d);
+// Validates the C ABI's dims and fills the kernels' form (every entry point's first step).
+swimba_status make_dims(const swimba_dims* in, Dims* d);
+// Device address of the current device's status word (looked up once per device; null on a CUDA error).
+unsigned* device_status();
 
 // ---------------------------------------------------------------------------------------------
 // Kernel launchers (defined in the .cu files next to their kernels).  All return cudaError_t of the
@@ -105,9 +109,10 @@ cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w,
 bool router_tc_supported(const Dims& d);
 cudaError_t launch_router_tc(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
                              float* dt, int32_t* counts, unsigned* st, cudaStream_t s);
-// rowmeta (nullable): per sorted row, (pair index p, router weight of p as float bits; 0 without topk_w)
+// rowmeta (nullable): per sorted row, (pair index p, router weight of p as float bits; 0 without topk_w).
+// Pairs whose index lies outside [0, E) are left out of the sort and raise ST_INDEX in *st.
 cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
-                            int32_t* perm, int2* rowmeta, const float* topk_w, cudaStream_t s);
+                            int32_t* perm, int2* rowmeta, const float* topk_w, unsigned* st, cudaStream_t s);
 // bf16 layers: the same dispatch with the gather of X rows into expert-major order (xsorted) fused in.
 cudaError_t launch_dispatch_gather(const Dims& d, const int32_t* idx, const int32_t* counts, const WsPlan& p, char* ws,
                                    int32_t* offsets, int32_t* perm, const float* topk_w, const void* X,

@@ -18,17 +18,25 @@ namespace swimba {
 
 constexpr int kDispatchThreads = 1024;
 
+// Caller-given indices outside [0, E) are skipped (and reported through the status word) so that no
+// shared-memory table is indexed out of bounds.
 __global__ void __launch_bounds__(kDispatchThreads)
-dispatch_count_kernel(Dims d, const int32_t* __restrict__ idx, int32_t* __restrict__ counts) {
+dispatch_count_kernel(Dims d, const int32_t* __restrict__ idx, int32_t* __restrict__ counts, unsigned* st) {
   __shared__ int c_s[64];
   const int tile = blockIdx.x;
   if (threadIdx.x < 64) c_s[threadIdx.x] = 0;
   __syncthreads();
   const int total = d.M * d.k;
+  bool bad = false;
   for (int i = threadIdx.x; i < kDispatchTile; i += blockDim.x) {
     int p = tile * kDispatchTile + i;
-    if (p < total) atomicAdd(&c_s[idx[p]], 1);
+    if (p < total) {
+      const int e = idx[p];
+      if (e >= 0 && e < d.E) atomicAdd(&c_s[e], 1);
+      else bad = true;
+    }
   }
+  if (bad) atomicOr(st, ST_INDEX);
   __syncthreads();
   if (threadIdx.x < d.E) counts[tile * d.E + threadIdx.x] = c_s[threadIdx.x];
 }
@@ -80,8 +88,9 @@ dispatch_scatter_kernel(Dims d, const int32_t* __restrict__ idx, const int32_t* 
   for (int x = threadIdx.x; x < (kDispatchThreads / 32) * 64; x += blockDim.x) (&wc_s[0][0])[x] = 0;
   __syncthreads();
   const int p = tile * kDispatchTile + threadIdx.x;  // kDispatchTile == blockDim.x
-  const bool valid = p < total;
-  const int e = valid ? idx[p] : -1 - lane;          // distinct sentinels never match a real expert
+  const int raw = p < total ? idx[p] : 0;
+  const bool valid = p < total && raw >= 0 && raw < d.E;  // out-of-range indices were reported by the count
+  const int e = valid ? raw : -1 - lane;             // distinct sentinels never match a real expert
   const unsigned peers = __match_any_sync(0xffffffffu, e);
   const int rank = __popc(peers & ((1u << lane) - 1u));
   if (valid && rank == 0) wc_s[warp][e] = __popc(peers);
@@ -283,11 +292,11 @@ __global__ void gather_rows_kernel(Dims d, const T* __restrict__ X, const int32_
 }
 
 cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,
-                            int32_t* perm, int2* rowmeta, const float* topk_w, cudaStream_t s) {
+                            int32_t* perm, int2* rowmeta, const float* topk_w, unsigned* st, cudaStream_t s) {
   const int nt = dispatch_tiles(d);
   int32_t* counts = (int32_t*)(ws + p.dcounts);
   int32_t* base = (int32_t*)(ws + p.dbase);
-  dispatch_count_kernel<<<nt, kDispatchThreads, 0, s>>>(d, idx, counts);
+  dispatch_count_kernel<<<nt, kDispatchThreads, 0, s>>>(d, idx, counts, st);
   dispatch_offsets_kernel<<<1, 1024, 0, s>>>(d, nt, counts, base, offsets, (int32_t*)(ws + p.tiles),
                                              (int32_t*)(ws + p.ntiles));
   dispatch_scatter_kernel<<<nt, kDispatchThreads, 0, s>>>(d, idx, base, perm, rowmeta, topk_w);

@@ -9,7 +9,8 @@
 // The array is a file-scope __device__ variable: every GPU that loads the library holds kScratchBytes of
 // it until the process exits.  In host code its name is only a host-side stand-in, so the device address
 // is fetched with cudaGetSymbolAddress once per device (the first call on a device does it, with that
-// device current) and handed to the kernels.  All calls share the array and it keeps the last call's
+// device current) and handed to the kernels.  The address is kept for the life of the process, so a
+// device reset (cudaDeviceReset) between calls is not supported.  All calls share the array and it keeps the last call's
 // contents; every word the kernels read is written earlier in the same call, so nothing has to be
 // cleared.  Two calls whose work overlaps on the GPU (different streams, or different host threads
 // without ordering) race on the array.
@@ -63,22 +64,20 @@ using namespace swimba;
 
 extern "C" swimba_status swimba_dispatch_noalloc(const swimba_dims* dims, const int32_t* topk_idx,
                                                  int32_t* expert_offsets, int32_t* perm, void* stream) {
-  if (!dims || !topk_idx || !expert_offsets || !perm) return SWIMBA_ERR_INVALID_ARG;
-  if (((uintptr_t)topk_idx | (uintptr_t)expert_offsets | (uintptr_t)perm) & 15u) return SWIMBA_ERR_INVALID_ARG;
-  // the same shape rules as every other entry point (swimba_workspace_size returns 0 on invalid dims)
-  if (swimba_workspace_size(dims) == 0) return SWIMBA_ERR_UNSUPPORTED;
-  const swimba_dims& s = *dims;
+  // the same dims rules and status codes as swimba_dispatch
   Dims d{};
-  d.Bsz = s.batch; d.T = s.seqlen; d.D = s.d_model; d.H = s.nheads; d.P = s.headdim; d.N = s.dstate;
-  d.G = s.ngroups; d.E = s.n_experts; d.k = s.top_k; d.Q = s.chunk; d.dtype = s.dtype;
-  d.M = s.batch * s.seqlen; d.HP = s.nheads * s.headdim; d.GN = s.ngroups * s.dstate; d.We = d.HP + 2 * d.GN;
-  d.nc = ceil_div(s.seqlen, s.chunk); d.hpg = s.nheads / s.ngroups;
+  const swimba_status ds = make_dims(dims, &d);
+  if (ds != SWIMBA_OK) return ds;
+  if (!topk_idx || !expert_offsets || !perm) return SWIMBA_ERR_INVALID_ARG;
+  if (((uintptr_t)topk_idx | (uintptr_t)expert_offsets | (uintptr_t)perm) & 15u) return SWIMBA_ERR_INVALID_ARG;
   WsPlan p;
   if (!scratch_plan(d, &p)) return SWIMBA_ERR_WORKSPACE;  // needs more than the fixed 1 MiB scratch
   char* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return SWIMBA_ERR_CUDA;
-  return launch_dispatch(d, topk_idx, p, scratch, expert_offsets, perm, nullptr, nullptr, (cudaStream_t)stream) ==
-                 cudaSuccess
+  unsigned* st = device_status();
+  if (!st) return SWIMBA_ERR_CUDA;
+  return launch_dispatch(d, topk_idx, p, scratch, expert_offsets, perm, nullptr, nullptr, st,
+                         (cudaStream_t)stream) == cudaSuccess
              ? SWIMBA_OK
              : SWIMBA_ERR_CUDA;
 }

@@ -13,7 +13,9 @@ namespace swimba {
 // swimba_check_device_status.  Host code only ever uses its device address (device_status()).
 __device__ unsigned g_status_word;
 
-static unsigned* device_status() {
+// The address is looked up once per device and kept for the life of the process (a device reset between
+// calls is not supported: it would reload the module and leave the kept address stale).
+unsigned* device_status() {
   static std::mutex mu;
   static unsigned* addr[64] = {};
   int dev = 0;
@@ -107,7 +109,7 @@ WsPlan plan_workspace(const Dims& d) {
 
 static bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
 
-static swimba_status make_dims(const swimba_dims* in, Dims* d) {
+swimba_status make_dims(const swimba_dims* in, Dims* d) {
   if (!in) return SWIMBA_ERR_INVALID_ARG;
   const swimba_dims& s = *in;
   if (s.batch < 1 || s.seqlen < 1 || s.d_model < 1 || s.nheads < 1 || s.headdim < 1 || s.dstate < 1 ||
@@ -269,8 +271,10 @@ swimba_status swimba_dispatch(const swimba_dims* dims, const int32_t* topk_idx, 
   if (!ok_ptr(topk_idx) || !ok_ptr(expert_offsets) || !ok_ptr(perm)) return SWIMBA_ERR_INVALID_ARG;
   SW_TRY(check_ws(d, ws, ws_bytes));
   WsPlan p = plan_workspace(d);
+  unsigned* st = device_status();
+  if (!st) return SWIMBA_ERR_CUDA;
   return cuda_status(
-      launch_dispatch(d, topk_idx, p, (char*)ws, expert_offsets, perm, nullptr, nullptr, (cudaStream_t)stream));
+      launch_dispatch(d, topk_idx, p, (char*)ws, expert_offsets, perm, nullptr, nullptr, st, (cudaStream_t)stream));
 }
 
 swimba_status swimba_expert_proj(const swimba_dims* dims, const void* X, const swimba_weights* w,
@@ -285,8 +289,10 @@ swimba_status swimba_expert_proj(const swimba_dims* dims, const void* X, const s
   cudaStream_t s = (cudaStream_t)stream;
   int32_t* offsets = (int32_t*)(b + p.offsets);
   int32_t* perm = (int32_t*)(b + p.perm);
-  SW_CUDA(launch_dispatch(d, topk_idx, p, b, offsets, perm, (int2*)(b + p.rowmeta), nullptr, s));
-  return run_proj(d, X, w->w_exp, b, p, nullptr, 2, nullptr, nullptr, nullptr, Z, device_status(), s);
+  unsigned* st = device_status();
+  if (!st) return SWIMBA_ERR_CUDA;
+  SW_CUDA(launch_dispatch(d, topk_idx, p, b, offsets, perm, (int2*)(b + p.rowmeta), nullptr, st, s));
+  return run_proj(d, X, w->w_exp, b, p, nullptr, 2, nullptr, nullptr, nullptr, Z, st, s);
 }
 
 swimba_status swimba_mix(const swimba_dims* dims, const float* Z, const float* topk_w, int32_t flags, void* Bpi,
@@ -510,6 +516,7 @@ swimba_status swimba_check_device_status(void* stream) {
   if (v && cudaMemset(st, 0, sizeof(v)) != cudaSuccess) return SWIMBA_ERR_CUDA;
   if (v & ST_TIMEOUT) return SWIMBA_ERR_TIMEOUT;
   if (v & ST_RANGE) return SWIMBA_ERR_RANGE;
+  if (v & ST_INDEX) return SWIMBA_ERR_INDEX;
   return SWIMBA_OK;
 }
 
@@ -548,6 +555,7 @@ const char* swimba_status_string(swimba_status s) {
     case SWIMBA_ERR_WORKSPACE: return "SWIMBA_ERR_WORKSPACE";
     case SWIMBA_ERR_TIMEOUT: return "SWIMBA_ERR_TIMEOUT";
     case SWIMBA_ERR_RANGE: return "SWIMBA_ERR_RANGE";
+    case SWIMBA_ERR_INDEX: return "SWIMBA_ERR_INDEX";
   }
   return "SWIMBA_UNKNOWN_STATUS";
 }

@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libswimba.so")
 F32, BF16, F16 = 0, 1, 2
 MIX_UNSCALED_B = 1
 STATUS = {0: "SWIMBA_OK", 1: "SWIMBA_ERR_INVALID_ARG", 2: "SWIMBA_ERR_UNSUPPORTED", 3: "SWIMBA_ERR_CUDA",
-          4: "SWIMBA_ERR_WORKSPACE", 5: "SWIMBA_ERR_TIMEOUT", 6: "SWIMBA_ERR_RANGE"}
+          4: "SWIMBA_ERR_WORKSPACE", 5: "SWIMBA_ERR_TIMEOUT", 6: "SWIMBA_ERR_RANGE", 7: "SWIMBA_ERR_INDEX"}
 EXPORTS = ("swimba_workspace_size", "swimba_stream_dtype", "swimba_router_topk", "swimba_dispatch",
            "swimba_expert_proj", "swimba_mix", "swimba_ssd_scan", "swimba_layer_fwd", "swimba_step",
            "swimba_separated_scan", "swimba_check_device_status", "swimba_status_string",

@@ -82,6 +82,20 @@ def test_invalid_dims(L, kw):
     w = swimba.Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
     rc = L.swimba_router_topk(ctypes.byref(d), fake, ctypes.byref(w), fake, fake, fake, None)
     assert rc == 1
+    # both dispatch entry points give the same code for the same invalid dims
+    assert L.swimba_dispatch(ctypes.byref(d), fake, fake, fake, fake, 1 << 40, None) == 1
+    assert L.swimba_dispatch_noalloc(ctypes.byref(d), fake, fake, fake, None) == 1
+
+
+@pytest.mark.parametrize("kw", BAD_DIMS)
+def test_dispatch_entry_points_agree_on_unsupported_dims(L, kw):
+    base = dict(batch=1, seqlen=64, d_model=128, nheads=2, headdim=64, dstate=16, ngroups=2, n_experts=4, top_k=2,
+                chunk=64, dtype=swimba.BF16)
+    base.update(kw)
+    d = swimba.dims(**base)
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.swimba_dispatch(ctypes.byref(d), fake, fake, fake, fake, 1 << 40, None) == 2
+    assert L.swimba_dispatch_noalloc(ctypes.byref(d), fake, fake, fake, None) == 2
 
 
 def test_null_misaligned_and_workspace_errors(L):
