@@ -103,3 +103,15 @@ def oracle_heads(inp, w, X, heads, forced=None, init=None):
     s = head_slice(inp, w, heads)
     return O.layer_fwd(X, s["W_r"], s["W_dt"], s["b_dt"], s["A"], s["W_exp"], s["H"], w.headdim, w.dstate,
                        s["G"], w.top_k, init=init, forced_idx=forced)
+
+
+def oracle_heads_blocked(inp, w, X, heads, forced=None, init=None, block=16):
+    """oracle_heads over many heads, a block of heads at a time (bounded fp64 weight copies): y
+    [B,T,len(heads),P], final [B,len(heads),N,P].  init, when given, is [B,len(heads),N,P]."""
+    ys, fins = [], []
+    for i in range(0, len(heads), block):
+        hb = heads[i:i + block]
+        r = oracle_heads(inp, w, X, hb, forced, None if init is None else init[:, i:i + block])
+        ys.append(r["y"])
+        fins.append(r["final"])
+    return dict(y=np.concatenate(ys, axis=2), final=np.concatenate(fins, axis=1))

@@ -7,7 +7,8 @@ import torch
 from oracle import swimba_oracle as O
 from parameter_space_moe_b200 import configs, inputs, swimba
 
-from .parity import (check_topk, device_weights, f64, oracle_heads, out_dtype, rel, to_np, tol_of)
+from .parity import (check_topk, device_weights, f64, oracle_heads, oracle_heads_blocked, out_dtype, rel, to_np,
+                     tol_of)
 
 pytestmark = pytest.mark.gpu
 
@@ -94,10 +95,18 @@ def test_layer_esweep_sampled(E):
     g = O.router_logits(X.reshape(w.M, -1), f64(inp["W_r"]))
     fl, forced = check_topk(to_np(idx), g, w.top_k)
     heads = [0, 13, 23]
-    ref = oracle_heads(inp, w, X, heads, forced.reshape(w.batch, w.seqlen, w.top_k) if fl.any() else None)
+    fr = forced.reshape(w.batch, w.seqlen, w.top_k) if fl.any() else None
+    ref = oracle_heads(inp, w, X, heads, fr)
     yg = to_np(y).reshape(w.batch, w.seqlen, w.nheads, w.headdim)[:, :, heads]
     assert rel(yg, ref["y"]) <= 2e-3
     assert rel(to_np(fin)[:, heads], ref["final"]) <= 2e-3
+    # every head of two of the four sequences (sequences are independent)
+    seqs = [1, 3]
+    ws = w.with_(batch=len(seqs))
+    refa = oracle_heads_blocked(inp, ws, X[seqs], list(range(w.nheads)), None if fr is None else fr[seqs])
+    ya = to_np(y).reshape(w.batch, w.seqlen, w.nheads, w.headdim)[seqs]
+    assert rel(ya, refa["y"]) <= 2e-3
+    assert rel(to_np(fin)[seqs], refa["final"]) <= 2e-3
 
 
 def test_chunk_size_invariance():

@@ -28,6 +28,28 @@ TC_Q64 = configs.BASE.with_(name="tc_Q64_ragged", batch=3, seqlen=201, d_model=1
 PAIR_GEMM = configs.BASE.with_(name="pair_gemm_E2", batch=2, seqlen=1600, d_model=256, nheads=4, n_experts=2,
                                chunk=128, seed=86)
 STAGE_CFGS = [configs.TINY_F32, SMALL_BF16, SMALL_G, TC_P128, TC_Q64, PAIR_GEMM, configs.BASE]
+# tensor-core scan (P = 64, N = 128): one key slot, a single partial sub-chunk, one head whose 16 sub-chunks chain
+# through the hand-off, more (sequence, head) rows than SMs; and long hand-off chains (32 or more 128-token
+# sub-chunks per sequence): two key slots with a ragged tail, one key slot, a single head whose 40 sub-chunks
+# all chain, and more head rows than SMs
+SCAN_K1 = configs.BASE.with_(name="scan_k1_ragged", batch=2, seqlen=333, d_model=128, nheads=3, n_experts=3, top_k=1,
+                             chunk=128, seed=88)
+SCAN_SHORT = configs.BASE.with_(name="scan_one_partial_sub_chunk", batch=3, seqlen=50, d_model=128, nheads=2,
+                                n_experts=4, chunk=128, seed=89)
+SCAN_CHAIN = configs.BASE.with_(name="scan_one_head_16_sub_chunks", batch=1, seqlen=2000, d_model=128, nheads=1,
+                                n_experts=4, chunk=256, seed=90)
+SCAN_WIDE = configs.BASE.with_(name="scan_200_heads", batch=2, seqlen=300, d_model=128, nheads=100, n_experts=2,
+                               chunk=256, seed=91)
+LONGCHAIN_K2 = configs.BASE.with_(name="longchain_k2_ragged", batch=2, seqlen=4500, d_model=128, nheads=2,
+                                  n_experts=4, chunk=256, seed=92)
+LONGCHAIN_K1 = configs.BASE.with_(name="longchain_k1", batch=1, seqlen=4200, d_model=128, nheads=3, n_experts=3,
+                                  top_k=1, chunk=128, seed=93)
+LONGCHAIN_ONE_HEAD = configs.BASE.with_(name="longchain_one_head_40_sub_chunks", batch=1, seqlen=5100, d_model=128,
+                                        nheads=1, n_experts=4, chunk=256, seed=94)
+LONGCHAIN_WIDE = configs.BASE.with_(name="longchain_160_heads", batch=2, seqlen=4100, d_model=128, nheads=80,
+                                    n_experts=2, chunk=256, seed=95)
+SCAN_CFGS = STAGE_CFGS + [SCAN_K1, SCAN_SHORT, SCAN_CHAIN, SCAN_WIDE, LONGCHAIN_K2, LONGCHAIN_K1, LONGCHAIN_ONE_HEAD,
+                          LONGCHAIN_WIDE]
 _cache = {}
 
 
@@ -115,6 +137,30 @@ def test_dispatch_is_stable_sort(w):
     np.testing.assert_array_equal(to_np(off), np.concatenate([[0], np.cumsum(np.bincount(flat, minlength=w.n_experts))]))
 
 
+def test_dispatch_skips_out_of_range_indices():
+    """Caller-given indices outside [0, E) are left out of the sort and reported as SWIMBA_ERR_INDEX; the
+    valid pairs are still sorted stably (the kernels index no table with the bad values)."""
+    w = configs.BASE.with_(batch=1, seqlen=3000, n_experts=8, top_k=2)
+    rng = np.random.default_rng(5)
+    idx_np = np.stack([rng.permutation(w.n_experts)[:w.top_k] for _ in range(w.M)]).astype(np.int32)
+    bad = rng.choice(w.M * w.top_k, size=37, replace=False)
+    flat = idx_np.reshape(-1)
+    flat[bad[:20]] = 99
+    flat[bad[20:]] = -3
+    d = swimba.dims_of(w)
+    off = torch.empty(w.n_experts + 1, dtype=torch.int32, device="cuda")
+    perm = torch.full((w.M * w.top_k,), -7, dtype=torch.int32, device="cuda")
+    swimba.dispatch(d, torch.from_numpy(idx_np).cuda(), off, perm, _ws(d))
+    assert swimba.check_device_status() == 7
+    assert swimba.check_device_status() == 0
+    ok = (flat >= 0) & (flat < w.n_experts)
+    want = np.nonzero(ok)[0][np.argsort(flat[ok], kind="stable")]
+    n = int(ok.sum())
+    np.testing.assert_array_equal(to_np(off), np.concatenate([[0], np.cumsum(np.bincount(flat[ok], minlength=8))]))
+    np.testing.assert_array_equal(to_np(perm)[:n], want)
+    assert (to_np(perm)[n:] == -7).all()
+
+
 @pytest.mark.parametrize("w", STAGE_CFGS, ids=lambda w: w.name)
 def test_expert_proj_and_mix(w):
     inp, Xf, ref, dev = _setup(w)
@@ -151,7 +197,7 @@ def _oracle_streams_on_device(w, ref):
     return Bpi, Xs, Cpi, dt
 
 
-@pytest.mark.parametrize("w", STAGE_CFGS, ids=lambda w: w.name)
+@pytest.mark.parametrize("w", SCAN_CFGS, ids=lambda w: w.name)
 @pytest.mark.parametrize("with_init", [False, True])
 def test_ssd_scan(w, with_init):
     inp, Xf, ref, dev = _setup(w)
@@ -183,7 +229,7 @@ def test_ssd_scan(w, with_init):
         assert rel(to_np(cst)[b].transpose(1, 0, 2, 3), Hs) < state_tol_of(w)
 
 
-@pytest.mark.parametrize("w", [configs.TINY_F32, TC_P128, TC_Q64], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [configs.TINY_F32, TC_P128, TC_Q64, LONGCHAIN_K2], ids=lambda w: w.name)
 def test_separated_scan(w):
     """The separated design ("k scans"): k trajectories with unscaled injections, pi-scaled readouts."""
     inp, Xf, ref, dev = _setup(w)
@@ -207,13 +253,14 @@ def test_separated_scan(w):
         assert rel(to_np(fin)[:, b], hs) < state_tol_of(w)
 
 
-def test_scan_lost_predecessor_times_out_without_fault():
+@pytest.mark.parametrize("seqlen", [512, 4200], ids=["T512", "T4200"])
+def test_scan_lost_predecessor_times_out_without_fault(seqlen):
     """Failure detection: the first sub-chunk of every head is made to go missing, so the successors'
     flag waits can never succeed.  They give up after their bounded wait, the status word reports
     SWIMBA_ERR_TIMEOUT (no fault, no hang), and the context stays usable: the normal scan that follows
     is correct."""
     import time
-    w = configs.BASE.with_(name="lost_chunk", batch=1, seqlen=512, d_model=128, nheads=2, seed=87)
+    w = configs.BASE.with_(name=f"lost_chunk_T{seqlen}", batch=1, seqlen=seqlen, d_model=128, nheads=2, seed=87)
     inp, Xf, ref, dev = _setup(w)
     d = swimba.dims_of(w)
     Bpi, Xs, Cpi, dt = (t.cuda() for t in _oracle_streams_on_device(w, ref))
