@@ -8,6 +8,11 @@ layer B4 T2048 D768 H24 P64 N128 E8 k2 Q256 (bf16 weights and activations, fp32 
 (torchrun) every rank runs its own batch (weak scaling, no data-path collective; the process group only
 carries the barrier and the max-over-ranks of the timings).
 
+On one GPU the default run adds two nested measurements to the same JSON line, timed the same way:
+"decode" (swimba_step on 256 sequences, D2048 H64 N128 P64 E16 k2, state from a 512-token prefill; bound
+by HBM) and "esweep" (the base layer at E in {8, 16, 32, 64}: layer and scan-stage times, which the
+method's cost statement says are flat in E, plus the separated-trajectory scan that runs k trajectories).
+
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launching stream,
 with a write of 2x the L2 size between steps (outside the events) so every step reads its inputs from
 HBM.  A second pass of K steps with the library's own per-stage events on gives the stage breakdown and
@@ -46,10 +51,19 @@ def load_peaks():
 
 # ------------------------------------------------------------------------------------------ work model
 
+def scan_chunk_of(w):
+    """Chunk length the scan actually solves in: the tensor-core scan (bf16, N = 128, P in {64, 128})
+    always uses 128-token sub-chunks; the CUDA-core scan uses the workload's chunk."""
+    if w.dtype == "bf16" and w.dstate == 128 and w.headdim in (64, 128):
+        return 128
+    return w.chunk
+
+
 def ssd_flops(w, T=None):
-    """Algorithmic FLOPs of the chunked solve (causal half of the intra-chunk products counted)."""
+    """Algorithmic FLOPs of the chunked solve at the chunk length the kernel runs (causal half of the
+    intra-chunk products counted)."""
     T = T or w.seqlen
-    Q, k, N, P = w.chunk, w.top_k, w.dstate, w.headdim
+    Q, k, N, P = scan_chunk_of(w), w.top_k, w.dstate, w.headdim
     total = 0
     for c in range(math.ceil(T / Q)):
         L = min(Q, T - c * Q)
@@ -345,27 +359,10 @@ def job_throughput(tokens_per_rank, world, steps, total_ms):
     return tokens_per_rank * world * steps / (total_ms / 1e3)
 
 
-def run_gpu(args, w):
-    from parameter_space_moe_b200 import swimba
-    rank, world, local = rank_env()
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    swimba.lib()
-    wr = rank_workload(w, rank)
-    inp = inputs.make_inputs(wr)
-    sess = (DecodeSession if w.prefill else LayerSession)(w, dev, inp, swimba)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
+def measure(sess, args, flush, stream, dist, local, swimba, e2e=True):
+    """Warm-up, then K device-timed steps (L2 flushed between steps, outside the events), a second pass of K
+    steps with the library's stage events on (so the headline carries no profiling events), and K end-to-end
+    steps through the host-memory entry point.  Times are this rank's totals in milliseconds."""
     for _ in range(args.warmup):
         sess.step()
     torch.cuda.synchronize()
@@ -390,8 +387,6 @@ def run_gpu(args, w):
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     assert swimba.check_device_status() == 0
 
-    # per-stage breakdown: the same steps again with the library's stage events on (a separate pass, so
-    # the headline above carries no profiling events)
     stage_ms = {}
     swimba.profile_enable(True)
     for i in range(args.steps):
@@ -402,40 +397,108 @@ def run_gpu(args, w):
     torch.cuda.synchronize()
     swimba.profile_enable(False)
 
-    # end to end through the C ABI: pinned host input in, output back to pinned host, every step
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for _ in range(2):
-        sess.e2e_step()
-    torch.cuda.synchronize()
-    e2e_ms = 0.0
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        e0.record(stream)
-        sess.e2e_step()
-        e1.record(stream)
-        e1.synchronize()
-        e2e_ms += e0.elapsed_time(e1)
+    e2e_ms = None
+    if e2e:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(2):
+            sess.e2e_step()
+        torch.cuda.synchronize()
+        e2e_ms = 0.0
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            e0.record(stream)
+            sess.e2e_step()
+            e1.record(stream)
+            e1.synchronize()
+            e2e_ms += e0.elapsed_time(e1)
+    assert swimba.check_device_status() == 0
+    return {"total_ms": total_ms, "stage_ms": stage_ms, "launches": launches, "clocks": sampler.summary(),
+            "e2e_ms": e2e_ms}
+
+
+def esweep_measure(args, dev, flush, stream, swimba):
+    """The base layer at E in {8, 16, 32, 64}: per-step layer and stage times (the scan's work does not
+    depend on E), plus the separated-trajectory scan ("k scans") at E = 8 on the same streams."""
+    out = {"E": [], "layer_ms": [], "scan_ms": [], "expert_proj_ms": [], "scan_roofline_frac": []}
+    peaks, _ = load_peaks()
+    for E in configs.ESWEEP_E:
+        w = configs.esweep(E)
+        sess = LayerSession(w, dev, inputs.make_inputs(w), swimba)
+        m = measure(sess, args, flush, stream, None, dev.index or 0, swimba, e2e=False)
+        K = args.steps
+        scan_s = m["stage_ms"].get("ssd_scan", 0.0) / K / 1e3
+        out["E"].append(E)
+        out["layer_ms"].append(m["total_ms"] / K)
+        out["scan_ms"].append(scan_s * 1e3)
+        out["expert_proj_ms"].append(m["stage_ms"].get("expert_proj_mix", 0.0) / K)
+        out["scan_roofline_frac"].append(sess.work["ssd_scan"]["bytes"] / scan_s / 1e9 / peaks["hbm_gbs"])
+        if E == configs.ESWEEP_E[0]:
+            sep = sess.extras(stream, args.steps)
+            out["separated_scan_ms"] = sep["separated_scan_ms"]
+            out["trajectories"] = {"mixed": sep["mixed_trajectories"], "separated": sep["separated_trajectories"]}
+        del sess
+        torch.cuda.empty_cache()
+    out["scan_ms_spread"] = max(out["scan_ms"]) / min(out["scan_ms"]) - 1.0
+    return out
+
+
+def run_gpu(args, w):
+    from parameter_space_moe_b200 import swimba
+    rank, world, local = rank_env()
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    swimba.lib()
+    wr = rank_workload(w, rank)
+    inp = inputs.make_inputs(wr)
+    sess = (DecodeSession if w.prefill else LayerSession)(w, dev, inp, swimba)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    m = measure(sess, args, flush, stream, dist, local, swimba)
     extras = sess.extras(stream, args.steps) if args.separated else {}
 
-    t = max_over_ranks([total_ms, e2e_ms] + [stage_ms.get(n, 0.0) for n in sorted(stage_ms)], dist, dev)
-    total_ms, e2e_ms = t[0], t[1]
-    stage_ms = {n: t[2 + i] for i, n in enumerate(sorted(stage_ms))}
+    t = max_over_ranks([m["total_ms"], m["e2e_ms"]] + [m["stage_ms"].get(n, 0.0) for n in sorted(m["stage_ms"])],
+                       dist, dev)
+    m["total_ms"], m["e2e_ms"] = t[0], t[1]
+    m["stage_ms"] = {n: t[2 + i] for i, n in enumerate(sorted(m["stage_ms"]))}
+    out = summarize(args, w, sess, world, m, inp, extras)
+    # one GPU, default workload: the decode step and the expert-count sweep in the same line
+    if world == 1 and w.name == configs.BASE.name and not args.no_extras:
+        del sess
+        torch.cuda.empty_cache()
+        dw = configs.DECODE
+        dsess = DecodeSession(dw, dev, inputs.make_inputs(dw), swimba)
+        dm = measure(dsess, args, flush, stream, None, local, swimba)
+        d = summarize(args, dw, dsess, 1, dm, None, {})
+        out["decode"] = {k: d[k] for k in ("metric", "value", "unit", "ms_per_step", "config", "roofline",
+                                           "layer_roofline", "stages_ms_per_step", "e2e", "gpu_launches", "clocks")}
+        del dsess
+        torch.cuda.empty_cache()
+        out["esweep"] = esweep_measure(args, dev, flush, stream, swimba)
     if rank == 0:
-        report(args, w, sess, world, total_ms, e2e_ms, stage_ms, launches, sampler.summary(),
-               sess.Xh.numel() * sess.Xh.element_size(), sess.yh.numel() * sess.yh.element_size(), inp, extras)
+        if world == 1 and not args.no_cpu_baseline and not w.prefill:
+            v, sample = cpu_oracle_sample(w, inp)
+            out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                   "sample": sample}
+        print(json.dumps(out))
     if dist:
         dist.barrier()
         dist.destroy_process_group()
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, bytes per launch) of a stage's kernel from one
-# ncu capture of the current kernel build, with the summary it comes from; a stage/workload not listed
-# reports null.  An entry is removed whenever its kernel changes.
-PROFILED_TRAFFIC = {
-    ("base_B4_T2048_D768_H24_E8_k2", "expert_proj_mix"): (326.7e6, "profiles/proj_tc_base_B4_T2048_D768_H24_E8_k2.md"),
-    ("base_B4_T2048_D768_H24_E8_k2", "ssd_scan"): (304.2e6, "profiles/scan_tc_base_B4_T2048_D768_H24_E8_k2.md"),
-    ("base_B4_T2048_D768_H24_E8_k2", "router"): (12.7e6, "profiles/router_tc_base_B4_T2048_D768_H24_E8_k2.md"),
-}
+# ncu capture of the current kernel build; a stage/workload not listed reports null.  An entry is removed
+# whenever its kernel changes.
+PROFILED_TRAFFIC = {}
 
 
 def tensor_peak(peaks, clocks):
@@ -457,42 +520,40 @@ def stage_roofline(model, secs, peaks, tpeak):
     return "hbm", model["bytes"] / secs / 1e9, peaks["hbm_gbs"], "GB/s", model["bytes"]
 
 
-def report(args, w, sess, world, total_ms, e2e_ms, stage_ms, launches, clocks, h2d, d2h, inp, extras):
+def summarize(args, w, sess, world, m, inp, extras):
+    """The JSON object of one measured workload (the headline fields of the bench contract)."""
     peaks, src = load_peaks()
     wk = sess.work
     K = args.steps
+    total_ms, e2e_ms, stage_ms, clocks = m["total_ms"], m["e2e_ms"], m["stage_ms"], m["clocks"] or {}
     tokens = sess.tokens * world * K
     value = job_throughput(sess.tokens, world, K, total_ms)
     # dominant kernel stage (among those with a work model) and its roofline
     dom = max((n for n in stage_ms if n in wk), key=stage_ms.get)
     avg_s = stage_ms[dom] / K / 1e3
     tpeak, tkind = tensor_peak(peaks, clocks)
-    traffic = PROFILED_TRAFFIC.get((w.name, dom))
     bound, achieved, peak, unit, alg = stage_roofline(wk[dom], avg_s, peaks, tpeak)
     peak_note = (f"bf16 dense, {tkind}, {src}" if bound == "tensor" else f"HBM copy, {src}")
     roof_s = max(wk["layer"]["flops"] / (tpeak * 1e12), wk["layer"]["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    h2d = sess.Xh.numel() * sess.Xh.element_size()
+    d2h = sess.yh.numel() * sess.yh.element_size()
     out = {
         "metric": sess.metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic", "config": config_of(w),
         "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": traffic[0] if traffic else None,
-                     "traffic_source": traffic[1] if traffic else None, "peak_source": peak_note,
-                     "algorithmic": alg},
+                     "frac": achieved / peak, "traffic": PROFILED_TRAFFIC.get((w.name, dom)),
+                     "peak_source": peak_note, "algorithmic": alg},
         "layer_roofline": {"time_us": roof_s * 1e6, "frac": roof_s / (total_ms / K / 1e3),
                            "flops": wk["layer"]["flops"], "bytes": wk["layer"]["bytes"]},
         "stages_ms_per_step": {n: v / K for n, v in stage_ms.items()},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches,
-        "clocks": clocks,
+        "gpu_launches": m["launches"],
+        "clocks": m["clocks"],
     }
     out.update(extras)
-    if world == 1 and not args.no_cpu_baseline and not w.prefill:
-        v, sample = cpu_oracle_sample(w, inp)
-        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                               "sample": sample}
-    print(json.dumps(out))
+    return out
 
 
 def main():
@@ -505,6 +566,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--separated", action="store_true",
                     help="also time the separated-trajectory scan (k scans) on the layer's streams")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="default workload on one GPU: skip the nested decode and expert-count sweep measurements")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = configs.ALL[args.workload]
