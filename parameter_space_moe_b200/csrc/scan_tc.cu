@@ -132,6 +132,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__
     tc::mbar_init(hbar, 1);
     tc::mbar_init(fullC, 1);
     tc::fence_barrier_init();
+    // the ticket counter and flags are cleared by earlier work in the stream: the ticket is taken once the
+    // grid launched before this one has completed, so every earlier write is visible
+    griddep_wait();
     misc[1] = atomicAdd(a.ticket, 1u);
   }
   if (warp == 0) { tc::tmem_alloc(&misc[0], TMEM_COLS); tc::tmem_relinquish(); }
