@@ -477,9 +477,11 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       tc::fence_after_sync();
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 32 * ch0);
       drain_tile(a, taddr, ct * BN + 32 * ch0, nch, valid, meta, epi_stage, lane, range_bad);
+      // the accumulator's TMEM reads are complete (tcgen05.wait::ld) and ordered by the tcgen05 fence; the
+      // tile's global stores need not be visible to the even CTA, so the arrival is relaxed
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive_cluster(acc_empty0 + 8u * (uint32_t)buf);
+      if (lane == 0) tc::mbar_arrive_cluster_relaxed(acc_empty0 + 8u * (uint32_t)buf);
       if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
     }
     if (range_bad) atomicOr(a.st, ST_RANGE);
@@ -508,9 +510,10 @@ cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaError_t e;
-  // CTA pairs when experts average at least 3072 rows: each expert's last pair tile is partly past its
-  // rows, and below that the 256-row tiles waste more tensor time than the pairs save
-  if ((long long)d.M * d.k >= 3072LL * d.E) {
+  // CTA pairs when experts average at least 1536 rows: each expert's last pair tile is partly past its
+  // rows, and below that the 256-row tiles waste more tensor time than the pairs' lower operand traffic
+  // (a third less per FLOP from L2) saves
+  if ((long long)d.M * d.k >= 1536LL * d.E) {
     // CTA pairs: A boxes of 128 rows (the pair's two halves), B boxes of 128 weight rows
     CUtensorMap tb2;
     if (!encode_tmap_2d(&tb2, w_exp, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.E * d.We, (uint64_t)d.D * 2, BK, 128))

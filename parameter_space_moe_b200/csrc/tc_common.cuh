@@ -174,6 +174,12 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// The same arrival without release semantics: for signals that order only tcgen05 work (ordered by the
+// tcgen05 fences around the synchronisation), so that the arrival does not first wait for this thread's
+// outstanding global stores to become visible to the whole cluster.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 
 // ------------------------------------------------------------------------------------------ CTA pairs
 // tcgen05 with cta_group::2: the two CTAs of a cluster of 2 act as one pair.  TMEM is allocated and freed

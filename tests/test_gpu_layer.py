@@ -65,7 +65,7 @@ BF16_VARIANTS = [
     configs.BASE.with_(name="bf16_P128_N64", batch=1, seqlen=300, d_model=128, nheads=2, headdim=128, dstate=64,
                        chunk=64, seed=22),
     configs.BASE.with_(name="bf16_G2", batch=1, seqlen=400, d_model=256, nheads=4, ngroups=2, chunk=128, seed=23),
-    # CTA-pair expert GEMM (>= 3072 rows per expert on average); the second has a ragged last column tile
+    # CTA-pair expert GEMM (>= 1536 rows per expert on average); the second has a ragged last column tile
     configs.BASE.with_(name="bf16_pair_gemm", batch=2, seqlen=1600, d_model=256, nheads=4, n_experts=2, seed=24),
     configs.BASE.with_(name="bf16_pair_ragged_cols", batch=3, seqlen=3100, d_model=192, nheads=3, dstate=64,
                        ngroups=1, n_experts=3, top_k=1, chunk=128, seed=25),

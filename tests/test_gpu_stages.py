@@ -24,7 +24,7 @@ TC_P128 = configs.BASE.with_(name="tc_P128_k3_G2", batch=2, seqlen=333, d_model=
                              dstate=128, ngroups=2, n_experts=5, top_k=3, chunk=128, seed=79)
 TC_Q64 = configs.BASE.with_(name="tc_Q64_ragged", batch=3, seqlen=201, d_model=128, nheads=2, n_experts=4,
                             chunk=64, seed=80)
-# enough rows per expert (>= 3072 on average) for the CTA-pair expert GEMM, ragged expert tails
+# enough rows per expert (>= 1536 on average) for the CTA-pair expert GEMM, ragged expert tails
 PAIR_GEMM = configs.BASE.with_(name="pair_gemm_E2", batch=2, seqlen=1600, d_model=256, nheads=4, n_experts=2,
                                chunk=128, seed=86)
 STAGE_CFGS = [configs.TINY_F32, SMALL_BF16, SMALL_G, TC_P128, TC_Q64, PAIR_GEMM, configs.BASE]
