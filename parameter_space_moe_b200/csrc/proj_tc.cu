@@ -256,12 +256,10 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         if (!tc::mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
         const uint32_t sa = tc::smem_u32(stage_base + stage * kStageBytes);
-        const uint32_t sb = sa + kStageA;
+        const uint64_t da = tc::sdesc_kmajor_sw128(sa), db = tc::sdesc_kmajor_sw128(sa + kStageA);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          tc::mma_f16(dt, tc::sdesc_kmajor_sw128(sa + kk * 32), tc::sdesc_kmajor_sw128(sb + kk * 32), kIdesc,
-                      (kb | kk) != 0);
-        }
+        for (int kk = 0; kk < BK / 16; ++kk)  // K16 step: +32 bytes = +2 in the descriptor's address field
+          tc::mma_f16(dt, da + 2 * kk, db + 2 * kk, kIdesc, (kb | kk) != 0);
         tc::mma_commit(&empty[stage]);
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
@@ -432,12 +430,10 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         if (!tc::mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
         tc::fence_after_sync();
         const uint32_t sa = tc::smem_u32(stage_base + stage * kPairStageBytes);
-        const uint32_t sb = sa + kPairStageA;
+        const uint64_t da = tc::sdesc_kmajor_sw128(sa), db = tc::sdesc_kmajor_sw128(sa + kPairStageA);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          tc::mma_f16_pair(dt, tc::sdesc_kmajor_sw128(sa + kk * 32), tc::sdesc_kmajor_sw128(sb + kk * 32), kPairIdesc,
-                           (kb | kk) != 0);
-        }
+        for (int kk = 0; kk < BK / 16; ++kk)  // K16 step: +32 bytes = +2 in the descriptor's address field
+          tc::mma_f16_pair(dt, da + 2 * kk, db + 2 * kk, kPairIdesc, (kb | kk) != 0);
         tc::mma_commit_pair(&empty[stage], 0x3);
         if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
       }
