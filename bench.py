@@ -10,8 +10,9 @@ carries the barrier and the max-over-ranks of the timings).
 
 On one GPU the default run adds two nested measurements to the same JSON line, timed the same way:
 "decode" (swimba_step on 256 sequences, D2048 H64 N128 P64 E16 k2, state from a 512-token prefill; bound
-by HBM) and "esweep" (the base layer at E in {8, 16, 32, 64}: layer and scan-stage times, which the
-method's cost statement says are flat in E, plus the separated-trajectory scan that runs k trajectories).
+by HBM), "esweep" (the base layer at E in {8, 16, 32, 64}: layer and scan-stage times, which the
+method's cost statement says are flat in E, plus the separated-trajectory scan that runs k trajectories) and
+"out_proj" (the output projection y W_out^T on the base layer's y, bound by the tensor cores).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launching stream,
 with a write of 2x the L2 size between steps (outside the events) so every step reads its inputs from
@@ -442,6 +443,37 @@ def esweep_measure(args, dev, flush, stream, swimba):
     return out
 
 
+def out_proj_measure(args, sess, inp, flush, stream, swimba):
+    """The output projection out = y W_out^T (swimba_out_proj) on the layer's own y, timed alone: K launches
+    between L2 flushes, against the burst bf16 peak (a kernel timed alone)."""
+    w = sess.w
+    W_out = inp["W_out"].to(sess.X.device)
+    out = torch.empty(w.M, w.d_model, dtype=sess.y.dtype, device=sess.X.device)
+    for _ in range(max(args.warmup, 3)):
+        swimba.out_proj(sess.d, sess.y, W_out, out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tot = 0.0
+    for _ in range(args.steps):
+        flush.fill_(1)
+        e0.record(stream)
+        swimba.out_proj(sess.d, sess.y, W_out, out)
+        e1.record(stream)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    if swimba.check_device_status() != 0:
+        raise RuntimeError("swimba_out_proj raised a device status")
+    peaks, src = load_peaks()
+    HP = w.nheads * w.headdim
+    flops = 2.0 * w.M * w.d_model * HP
+    nbytes = (w.M * HP + w.d_model * HP + w.M * w.d_model) * out.element_size()
+    secs = tot / args.steps / 1e3
+    return {"ms": secs * 1e3, "shape": f"[{w.M} x {HP}] x [{HP} x {w.d_model}]", "flops": flops, "bytes": nbytes,
+            "roofline": {"bound": "tensor", "achieved": flops / secs / 1e12, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": flops / secs / 1e12 / peaks["bf16_tflops"],
+                         "peak_source": f"bf16 dense, burst, {src}"}}
+
+
 def run_gpu(args, w):
     from parameter_space_moe_b200 import swimba
     rank, world, local = rank_env()
@@ -473,6 +505,7 @@ def run_gpu(args, w):
     out = summarize(args, w, sess, world, m, inp, extras)
     # one GPU, default workload: the decode step and the expert-count sweep in the same line
     if world == 1 and w.name == configs.BASE.name and not args.no_extras:
+        out["out_proj"] = out_proj_measure(args, sess, inp, flush, stream, swimba)
         del sess
         torch.cuda.empty_cache()
         dw = configs.DECODE

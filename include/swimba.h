@@ -204,6 +204,18 @@ swimba_status swimba_separated_scan(const swimba_dims* dims, const void* B, cons
                                     const float* dt, const float* A, const float* init_states, void* y,
                                     float* final_states, void* ws, size_t ws_bytes, void* stream);
 
+/* The layer's output projection: out = y W_out^T, one projection shared by every expert (the layer has one
+ * recurrence and one readout).  Paper: gist.science Technical Summary, Architecture Details (the shared
+ * recurrence "followed by a single output projection").
+ *   y      [M][H*P] dtype in, as written by swimba_layer_fwd / swimba_ssd_scan / swimba_step
+ *   w_out  [D][H*P] dtype in (D = d_model)
+ *   out    [M][D] dtype out
+ * Only batch*seqlen, nheads*headdim, d_model and dtype are read from `dims`; the other fields must still be
+ * valid.  bf16: tensor cores, bf16 operands, fp32 accumulation, one rounding to bf16 per output.  fp32: CUDA
+ * cores in fp32.  Needs no workspace; y and out must not overlap.  Pointers must be non-NULL and 16-byte
+ * aligned (SWIMBA_ERR_INVALID_ARG otherwise). */
+swimba_status swimba_out_proj(const swimba_dims* dims, const void* y, const void* w_out, void* out, void* stream);
+
 /* Synchronises `stream`, then reads and clears the current device's status word: SWIMBA_OK,
  * SWIMBA_ERR_TIMEOUT, SWIMBA_ERR_RANGE or SWIMBA_ERR_INDEX, in that order of precedence (SWIMBA_ERR_CUDA
  * if the stream reports an error).  The word is sticky: it collects every flag raised on this device

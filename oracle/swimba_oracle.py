@@ -288,6 +288,17 @@ def layer_fwd(X, W_r, W_dt, b_dt, A, W_exp, H, P, N, G, k, init=None, forced_idx
     return dict(y=y, final=final, g=g, dt=dt, idx=idx, w=w, z=z, Bpi=Bpi, Xs=Xs, Ct=Ct, Cpi=Cpi)
 
 
+def out_proj(y, W_out):
+    """out_t = W_out y_t: the one output projection that follows the shared recurrence's readout
+    ([gist] Architecture Details).  There is one recurrence, so one projection, shared by all experts.
+
+    y [..., H*P] with the heads flattened head-major (y[..., h*P + p]), W_out [D, H*P]; returns [..., D].
+    Reading: a plain linear map without bias, applied to y as the readout returns it; the pages name no
+    gate, normalisation or skip term before it, so none is applied.
+    """
+    return np.asarray(y) @ np.asarray(W_out).T
+
+
 def step(Xt, W_r, W_dt, b_dt, A, W_exp, H, P, N, G, k, state, forced_idx=None, decision_dtype=np.float32):
     """One recurrent decode step per sequence: the layer applied to a single new token X_t [B,D]
     with the cached state [B,H,N,P] (the recurrence of [notes] key design 1 advanced by one token).

@@ -130,6 +130,8 @@ cudaError_t launch_proj_simt(const Dims& d, const void* X, const void* w_exp, co
 cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int2* rowmeta,
                            const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, int mode, void* bpi,
                            void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s);
+cudaError_t launch_out_proj(const Dims& d, const void* y, const void* w_out, void* out, unsigned* st,
+                            cudaStream_t s);
 cudaError_t launch_mix(const Dims& d, const float* Z, const float* topk_w, int flags, void* bpi, void* xs, void* cpi,
                        unsigned* st, cudaStream_t s);
 // Chunked scan.  Slot ranges select which of the k per-token keys feed one trajectory and which

@@ -42,12 +42,14 @@ struct TcArgs {
   const int32_t* tiles;
   const int32_t* ntiles;
   const int32_t* offsets;
-  int mode;  // 0 mix, 1 mix with unscaled B, 2 raw fp32 Z
+  int mode;  // 0 mix, 1 mix with unscaled B, 2 raw fp32 Z, 3 plain bf16 product (the output projection)
+  int dense;  // 1: one operand group over rows 0 .. M-1 in order (no dispatch schedule, offsets or row metadata)
   __half* bpi;
   __half* xs;
   __half* cpi;
   float* Z;
   unsigned* st;
+  __nv_bfloat16* out;  // mode 3: [M][We] bf16
 };
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
@@ -149,6 +151,41 @@ __device__ __forceinline__ void store_group32(const TcArgs& a, uint8_t* stage, i
   __syncwarp();
 }
 
+// Mode 3: one warp stores 32 columns of its 32 rows of the plain product as bf16 (row-major [M][We]), staged
+// through shared memory so that every store instruction writes 8 whole 64-byte row segments; a ragged last
+// column group is stored per thread.
+__device__ __forceinline__ void store_dense32(const TcArgs& a, uint8_t* stage, int lane, bool valid, int row, int c0,
+                                              const uint32_t (&r)[32]) {
+  const int N = a.d.We;
+  if (c0 + 32 > N) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)  // constant indices keep r in registers
+      if (valid && c0 + i < N) a.out[(size_t)row * N + c0 + i] = __float2bfloat16_rn(u2f(r[i]));
+    return;
+  }
+  uint8_t* my = stage + lane * kStageRow;
+#pragma unroll
+  for (int i = 0; i < 32; i += 8) {
+    uint4 v;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(u2f(r[i + 2 * q]), u2f(r[i + 2 * q + 1]));
+      w[q] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(my + 2 * i) = v;
+  }
+  __syncwarp();
+  const unsigned long long dptr = valid ? reinterpret_cast<unsigned long long>(a.out + (size_t)row * N + c0) : 0ull;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int rr = 8 * it + (lane >> 2), chunk = lane & 3;
+    const unsigned long long rd = __shfl_sync(0xffffffffu, dptr, rr);
+    if (rd) *reinterpret_cast<uint4*>(rd + 16 * chunk) = *reinterpret_cast<const uint4*>(stage + rr * kStageRow + 16 * chunk);
+  }
+  __syncwarp();
+}
+
 // One epilogue warp drains its 32 accumulator rows x nch 32-column chunks (starting at output column col0)
 // of a tile: the TMEM load of the next chunk is in flight while the current one is converted and stored.
 __device__ __forceinline__ void drain_tile(const TcArgs& a, uint32_t taddr, int col0, int nch, bool valid, int2 meta,
@@ -165,6 +202,10 @@ __device__ __forceinline__ void drain_tile(const TcArgs& a, uint32_t taddr, int 
     tc::tmem_ld_wait(cur);
     if (c + 1 < nch) tc::tmem_ld_32x32b_x32(taddr + 32 * (c + 1), nxt);
     const int c0 = col0 + 32 * c;
+    if (a.mode == 3) {
+      store_dense32(a, stage, lane, valid, meta.x, c0, cur);
+      continue;
+    }
     float sc_probe;
     // fast path: the warp's 32-column group lies in one fp16 stream for every valid row
     const bool fast = a.mode != 2 && c0 + 32 <= d.We &&
@@ -193,7 +234,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Dims& d = a.d;
   const int nct = ceil_div(d.We, BN);
-  const int nkb = d.D / BK;
+  const int nkb = ceil_div(d.D, BK);  // a dense product's ragged K tail is zero-filled by TMA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
@@ -207,12 +248,16 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
   griddep_launch_dependents();
   if (warp == 1) { tc::tmem_alloc(tmem_slot, kTmemCols); tc::tmem_relinquish(); }
   griddep_wait();  // the dispatch's offsets and schedule, the gathered rows
-  for (int e = threadIdx.x; e <= d.E; e += blockDim.x) off_s[e] = a.offsets[e];
+  if (a.dense) {
+    if (threadIdx.x == 0) { off_s[0] = 0; off_s[1] = d.M; }
+  } else {
+    for (int e = threadIdx.x; e <= d.E; e += blockDim.x) off_s[e] = a.offsets[e];
+  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int total = *a.ntiles * nct;
+  const int total = (a.dense ? ceil_div(d.M, BM) : *a.ntiles) * nct;
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -222,7 +267,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const int rt = t / nct, ct = t % nct;
-      const int e = a.tiles[2 * rt], row0 = a.tiles[2 * rt + 1];
+      const int e = a.dense ? 0 : a.tiles[2 * rt], row0 = a.dense ? rt * BM : a.tiles[2 * rt + 1];
       const int wrow = e * d.We + ct * BN;
       for (int kb = 0; kb < nkb; ++kb) {
         if (!tc::mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
@@ -282,14 +327,17 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     uint32_t acc_phase = 0;
     bool range_bad = false;
     int t = blockIdx.x;
-    int2 tinfo = t < total ? *reinterpret_cast<const int2*>(a.tiles + 2 * (t / nct)) : make_int2(0, 0);
+    auto tile_info = [&](int tt) {
+      return a.dense ? make_int2(0, (tt / nct) * BM) : *reinterpret_cast<const int2*>(a.tiles + 2 * (tt / nct));
+    };
+    int2 tinfo = t < total ? tile_info(t) : make_int2(0, 0);
     for (; t < total; t += gridDim.x) {
       const int ct = t % nct;
       const int e = tinfo.x, row0 = tinfo.y;
       const bool valid = row0 + row_local < off_s[e + 1];
-      const int2 meta = valid ? a.rowmeta[row0 + row_local] : make_int2(0, 0);
+      const int2 meta = !valid ? make_int2(0, 0) : (a.dense ? make_int2(row0 + row_local, 0) : a.rowmeta[row0 + row_local]);
       const int tn = t + gridDim.x;
-      if (tn < total) tinfo = *reinterpret_cast<const int2*>(a.tiles + 2 * (tn / nct));
+      if (tn < total) tinfo = tile_info(tn);
       if (!tc::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) {
         *abort_flag = 1;
         atomicOr(a.st, ST_TIMEOUT);
@@ -501,7 +549,7 @@ cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp
     return cudaErrorInvalidValue;
   if (!encode_tmap_2d(&tb, w_exp, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.E * d.We, (uint64_t)d.D * 2, BK, BN))
     return cudaErrorInvalidValue;
-  TcArgs a{d, rowmeta, tiles, ntiles, offsets, mode, (__half*)bpi, (__half*)xs, (__half*)cpi, Z, st};
+  TcArgs a{d, rowmeta, tiles, ntiles, offsets, mode, 0, (__half*)bpi, (__half*)xs, (__half*)cpi, Z, st, nullptr};
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -549,6 +597,29 @@ cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp
   const int max_tiles = max_row_tiles(d) * ceil_div(d.We, BN);
   const int grid = max_tiles < sms ? max_tiles : sms;
   e = launch_dependent(proj_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, s, 1, ta, tb, a);
+  count_launches(1);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// The output projection out = y W_out^T as one dense product on the one-CTA kernel: A = y [M][K] (K = H*P),
+// B = W_out [N][K] (N = d_model), out [M][N] bf16.  K must be a multiple of 64, N of 8.
+cudaError_t launch_out_proj_tc(int M, int K, int N, const void* y, const void* w_out, void* out, unsigned* st,
+                               cudaStream_t s) {
+  CUtensorMap ta, tb;
+  if (!encode_tmap_2d(&ta, y, SWIMBA_BF16, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK, BM))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(&tb, w_out, SWIMBA_BF16, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, BN))
+    return cudaErrorInvalidValue;
+  Dims d{};
+  d.M = M; d.D = K; d.We = N; d.E = 1; d.k = 1; d.dtype = SWIMBA_BF16;
+  TcArgs a{d, nullptr, nullptr, nullptr, nullptr, 3, 1, nullptr, nullptr, nullptr, nullptr, st,
+           (__nv_bfloat16*)out};
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t e = set_max_dynamic_smem((const void*)proj_tc_kernel, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int tiles = ceil_div(M, BM) * ceil_div(N, BN);
+  e = launch_dependent(proj_tc_kernel, dim3(tiles < sms ? tiles : sms), dim3(kThreads), kSmemBytes, s, 1, ta, tb, a);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

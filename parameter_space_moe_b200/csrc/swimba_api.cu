@@ -507,6 +507,15 @@ swimba_status swimba_separated_scan(const swimba_dims* dims, const void* B, cons
   return SWIMBA_OK;
 }
 
+swimba_status swimba_out_proj(const swimba_dims* dims, const void* y, const void* w_out, void* out, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  if (!ok_ptr(y) || !ok_ptr(w_out) || !ok_ptr(out)) return SWIMBA_ERR_INVALID_ARG;
+  unsigned* st = device_status();
+  if (!st) return SWIMBA_ERR_CUDA;
+  return cuda_status(launch_out_proj(d, y, w_out, out, st, (cudaStream_t)stream));
+}
+
 swimba_status swimba_check_device_status(void* stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SWIMBA_ERR_CUDA;
   unsigned* st = device_status();

@@ -21,7 +21,7 @@ EXPORTS = ("swimba_workspace_size", "swimba_stream_dtype", "swimba_router_topk",
            "swimba_expert_proj", "swimba_mix", "swimba_ssd_scan", "swimba_layer_fwd", "swimba_step",
            "swimba_separated_scan", "swimba_check_device_status", "swimba_status_string",
            "swimba_profile_enable", "swimba_profile_read", "swimba_launch_count", "swimba_dispatch_noalloc",
-           "swimba_layer_fwd_host", "swimba_debug_scan_lost_first_chunk")
+           "swimba_layer_fwd_host", "swimba_debug_scan_lost_first_chunk", "swimba_out_proj")
 
 
 class SwimbaError(RuntimeError):
@@ -70,6 +70,7 @@ def lib():
             "swimba_debug_scan_lost_first_chunk": [P(Dims), vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_step": [P(Dims), vp, P(Weights), vp, vp, vp, vp, sz, vp],
             "swimba_separated_scan": [P(Dims), vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "swimba_out_proj": [P(Dims), vp, vp, vp, vp],
             "swimba_check_device_status": [vp],
         }
         L.swimba_profile_enable.restype = ctypes.c_int
@@ -184,6 +185,10 @@ def separated_scan(d, B, Xs, Cpi, dt, A, init_states, y, final_states, ws, strea
                                                                  _p(A), _p(init_states), _p(y), _p(final_states),
                                                                  _p(ws), ws.numel() * ws.element_size(),
                                                                  _stream(stream)))
+
+
+def out_proj(d, y, w_out, out, stream=None):
+    _check("swimba_out_proj", lib().swimba_out_proj(ctypes.byref(d), _p(y), _p(w_out), _p(out), _stream(stream)))
 
 
 def debug_scan_lost_first_chunk(d, Bpi, Xs, Cpi, dt, A, y, ws, stream=None):

@@ -85,6 +85,7 @@ def test_invalid_dims(L, kw):
     # both dispatch entry points give the same code for the same invalid dims
     assert L.swimba_dispatch(ctypes.byref(d), fake, fake, fake, fake, 1 << 40, None) == 1
     assert L.swimba_dispatch_noalloc(ctypes.byref(d), fake, fake, fake, None) == 1
+    assert L.swimba_out_proj(ctypes.byref(d), fake, fake, fake, None) == 1
 
 
 @pytest.mark.parametrize("kw", BAD_DIMS)
@@ -96,6 +97,7 @@ def test_dispatch_entry_points_agree_on_unsupported_dims(L, kw):
     fake = ctypes.c_void_p(1 << 20)
     assert L.swimba_dispatch(ctypes.byref(d), fake, fake, fake, fake, 1 << 40, None) == 2
     assert L.swimba_dispatch_noalloc(ctypes.byref(d), fake, fake, fake, None) == 2
+    assert L.swimba_out_proj(ctypes.byref(d), fake, fake, fake, None) == 2
 
 
 def test_null_misaligned_and_workspace_errors(L):
@@ -118,6 +120,11 @@ def test_null_misaligned_and_workspace_errors(L):
     assert L.swimba_step(ctypes.byref(d), fake, ctypes.byref(w), fake, fake, None, fake, need, None) == 1
     # mix rejects unknown flags
     assert L.swimba_mix(ctypes.byref(d), fake, fake, 8, fake, fake, fake, None) == 1
+    # output projection: every pointer non-null and 16-byte aligned
+    assert L.swimba_out_proj(ctypes.byref(d), None, fake, fake, None) == 1
+    assert L.swimba_out_proj(ctypes.byref(d), fake, odd, fake, None) == 1
+    assert L.swimba_out_proj(ctypes.byref(d), fake, fake, None, None) == 1
+    assert L.swimba_out_proj(None, fake, fake, fake, None) == 1
 
 
 def test_host_pipeline_and_debug_hook_validation(L):

@@ -5,7 +5,8 @@ Mistakes planted: no renormalisation over the winners, ties broken toward the hi
 dt clamp dropped, every slot projected with its first slot's expert, B and C swapped in the stream
 split, C~ summed without the router weights, the injection added before the decay, the decay's sign
 flipped, the chunked form's causal mask shifted by one, the chunk-state decay taken from the chunk
-start instead of its end, and the separated-E design advancing only the active experts."""
+start instead of its end, the separated-E design advancing only the active experts, and the output
+projection applied with its matrix transposed."""
 import numpy as np
 import pytest
 
@@ -145,9 +146,14 @@ def _chunked_state_decay_from_start(Bpi, Xs, Ct, dt, A, Q, init=None):
     return y, Hs, Hc
 
 
+def _out_proj_transposed(y, W_out):
+    # the projection matrix applied transposed (shapes permitting: D == H*P)
+    return np.asarray(y) @ np.asarray(W_out)
+
+
 ORIG = {name: getattr(O, name) for name in
         ("topk_weights", "topk_select", "dt_proj", "expert_proj", "split_streams", "mix", "scan_sequential",
-         "scan_chunked", "scan_separated_dense")}
+         "scan_chunked", "scan_separated_dense", "out_proj")}
 
 # every pin, called with the parameters its decorator gives
 ALL_PINS = [
@@ -160,7 +166,8 @@ ALL_PINS = [
     pins.test_groups_equal_replicated_heads, lambda: pins.test_chunked_equals_sequential(70, 16),
     pins.test_thm33_bibo_bound, pins.test_thm34_static_routing_equivalence_and_counts,
     pins.test_thm34_dynamic_routing_bound, pins.test_layer_fwd_state_handoff, pins.test_steps_equal_layer_fwd,
-    pins.test_forced_routing_replays_given_indices,
+    pins.test_forced_routing_replays_given_indices, pins.test_out_proj_matches_elementwise_dot_products,
+    pins.test_out_proj_identity_and_selection,
 ]
 
 MUTATIONS = {
@@ -175,6 +182,7 @@ MUTATIONS = {
     "causal_mask_shifted": ("scan_chunked", _chunked_strict_mask),
     "chunk_state_decay_from_start": ("scan_chunked", _chunked_state_decay_from_start),
     "dense_skips_inactive_experts": ("scan_separated_dense", _dense_skips_inactive_experts),
+    "out_proj_transposed": ("out_proj", _out_proj_transposed),
 }
 
 

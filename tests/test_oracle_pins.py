@@ -126,6 +126,31 @@ def test_expert_proj_matches_elementwise_dot_products():
                 assert abs(z[t, j, c] - sum(W_exp[idx[t, j], c, d] * X[t, d] for d in range(D))) < 1e-12
 
 
+def test_out_proj_matches_elementwise_dot_products():
+    # out[m][d] = sum_c y[m][c] W_out[d][c], written out term by term; a transposed W_out fails the shapes
+    # (D != H*P) and, for a square W_out, the values
+    rng = np.random.default_rng(5)
+    for M, HP, D in ((7, 6, 5), (4, 5, 5)):
+        y = rng.standard_normal((M, HP))
+        W_out = rng.standard_normal((D, HP))
+        out = O.out_proj(y, W_out)
+        assert out.shape == (M, D)
+        for m in range(M):
+            for d in range(D):
+                assert abs(out[m, d] - sum(y[m, c] * W_out[d, c] for c in range(HP))) < 1e-12
+
+
+def test_out_proj_identity_and_selection():
+    # W_out = I returns y; a row-selection W_out returns the selected columns of y, in W_out's row order
+    rng = np.random.default_rng(6)
+    y = rng.standard_normal((3, 2, 8))
+    np.testing.assert_array_equal(O.out_proj(y, np.eye(8)), y)
+    sel = [5, 0, 7]
+    W_out = np.zeros((3, 8))
+    W_out[np.arange(3), sel] = 1.0
+    np.testing.assert_array_equal(O.out_proj(y, W_out), y[..., sel])
+
+
 def test_split_streams_layout():
     H, P, G, N = 2, 3, 1, 2
     z = np.arange(H * P + 2 * G * N, dtype=float)
