@@ -12,7 +12,8 @@ On one GPU the default run adds two nested measurements to the same JSON line, t
 "decode" (swimba_step on 256 sequences, D2048 H64 N128 P64 E16 k2, state from a 512-token prefill; bound
 by HBM), "esweep" (the base layer at E in {8, 16, 32, 64}: layer and scan-stage times, which the
 method's cost statement says are flat in E, plus the separated-trajectory scan that runs k trajectories) and
-"out_proj" (the output projection y W_out^T on the base layer's y, bound by the tensor cores).
+"out_proj" (the output projection y W_out^T on the base layer's y, bound by the tensor cores) and "mixed_A"
+(the base layer with the expert-mixed transition A~ = sum_j pi_j A_exp[K_j]).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launching stream,
 with a write of 2x the L2 size between steps (outside the events) so every step reads its inputs from
@@ -243,10 +244,11 @@ def config_of(w):
 class LayerSession:
     """Forward-pass workloads: one step = swimba_layer_fwd over B x T tokens."""
 
-    def __init__(self, w, dev, inp, swimba):
+    def __init__(self, w, dev, inp, swimba, mixed_A=False):
         self.w, self.sw = w, swimba
         self.d = swimba.dims_of(w)
-        self.W = swimba.WeightSet(*(inp[k].to(dev) for k in ("W_r", "W_dt", "b_dt", "A", "W_exp")))
+        self.W = swimba.WeightSet(*(inp[k].to(dev) for k in ("W_r", "W_dt", "b_dt", "A", "W_exp")),
+                                  A_exp=inp["A_exp"].to(dev) if mixed_A else None)
         self.X = inp["X"].to(dev).reshape(w.M, w.d_model)
         odt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
         self.y = torch.empty(w.M, w.nheads * w.headdim, dtype=odt, device=dev)
@@ -507,6 +509,12 @@ def run_gpu(args, w):
     if world == 1 and w.name == configs.BASE.name and not args.no_extras:
         out["out_proj"] = out_proj_measure(args, sess, inp, flush, stream, swimba)
         del sess
+        torch.cuda.empty_cache()
+        msess = LayerSession(w, dev, inp, swimba, mixed_A=True)
+        mm = measure(msess, args, flush, stream, None, local, swimba, e2e=False)
+        out["mixed_A"] = {"layer_ms": mm["total_ms"] / args.steps,
+                          "stages_ms_per_step": {n: v / args.steps for n, v in mm["stage_ms"].items()}}
+        del msess
         torch.cuda.empty_cache()
         dw = configs.DECODE
         dsess = DecodeSession(dw, dev, inputs.make_inputs(dw), swimba)

@@ -53,7 +53,8 @@ typedef enum {
   SWIMBA_ERR_WORKSPACE = 4,    /* ws is NULL or smaller than swimba_workspace_size() */
   SWIMBA_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up (read via swimba_check_device_status) */
   SWIMBA_ERR_RANGE = 6,        /* device: a mixed-stream value did not fit the stream dtype */
-  SWIMBA_ERR_INDEX = 7         /* device: a caller-given expert index lay outside [0, E) */
+  SWIMBA_ERR_INDEX = 7,        /* device: a caller-given expert index lay outside [0, E) */
+  SWIMBA_ERR_UNSTABLE = 8      /* device: an expert-mixed transition A~ was not negative (no contraction) */
 } swimba_status;
 
 typedef enum { SWIMBA_F32 = 0, SWIMBA_BF16 = 1, SWIMBA_F16 = 2 } swimba_dtype;
@@ -78,6 +79,14 @@ typedef struct {
   const float* b_dt;     /* [H] fp32 */
   const float* A;        /* [H] fp32, negative: a_t = exp(dt_t A_h) */
   const void* w_exp;     /* [E][W_e][D] dtype: expert projections, rows [x: H*P | B: G*N | C: G*N] */
+  /* [E][H] fp32 or NULL.  When given, the transition is mixed in parameter space like B and C
+   * (notes, limitations and outlook: the mixing extended to the diagonal of A under Lyapunov stability):
+   * A~_t,h = sum_j pi_tj A_exp[K_tj][h] and a_t = exp(dt_t A~_t,h); A is then not read.  Every entry must
+   * be negative, so that each A~ is negative and 0 < a_t < 1 (one contracting trajectory); an A~ that is
+   * not negative is recorded as SWIMBA_ERR_UNSTABLE.  Read by swimba_layer_fwd, swimba_layer_fwd_host and
+   * swimba_step; the stage entry points (swimba_ssd_scan, swimba_separated_scan) take the shared form
+   * dt * A only: pass dt_t * A~_t as dt with A = 1 there. */
+  const float* A_exp;
 } swimba_weights;
 
 /* Bytes of workspace that every entry point taking `ws` needs for these dims (0 if the dims are
@@ -217,8 +226,8 @@ swimba_status swimba_separated_scan(const swimba_dims* dims, const void* B, cons
 swimba_status swimba_out_proj(const swimba_dims* dims, const void* y, const void* w_out, void* out, void* stream);
 
 /* Synchronises `stream`, then reads and clears the current device's status word: SWIMBA_OK,
- * SWIMBA_ERR_TIMEOUT, SWIMBA_ERR_RANGE or SWIMBA_ERR_INDEX, in that order of precedence (SWIMBA_ERR_CUDA
- * if the stream reports an error).  The word is sticky: it collects every flag raised on this device
+ * SWIMBA_ERR_TIMEOUT, SWIMBA_ERR_RANGE, SWIMBA_ERR_INDEX or SWIMBA_ERR_UNSTABLE, in that order of
+ * precedence (SWIMBA_ERR_CUDA if the stream reports an error).  The word is sticky: it collects every flag raised on this device
  * since the previous check.  Its device address is looked up once per device; a device reset between
  * calls into the library is not supported. */
 swimba_status swimba_check_device_status(void* stream);

@@ -122,6 +122,17 @@ def mix(z, w, H, P, G, N):
     return Bpi, x, Cpi.sum(axis=1), Cpi
 
 
+def mixed_A(idx, w, A_exp):
+    """Expert-mixed diagonal transition ([notes] limitations and outlook: parameter-space mixing carried over
+    to the diagonal of the transition A, with Lyapunov stability kept):
+        A~_t,h = sum_j pi_tj A^(K_tj)_h,        a_t = exp(dt_t A~_t)  for every head.
+    Reading: one A^(e) per expert and head (Mamba-2's scalar-per-head diagonal), mixed with the same router
+    weights as B and C; dt stays the one shared projection.  Every A^(e) < 0 makes A~_t a convex combination
+    of negative values, so 0 < a_t < 1: the transition stays a contraction and the recurrence is still one
+    trajectory.  idx [M,k], w [M,k], A_exp [E,H]; returns A~ [M,H]."""
+    return np.einsum("mj,mjh->mh", w, np.asarray(A_exp)[idx])
+
+
 # ----------------------------------------------------------------------------- the single recurrence
 
 def group_of(H, G):
@@ -134,13 +145,20 @@ def _count_update(stats):
         stats["updates"] = stats.get("updates", 0) + 1
 
 
+def log_decay(dt, A):
+    """dt_t A_h per token and head, [T,H]: A is the shared [H] vector, or a per-token [T,H] array (the
+    expert-mixed A~ of mixed_A)."""
+    return np.asarray(dt) * np.asarray(A)
+
+
 def scan_sequential(Bpi, Xs, Ct, dt, A, init=None, stats=None):
     """The single-trajectory recurrence, token by token ([notes] key design 1, second display
     equation; [gist] "h_t = A h_{t-1} + sum pi B X"):
         h_t = a_t h_{t-1} + sum_j Bpi_tj (x) Xs_tj,     y_t = C~_t^T h_t,     a_t = exp(dt_t A_h).
     Reading: no dt factor on the injection (the pages' equation has none).
 
-    One batch row: Bpi [T,k,G,N], Xs [T,k,H,P], Ct [T,G,N], dt [T,H], A [H], init [H,N,P] or None.
+    One batch row: Bpi [T,k,G,N], Xs [T,k,H,P], Ct [T,G,N], dt [T,H], A [H] (or [T,H], see log_decay),
+    init [H,N,P] or None.
     Returns y [T,H,P] and the final state [H,N,P].  stats (optional dict): "updates" is increased by one
     for every state update, so a T-token call adds T (one trajectory).
     """
@@ -149,8 +167,9 @@ def scan_sequential(Bpi, Xs, Ct, dt, A, init=None, stats=None):
     g = group_of(H, G)
     h = np.zeros((H, N, P)) if init is None else np.array(init, dtype=np.float64)
     y = np.zeros((T, H, P))
+    dA = log_decay(dt, A)
     for t in range(T):
-        a = np.exp(dt[t] * A)                                           # [H]
+        a = np.exp(dA[t])                                               # [H]
         U = np.einsum("jhn,jhp->hnp", Bpi[t][:, g], Xs[t])              # rank-k injection per head
         h = a[:, None, None] * h + U
         _count_update(stats)
@@ -165,7 +184,7 @@ def scan_bruteforce(Bpi, Xs, Ct, dt, A, init=None):
     whose input-output map is this lower-triangular matrix.  For tiny T only."""
     T, k, H, P = Xs.shape
     g = group_of(H, G=Bpi.shape[2])
-    dA = dt * A                                                        # [T,H]
+    dA = log_decay(dt, A)                                              # [T,H]
     y = np.zeros((T, H, P))
     for t in range(T):
         for s in range(t + 1):
@@ -192,12 +211,13 @@ def scan_chunked(Bpi, Xs, Ct, dt, A, Q, init=None):
     G, N = Bpi.shape[2], Bpi.shape[3]
     g = group_of(H, G)
     nc = (T + Q - 1) // Q
+    dA = log_decay(dt, A) * np.ones((T, H))
     Hc = np.zeros((H, N, P)) if init is None else np.array(init, dtype=np.float64)
     Hs = np.zeros((nc, H, N, P))
     y = np.zeros((T, H, P))
     for c in range(nc):
         t0, t1 = c * Q, min(T, (c + 1) * Q)
-        cs = np.cumsum(dt[t0:t1] * A, axis=0)                          # [L,H]
+        cs = np.cumsum(dA[t0:t1], axis=0)                              # [L,H]
         Cg = Ct[t0:t1][:, g]                                           # [L,H,N]
         Bg = Bpi[t0:t1][:, :, g]                                       # [L,k,H,N]
         Xc = Xs[t0:t1]                                                 # [L,k,H,P]
@@ -266,26 +286,28 @@ def scan_separated_dense(xE, BE, CE, pi_dense, dt, A):
 # ----------------------------------------------------------------------------- the layer
 
 def layer_fwd(X, W_r, W_dt, b_dt, A, W_exp, H, P, N, G, k, init=None, forced_idx=None,
-              decision_dtype=np.float32):
+              decision_dtype=np.float32, A_exp=None):
     """Forward pass of one Swimba token-mixer layer ([notes] Method flowchart: router -> expert
     projections -> parameter-space mixing -> one recurrence with the shared transition -> readout).
 
-    X [B,T,D]; init [B,H,N,P] or None; forced_idx [B,T,k] or None (see router).
+    X [B,T,D]; init [B,H,N,P] or None; forced_idx [B,T,k] or None (see router); A_exp [E,H] or None:
+    with it the transition is the expert-mixed A~ of mixed_A (A is then not used).
     Returns a dict: y [B,T,H,P], final [B,H,N,P] and the stage values (g, dt, idx, w, z, Bpi, Xs,
-    Ct, Cpi) flattened over tokens (row = b*T + t)."""
+    Ct, Cpi, At = the [M,H] or [H] transition used) flattened over tokens (row = b*T + t)."""
     Bsz, T, D = X.shape
     Xf = X.reshape(Bsz * T, D)
     fidx = None if forced_idx is None else forced_idx.reshape(Bsz * T, k)
     g, dt, idx, w = router(Xf, W_r, W_dt, b_dt, k, decision_dtype, fidx)
     z = expert_proj(Xf, W_exp, idx)
     Bpi, Xs, Ct, Cpi = mix(z, w, H, P, G, N)
+    At = A if A_exp is None else mixed_A(idx, w, A_exp)
     y = np.zeros((Bsz, T, H, P))
     final = np.zeros((Bsz, H, N, P))
     for b in range(Bsz):
         r = slice(b * T, (b + 1) * T)
-        y[b], final[b] = scan_sequential(Bpi[r], Xs[r], Ct[r], dt[r], A,
+        y[b], final[b] = scan_sequential(Bpi[r], Xs[r], Ct[r], dt[r], At if A_exp is None else At[r],
                                          None if init is None else init[b])
-    return dict(y=y, final=final, g=g, dt=dt, idx=idx, w=w, z=z, Bpi=Bpi, Xs=Xs, Ct=Ct, Cpi=Cpi)
+    return dict(y=y, final=final, g=g, dt=dt, idx=idx, w=w, z=z, Bpi=Bpi, Xs=Xs, Ct=Ct, Cpi=Cpi, At=At)
 
 
 def out_proj(y, W_out):
@@ -299,15 +321,16 @@ def out_proj(y, W_out):
     return np.asarray(y) @ np.asarray(W_out).T
 
 
-def step(Xt, W_r, W_dt, b_dt, A, W_exp, H, P, N, G, k, state, forced_idx=None, decision_dtype=np.float32):
+def step(Xt, W_r, W_dt, b_dt, A, W_exp, H, P, N, G, k, state, forced_idx=None, decision_dtype=np.float32,
+         A_exp=None):
     """One recurrent decode step per sequence: the layer applied to a single new token X_t [B,D]
-    with the cached state [B,H,N,P] (the recurrence of [notes] key design 1 advanced by one token).
-    Returns (y [B,H,P], new state [B,H,N,P], idx)."""
+    with the cached state [B,H,N,P] (the recurrence of [notes] key design 1 advanced by one token);
+    A_exp [E,H] or None as in layer_fwd.  Returns (y [B,H,P], new state [B,H,N,P], idx)."""
     g, dt, idx, w = router(Xt, W_r, W_dt, b_dt, k, decision_dtype, forced_idx)
     z = expert_proj(Xt, W_exp, idx)
     Bpi, Xs, Ct, _ = mix(z, w, H, P, G, N)
     gh = group_of(H, G)
-    a = np.exp(dt * A)                                                  # [B,H]
+    a = np.exp(log_decay(dt, A if A_exp is None else mixed_A(idx, w, A_exp)))   # [B,H]
     U = np.einsum("bjhn,bjhp->bhnp", Bpi[:, :, gh], Xs)
     new = a[:, :, None, None] * state + U
     y = np.einsum("bhn,bhnp->bhp", Ct[:, gh], new)

@@ -12,7 +12,7 @@
 namespace swimba {
 
 // Bits of the device status word.
-enum : unsigned { ST_TIMEOUT = 1u, ST_RANGE = 2u, ST_INDEX = 4u };
+enum : unsigned { ST_TIMEOUT = 1u, ST_RANGE = 2u, ST_INDEX = 4u, ST_UNSTABLE = 8u };
 
 // Largest finite fp16 value: mixed streams stored as fp16 must stay below it.
 constexpr float kF16Max = 65504.f;
@@ -64,6 +64,8 @@ struct WsPlan {
   size_t topk_idx;    // int32 [M][k]
   size_t topk_w;      // f32 [M][k]
   size_t dt;          // f32 [M][H]
+  size_t dA;          // f32 [M][H]  dt * A~ of the expert-mixed transition, and A = 1 [H] after it
+  size_t ones;
   size_t dcounts;     // int32 [ndt][E]  per dispatch tile expert counts
   size_t dbase;       // int32 [ndt][E]  first sorted position of each (tile, expert)
   size_t offsets;     // int32 [E+1]
@@ -130,6 +132,8 @@ cudaError_t launch_proj_simt(const Dims& d, const void* X, const void* w_exp, co
 cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int2* rowmeta,
                            const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, int mode, void* bpi,
                            void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s);
+cudaError_t launch_mixed_a(const Dims& d, const int32_t* idx, const float* wts, const float* A_exp, const float* dt,
+                           float* dA, float* ones, unsigned* st, cudaStream_t s);
 cudaError_t launch_out_proj(const Dims& d, const void* y, const void* w_out, void* out, unsigned* st,
                             cudaStream_t s);
 cudaError_t launch_mix(const Dims& d, const float* Z, const float* topk_w, int flags, void* bpi, void* xs, void* cpi,

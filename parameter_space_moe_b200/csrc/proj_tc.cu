@@ -406,7 +406,7 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
   const Dims& d = a.d;
   const int nct = ceil_div(d.We, BN);
-  const int nkb = d.D / BK;
+  const int nkb = ceil_div(d.D, BK);  // a dense product's ragged K tail is zero-filled by TMA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
@@ -420,7 +420,11 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
   griddep_launch_dependents();
   if (warp == 1) { tc::tmem_alloc_pair(tmem_slot, kTmemCols); tc::tmem_relinquish_pair(); }
   griddep_wait();  // the dispatch's offsets, the gathered rows
-  for (int e = threadIdx.x; e <= d.E; e += blockDim.x) off_s[e] = a.offsets[e];
+  if (a.dense) {
+    if (threadIdx.x == 0) { off_s[0] = 0; off_s[1] = d.M; }
+  } else {
+    for (int e = threadIdx.x; e <= d.E; e += blockDim.x) off_s[e] = a.offsets[e];
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     int acc = 0;
@@ -512,7 +516,7 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       const int rt = t / nct, ct = t % nct;
       const int2 tl = pair_tile(off_s, pt_s, d.E, rt);
       const bool valid = tl.y + row_local < off_s[tl.x + 1];
-      const int2 meta = valid ? a.rowmeta[tl.y + row_local] : make_int2(0, 0);
+      const int2 meta = !valid ? make_int2(0, 0) : (a.dense ? make_int2(tl.y + row_local, 0) : a.rowmeta[tl.y + row_local]);
       if (!tc::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) {
         *abort_flag = 1;
         atomicOr(a.st, ST_TIMEOUT);
@@ -541,6 +545,33 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
 }  // namespace
 
 // Host side --------------------------------------------------------------------------------------
+// The CTA-pair kernel, persistent: as many pairs as can be resident at once, at most one per pair tile.
+static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb2, const TcArgs& a, int max_pairs, int sms,
+                               cudaStream_t s) {
+  cudaError_t e = set_max_dynamic_smem((const void*)proj_tc_pair_kernel, kPairSmemBytes);
+  if (e != cudaSuccess) return e;
+  static int resident = 0;
+  if (resident == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3((unsigned)sms);
+    int n = 0;
+    resident = cudaOccupancyMaxActiveClusters(&n, proj_tc_pair_kernel, &cfg) == cudaSuccess && n > 0 ? n : sms / 2;
+  }
+  const int pairs = resident < max_pairs ? resident : max_pairs;
+  return launch_dependent(proj_tc_pair_kernel, dim3((unsigned)(2 * pairs)), dim3(kThreads), kPairSmemBytes, s, 2, ta,
+                          tb2, a);
+}
+
 cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int2* rowmeta,
                            const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, int mode, void* bpi,
                            void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s) {
@@ -562,30 +593,7 @@ cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp
     CUtensorMap tb2;
     if (!encode_tmap_2d(&tb2, w_exp, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.E * d.We, (uint64_t)d.D * 2, BK, 128))
       return cudaErrorInvalidValue;
-    e = set_max_dynamic_smem((const void*)proj_tc_pair_kernel, kPairSmemBytes);
-    if (e != cudaSuccess) return e;
-    // persistent: as many pairs as can be resident at once (at most one per tile)
-    static int resident = 0;
-    if (resident == 0) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.blockDim = dim3(kThreads);
-      cfg.dynamicSmemBytes = kPairSmemBytes;
-      cfg.stream = s;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = 2;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      cfg.gridDim = dim3((unsigned)sms);
-      int n = 0;
-      resident = cudaOccupancyMaxActiveClusters(&n, proj_tc_pair_kernel, &cfg) == cudaSuccess && n > 0 ? n : sms / 2;
-    }
-    const int max_pairs = (ceil_div(d.M * d.k, kPairRows) + d.E) * ceil_div(d.We, BN);
-    const int pairs = resident < max_pairs ? resident : max_pairs;
-    e = launch_dependent(proj_tc_pair_kernel, dim3((unsigned)(2 * pairs)), dim3(kThreads), kPairSmemBytes, s, 2, ta, tb2,
-                         a);
+    e = launch_pair(ta, tb2, a, (ceil_div(d.M * d.k, kPairRows) + d.E) * ceil_div(d.We, BN), sms, s);
     if (e == cudaSuccess) {
       count_launches(1);
       return cudaGetLastError();
@@ -616,7 +624,20 @@ cudaError_t launch_out_proj_tc(int M, int K, int N, const void* y, const void* w
            (__nv_bfloat16*)out};
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaError_t e = set_max_dynamic_smem((const void*)proj_tc_kernel, kSmemBytes);
+  cudaError_t e;
+  // CTA pairs (256-row tiles, half the operand bytes per FLOP) once there are rows for a few pair tiles
+  if (M >= 4 * kPairRows) {
+    CUtensorMap tb2;
+    if (!encode_tmap_2d(&tb2, w_out, SWIMBA_BF16, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, 128))
+      return cudaErrorInvalidValue;
+    e = launch_pair(ta, tb2, a, ceil_div(M, kPairRows) * ceil_div(N, BN), sms, s);
+    if (e == cudaSuccess) {
+      count_launches(1);
+      return cudaGetLastError();
+    }
+    (void)cudaGetLastError();  // pairs could not be launched: the one-CTA kernel below does the work
+  }
+  e = set_max_dynamic_smem((const void*)proj_tc_kernel, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int tiles = ceil_div(M, BM) * ceil_div(N, BN);
   e = launch_dependent(proj_tc_kernel, dim3(tiles < sms ? tiles : sms), dim3(kThreads), kSmemBytes, s, 1, ta, tb, a);

@@ -83,6 +83,8 @@ WsPlan plan_workspace(const Dims& d) {
   p.topk_idx = take(Mk * 4);
   p.topk_w = take(Mk * 4);
   p.dt = take((size_t)d.M * d.H * 4);
+  p.dA = take((size_t)d.M * d.H * 4);
+  p.ones = take((size_t)d.H * 4);
   p.dcounts = take((size_t)dispatch_tiles(d) * d.E * 4);
   const size_t nsub = (size_t)scan_tc_subchunks(d);
   p.lb_bytes = 256 + (size_t)d.Bsz * d.H * nsub * 4;
@@ -138,7 +140,8 @@ static bool ok_opt(const void* p) { return !p || aligned(p); }
 
 static swimba_status check_weights(const swimba_weights* w, bool need_router, bool need_exp) {
   if (!w) return SWIMBA_ERR_INVALID_ARG;
-  if (need_router && (!ok_ptr(w->w_router) || !ok_ptr(w->w_dt) || !w->b_dt || !w->A)) return SWIMBA_ERR_INVALID_ARG;
+  if (need_router && (!ok_ptr(w->w_router) || !ok_ptr(w->w_dt) || !w->b_dt || (!w->A && !w->A_exp)))
+    return SWIMBA_ERR_INVALID_ARG;
   if (need_exp && !ok_ptr(w->w_exp)) return SWIMBA_ERR_INVALID_ARG;
   return SWIMBA_OK;
 }
@@ -217,6 +220,20 @@ static swimba_status run_scan(const Dims& d, const ScanArgs& a, char* ws, const 
   } else {
     SW_CUDA(launch_scan_simt(d, a, s));
   }
+  return SWIMBA_OK;
+}
+
+// Expert-mixed transition (weights.A_exp given): dA = dt * A~ per token and head and A = 1, which the scan
+// and the decode step read in place of dt and the shared A (dt * 1 is exact).
+static swimba_status run_mixed_a(const Dims& d, const swimba_weights* w, const int32_t* idx, const float* wts,
+                                 char* ws, const WsPlan& p, const float** dt, const float** A, cudaStream_t s) {
+  if (!w->A_exp) return SWIMBA_OK;
+  float* dA = (float*)(ws + p.dA);
+  float* ones = (float*)(ws + p.ones);
+  SW_CUDA(launch_mixed_a(d, idx, wts, w->A_exp, *dt, dA, ones, device_status(), s));
+  prof_mark(s, "mixed_A");
+  *dt = dA;
+  *A = ones;
   return SWIMBA_OK;
 }
 
@@ -366,8 +383,9 @@ swimba_status swimba_layer_fwd(const swimba_dims* dims, const void* X, const swi
   float* wts = topk_w_out ? topk_w_out : (float*)(b + p.topk_w);
   prof_begin(s);
   SW_TRY(run_front(d, X, w, b, p, idx, wts, 0, device_status(), s));
-  ScanArgs a = mixed_scan_args(d, b, p, b + p.bpi, b + p.xs, b + p.cpi, (float*)(b + p.dt), w->A, init_state, y,
-                               final_state, nullptr);
+  const float *dt = (float*)(b + p.dt), *A = w->A;
+  SW_TRY(run_mixed_a(d, w, idx, wts, b, p, &dt, &A, s));
+  ScanArgs a = mixed_scan_args(d, b, p, b + p.bpi, b + p.xs, b + p.cpi, dt, A, init_state, y, final_state, nullptr);
   SW_TRY(run_scan(d, a, b, p, s, /*lb_clear=*/true));  // run_front already cleared the hand-off flags
   prof_mark(s, "ssd_scan");
   return SWIMBA_OK;
@@ -479,7 +497,9 @@ swimba_status swimba_step(const swimba_dims* dims, const void* X, const swimba_w
   float* wts = (float*)(b + p.topk_w);
   prof_begin(s);
   SW_TRY(run_front(d, X, w, b, p, idx, wts, 0, device_status(), s));
-  SW_CUDA(launch_step_update(d, b + p.bpi, b + p.xs, b + p.cpi, (float*)(b + p.dt), w->A, state, y, s));
+  const float *dt = (float*)(b + p.dt), *A = w->A;
+  SW_TRY(run_mixed_a(d, w, idx, wts, b, p, &dt, &A, s));
+  SW_CUDA(launch_step_update(d, b + p.bpi, b + p.xs, b + p.cpi, dt, A, state, y, s));
   prof_mark(s, "state_update");
   return SWIMBA_OK;
 }
@@ -526,6 +546,7 @@ swimba_status swimba_check_device_status(void* stream) {
   if (v & ST_TIMEOUT) return SWIMBA_ERR_TIMEOUT;
   if (v & ST_RANGE) return SWIMBA_ERR_RANGE;
   if (v & ST_INDEX) return SWIMBA_ERR_INDEX;
+  if (v & ST_UNSTABLE) return SWIMBA_ERR_UNSTABLE;
   return SWIMBA_OK;
 }
 
@@ -565,6 +586,7 @@ const char* swimba_status_string(swimba_status s) {
     case SWIMBA_ERR_TIMEOUT: return "SWIMBA_ERR_TIMEOUT";
     case SWIMBA_ERR_RANGE: return "SWIMBA_ERR_RANGE";
     case SWIMBA_ERR_INDEX: return "SWIMBA_ERR_INDEX";
+    case SWIMBA_ERR_UNSTABLE: return "SWIMBA_ERR_UNSTABLE";
   }
   return "SWIMBA_UNKNOWN_STATUS";
 }

@@ -13,8 +13,10 @@ Recipe (one numpy PCG64 stream per workload seed, tensors drawn in this order):
   A     = -exp(U[log 1, log 16])          [H]        negative, shared by all experts
   W_exp ~ N(0, 1/D)                       [E, W_e, D] rows ordered [x: H*P | B: G*N | C: G*N]
   (decode workloads then draw X_step ~ N(0,1) [B, D]; X above is the prefill, [B, prefill, D])
-  W_out ~ N(0, 1/(H*P))                   [D, H*P]   output projection (drawn last, so the draws above
-                                                     are the same with or without it)
+  W_out ~ N(0, 1/(H*P))                   [D, H*P]   output projection (drawn after the layer's own
+                                                     tensors, so those are the same with or without it)
+  A_exp = -exp(U[log 1, log 16])          [E, H]     per-expert transitions for the expert-mixed A~
+                                                     (drawn last; fp32)
 In bf16 workloads X, W_r, W_dt, W_exp and W_out are rounded to bf16 (round to nearest even) once, here;
 b_dt and A stay fp32.  Both sides then read the same rounded values.
 """
@@ -59,6 +61,7 @@ def make_inputs(w: Workload, with_x=True):
         out["X_step"] = _store(_normal(rng, (w.batch, D), 1.0), w.dtype)
     HP = H * w.headdim
     out["W_out"] = _store(_normal(rng, (D, HP), 1.0 / math.sqrt(HP)), w.dtype)
+    out["A_exp"] = torch.from_numpy((-np.exp(rng.uniform(0.0, math.log(16.0), size=(E, H)))).astype(np.float32))
     return out
 
 

@@ -16,7 +16,8 @@ LIB_PATH = os.path.join(_HERE, "libswimba.so")
 F32, BF16, F16 = 0, 1, 2
 MIX_UNSCALED_B = 1
 STATUS = {0: "SWIMBA_OK", 1: "SWIMBA_ERR_INVALID_ARG", 2: "SWIMBA_ERR_UNSUPPORTED", 3: "SWIMBA_ERR_CUDA",
-          4: "SWIMBA_ERR_WORKSPACE", 5: "SWIMBA_ERR_TIMEOUT", 6: "SWIMBA_ERR_RANGE", 7: "SWIMBA_ERR_INDEX"}
+          4: "SWIMBA_ERR_WORKSPACE", 5: "SWIMBA_ERR_TIMEOUT", 6: "SWIMBA_ERR_RANGE", 7: "SWIMBA_ERR_INDEX",
+          8: "SWIMBA_ERR_UNSTABLE"}
 EXPORTS = ("swimba_workspace_size", "swimba_stream_dtype", "swimba_router_topk", "swimba_dispatch",
            "swimba_expert_proj", "swimba_mix", "swimba_ssd_scan", "swimba_layer_fwd", "swimba_step",
            "swimba_separated_scan", "swimba_check_device_status", "swimba_status_string",
@@ -37,7 +38,7 @@ class Dims(ctypes.Structure):
 
 class Weights(ctypes.Structure):
     _fields_ = [("w_router", ctypes.c_void_p), ("w_dt", ctypes.c_void_p), ("b_dt", ctypes.c_void_p),
-                ("A", ctypes.c_void_p), ("w_exp", ctypes.c_void_p)]
+                ("A", ctypes.c_void_p), ("w_exp", ctypes.c_void_p), ("A_exp", ctypes.c_void_p)]
 
 
 _lib = None
@@ -114,8 +115,8 @@ def _check(fn, code):
 class WeightSet:
     """Device weights plus the C struct pointing at them (keeps the tensors alive)."""
 
-    def __init__(self, w_router, w_dt, b_dt, A, w_exp):
-        self.tensors = (w_router, w_dt, b_dt, A, w_exp)
+    def __init__(self, w_router, w_dt, b_dt, A, w_exp, A_exp=None):
+        self.tensors = (w_router, w_dt, b_dt, A, w_exp, A_exp)
         self.c = Weights(*(None if t is None else t.data_ptr() for t in self.tensors))
 
 

@@ -112,6 +112,10 @@ def test_null_misaligned_and_workspace_errors(L):
     assert L.swimba_layer_fwd(*args(fake, None, need)) == 4           # no workspace
     assert L.swimba_layer_fwd(*args(fake, fake, need - 1)) == 4       # workspace too small
     assert L.swimba_layer_fwd(*args(fake, odd, need)) == 4            # misaligned workspace
+    # A may be left out only when the expert-mixed A_exp is given
+    wnoA = swimba.Weights(1 << 20, 1 << 20, 1 << 20, None, 1 << 20)
+    assert L.swimba_layer_fwd(ctypes.byref(d), fake, ctypes.byref(wnoA), None, fake, None, None, None, fake, need,
+                              None) == 1
     wnull = swimba.Weights(1 << 20, None, 1 << 20, 1 << 20, 1 << 20)
     assert L.swimba_layer_fwd(ctypes.byref(d), fake, ctypes.byref(wnull), None, fake, None, None, None, fake, need,
                               None) == 1

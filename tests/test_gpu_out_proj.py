@@ -1,8 +1,9 @@
 """Parity of the output projection (swimba_out_proj) against the fp64 oracle, through the C ABI.
 
 The projection reads y as the layer writes it ([M][H*P], dtype) and W_out [D][H*P].  Shapes cover several
-128-row and 256-column tiles with ragged tails, a K that is not a multiple of the 64-wide K step, a single
-row, the fp32 CUDA-core kernel, the full base workload, and the layer and projection chained."""
+128-row (one-CTA kernel) and 256-row (CTA-pair kernel) tiles and 256-column tiles with ragged tails, a K
+that is not a multiple of the 64-wide K step, a single row, the fp32 CUDA-core kernel, the full base
+workload, and the layer and projection chained."""
 import numpy as np
 import pytest
 import torch
@@ -20,6 +21,10 @@ CASES = [
     # 333 rows (3 row tiles, ragged), K = 48 (one partial K step), D = 320 (a full and a partial column tile)
     configs.BASE.with_(name="bf16_ragged_K48_D320", batch=3, seqlen=111, d_model=320, nheads=3, headdim=16,
                        seed=102),
+    # the CTA-pair kernel (from 1024 rows) on ragged sizes: 1500 rows (6 pair tiles, the last partial), K = 48,
+    # D = 320
+    configs.BASE.with_(name="bf16_pair_ragged_K48_D320", batch=3, seqlen=500, d_model=320, nheads=3, headdim=16,
+                       seed=106),
     # one row; K = 320 (five K steps); D = 192 (less than one column tile)
     configs.BASE.with_(name="bf16_one_row", batch=1, seqlen=1, d_model=192, nheads=5, headdim=64, seed=103),
     # more tiles than SMs: 4000 x 1536 with K = 1536 (32 row tiles x 6 column tiles)

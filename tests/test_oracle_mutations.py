@@ -5,8 +5,9 @@ Mistakes planted: no renormalisation over the winners, ties broken toward the hi
 dt clamp dropped, every slot projected with its first slot's expert, B and C swapped in the stream
 split, C~ summed without the router weights, the injection added before the decay, the decay's sign
 flipped, the chunked form's causal mask shifted by one, the chunk-state decay taken from the chunk
-start instead of its end, the separated-E design advancing only the active experts, and the output
-projection applied with its matrix transposed."""
+start instead of its end, the separated-E design advancing only the active experts, the output
+projection applied with its matrix transposed, and the expert-mixed transition summed without the router
+weights or taken from the first active expert alone."""
 import numpy as np
 import pytest
 
@@ -146,6 +147,16 @@ def _chunked_state_decay_from_start(Bpi, Xs, Ct, dt, A, Q, init=None):
     return y, Hs, Hc
 
 
+def _mixed_A_unweighted(idx, w, A_exp):
+    # the active experts' A summed without the router weights
+    return np.asarray(A_exp)[idx].sum(axis=1)
+
+
+def _mixed_A_first_slot(idx, w, A_exp):
+    # the transition of the first active expert alone
+    return np.asarray(A_exp)[idx[:, 0]]
+
+
 def _out_proj_transposed(y, W_out):
     # the projection matrix applied transposed (shapes permitting: D == H*P)
     return np.asarray(y) @ np.asarray(W_out)
@@ -153,7 +164,7 @@ def _out_proj_transposed(y, W_out):
 
 ORIG = {name: getattr(O, name) for name in
         ("topk_weights", "topk_select", "dt_proj", "expert_proj", "split_streams", "mix", "scan_sequential",
-         "scan_chunked", "scan_separated_dense", "out_proj")}
+         "scan_chunked", "scan_separated_dense", "out_proj", "mixed_A")}
 
 # every pin, called with the parameters its decorator gives
 ALL_PINS = [
@@ -167,7 +178,9 @@ ALL_PINS = [
     pins.test_thm33_bibo_bound, pins.test_thm34_static_routing_equivalence_and_counts,
     pins.test_thm34_dynamic_routing_bound, pins.test_layer_fwd_state_handoff, pins.test_steps_equal_layer_fwd,
     pins.test_forced_routing_replays_given_indices, pins.test_out_proj_matches_elementwise_dot_products,
-    pins.test_out_proj_identity_and_selection,
+    pins.test_out_proj_identity_and_selection, pins.test_mixed_A_is_the_router_weighted_mean,
+    pins.test_mixed_A_with_equal_experts_is_the_shared_layer, pins.test_mixed_A_decay_closed_form,
+    pins.test_mixed_A_steps_equal_layer_fwd, pins.test_chunked_with_per_token_A_equals_sequential,
 ]
 
 MUTATIONS = {
@@ -183,6 +196,8 @@ MUTATIONS = {
     "chunk_state_decay_from_start": ("scan_chunked", _chunked_state_decay_from_start),
     "dense_skips_inactive_experts": ("scan_separated_dense", _dense_skips_inactive_experts),
     "out_proj_transposed": ("out_proj", _out_proj_transposed),
+    "mixed_A_without_weights": ("mixed_A", _mixed_A_unweighted),
+    "mixed_A_first_slot_only": ("mixed_A", _mixed_A_first_slot),
 }
 
 

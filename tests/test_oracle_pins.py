@@ -126,6 +126,88 @@ def test_expert_proj_matches_elementwise_dot_products():
                 assert abs(z[t, j, c] - sum(W_exp[idx[t, j], c, d] * X[t, d] for d in range(D))) < 1e-12
 
 
+# ----------------------------------------------------------------------------- expert-mixed transition
+
+def test_mixed_A_is_the_router_weighted_mean():
+    # A~[t,h] = sum_j pi_tj A_exp[K_tj, h], written out term by term
+    rng = np.random.default_rng(8)
+    M, k, E, H = 6, 3, 5, 4
+    idx = np.array([rng.permutation(E)[:k] for _ in range(M)])
+    w = rng.dirichlet(np.ones(k), size=M)
+    A_exp = -np.exp(rng.uniform(0, math.log(16), size=(E, H)))
+    At = O.mixed_A(idx, w, A_exp)
+    for t in range(M):
+        for h in range(H):
+            assert abs(At[t, h] - sum(w[t, j] * A_exp[idx[t, j], h] for j in range(k))) < 1e-12
+    # a convex combination of negative values: strictly between the most and least negative expert values
+    assert (At < 0).all()
+    assert (At >= A_exp.min(axis=0) - 1e-12).all() and (At <= A_exp.max(axis=0) + 1e-12).all()
+
+
+def test_mixed_A_with_equal_experts_is_the_shared_layer():
+    # every expert carrying the same A row reduces the mixed transition to the shared one (the weights sum to 1)
+    L = _small_layer(np.random.default_rng(9), E=4, k=2)
+    E = L["W_exp"].shape[0]
+    ref = _fwd(L)
+    mixed = O.layer_fwd(L["X"], L["W_r"], L["W_dt"], L["b_dt"], None, L["W_exp"], L["H"], L["P"], L["N"], L["G"],
+                        L["k"], A_exp=np.tile(L["A"], (E, 1)))
+    np.testing.assert_allclose(mixed["y"], ref["y"], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(mixed["final"], ref["final"], rtol=1e-11, atol=1e-12)
+
+
+def test_mixed_A_decay_closed_form():
+    # a carried state with no injection (the B rows of every expert are zero) decays by
+    # prod_t exp(dt_t (pi_t0 A_e0 + pi_t1 A_e1)), read out by C~; checked against that product
+    rng = np.random.default_rng(10)
+    L = _small_layer(rng, B=1, T=5, E=3, k=2)
+    H, P, N, G = L["H"], L["P"], L["N"], L["G"]
+    L["W_exp"][:, H * P:H * P + G * N] = 0.0
+    E = L["W_exp"].shape[0]
+    A_exp = -np.exp(rng.uniform(0, math.log(16), size=(E, H)))
+    init = rng.standard_normal((1, H, N, P))
+    out = O.layer_fwd(L["X"], L["W_r"], L["W_dt"], L["b_dt"], None, L["W_exp"], H, P, N, G, L["k"], init=init,
+                      A_exp=A_exp)
+    g = L["X"][0] @ L["W_r"].T
+    dt = np.clip(np.log1p(np.exp(L["X"][0] @ L["W_dt"].T + L["b_dt"])), 1e-3, 0.1)
+    decay = np.ones(H)
+    for t in range(5):
+        top = np.argsort(-g[t].astype(np.float32), kind="stable")[:2]
+        e0, e1 = top
+        p1 = 1.0 / (1.0 + np.exp(g[t, e0] - g[t, e1]))
+        decay = decay * np.exp(dt[t] * ((1 - p1) * A_exp[e0] + p1 * A_exp[e1]))
+    np.testing.assert_allclose(out["final"][0], decay[:, None, None] * init[0], rtol=1e-12)
+    gh = O.group_of(H, G)
+    Ct = out["Ct"][4]
+    np.testing.assert_allclose(out["y"][0, 4], np.einsum("hn,hnp->hp", Ct[gh], decay[:, None, None] * init[0]),
+                               rtol=1e-10, atol=1e-12)
+
+
+def test_mixed_A_steps_equal_layer_fwd():
+    rng = np.random.default_rng(11)
+    L = _small_layer(rng, B=2, T=6, E=4, k=2)
+    A_exp = -np.exp(rng.uniform(0, math.log(16), size=(4, L["H"])))
+    full = O.layer_fwd(L["X"], L["W_r"], L["W_dt"], L["b_dt"], None, L["W_exp"], L["H"], L["P"], L["N"], L["G"],
+                       L["k"], A_exp=A_exp)
+    state = np.zeros((2, L["H"], L["N"], L["P"]))
+    for t in range(6):
+        y, state, _ = O.step(L["X"][:, t], L["W_r"], L["W_dt"], L["b_dt"], None, L["W_exp"], L["H"], L["P"], L["N"],
+                             L["G"], L["k"], state, A_exp=A_exp)
+        np.testing.assert_allclose(y, full["y"][:, t], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(state, full["final"], rtol=1e-11, atol=1e-12)
+
+
+def test_chunked_with_per_token_A_equals_sequential():
+    rng = np.random.default_rng(12)
+    Bpi, Xs, Ct, dt, A = _rand_streams(rng, 37, 2, 3, 4, 3, 5)
+    At = -np.exp(rng.uniform(0, math.log(16), size=(37, 3)))
+    ys, hs = O.scan_sequential(Bpi, Xs, Ct, dt, At)
+    yc, Hs, hc = O.scan_chunked(Bpi, Xs, Ct, dt, At, 16)
+    np.testing.assert_allclose(yc, ys, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(hc, hs, rtol=1e-10, atol=1e-12)
+    yb = O.scan_bruteforce(Bpi, Xs, Ct, dt, At)
+    np.testing.assert_allclose(yb, ys, rtol=1e-10, atol=1e-12)
+
+
 def test_out_proj_matches_elementwise_dot_products():
     # out[m][d] = sum_c y[m][c] W_out[d][c], written out term by term; a transposed W_out fails the shapes
     # (D != H*P) and, for a square W_out, the values
