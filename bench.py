@@ -12,8 +12,9 @@ On one GPU the default run adds two nested measurements to the same JSON line, t
 "decode" (swimba_step on 256 sequences, D2048 H64 N128 P64 E16 k2, state from a 512-token prefill; bound
 by HBM), "esweep" (the base layer at E in {8, 16, 32, 64}: layer and scan-stage times, which the
 method's cost statement says are flat in E, plus the separated-trajectory scan that runs k trajectories) and
-"out_proj" (the output projection y W_out^T on the base layer's y, bound by the tensor cores) and "mixed_A"
-(the base layer with the expert-mixed transition A~ = sum_j pi_j A_exp[K_j]).
+"out_proj" (the output projection y W_out^T on the base layer's y, bound by the tensor cores), "mixed_A"
+(the base layer with the expert-mixed transition A~ = sum_j pi_j A_exp[K_j]) and "groups" (the base layer
+with B and C shared by G in {H, H/4, 1} groups of heads: layer and scan times).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launching stream,
 with a write of 2x the L2 size between steps (outside the events) so every step reads its inputs from
@@ -315,6 +316,7 @@ class DecodeSession:
         swimba.layer_fwd(dp, inp["X"].to(dev).reshape(Mp, w.d_model), self.W, None, yp, self.state, None, None, wsp)
         torch.cuda.synchronize()
         del wsp, yp
+        torch.cuda.empty_cache()  # the prefill's workspace goes back to the driver: the step needs far less
         self.d = swimba.dims_of(w, seqlen=1)
         self.X = inp["X_step"].to(dev)
         self.y = torch.empty(w.batch, w.nheads * w.headdim, dtype=torch.bfloat16, device=dev)
@@ -476,6 +478,24 @@ def out_proj_measure(args, sess, inp, flush, stream, swimba):
                          "peak_source": f"bf16 dense, burst, {src}"}}
 
 
+def groups_measure(args, dev, flush, stream, swimba, base_out):
+    """The base layer with B and C shared by groups of heads, G in {H, H/4, 1}: per-step layer and scan
+    times (the heads of a group read the same B and C rows, which L2 then serves)."""
+    w0 = configs.BASE
+    res = {"G": [w0.G], "layer_ms": [base_out["ms_per_step"]],
+           "scan_ms": [base_out["stages_ms_per_step"].get("ssd_scan")]}
+    for w in (configs.BASE_G6, configs.BASE_G1):
+        G = w.G
+        torch.cuda.empty_cache()
+        sess = LayerSession(w, dev, inputs.make_inputs(w), swimba)
+        m = measure(sess, args, flush, stream, None, dev.index or 0, swimba, e2e=False)
+        res["G"].append(G)
+        res["layer_ms"].append(m["total_ms"] / args.steps)
+        res["scan_ms"].append(m["stage_ms"].get("ssd_scan", 0.0) / args.steps)
+        del sess
+    return res
+
+
 def run_gpu(args, w):
     from parameter_space_moe_b200 import swimba
     rank, world, local = rank_env()
@@ -515,6 +535,7 @@ def run_gpu(args, w):
         out["mixed_A"] = {"layer_ms": mm["total_ms"] / args.steps,
                           "stages_ms_per_step": {n: v / args.steps for n, v in mm["stage_ms"].items()}}
         del msess
+        out["groups"] = groups_measure(args, dev, flush, stream, swimba, out)
         torch.cuda.empty_cache()
         dw = configs.DECODE
         dsess = DecodeSession(dw, dev, inputs.make_inputs(dw), swimba)

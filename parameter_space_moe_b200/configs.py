@@ -71,4 +71,8 @@ LONG = Workload("long_B1_T32768_D2048_H64_E16_k2", batch=1, seqlen=32768, d_mode
 DECODE = Workload("decode_B256_D2048_H64_E16_k2", batch=256, seqlen=1, d_model=2048, nheads=64, headdim=64,
                   dstate=128, n_experts=16, top_k=2, chunk=256, dtype=BF16, seed=SEED0 + 4, prefill=512)
 
-ALL = {w.name: w for w in (TINY_F32, BASE, *(esweep(e) for e in ESWEEP_E), LONG, DECODE)}
+# The base layer with B and C shared by groups of heads (G = H/4 and G = 1, Mamba-2 style groups).
+BASE_G6 = BASE.with_(name="base_G6_B4_T2048_D768_H24_E8_k2", ngroups=6, seed=SEED0 + 5)
+BASE_G1 = BASE.with_(name="base_G1_B4_T2048_D768_H24_E8_k2", ngroups=1, seed=SEED0 + 6)
+
+ALL = {w.name: w for w in (TINY_F32, BASE, *(esweep(e) for e in ESWEEP_E), LONG, DECODE, BASE_G6, BASE_G1)}

@@ -88,7 +88,8 @@ def head_slice(inp, w, heads):
     H, P, N, G = w.nheads, w.headdim, w.dstate, w.G
     hpg = H // G
     groups = sorted({h // hpg for h in heads})
-    assert len(groups) == len(heads) or G == H, "sample whole groups or G == H"
+    whole = list(heads) == sorted(heads) and all(sum(1 for h in heads if h // hpg == g) == hpg for g in groups)
+    assert len(groups) == len(heads) or G == H or whole, "sample one head per group, or whole groups in order"
     W = inp["W_exp"]
     xcols = np.concatenate([np.arange(h * P, (h + 1) * P) for h in heads])
     bcols = np.concatenate([H * P + np.arange(g * N, (g + 1) * N) for g in groups])

@@ -65,6 +65,9 @@ BF16_VARIANTS = [
     configs.BASE.with_(name="bf16_P128_N64", batch=1, seqlen=300, d_model=128, nheads=2, headdim=128, dstate=64,
                        chunk=64, seed=22),
     configs.BASE.with_(name="bf16_G2", batch=1, seqlen=400, d_model=256, nheads=4, ngroups=2, chunk=128, seed=23),
+    # B and C shared by all 8 heads (G = 1), ragged, k = 3
+    configs.BASE.with_(name="bf16_H8_G1_k3", batch=2, seqlen=777, d_model=256, nheads=8, ngroups=1, n_experts=6,
+                       top_k=3, chunk=128, seed=26),
     # CTA-pair expert GEMM (>= 1536 rows per expert on average); the second has a ragged last column tile
     configs.BASE.with_(name="bf16_pair_gemm", batch=2, seqlen=1600, d_model=256, nheads=4, n_experts=2, seed=24),
     configs.BASE.with_(name="bf16_pair_ragged_cols", batch=3, seqlen=3100, d_model=192, nheads=3, dstate=64,
@@ -76,6 +79,27 @@ BF16_VARIANTS = [
 def test_layer_bf16_small(w):
     ey, ef, nfl = full_parity(w)
     assert ey <= 2e-3 and ef <= 2e-3, (ey, ef, nfl)
+
+
+@pytest.mark.parametrize("G", [6, 1])
+def test_layer_base_groups(G):
+    """Base sizes with B and C shared by groups of heads (G = H/4 and G = 1).  Every head of two of the four
+    sequences against the oracle."""
+    w = {6: configs.BASE_G6, 1: configs.BASE_G1}[G]
+    inp = inputs.make_inputs(w)
+    y, fin, idx = run_layer(w, inp)
+    X = f64(inp["X"])
+    g = O.router_logits(X.reshape(w.M, -1), f64(inp["W_r"]))
+    fl, forced = check_topk(to_np(idx), g, w.top_k)
+    fr = forced.reshape(w.batch, w.seqlen, w.top_k) if fl.any() else None
+    seqs = [0, 2]
+    ws = w.with_(batch=len(seqs))
+    ref = oracle_heads_blocked(inp, ws, X[seqs], list(range(w.nheads)), None if fr is None else fr[seqs],
+                               block=max(16 // (w.nheads // G), 1) * (w.nheads // G))
+    ya = to_np(y).reshape(w.batch, w.seqlen, w.nheads, w.headdim)[seqs]
+    ey, ef = rel(ya, ref["y"]), rel(to_np(fin)[seqs], ref["final"])
+    print(f"base G={G}: rel err y {ey:.3e} final {ef:.3e}")
+    assert ey <= 2e-3 and ef <= 2e-3
 
 
 def test_layer_base_full():

@@ -48,8 +48,19 @@ LONGCHAIN_ONE_HEAD = configs.BASE.with_(name="longchain_one_head_40_sub_chunks",
                                         nheads=1, n_experts=4, chunk=256, seed=94)
 LONGCHAIN_WIDE = configs.BASE.with_(name="longchain_160_heads", batch=2, seqlen=4100, d_model=128, nheads=80,
                                     n_experts=2, chunk=256, seed=95)
+# B and C shared by groups of heads: G = H / 4 with a ragged tail, G = 1 over 6 heads with k = 3, G = H / 2 on a
+# long hand-off chain, and 400 (sequence, head) rows in 200 groups
+SCAN_G4 = configs.BASE.with_(name="scan_H8_G2_ragged", batch=2, seqlen=333, d_model=128, nheads=8, ngroups=2,
+                             n_experts=4, chunk=128, seed=96)
+SCAN_G1_K3 = configs.BASE.with_(name="scan_H6_G1_k3", batch=1, seqlen=700, d_model=128, nheads=6, ngroups=1,
+                                n_experts=5, top_k=3, chunk=256, seed=97)
+LONGCHAIN_G = configs.BASE.with_(name="longchain_H4_G2", batch=1, seqlen=4300, d_model=128, nheads=4, ngroups=2,
+                                 n_experts=4, chunk=256, seed=98)
+SCAN_G_WIDE = configs.BASE.with_(name="scan_400_heads_G100", batch=2, seqlen=300, d_model=128, nheads=200,
+                                 ngroups=100, n_experts=2, chunk=256, seed=99)
+SCAN_GROUPED = [SCAN_G4, SCAN_G1_K3, LONGCHAIN_G, SCAN_G_WIDE]
 SCAN_CFGS = STAGE_CFGS + [SCAN_K1, SCAN_SHORT, SCAN_CHAIN, SCAN_WIDE, LONGCHAIN_K2, LONGCHAIN_K1, LONGCHAIN_ONE_HEAD,
-                          LONGCHAIN_WIDE]
+                          LONGCHAIN_WIDE] + SCAN_GROUPED
 _cache = {}
 
 
@@ -229,7 +240,8 @@ def test_ssd_scan(w, with_init):
         assert rel(to_np(cst)[b].transpose(1, 0, 2, 3), Hs) < state_tol_of(w)
 
 
-@pytest.mark.parametrize("w", [configs.TINY_F32, TC_P128, TC_Q64, LONGCHAIN_K2], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [configs.TINY_F32, TC_P128, TC_Q64, LONGCHAIN_K2, SCAN_G4, SCAN_G1_K3],
+                         ids=lambda w: w.name)
 def test_separated_scan(w):
     """The separated design ("k scans"): k trajectories with unscaled injections, pi-scaled readouts."""
     inp, Xf, ref, dev = _setup(w)
@@ -253,14 +265,15 @@ def test_separated_scan(w):
         assert rel(to_np(fin)[:, b], hs) < state_tol_of(w)
 
 
-@pytest.mark.parametrize("seqlen", [512, 4200], ids=["T512", "T4200"])
-def test_scan_lost_predecessor_times_out_without_fault(seqlen):
+@pytest.mark.parametrize("seqlen,groups", [(512, 0), (4200, 0), (512, 1)], ids=["T512", "T4200", "T512_G1"])
+def test_scan_lost_predecessor_times_out_without_fault(seqlen, groups):
     """Failure detection: the first sub-chunk of every head is made to go missing, so the successors'
     flag waits can never succeed.  They give up after their bounded wait, the status word reports
     SWIMBA_ERR_TIMEOUT (no fault, no hang), and the context stays usable: the normal scan that follows
     is correct."""
     import time
-    w = configs.BASE.with_(name=f"lost_chunk_T{seqlen}", batch=1, seqlen=seqlen, d_model=128, nheads=2, seed=87)
+    w = configs.BASE.with_(name=f"lost_chunk_T{seqlen}_G{groups}", batch=1, seqlen=seqlen, d_model=128, nheads=2,
+                           ngroups=groups, seed=87)
     inp, Xf, ref, dev = _setup(w)
     d = swimba.dims_of(w)
     Bpi, Xs, Cpi, dt = (t.cuda() for t in _oracle_streams_on_device(w, ref))
