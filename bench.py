@@ -560,7 +560,10 @@ def run_gpu(args, w):
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, bytes per launch) of a stage's kernel from one
 # ncu capture of the current kernel build; a stage/workload not listed reports null.  An entry is removed
 # whenever its kernel changes.
-PROFILED_TRAFFIC = {}
+PROFILED_TRAFFIC = {
+    ("base_B4_T2048_D768_H24_E8_k2", "expert_proj_mix"): 120178688 + 205011456,     # proj_tc_pair_kernel
+    ("decode_B256_D2048_H64_E16_k2", "expert_proj_mix"): 1347068672 + 21526528,     # proj_tc_kernel
+}
 
 
 def tensor_peak(peaks, clocks):
