@@ -265,8 +265,8 @@ class LayerSession:
         self.sw.layer_fwd(self.d, self.X, self.W, None, self.y, self.fin, None, None, self.ws)
 
     def e2e_step(self):
-        """Host X in, host y out through swimba_layer_fwd_host (copies of one group of sequences overlap
-        the compute of another)."""
+        """Host X in, host y out through swimba_layer_fwd_host: 4 time segments of every sequence chained
+        through the final state, each segment's copies overlapping another segment's compute."""
         self.sw.layer_fwd_host(self.d, self.Xh, self.W, None, self.yh, self.fin, self.X, self.y, self.ws, chunks=4)
 
     def extras(self, stream, steps):

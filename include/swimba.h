@@ -186,8 +186,9 @@ swimba_status swimba_layer_fwd(const swimba_dims* dims, const void* X, const swi
  *   X_dev, y_dev: device staging buffers of the same sizes (caller-owned)
  *   init_state / final_state: device [B][H][N][P] fp32 or NULL, as for swimba_layer_fwd
  *   ws: workspace sized for the full dims; chunks in [1, 16], clamped to the batch
- * A single sequence (batch 1) with final_state given is split along time instead, into segments of whole
- * 128-token sub-chunks chained through final_state (which then also carries the state between segments).
+ * With final_state given the groups are time segments instead: whole 128-token sub-chunks of every
+ * sequence, chained through final_state (which then also carries the state between segments); the staging
+ * buffers then hold the groups one after another ([batch][segment] rows each).
  * Returns SWIMBA_ERR_INVALID_ARG for null or misaligned pointers; the result is complete once `stream`
  * reaches the point after this call (synchronise `stream` before reading y_host).  The copy streams are
  * shared by all calls on a device: calls that may overlap in time must come from one host thread. */

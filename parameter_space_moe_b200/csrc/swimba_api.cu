@@ -437,10 +437,11 @@ swimba_status swimba_layer_fwd_host(const swimba_dims* dims, const void* X_host,
   const int want = chunks < kMaxHostChunks ? chunks : kMaxHostChunks;
   const size_t xrow = (size_t)d.D * elem_bytes(d.dtype), yrow = (size_t)d.HP * elem_bytes(d.dtype);
   const size_t state = (size_t)d.H * d.N * d.P;
-  // A single sequence is split along time instead, into segments of whole 128-token sub-chunks chained
-  // through final_state (segment c starts from segment c - 1's final state), when final_state is given.
+  // With final_state given the groups are time segments of whole 128-token sub-chunks of every sequence,
+  // chained through final_state (segment c starts from segment c - 1's final state): each group keeps all
+  // (sequence, head) rows, so the scan's hand-off chains stay short.  Otherwise groups of whole sequences.
   const int max_seg = ceil_div(d.T, 128);
-  const bool by_time = d.Bsz == 1 && want > 1 && final_state != nullptr && max_seg > 1;
+  const bool by_time = want > 1 && final_state != nullptr && max_seg > 1;
   const int nch = by_time ? (want < max_seg ? want : max_seg) : (want < d.Bsz ? want : d.Bsz);
   // the copies start after the work already queued on `stream`
   SW_CUDA(cudaEventRecord(q->start, s));
@@ -448,34 +449,40 @@ swimba_status swimba_layer_fwd_host(const swimba_dims* dims, const void* X_host,
   SW_CUDA(cudaStreamWaitEvent(q->d2h, q->start, 0));
   for (int c = 0; c < nch; ++c) {
     swimba_dims dc = *dims;
-    size_t r0, rows;
+    size_t r0;          // the group's first row in the staging buffers (group-major: [batch][len] of the group)
+    size_t h0, len, n;  // host side: n blocks of len rows, block b at row h0 + b * T
     const float* init_c;
     float* fin_c;
-    if (by_time) {  // sub-chunk-aligned time segments of the one sequence
+    if (by_time) {  // sub-chunk-aligned time segments of every sequence
       const int s0 = (int)((long long)max_seg * c / nch) * 128, s1 = c + 1 == nch ? d.T : (int)((long long)max_seg * (c + 1) / nch) * 128;
-      r0 = (size_t)s0;
-      rows = (size_t)(s1 - s0);
+      len = (size_t)(s1 - s0);
+      n = (size_t)d.Bsz;
+      h0 = (size_t)s0;
+      r0 = (size_t)d.Bsz * s0;
       dc.seqlen = s1 - s0;
       init_c = c == 0 ? init_state : final_state;
       fin_c = final_state;
     } else {  // groups of whole sequences
       const int b0 = (int)((long long)d.Bsz * c / nch), b1 = (int)((long long)d.Bsz * (c + 1) / nch);
-      r0 = (size_t)b0 * d.T;
-      rows = (size_t)(b1 - b0) * d.T;
+      len = (size_t)(b1 - b0) * d.T;
+      n = 1;
+      h0 = (size_t)b0 * d.T;
+      r0 = h0;
       dc.batch = b1 - b0;
       init_c = init_state ? init_state + (size_t)b0 * state : nullptr;
       fin_c = final_state ? final_state + (size_t)b0 * state : nullptr;
     }
-    SW_CUDA(cudaMemcpyAsync((char*)X_dev + r0 * xrow, (const char*)X_host + r0 * xrow, rows * xrow,
-                            cudaMemcpyHostToDevice, q->h2d));
+    const size_t hstride = n > 1 ? (size_t)d.T : len;  // host rows from one block to the next
+    SW_CUDA(cudaMemcpy2DAsync((char*)X_dev + r0 * xrow, len * xrow, (const char*)X_host + h0 * xrow, hstride * xrow,
+                              len * xrow, n, cudaMemcpyHostToDevice, q->h2d));
     SW_CUDA(cudaEventRecord(q->in[c], q->h2d));
     SW_CUDA(cudaStreamWaitEvent(s, q->in[c], 0));
     SW_TRY(swimba_layer_fwd(&dc, (const char*)X_dev + r0 * xrow, w, init_c, (char*)y_dev + r0 * yrow, fin_c, nullptr,
                             nullptr, ws, ws_bytes, stream));
     SW_CUDA(cudaEventRecord(q->out[c], s));
     SW_CUDA(cudaStreamWaitEvent(q->d2h, q->out[c], 0));
-    SW_CUDA(cudaMemcpyAsync((char*)y_host + r0 * yrow, (const char*)y_dev + r0 * yrow, rows * yrow,
-                            cudaMemcpyDeviceToHost, q->d2h));
+    SW_CUDA(cudaMemcpy2DAsync((char*)y_host + h0 * yrow, hstride * yrow, (const char*)y_dev + r0 * yrow, len * yrow,
+                              len * yrow, n, cudaMemcpyDeviceToHost, q->d2h));
   }
   SW_CUDA(cudaEventRecord(q->done, q->d2h));
   SW_CUDA(cudaStreamWaitEvent(s, q->done, 0));
