@@ -177,6 +177,48 @@ def scan_sequential(Bpi, Xs, Ct, dt, A, init=None, stats=None):
     return y, h
 
 
+def scan_backward(Bpi, Xs, Ct, dt, A, dy, init=None):
+    """Gradients of L = sum_t <dy_t, y_t> for one batch row of scan_sequential, by the adjoint recurrence
+    run backwards in time (reverse-mode differentiation of [notes] key design 1's second display equation):
+        lam_t    = dL/dh_t = C~_t (x) dy_t + a_{t+1} lam_{t+1}          (lam = 0 after the last token)
+        dBpi_tj  = lam_t Xs_tj          dXs_tj = lam_t^T Bpi_tj          dC~_t = h_t dy_t
+        g_t      = a_t <lam_t, h_{t-1}>  (the gradient of the log-decay dA_t = dt_t A)
+        d dt_t   = g_t A_h,   dA_h = sum_t g_t dt_t,   d init = a_0 lam_0 (with h_{-1} = init).
+    With G < H groups the B and C~ gradients sum over the heads of a group.  A may be [H] or [T,H] (then dA
+    is [T,H], the gradient of each token's transition).
+    Returns a dict: dBpi [T,k,G,N], dXs [T,k,H,P], dCt [T,G,N], ddt [T,H], dA, dinit [H,N,P]."""
+    T, k, H, P = Xs.shape
+    G, N = Bpi.shape[2], Bpi.shape[3]
+    g = group_of(H, G)
+    dAt = log_decay(dt, A) * np.ones((T, H))
+    a = np.exp(dAt)                                                    # [T,H]
+    hs = np.zeros((T + 1, H, N, P))                                    # hs[t + 1] = h_t, hs[0] = init
+    if init is not None:
+        hs[0] = init
+    for t in range(T):
+        U = np.einsum("jhn,jhp->hnp", Bpi[t][:, g], Xs[t])
+        hs[t + 1] = a[t][:, None, None] * hs[t] + U
+    dBpi = np.zeros(Bpi.shape)
+    dXs = np.zeros(Xs.shape)
+    dCt = np.zeros(Ct.shape)
+    gdA = np.zeros((T, H))
+    lam = np.zeros((H, N, P))
+    for t in range(T - 1, -1, -1):
+        if t + 1 < T:
+            lam = a[t + 1][:, None, None] * lam
+        lam = lam + np.einsum("hn,hp->hnp", Ct[t][g], dy[t])
+        for gi in range(G):
+            heads = np.nonzero(g == gi)[0]
+            dBpi[t, :, gi] = np.einsum("hnp,jhp->jn", lam[heads], Xs[t][:, heads])
+            dCt[t, gi] = np.einsum("hnp,hp->n", hs[t + 1][heads], dy[t][heads])
+        dXs[t] = np.einsum("hnp,jhn->jhp", lam, Bpi[t][:, g])
+        gdA[t] = a[t] * np.einsum("hnp,hnp->h", lam, hs[t])
+    ddt = gdA * (np.ones((T, H)) * np.asarray(A))
+    dA = (gdA * dt).sum(axis=0) if np.ndim(A) == 1 else gdA * dt
+    dinit = a[0][:, None, None] * lam
+    return dict(dBpi=dBpi, dXs=dXs, dCt=dCt, ddt=ddt, dA=dA, dinit=dinit)
+
+
 def scan_bruteforce(Bpi, Xs, Ct, dt, A, init=None):
     """The same layer as one materialised semiseparable matrix product (quadratic in T):
         y_t = sum_{s<=t} (prod_{r=s+1..t} a_r) sum_j (C~_t . Bpi_sj) Xs_sj  +  (prod_{r<=t} a_r) C~_t^T h_init.

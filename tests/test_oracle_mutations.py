@@ -6,8 +6,9 @@ dt clamp dropped, every slot projected with its first slot's expert, B and C swa
 split, C~ summed without the router weights, the injection added before the decay, the decay's sign
 flipped, the chunked form's causal mask shifted by one, the chunk-state decay taken from the chunk
 start instead of its end, the separated-E design advancing only the active experts, the output
-projection applied with its matrix transposed, and the expert-mixed transition summed without the router
-weights or taken from the first active expert alone."""
+projection applied with its matrix transposed, the expert-mixed transition summed without the router
+weights or taken from the first active expert alone, and the scan's adjoint recurrence without its decay or
+with the decay gradient taken one state late."""
 import numpy as np
 import pytest
 
@@ -157,6 +158,45 @@ def _mixed_A_first_slot(idx, w, A_exp):
     return np.asarray(A_exp)[idx[:, 0]]
 
 
+def _backward_mutant(Bpi, Xs, Ct, dt, A, dy, init=None, decay_adjoint=True, h_shift=0):
+    # the adjoint recurrence with one planted change: no decay between adjoint steps, or the log-decay
+    # gradient taken against h_t instead of h_{t-1}
+    T, k, H, P = Xs.shape
+    G, N = Bpi.shape[2], Bpi.shape[3]
+    g = O.group_of(H, G)
+    a = np.exp(O.log_decay(dt, A) * np.ones((T, H)))
+    hs = np.zeros((T + 1, H, N, P))
+    if init is not None:
+        hs[0] = init
+    for t in range(T):
+        hs[t + 1] = a[t][:, None, None] * hs[t] + np.einsum("jhn,jhp->hnp", Bpi[t][:, g], Xs[t])
+    out = {n: np.zeros(v.shape) for n, v in (("dBpi", Bpi), ("dXs", Xs), ("dCt", Ct))}
+    gdA = np.zeros((T, H))
+    lam = np.zeros((H, N, P))
+    for t in range(T - 1, -1, -1):
+        if t + 1 < T and decay_adjoint:
+            lam = a[t + 1][:, None, None] * lam
+        lam = lam + np.einsum("hn,hp->hnp", Ct[t][g], dy[t])
+        for gi in range(G):
+            heads = np.nonzero(g == gi)[0]
+            out["dBpi"][t, :, gi] = np.einsum("hnp,jhp->jn", lam[heads], Xs[t][:, heads])
+            out["dCt"][t, gi] = np.einsum("hnp,hp->n", hs[t + 1][heads], dy[t][heads])
+        out["dXs"][t] = np.einsum("hnp,jhn->jhp", lam, Bpi[t][:, g])
+        gdA[t] = a[t] * np.einsum("hnp,hnp->h", lam, hs[t + h_shift])
+    out["ddt"] = gdA * (np.ones((T, H)) * np.asarray(A))
+    out["dA"] = (gdA * dt).sum(axis=0) if np.ndim(A) == 1 else gdA * dt
+    out["dinit"] = a[0][:, None, None] * lam
+    return out
+
+
+def _backward_no_adjoint_decay(Bpi, Xs, Ct, dt, A, dy, init=None):
+    return _backward_mutant(Bpi, Xs, Ct, dt, A, dy, init, decay_adjoint=False)
+
+
+def _backward_decay_gradient_off_by_one(Bpi, Xs, Ct, dt, A, dy, init=None):
+    return _backward_mutant(Bpi, Xs, Ct, dt, A, dy, init, h_shift=1)
+
+
 def _out_proj_transposed(y, W_out):
     # the projection matrix applied transposed (shapes permitting: D == H*P)
     return np.asarray(y) @ np.asarray(W_out)
@@ -164,7 +204,7 @@ def _out_proj_transposed(y, W_out):
 
 ORIG = {name: getattr(O, name) for name in
         ("topk_weights", "topk_select", "dt_proj", "expert_proj", "split_streams", "mix", "scan_sequential",
-         "scan_chunked", "scan_separated_dense", "out_proj", "mixed_A")}
+         "scan_chunked", "scan_separated_dense", "out_proj", "mixed_A", "scan_backward")}
 
 # every pin, called with the parameters its decorator gives
 ALL_PINS = [
@@ -181,6 +221,7 @@ ALL_PINS = [
     pins.test_out_proj_identity_and_selection, pins.test_mixed_A_is_the_router_weighted_mean,
     pins.test_mixed_A_with_equal_experts_is_the_shared_layer, pins.test_mixed_A_decay_closed_form,
     pins.test_mixed_A_steps_equal_layer_fwd, pins.test_chunked_with_per_token_A_equals_sequential,
+    lambda: pins.test_scan_backward_matches_finite_differences(2), pins.test_scan_backward_per_token_transition,
 ]
 
 MUTATIONS = {
@@ -198,6 +239,8 @@ MUTATIONS = {
     "out_proj_transposed": ("out_proj", _out_proj_transposed),
     "mixed_A_without_weights": ("mixed_A", _mixed_A_unweighted),
     "mixed_A_first_slot_only": ("mixed_A", _mixed_A_first_slot),
+    "adjoint_without_decay": ("scan_backward", _backward_no_adjoint_decay),
+    "decay_gradient_off_by_one": ("scan_backward", _backward_decay_gradient_off_by_one),
 }
 
 

@@ -126,6 +126,53 @@ def test_expert_proj_matches_elementwise_dot_products():
                 assert abs(z[t, j, c] - sum(W_exp[idx[t, j], c, d] * X[t, d] for d in range(D))) < 1e-12
 
 
+# ----------------------------------------------------------------------------- scan gradients
+
+def _loss(Bpi, Xs, Ct, dt, A, dy, init):
+    y, _ = O.scan_sequential(Bpi, Xs, Ct, dt, A, init)
+    return float((dy * y).sum())
+
+
+@pytest.mark.parametrize("G", [2, 1])
+def test_scan_backward_matches_finite_differences(G):
+    # every gradient of L = sum <dy, y> against central differences of the forward recurrence, entry by entry
+    rng = np.random.default_rng(13 + G)
+    T, k, H, P, N = 6, 2, 2, 3, 2
+    Bpi, Xs, Ct, dt, A = _rand_streams(rng, T, k, H, P, G, N)
+    dy = rng.standard_normal((T, H, P))
+    init = rng.standard_normal((H, N, P))
+    got = O.scan_backward(Bpi, Xs, Ct, dt, A, dy, init)
+    args = dict(Bpi=Bpi, Xs=Xs, Ct=Ct, dt=dt, A=A, init=init)
+    names = dict(Bpi="dBpi", Xs="dXs", Ct="dCt", dt="ddt", A="dA", init="dinit")
+    eps = 1e-6
+    for name, arr in args.items():
+        num = np.zeros(arr.shape)
+        for idx in np.ndindex(arr.shape):
+            hi = {n: v.copy() for n, v in args.items()}
+            lo = {n: v.copy() for n, v in args.items()}
+            hi[name][idx] += eps
+            lo[name][idx] -= eps
+            num[idx] = (_loss(dy=dy, **hi) - _loss(dy=dy, **lo)) / (2 * eps)
+        np.testing.assert_allclose(got[names[name]], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_scan_backward_per_token_transition():
+    # with a [T,H] transition the dA gradient is per token; central differences on each entry
+    rng = np.random.default_rng(17)
+    T, k, H, P, N = 5, 1, 2, 2, 3
+    Bpi, Xs, Ct, dt, _ = _rand_streams(rng, T, k, H, P, 2, N)
+    At = -np.exp(rng.uniform(0, math.log(16), size=(T, H)))
+    dy = rng.standard_normal((T, H, P))
+    got = O.scan_backward(Bpi, Xs, Ct, dt, At, dy)
+    eps = 1e-6
+    for idx in np.ndindex(At.shape):
+        hi, lo = At.copy(), At.copy()
+        hi[idx] += eps
+        lo[idx] -= eps
+        num = (_loss(Bpi, Xs, Ct, dt, hi, dy, None) - _loss(Bpi, Xs, Ct, dt, lo, dy, None)) / (2 * eps)
+        assert abs(got["dA"][idx] - num) <= 1e-6 * max(1.0, abs(num))
+
+
 # ----------------------------------------------------------------------------- expert-mixed transition
 
 def test_mixed_A_is_the_router_weighted_mean():
