@@ -13,8 +13,9 @@ On one GPU the default run adds two nested measurements to the same JSON line, t
 by HBM), "esweep" (the base layer at E in {8, 16, 32, 64}: layer and scan-stage times, which the
 method's cost statement says are flat in E, plus the separated-trajectory scan that runs k trajectories) and
 "out_proj" (the output projection y W_out^T on the base layer's y, bound by the tensor cores), "mixed_A"
-(the base layer with the expert-mixed transition A~ = sum_j pi_j A_exp[K_j]) and "groups" (the base layer
-with B and C shared by G in {H, H/4, 1} groups of heads: layer and scan times).
+(the base layer with the expert-mixed transition A~ = sum_j pi_j A_exp[K_j]), "groups" (the base layer
+with B and C shared by G in {H, H/4, 1} groups of heads: layer and scan times) and "scan_bwd" (the scan
+gradients at the base sizes, bound by fp32 CUDA-core arithmetic).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launching stream,
 with a write of 2x the L2 size between steps (outside the events) so every step reads its inputs from
@@ -146,7 +147,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self.ok:
@@ -447,6 +448,67 @@ def esweep_measure(args, dev, flush, stream, swimba):
     return out
 
 
+def scan_bwd_flops(w):
+    """FLOPs the scan-gradient kernels execute (2 per FMA), 64-token sub-chunks of L tokens, T2 = L (L + 1) / 2
+    causal pairs: per sub-chunk and head k [3 L N P + T2 (3 N + 2 P)] + 2 L N P FMAs (end states, the carried-
+    state terms, the score tiles, and the Xs, Bpi and C~ contractions)."""
+    N, P, k = w.dstate, w.headdim, w.top_k
+    total = 0
+    for t0 in range(0, w.seqlen, 64):
+        L = min(64, w.seqlen - t0)
+        T2 = L * (L + 1) // 2
+        total += k * (3 * L * N * P + T2 * (3 * N + 2 * P)) + 2 * L * N * P
+    return 2.0 * total * w.batch * w.nheads
+
+
+def scan_bwd_measure(args, dev, flush, stream, swimba):
+    """The scan gradients (swimba_ssd_scan_bwd) at the base layer's sizes on seeded streams, timed alone; bound by
+    the fp32 CUDA-core arithmetic, against 148 SMs x 128 fp32 lanes x 2 FLOP x the maximum SM clock."""
+    w = configs.BASE
+    g = torch.Generator().manual_seed(131)
+    M, k, H, P, N = w.M, w.top_k, w.nheads, w.headdim, w.dstate
+    Bpi = (0.5 * torch.randn(M, k, H, N, generator=g)).half().to(dev)
+    Xs = torch.randn(M, k, H, P, generator=g).half().to(dev)
+    Cpi = (0.5 * torch.randn(M, k, H, N, generator=g)).half().to(dev)
+    dt = (1e-3 + 0.099 * torch.rand(M, H, generator=g)).to(dev)
+    A = inputs.make_inputs(w, with_x=False)["A"].to(dev)
+    dy = torch.randn(M, H, P, generator=g).to(dev)
+    outs = [torch.empty(M, k, H, N, device=dev), torch.empty(M, k, H, P, device=dev), torch.empty(M, H, N, device=dev),
+            torch.empty(M, H, device=dev), torch.empty(H, device=dev)]
+    d = swimba.dims_of(w)
+    ws = torch.empty(swimba.workspace_size(d), dtype=torch.uint8, device=dev)
+    call = lambda: swimba.ssd_scan_bwd(d, Bpi, Xs, Cpi, dt, A, None, dy, *outs, None, ws)
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tot = 0.0
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    if swimba.check_device_status() != 0:
+        raise RuntimeError("swimba_ssd_scan_bwd raised a device status")
+    secs = tot / args.steps / 1e3
+    flops = scan_bwd_flops(w)
+    mhz = 1965.0
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(pynvml.nvmlDeviceGetHandleByIndex(dev.index or 0),
+                                                     pynvml.NVML_CLOCK_SM))
+    except Exception:
+        pass
+    peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    return {"ms": secs * 1e3, "flops": flops,
+            "roofline": {"bound": "alu", "achieved": flops / secs / 1e12, "peak": peak, "unit": "TFLOP/s",
+                         "frac": flops / secs / 1e12 / peak,
+                         "peak_source": f"148 SMs x 128 fp32 lanes x 2 FLOP x {mhz:.0f} MHz (max SM clock)"}}
+
+
 def out_proj_measure(args, sess, inp, flush, stream, swimba):
     """The output projection out = y W_out^T (swimba_out_proj) on the layer's own y, timed alone: K launches
     between L2 flushes, against the burst bf16 peak (a kernel timed alone)."""
@@ -536,6 +598,8 @@ def run_gpu(args, w):
                           "stages_ms_per_step": {n: v / args.steps for n, v in mm["stage_ms"].items()}}
         del msess
         out["groups"] = groups_measure(args, dev, flush, stream, swimba, out)
+        torch.cuda.empty_cache()
+        out["scan_bwd"] = scan_bwd_measure(args, dev, flush, stream, swimba)
         torch.cuda.empty_cache()
         dw = configs.DECODE
         dsess = DecodeSession(dw, dev, inputs.make_inputs(dw), swimba)

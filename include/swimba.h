@@ -214,6 +214,23 @@ swimba_status swimba_separated_scan(const swimba_dims* dims, const void* B, cons
                                     const float* dt, const float* A, const float* init_states, void* y,
                                     float* final_states, void* ws, size_t ws_bytes, void* stream);
 
+/* Gradients of the chunked scan (swimba_ssd_scan over all k key and read slots) for the loss
+ * L = sum_t <dy_t, y_t>, i.e. the vector-Jacobian product with an upstream gradient dy.  Paper: notes,
+ * key design 1, second display equation differentiated in reverse (the notes train the model: loss
+ * function / training strategy); the adjoint state runs backwards through the same transition a_t.
+ *   Bpi, Xs, Cpi, dt, A, init_state  as for swimba_ssd_scan (init_state may be NULL: zero)
+ *   dy      [M][H][P] fp32: upstream gradient of y
+ *   dBpi    [M][k][G][N] fp32 out     dXs [M][k][H][P] fp32 out
+ *   dCt     [M][G][N] fp32 out: gradient of C~ = sum_j Cpi_j (every slot's Cpi receives it)
+ *   d_dt    [M][H] fp32 out           dA [H] fp32 out (summed over tokens and sequences)
+ *   d_init  [B][H][N][P] fp32 out or NULL
+ * CUDA cores in fp32 over 64-token sub-chunks (the gradient kernel takes up to 226 KB of shared memory at
+ * N = P = 128); needs the layer workspace (the same dims' swimba_workspace_size). */
+swimba_status swimba_ssd_scan_bwd(const swimba_dims* dims, const void* Bpi, const void* Xs, const void* Cpi,
+                                  const float* dt, const float* A, const float* init_state, const float* dy,
+                                  float* dBpi, float* dXs, float* dCt, float* d_dt, float* dA, float* d_init,
+                                  void* ws, size_t ws_bytes, void* stream);
+
 /* The layer's output projection: out = y W_out^T, one projection shared by every expert (the layer has one
  * recurrence and one readout).  Paper: gist.science Technical Summary, Architecture Details (the shared
  * recurrence "followed by a single output projection").

@@ -132,6 +132,13 @@ cudaError_t launch_proj_simt(const Dims& d, const void* X, const void* w_exp, co
 cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int2* rowmeta,
                            const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, int mode, void* bpi,
                            void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s);
+// Scan gradients (CUDA cores, 64-token sub-chunks): states of every sub-chunk in hstart/work, cs ends in cse.
+int scan_bwd_subchunks(const Dims& d);
+size_t scan_bwd_smem(const Dims& d);
+cudaError_t launch_scan_bwd(const Dims& d, const void* bpi, const void* xs, const void* cpi, const float* dt,
+                            const float* A, const float* init, const float* dy, float* dbpi, float* dxs, float* dct,
+                            float* ddt, float* dA, float* dinit, float* hstart, float* work, float* cse,
+                            cudaStream_t s);
 cudaError_t launch_mixed_a(const Dims& d, const int32_t* idx, const float* wts, const float* A_exp, const float* dt,
                            float* dA, float* ones, unsigned* st, cudaStream_t s);
 cudaError_t launch_out_proj(const Dims& d, const void* y, const void* w_out, void* out, unsigned* st,

@@ -78,7 +78,9 @@ WsPlan plan_workspace(const Dims& d) {
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
   const size_t Mk = (size_t)d.M * d.k;
   const size_t sb = elem_bytes(stream_dtype_of(d.dtype));
-  const size_t states = (size_t)d.Bsz * d.H * d.nc * d.N * d.P * 4;
+  // chunk states: per Q-token chunk for the CUDA-core scan, per 64-token sub-chunk for the scan gradients
+  const size_t nst = (size_t)scan_bwd_subchunks(d) > (size_t)d.nc ? (size_t)scan_bwd_subchunks(d) : (size_t)d.nc;
+  const size_t states = (size_t)d.Bsz * d.H * nst * d.N * d.P * 4;
   p.status = take(256);
   p.topk_idx = take(Mk * 4);
   p.topk_w = take(Mk * 4);
@@ -103,7 +105,7 @@ WsPlan plan_workspace(const Dims& d) {
   p.ysum = take((size_t)d.M * d.HP * 4);
   p.schunk = take(states);
   p.hstart = take(states);
-  p.cslast = take((size_t)d.Bsz * d.H * d.nc * 4);
+  p.cslast = take((size_t)d.Bsz * d.H * nst * 4);
   p.exch = take((size_t)d.Bsz * d.H * nsub * d.N * d.P * 4);
   p.total = o;
   return p;
@@ -541,6 +543,27 @@ swimba_status swimba_out_proj(const swimba_dims* dims, const void* y, const void
   unsigned* st = device_status();
   if (!st) return SWIMBA_ERR_CUDA;
   return cuda_status(launch_out_proj(d, y, w_out, out, st, (cudaStream_t)stream));
+}
+
+swimba_status swimba_ssd_scan_bwd(const swimba_dims* dims, const void* Bpi, const void* Xs, const void* Cpi,
+                                  const float* dt, const float* A, const float* init_state, const float* dy,
+                                  float* dBpi, float* dXs, float* dCt, float* d_dt, float* dA, float* d_init,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  if (!ok_ptr(Bpi) || !ok_ptr(Xs) || !ok_ptr(Cpi) || !ok_ptr(dt) || !A || !ok_ptr(dy) || !ok_ptr(dBpi) ||
+      !ok_ptr(dXs) || !ok_ptr(dCt) || !ok_ptr(d_dt) || !dA || !ok_opt(init_state) || !ok_opt(d_init))
+    return SWIMBA_ERR_INVALID_ARG;
+  if (scan_bwd_smem(d) > (size_t)227 * 1024) return SWIMBA_ERR_UNSUPPORTED;
+  SW_TRY(check_ws(d, ws, ws_bytes));
+  WsPlan p = plan_workspace(d);
+  char* b = (char*)ws;
+  cudaStream_t s = (cudaStream_t)stream;
+  prof_begin(s);
+  SW_CUDA(launch_scan_bwd(d, Bpi, Xs, Cpi, dt, A, init_state, dy, dBpi, dXs, dCt, d_dt, dA, d_init,
+                          (float*)(b + p.hstart), (float*)(b + p.schunk), (float*)(b + p.cslast), s));
+  prof_mark(s, "ssd_scan_bwd");
+  return SWIMBA_OK;
 }
 
 swimba_status swimba_check_device_status(void* stream) {

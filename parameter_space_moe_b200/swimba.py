@@ -22,7 +22,8 @@ EXPORTS = ("swimba_workspace_size", "swimba_stream_dtype", "swimba_router_topk",
            "swimba_expert_proj", "swimba_mix", "swimba_ssd_scan", "swimba_layer_fwd", "swimba_step",
            "swimba_separated_scan", "swimba_check_device_status", "swimba_status_string",
            "swimba_profile_enable", "swimba_profile_read", "swimba_launch_count", "swimba_dispatch_noalloc",
-           "swimba_layer_fwd_host", "swimba_debug_scan_lost_first_chunk", "swimba_out_proj")
+           "swimba_layer_fwd_host", "swimba_debug_scan_lost_first_chunk", "swimba_out_proj",
+           "swimba_ssd_scan_bwd")
 
 
 class SwimbaError(RuntimeError):
@@ -72,6 +73,7 @@ def lib():
             "swimba_step": [P(Dims), vp, P(Weights), vp, vp, vp, vp, sz, vp],
             "swimba_separated_scan": [P(Dims), vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_out_proj": [P(Dims), vp, vp, vp, vp],
+            "swimba_ssd_scan_bwd": [P(Dims), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_check_device_status": [vp],
         }
         L.swimba_profile_enable.restype = ctypes.c_int
@@ -186,6 +188,12 @@ def separated_scan(d, B, Xs, Cpi, dt, A, init_states, y, final_states, ws, strea
                                                                  _p(A), _p(init_states), _p(y), _p(final_states),
                                                                  _p(ws), ws.numel() * ws.element_size(),
                                                                  _stream(stream)))
+
+
+def ssd_scan_bwd(d, Bpi, Xs, Cpi, dt, A, init_state, dy, dBpi, dXs, dCt, d_dt, dA, d_init, ws, stream=None):
+    _check("swimba_ssd_scan_bwd", lib().swimba_ssd_scan_bwd(
+        ctypes.byref(d), _p(Bpi), _p(Xs), _p(Cpi), _p(dt), _p(A), _p(init_state), _p(dy), _p(dBpi), _p(dXs),
+        _p(dCt), _p(d_dt), _p(dA), _p(d_init), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def out_proj(d, y, w_out, out, stream=None):

@@ -98,6 +98,8 @@ def test_dispatch_entry_points_agree_on_unsupported_dims(L, kw):
     assert L.swimba_dispatch(ctypes.byref(d), fake, fake, fake, fake, 1 << 40, None) == 2
     assert L.swimba_dispatch_noalloc(ctypes.byref(d), fake, fake, fake, None) == 2
     assert L.swimba_out_proj(ctypes.byref(d), fake, fake, fake, None) == 2
+    assert L.swimba_ssd_scan_bwd(ctypes.byref(d), fake, fake, fake, fake, fake, None, fake, fake, fake, fake, fake,
+                                 fake, None, fake, 1 << 40, None) == 2
 
 
 def test_null_misaligned_and_workspace_errors(L):
@@ -124,6 +126,12 @@ def test_null_misaligned_and_workspace_errors(L):
     assert L.swimba_step(ctypes.byref(d), fake, ctypes.byref(w), fake, fake, None, fake, need, None) == 1
     # mix rejects unknown flags
     assert L.swimba_mix(ctypes.byref(d), fake, fake, 8, fake, fake, fake, None) == 1
+    # scan gradients: null and misaligned pointers, workspace too small
+    bwd = lambda dy, ws=fake, n=need: L.swimba_ssd_scan_bwd(ctypes.byref(d), fake, fake, fake, fake, fake, None, dy,
+                                                         fake, fake, fake, fake, fake, None, ws, n, None)
+    assert bwd(None) == 1
+    assert bwd(odd) == 1
+    assert bwd(fake, n=need - 1) == 4
     # output projection: every pointer non-null and 16-byte aligned
     assert L.swimba_out_proj(ctypes.byref(d), None, fake, fake, None) == 1
     assert L.swimba_out_proj(ctypes.byref(d), fake, odd, fake, None) == 1
