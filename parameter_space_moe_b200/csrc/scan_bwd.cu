@@ -14,7 +14,8 @@
 //               - e^{cs_end - cs_t} sum_j Bpi_tj . Lam_{c+1} Xs_tj   (+ at the last token: e^{cs_end} <Lam, H_c>
 //               + sum_{s,j} e^{cs_end - cs_s} Bpi_sj . Lam_{c+1} Xs_sj)
 //     dA_r    = sum_{t >= r} q_t,   d dt_r = dA_r A_h,   dA_h = sum_r dA_r dt_r,   d init = Lam_0.
-// With G < H the Bpi and C~ gradients of a group's heads are summed (atomic adds into zeroed outputs).
+// With G < H the Bpi and C~ gradients of a group's heads are summed (atomic adds into zeroed outputs); with
+// G = H every output element is written by exactly one CTA.
 #include "common.cuh"
 
 namespace swimba {
@@ -34,25 +35,77 @@ struct BwdArgs {
   float* cse;              // [B][H][nc]        cs at each sub-chunk's last token
 };
 
-// cs[i] = sum_{r <= i} dt_r A_h over the sub-chunk (thread 0, L <= 64)
+// cs[i] = sum_{r <= i} dt_r A_h over the sub-chunk (warp 0: two tokens per lane, shuffle scans; L <= 64)
 __device__ __forceinline__ void sub_cumsum(const BwdArgs& a, int b, int h, int t0, int L, float* cs) {
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
     const Dims& d = a.d;
-    float run = 0.f;
-    for (int i = 0; i < L; ++i) {
-      run += a.dt[(size_t)(b * d.T + t0 + i) * d.H + h] * a.A[h];
-      cs[i] = run;
+    const int lane = threadIdx.x;
+    const float Ah = a.A[h];
+    float v0 = lane < L ? a.dt[(size_t)(b * d.T + t0 + lane) * d.H + h] * Ah : 0.f;
+    float v1 = lane + 32 < L ? a.dt[(size_t)(b * d.T + t0 + lane + 32) * d.H + h] * Ah : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u0 = __shfl_up_sync(0xffffffffu, v0, o), u1 = __shfl_up_sync(0xffffffffu, v1, o);
+      if (lane >= o) { v0 += u0; v1 += u1; }
     }
+    const float first = __shfl_sync(0xffffffffu, v0, 31);
+    cs[lane] = v0;
+    cs[lane + 32] = v1 + first;
   }
 }
 
+// acc[i][jj] += sum_{k < K} X(k, r_i) Y(k, c_jj) for rows r_i = ty + 16 i (i < 4) and columns c_jj = tx + 16 jj
+// (jj < nj); X(k, r) = X[k * xk + r * xr], Y(k, c) = Y[k * yk + c * yc].  A 16 x 16 thread grid over a 64-row
+// output, every thread with 4 x nj independent accumulators.
+template <int MJ, int MI = 4>
+__device__ __forceinline__ void tile_mac(float (&acc)[MI][MJ], int nj, int K, const float* X, int xk, int xr,
+                                         const float* Y, int yk, int yc, int ty, int tx, int ni = MI) {
+  for (int k = 0; k < K; ++k) {
+    float xv[MI], yv[MJ];
+#pragma unroll
+    for (int i = 0; i < MI; ++i) xv[i] = i < ni ? X[k * xk + (ty + 16 * i) * xr] : 0.f;
+#pragma unroll
+    for (int jj = 0; jj < MJ; ++jj) yv[jj] = jj < nj ? Y[k * yk + (tx + 16 * jj) * yc] : 0.f;
+#pragma unroll
+    for (int i = 0; i < MI; ++i)
+#pragma unroll
+      for (int jj = 0; jj < MJ; ++jj) acc[i][jj] = fmaf(xv[i], yv[jj], acc[i][jj]);
+  }
+}
+
+__device__ __forceinline__ void widen(const uint4& q, float (&f)[8]) {
+  const __half2* h = reinterpret_cast<const __half2*>(&q);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 v = __half22float2(h[e]);
+    f[2 * e] = v.x;
+    f[2 * e + 1] = v.y;
+  }
+}
+__device__ __forceinline__ void widen(const uint4& q, float (&f)[4]) {
+  const float* v = reinterpret_cast<const float*>(&q);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) f[e] = v[e];
+}
+
+// dst[i][c] = src[((m0 + i) * k + slot) * stride_row + col0 + c] for i < BL, c < width, zero past the
+// sub-chunk; 16-byte loads (width, stride_row and col0 are multiples of 8 elements, the rows 16-byte aligned)
 template <class S>
 __device__ __forceinline__ void load_rows(const S* src, size_t m0, int k, int slot, int width, size_t stride_row,
                                           size_t col0, int L, float* dst, int ld) {
-  // dst[i][c] = src[((m0 + i) * k + slot) * stride_row + col0 + c], zero past the sub-chunk
-  for (int x = threadIdx.x; x < BL * width; x += blockDim.x) {
-    const int i = x / width, c = x % width;
-    dst[i * ld + c] = i < L ? to_f32(src[((m0 + i) * k + slot) * stride_row + col0 + c]) : 0.f;
+  constexpr int V = 16 / sizeof(S);
+  const int per_row = width / V;
+  for (int x = threadIdx.x; x < BL * per_row; x += blockDim.x) {
+    const int i = x / per_row, c = (x - i * per_row) * V;
+    float f[V];
+    if (i < L) {
+      widen(*reinterpret_cast<const uint4*>(src + ((m0 + i) * k + slot) * stride_row + col0 + c), f);
+    } else {
+#pragma unroll
+      for (int e = 0; e < V; ++e) f[e] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < V; ++e) dst[i * ld + c + e] = f[e];
   }
 }
 
@@ -70,11 +123,13 @@ __global__ void __launch_bounds__(kBT) bwd_fwd_chunk_kernel(BwdArgs a) {
   __syncthreads();
   const size_t m0 = (size_t)b * d.T + t0;
   const int NP = d.N * d.P;
-  constexpr int kMaxAcc = (128 * 128) / kBT;
-  float acc[kMaxAcc];
-  const int per = NP / kBT;  // N * P is a multiple of 256 for N, P in {16 .. 128}
+  // thread (ty, tx) of a 16 x 16 grid holds S_c[n][p] for n = ty + 16 i, p = tx + 16 jj
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4, ni = d.N / 16, nj = d.P / 16;
+  float acc[8][8];
 #pragma unroll
-  for (int r = 0; r < kMaxAcc; ++r) acc[r] = 0.f;
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
   for (int j = 0; j < d.k; ++j) {
     load_rows<S>((const S*)a.bpi, m0, d.k, j, d.N, d.GN, (size_t)g * d.N, L, Bs, d.N);
     load_rows<S>((const S*)a.xs, m0, d.k, j, d.P, d.HP, (size_t)h * d.P, L, Xv, d.P);
@@ -84,20 +139,15 @@ __global__ void __launch_bounds__(kBT) bwd_fwd_chunk_kernel(BwdArgs a) {
       if (i < L) Xv[x] *= expf(cs[L - 1] - cs[i]);
     }
     __syncthreads();
-#pragma unroll
-    for (int r = 0; r < kMaxAcc; ++r) {
-      if (r >= per) break;
-      const int e = threadIdx.x + r * kBT, n = e / d.P, p = e % d.P;
-      float v = acc[r];
-      for (int i = 0; i < L; ++i) v = fmaf(Bs[i * d.N + n], Xv[i * d.P + p], v);
-      acc[r] = v;
-    }
+    tile_mac<8, 8>(acc, nj, L, Bs, d.N, 1, Xv, d.P, 1, ty, tx, ni);
     __syncthreads();
   }
   const size_t base = (((size_t)b * d.H + h) * a.nc + c) * NP;
 #pragma unroll
-  for (int r = 0; r < kMaxAcc; ++r)
-    if (r < per) a.work[base + threadIdx.x + r * kBT] = acc[r];
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+      if (i < ni && jj < nj) a.work[base + (size_t)(ty + 16 * i) * d.P + tx + 16 * jj] = acc[i][jj];
   if (threadIdx.x == 0) a.cse[((size_t)b * d.H + h) * a.nc + c] = cs[L - 1];
 }
 
@@ -148,12 +198,18 @@ __global__ void __launch_bounds__(kBT) bwd_d_kernel(BwdArgs a) {
   __syncthreads();
   const int NP = d.N * d.P;
   const size_t base = (((size_t)b * d.H + h) * a.nc + c) * NP;
-  for (int e = threadIdx.x; e < NP; e += blockDim.x) {
-    const int n = e / d.P, p = e % d.P;
-    float v = 0.f;
-    for (int i = 0; i < L; ++i) v = fmaf(Cs[i * d.N + n], Dy[i * d.P + p], v);
-    a.work[base + e] = v;
-  }
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4, ni = d.N / 16, nj = d.P / 16;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
+  tile_mac<8, 8>(acc, nj, L, Cs, d.N, 1, Dy, d.P, 1, ty, tx, ni);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+      if (i < ni && jj < nj) a.work[base + (size_t)(ty + 16 * i) * d.P + tx + 16 * jj] = acc[i][jj];
 }
 
 // 4. Lam_{c+1} for every sub-chunk (into work, replacing D_c), and d init = Lam_0
@@ -165,9 +221,11 @@ __global__ void bwd_adj_pass_kernel(BwdArgs a) {
   if (e >= NP) return;
   const size_t bh = (size_t)b * d.H + h;
   float lam = 0.f;
+  float Dnext = a.work[(bh * a.nc + a.nc - 1) * NP + e];
   for (int c = a.nc - 1; c >= 0; --c) {
     const size_t o = (bh * a.nc + c) * NP + e;
-    const float Dc = a.work[o];
+    const float Dc = Dnext;
+    if (c > 0) Dnext = a.work[o - NP];
     a.work[o] = lam;
     lam = fmaf(expf(a.cse[bh * a.nc + c]), lam, Dc);
   }
@@ -175,24 +233,25 @@ __global__ void bwd_adj_pass_kernel(BwdArgs a) {
 }
 
 // Shared-memory plan of the gradient kernel (floats): per sub-chunk C~, dy, then per slot keys, values,
-// the two score tiles, and the end adjoint Lam_{c+1} (with H_c first, for the carried-state terms).
+// the two score tiles, and the end adjoint Lam_{c+1} (with H_c first, for the carried-state terms).  Rows of
+// N or P floats are padded by one so that column walks across rows hit distinct banks.
 struct GradSmem {
-  int N, P, ldS;
+  int N, P, ldN, ldP;
   size_t cs, eend, q, bv, red, C, Dy, B, X, S1, S2, Lam, total;
-  __host__ __device__ GradSmem(int n, int p) : N(n), P(p), ldS(BL + 1) {
+  __host__ __device__ GradSmem(int n, int p) : N(n), P(p), ldN(n + 1), ldP(p + 1) {
     size_t o = 0;
     cs = o; o += BL;
     eend = o; o += BL;
     q = o; o += BL;
     bv = o; o += BL;
     red = o; o += 4;
-    C = o; o += (size_t)BL * N;
-    Dy = o; o += (size_t)BL * P;
-    B = o; o += (size_t)BL * N;
-    X = o; o += (size_t)BL * P;
-    S1 = o; o += (size_t)BL * ldS;
-    S2 = o; o += (size_t)BL * ldS;
-    Lam = o; o += (size_t)N * P;
+    C = o; o += (size_t)BL * ldN;
+    Dy = o; o += (size_t)BL * ldP;
+    B = o; o += (size_t)BL * ldN;
+    X = o; o += (size_t)BL * ldP;
+    S1 = o; o += (size_t)BL * BL;
+    S2 = o; o += (size_t)BL * BL;
+    Lam = o; o += (size_t)N * ldP;
     total = o;
   }
 };
@@ -203,7 +262,7 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
   extern __shared__ float sm[];
   const Dims& d = a.d;
   const GradSmem Ls(d.N, d.P);
-  const int N = d.N, P = d.P, ldS = Ls.ldS;
+  const int N = d.N, P = d.P, ldN = Ls.ldN, ldP = Ls.ldP;
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / d.hpg;
   const int t0 = c * BL, L = min(BL, d.T - t0);
   float* cs = sm + Ls.cs;
@@ -232,96 +291,163 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
     float v = 0.f;
     if (i < L)
       for (int j = 0; j < d.k; ++j) v += to_f32(((const S*)a.cpi)[((m0 + i) * d.k + j) * d.GN + (size_t)g * N + n]);
-    C[x] = v;
+    C[i * ldN + n] = v;
   }
   for (int x = tid; x < BL * P; x += blockDim.x) {
     const int i = x / P, p = x % P;
-    Dy[x] = i < L ? a.dy[(m0 + i) * d.HP + (size_t)h * P + p] : 0.f;
+    Dy[i * ldP + p] = i < L ? a.dy[(m0 + i) * d.HP + (size_t)h * P + p] : 0.f;
   }
   // H_c into the Lam buffer first; e^{cs_end} <Lam_{c+1}, H_c> on the way
   float part = 0.f;
   for (int e = tid; e < NP; e += blockDim.x) {
     const float hv = a.hstart[sbase + e];
-    Lam[e] = hv;
+    Lam[(e / P) * ldP + e % P] = hv;
     part = fmaf(a.work[sbase + e], hv, part);
   }
   atomicAdd(&red[0], part);
   __syncthreads();
   const float cs_end = cs[L - 1];
   for (int i = tid; i < BL; i += blockDim.x) eend[i] = i < L ? expf(cs_end - cs[i]) : 0.f;
-  // carried-state terms: dC~_t = e^{cs_t} H_c dy_t (kept per thread over the slots), q_t = C~_t . that
-  constexpr int kMaxPer = (BL * 128) / kBT;
-  float dC[kMaxPer];
-  const int perC = (BL * N) / kBT;
+  // carried-state terms: dC~_t = e^{cs_t} H_c dy_t, kept per thread over the slots as a 4 x N/16 tile of
+  // (t = ty + 16 i, n = tx + 16 jj); q_t = C~_t . that (the 16 lanes of a half-warp share t)
+  const int tx = tid & 15, ty = tid >> 4;
+  const int nN = N / 16, nP = P / 16;
+  float dC[4][8];
 #pragma unroll
-  for (int r = 0; r < kMaxPer; ++r) {
-    if (r >= perC) break;
-    const int x = tid + r * kBT, i = x / N, n = x % N;
-    float v = 0.f;
-    if (i < L) {
-      for (int p = 0; p < P; ++p) v = fmaf(Lam[n * P + p], Dy[i * P + p], v);
-      v *= expf(cs[i]);
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) dC[i][jj] = 0.f;
+  tile_mac<8>(dC, nN, P, Dy, 1, ldP, Lam, 1, ldP, ty, tx);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = ty + 16 * i;
+    const float e = t < L ? expf(cs[t]) : 0.f;
+    float qp = 0.f;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      if (jj >= nN) break;
+      dC[i][jj] *= e;
+      qp = fmaf(C[t * ldN + tx + 16 * jj], dC[i][jj], qp);
     }
-    dC[r] = v;
-    if (i < L) atomicAdd(&q[i], C[i * N + n] * v);
+    for (int o = 8; o > 0; o >>= 1) qp += __shfl_xor_sync(0xffffffffu, qp, o);
+    if (tx == 0 && t < L) atomicAdd(&q[t], qp);
   }
   __syncthreads();
   // the end adjoint Lam_{c+1}
-  for (int e = tid; e < NP; e += blockDim.x) Lam[e] = a.work[sbase + e];
+  for (int e = tid; e < NP; e += blockDim.x) Lam[(e / P) * ldP + e % P] = a.work[sbase + e];
   __syncthreads();
 
   for (int j = 0; j < d.k; ++j) {
-    load_rows<S>((const S*)a.bpi, m0, d.k, j, N, d.GN, (size_t)g * N, L, Bs, N);
-    load_rows<S>((const S*)a.xs, m0, d.k, j, P, d.HP, (size_t)h * P, L, Xs, P);
+    load_rows<S>((const S*)a.bpi, m0, d.k, j, N, d.GN, (size_t)g * N, L, Bs, ldN);
+    load_rows<S>((const S*)a.xs, m0, d.k, j, P, d.HP, (size_t)h * P, L, Xs, ldP);
     __syncthreads();
-    // score tiles with the causal decay: K1 = W S1 (into S1), K2 = W S2 (into S2); M = W S1 S2 into q
-    for (int x = tid; x < BL * BL; x += blockDim.x) {
-      const int t = x / BL, s = x % BL;
-      float k1 = 0.f, k2 = 0.f;
-      if (s <= t && t < L) {
-        float s1 = 0.f, s2 = 0.f;
-        for (int n = 0; n < N; ++n) s1 = fmaf(C[t * N + n], Bs[s * N + n], s1);
-        for (int p = 0; p < P; ++p) s2 = fmaf(Dy[t * P + p], Xs[s * P + p], s2);
-        const float w = expf(cs[t] - cs[s]);
-        k1 = w * s1;
-        k2 = w * s2;
-        const float m = k1 * s2;
-        atomicAdd(&q[t], m);
-        atomicAdd(&q[s], -m);
+    // score tiles with the causal decay, 4 x 4 (t, s) pairs per thread: K1 = W S1 (into S1), K2 = W S2 (into S2);
+    // M = W S1 S2 adds its row sums to q and takes its column sums from it
+    {
+      const int tx = tid & 15, ty = tid >> 4;
+      float s1[4][4], s2[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) { s1[i][jj] = 0.f; s2[i][jj] = 0.f; }
+      for (int n = 0; n < N; ++n) {
+        float cv[4], bw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { cv[i] = C[(ty + 16 * i) * ldN + n]; bw[i] = Bs[(tx + 16 * i) * ldN + n]; }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) s1[i][jj] = fmaf(cv[i], bw[jj], s1[i][jj]);
       }
-      S1[t * ldS + s] = k1;
-      S2[t * ldS + s] = k2;
+      for (int p = 0; p < P; ++p) {
+        float dv[4], xv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { dv[i] = Dy[(ty + 16 * i) * ldP + p]; xv[i] = Xs[(tx + 16 * i) * ldP + p]; }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) s2[i][jj] = fmaf(dv[i], xv[jj], s2[i][jj]);
+      }
+      float rowp[4] = {0.f, 0.f, 0.f, 0.f}, colp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int t = ty + 16 * i, s = tx + 16 * jj;
+          float k1 = 0.f, k2 = 0.f;
+          if (s <= t && t < L) {
+            const float w = expf(cs[t] - cs[s]);
+            k1 = w * s1[i][jj];
+            k2 = w * s2[i][jj];
+            const float m = k1 * s2[i][jj];
+            rowp[i] += m;
+            colp[jj] += m;
+          }
+          S1[t * BL + s] = k1;
+          S2[t * BL + s] = k2;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        atomicAdd(&q[ty + 16 * i], rowp[i]);
+        atomicAdd(&q[tx + 16 * i], -colp[i]);
+      }
     }
     __syncthreads();
-    // dXs_s = sum_t K1[t][s] dy_t + e^{cs_end - cs_s} Lam^T B_s
-    for (int x = tid; x < BL * P; x += blockDim.x) {
-      const int s = x / P, p = x % P;
+    float acc[4][8];
+    // dXs_s = e^{cs_end - cs_s} Lam^T B_s + sum_t K1[t][s] dy_t   (tile of s = ty + 16 i, p = tx + 16 jj)
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
+    tile_mac<8>(acc, nP, N, Bs, 1, ldN, Lam, ldP, 1, ty, tx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) acc[i][jj] *= eend[ty + 16 * i];
+    tile_mac<8>(acc, nP, L, S1, BL, 1, Dy, ldP, 1, ty, tx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int s = ty + 16 * i;
       if (s >= L) continue;
-      float v = 0.f, u = 0.f;
-      for (int t = s; t < L; ++t) v = fmaf(S1[t * ldS + s], Dy[t * P + p], v);
-      for (int n = 0; n < N; ++n) u = fmaf(Lam[n * P + p], Bs[s * N + n], u);
-      a.dxs[((m0 + s) * d.k + j) * d.HP + (size_t)h * P + p] = fmaf(eend[s], u, v);
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj)
+        if (jj < nP) a.dxs[((m0 + s) * d.k + j) * d.HP + (size_t)h * P + tx + 16 * jj] = acc[i][jj];
     }
-    // dBpi_s = sum_t K2[t][s] C~_t + e^{cs_end - cs_s} Lam x_s;  bv_s += B_s . Lam x_s
-    for (int x = tid; x < BL * N; x += blockDim.x) {
-      const int s = x / N, n = x % N;
+    // dBpi_s = e^{cs_end - cs_s} Lam x_s + sum_t K2[t][s] C~_t   (tile of s, n = tx + 16 jj); bv_s += B_s . Lam x_s
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
+    tile_mac<8>(acc, nN, P, Xs, 1, ldP, Lam, 1, ldP, ty, tx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int s = ty + 16 * i;
+      float bp = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        if (jj >= nN) break;
+        bp = fmaf(Bs[s * ldN + tx + 16 * jj], acc[i][jj], bp);
+        acc[i][jj] *= eend[s];
+      }
+      for (int o = 8; o > 0; o >>= 1) bp += __shfl_xor_sync(0xffffffffu, bp, o);
+      if (tx == 0 && s < L) atomicAdd(&bv[s], bp);
+    }
+    tile_mac<8>(acc, nN, L, S2, BL, 1, C, ldN, 1, ty, tx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int s = ty + 16 * i;
       if (s >= L) continue;
-      float v = 0.f, u = 0.f;
-      for (int t = s; t < L; ++t) v = fmaf(S2[t * ldS + s], C[t * N + n], v);
-      for (int p = 0; p < P; ++p) u = fmaf(Lam[n * P + p], Xs[s * P + p], u);
-      atomicAdd(&a.dbpi[((m0 + s) * d.k + j) * d.GN + (size_t)g * N + n], fmaf(eend[s], u, v));
-      atomicAdd(&bv[s], Bs[s * N + n] * u);
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        if (jj >= nN) break;
+        float* o = &a.dbpi[((m0 + s) * d.k + j) * d.GN + (size_t)g * N + tx + 16 * jj];
+        if (d.hpg == 1) *o = acc[i][jj];
+        else atomicAdd(o, acc[i][jj]);
+      }
     }
     // dC~_t += sum_{s <= t} K2[t][s] B_s
-#pragma unroll
-    for (int r = 0; r < kMaxPer; ++r) {
-      if (r >= perC) break;
-      const int x = tid + r * kBT, t = x / N, n = x % N;
-      if (t >= L) continue;
-      float v = dC[r];
-      for (int s = 0; s <= t; ++s) v = fmaf(S2[t * ldS + s], Bs[s * N + n], v);
-      dC[r] = v;
-    }
+    tile_mac<8>(dC, nN, L, S2, 1, BL, Bs, ldN, 1, ty, tx);
     __syncthreads();
     // q_t -= e^{cs_end - cs_t} bv_t, and the last token takes sum_s e^{cs_end - cs_s} bv_s
     if (tid < L) {
@@ -333,10 +459,16 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
     __syncthreads();
   }
 #pragma unroll
-  for (int r = 0; r < kMaxPer; ++r) {
-    if (r >= perC) break;
-    const int x = tid + r * kBT, t = x / N, n = x % N;
-    if (t < L) atomicAdd(&a.dct[(m0 + t) * d.GN + (size_t)g * N + n], dC[r]);
+  for (int i = 0; i < 4; ++i) {
+    const int t = ty + 16 * i;
+    if (t >= L) continue;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      if (jj >= nN) break;
+      float* o = &a.dct[(m0 + t) * d.GN + (size_t)g * N + tx + 16 * jj];
+      if (d.hpg == 1) *o = dC[i][jj];
+      else atomicAdd(o, dC[i][jj]);
+    }
   }
   if (tid == 0) {
     q[L - 1] += expf(cs_end) * red[0] + red[1];
@@ -388,10 +520,10 @@ cudaError_t launch_scan_bwd(const Dims& d, const void* bpi, const void* xs, cons
                             cudaStream_t s) {
   BwdArgs a{d, scan_bwd_subchunks(d), bpi, xs, cpi, dt, A, init, dy, dbpi, dxs, dct, ddt, dA, dinit,
             hstart, work, cse};
-  // the Bpi, C~ and A gradients are accumulated
-  cudaError_t e = cudaMemsetAsync(dbpi, 0, (size_t)d.M * d.k * d.GN * 4, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dct, 0, (size_t)d.M * d.GN * 4, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dA, 0, (size_t)d.H * 4, s);
+  // the A gradient, and with G < H the Bpi and C~ gradients (summed over a group's heads), are accumulated
+  cudaError_t e = cudaMemsetAsync(dA, 0, (size_t)d.H * 4, s);
+  if (e == cudaSuccess && d.hpg > 1) e = cudaMemsetAsync(dbpi, 0, (size_t)d.M * d.k * d.GN * 4, s);
+  if (e == cudaSuccess && d.hpg > 1) e = cudaMemsetAsync(dct, 0, (size_t)d.M * d.GN * 4, s);
   if (e != cudaSuccess) return e;
   return d.dtype == SWIMBA_BF16 ? launch_bwd_typed<__half>(a, s) : launch_bwd_typed<float>(a, s);
 }
