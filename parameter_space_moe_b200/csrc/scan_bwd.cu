@@ -60,6 +60,7 @@ __device__ __forceinline__ void sub_cumsum(const BwdArgs& a, int b, int h, int t
 template <int MJ, int MI = 4>
 __device__ __forceinline__ void tile_mac(float (&acc)[MI][MJ], int nj, int K, const float* X, int xk, int xr,
                                          const float* Y, int yk, int yc, int ty, int tx, int ni = MI) {
+#pragma unroll 4
   for (int k = 0; k < K; ++k) {
     float xv[MI], yv[MJ];
 #pragma unroll
