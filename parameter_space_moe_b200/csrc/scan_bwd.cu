@@ -110,6 +110,30 @@ __device__ __forceinline__ void load_rows(const S* src, size_t m0, int k, int sl
   }
 }
 
+// dst[i][c] = sum_{j < k} src[((m0 + i) * k + j) * stride_row + col0 + c] (C~ from the per-slot readouts)
+template <class S>
+__device__ __forceinline__ void load_rows_sum(const S* src, size_t m0, int k, int width, size_t stride_row,
+                                              size_t col0, int L, float* dst, int ld) {
+  constexpr int V = 16 / sizeof(S);
+  const int per_row = width / V;
+  for (int x = threadIdx.x; x < BL * per_row; x += blockDim.x) {
+    const int i = x / per_row, c = (x - i * per_row) * V;
+    float acc[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    if (i < L) {
+      for (int j = 0; j < k; ++j) {
+        float f[V];
+        widen(*reinterpret_cast<const uint4*>(src + ((m0 + i) * k + j) * stride_row + col0 + c), f);
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] += f[e];
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < V; ++e) dst[i * ld + c + e] = acc[e];
+  }
+}
+
 // 1. sub-chunk end states S_c (keys of every slot) and cs at the last token
 template <class S>
 __global__ void __launch_bounds__(kBT) bwd_fwd_chunk_kernel(BwdArgs a) {
@@ -180,17 +204,8 @@ __global__ void __launch_bounds__(kBT) bwd_d_kernel(BwdArgs a) {
   float* Dy = Cs + BL * d.N;         // [BL][P]
   sub_cumsum(a, b, h, t0, L, cs);
   const size_t m0 = (size_t)b * d.T + t0;
-  for (int x = threadIdx.x; x < BL * d.N; x += blockDim.x) {
-    const int i = x / d.N, n = x % d.N;
-    float v = 0.f;
-    if (i < L)
-      for (int j = 0; j < d.k; ++j) v += to_f32(((const S*)a.cpi)[((m0 + i) * d.k + j) * d.GN + (size_t)g * d.N + n]);
-    Cs[x] = v;
-  }
-  for (int x = threadIdx.x; x < BL * d.P; x += blockDim.x) {
-    const int i = x / d.P, p = x % d.P;
-    Dy[x] = i < L ? a.dy[(m0 + i) * d.HP + (size_t)h * d.P + p] : 0.f;
-  }
+  load_rows_sum<S>((const S*)a.cpi, m0, d.k, d.N, d.GN, (size_t)g * d.N, L, Cs, d.N);
+  load_rows<float>(a.dy, m0, 1, 0, d.P, d.HP, (size_t)h * d.P, L, Dy, d.P);
   __syncthreads();
   for (int x = threadIdx.x; x < BL * d.N; x += blockDim.x) {
     const int i = x / d.N;
@@ -287,23 +302,16 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
   sub_cumsum(a, b, h, t0, L, cs);
   for (int i = tid; i < BL; i += blockDim.x) { q[i] = 0.f; bv[i] = 0.f; }
   if (tid < 4) red[tid] = 0.f;
-  for (int x = tid; x < BL * N; x += blockDim.x) {
-    const int i = x / N, n = x % N;
-    float v = 0.f;
-    if (i < L)
-      for (int j = 0; j < d.k; ++j) v += to_f32(((const S*)a.cpi)[((m0 + i) * d.k + j) * d.GN + (size_t)g * N + n]);
-    C[i * ldN + n] = v;
-  }
-  for (int x = tid; x < BL * P; x += blockDim.x) {
-    const int i = x / P, p = x % P;
-    Dy[i * ldP + p] = i < L ? a.dy[(m0 + i) * d.HP + (size_t)h * P + p] : 0.f;
-  }
-  // H_c into the Lam buffer first; e^{cs_end} <Lam_{c+1}, H_c> on the way
+  load_rows_sum<S>((const S*)a.cpi, m0, d.k, N, d.GN, (size_t)g * N, L, C, ldN);
+  load_rows<float>(a.dy, m0, 1, 0, P, d.HP, (size_t)h * P, L, Dy, ldP);
+  // H_c into the Lam buffer first; e^{cs_end} <Lam_{c+1}, H_c> on the way (16-byte loads of both)
   float part = 0.f;
-  for (int e = tid; e < NP; e += blockDim.x) {
-    const float hv = a.hstart[sbase + e];
-    Lam[(e / P) * ldP + e % P] = hv;
-    part = fmaf(a.work[sbase + e], hv, part);
+  for (int e = 4 * tid; e < NP; e += 4 * blockDim.x) {
+    const float4 hv = *reinterpret_cast<const float4*>(a.hstart + sbase + e);
+    const float4 lv = *reinterpret_cast<const float4*>(a.work + sbase + e);
+    float* dst = Lam + (e / P) * ldP + e % P;
+    dst[0] = hv.x; dst[1] = hv.y; dst[2] = hv.z; dst[3] = hv.w;
+    part = fmaf(lv.x, hv.x, fmaf(lv.y, hv.y, fmaf(lv.z, hv.z, fmaf(lv.w, hv.w, part))));
   }
   atomicAdd(&red[0], part);
   __syncthreads();
@@ -335,7 +343,11 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
   }
   __syncthreads();
   // the end adjoint Lam_{c+1}
-  for (int e = tid; e < NP; e += blockDim.x) Lam[(e / P) * ldP + e % P] = a.work[sbase + e];
+  for (int e = 4 * tid; e < NP; e += 4 * blockDim.x) {
+    const float4 lv = *reinterpret_cast<const float4*>(a.work + sbase + e);
+    float* dst = Lam + (e / P) * ldP + e % P;
+    dst[0] = lv.x; dst[1] = lv.y; dst[2] = lv.z; dst[3] = lv.w;
+  }
   __syncthreads();
 
   for (int j = 0; j < d.k; ++j) {
