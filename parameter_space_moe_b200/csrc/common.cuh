@@ -105,12 +105,17 @@ unsigned* device_status();
 // launch; `st` is the workspace status word.
 // counts (nullable): [dispatch tile][E] table, zeroed by the caller, that the router increments for the
 // (token, slot) pairs it routes (dispatch tile = pair index / kDispatchTile).
+// after_zero: the stream's previous kernel is launch_zero_u32 clearing `counts` (and nothing else the router
+// reads is produced by it): the tensor-core router then starts under programmatic dependent launch and waits
+// for that kernel only before its first count.
 cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
-                          float* dt, int32_t* counts, unsigned* st, cudaStream_t s);
+                          float* dt, int32_t* counts, unsigned* st, cudaStream_t s, bool after_zero = false);
 // The tensor-core (tcgen05) router that launch_router prefers where it applies.
 bool router_tc_supported(const Dims& d);
 cudaError_t launch_router_tc(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
-                             float* dt, int32_t* counts, unsigned* st, cudaStream_t s);
+                             float* dt, int32_t* counts, unsigned* st, cudaStream_t s, bool after_zero);
+// Zeroes n 32-bit words; lets the next kernel launch at once (it must wait before reading them).
+cudaError_t launch_zero_u32(unsigned* p, size_t n, cudaStream_t s);
 // rowmeta (nullable): per sorted row, (pair index p, router weight of p as float bits; 0 without topk_w).
 // Pairs whose index lies outside [0, E) are left out of the sort and raise ST_INDEX in *st.
 cudaError_t launch_dispatch(const Dims& d, const int32_t* idx, const WsPlan& p, char* ws, int32_t* offsets,

@@ -235,10 +235,10 @@ router_mma_kernel(Dims d, int RP, const __nv_bfloat16* __restrict__ X, const __n
 }  // namespace
 
 cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
-                          float* dt, int32_t* counts, unsigned* st, cudaStream_t s) {
+                          float* dt, int32_t* counts, unsigned* st, cudaStream_t s, bool after_zero) {
   const int R = d.E + d.H;
   if (st && router_tc_supported(d)) {
-    const cudaError_t e = launch_router_tc(d, X, w, idx, wts, dt, counts, st, s);
+    const cudaError_t e = launch_router_tc(d, X, w, idx, wts, dt, counts, st, s, after_zero);
     if (e != cudaErrorNotSupported) return e;
   }
   if (d.dtype == SWIMBA_BF16 && R <= 8 * kMaxNT) {
@@ -268,6 +268,20 @@ cudaError_t launch_router(const Dims& d, const void* X, const swimba_weights& w,
                                                                       counts);
     }
   }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+namespace {
+__global__ void zero_u32_kernel(unsigned* p, size_t n) {
+  griddep_launch_dependents();
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) p[i] = 0u;
+}
+}  // namespace
+
+cudaError_t launch_zero_u32(unsigned* p, size_t n, cudaStream_t s) {
+  const size_t blocks = (n + 255) / 256;
+  zero_u32_kernel<<<(unsigned)(blocks < 148 ? (blocks > 0 ? blocks : 1) : 148), 256, 0, s>>>(p, n);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -226,6 +226,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       if (i0 + u * 128 < rows * d.H) a.dt[(size_t)(m0 + r[u]) * d.H + h[u]] = fminf(fmaxf(sp, 1e-3f), 0.1f);
     }
   }
+  // the counts table was cleared by the kernel before this one (launched with programmatic dependent launch
+  // after it, this grid may have started early); without that launch mode the wait returns at once
+  griddep_wait();
   if (tid < rows) {
     const int m = m0 + tid;
     const float* gl = G + tid * L.gs;
@@ -281,7 +284,7 @@ bool router_tc_supported(const Dims& d) {
 // Returns cudaErrorNotSupported, with nothing launched, when a tensor map cannot be encoded (the caller
 // then takes another router kernel).
 cudaError_t launch_router_tc(const Dims& d, const void* X, const swimba_weights& w, int32_t* idx, float* wts,
-                             float* dt, int32_t* counts, unsigned* st, cudaStream_t s) {
+                             float* dt, int32_t* counts, unsigned* st, cudaStream_t s, bool after_zero) {
   const int eoff = (d.E + 7) / 8 * 8;
   const int RP = (eoff + d.H + 15) / 16 * 16;
   CUtensorMap tx, twr, twd;
@@ -308,13 +311,15 @@ cudaError_t launch_router_tc(const Dims& d, const void* X, const swimba_weights&
   cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = after_zero ? 2 : 1;
   e = cudaLaunchKernelEx(&cfg, router_tc_kernel, tx, twr, twd, a);
   count_launches(1);
   if (e != cudaSuccess) return e;

@@ -90,7 +90,7 @@ WsPlan plan_workspace(const Dims& d) {
   p.dcounts = take((size_t)dispatch_tiles(d) * d.E * 4);
   const size_t nsub = (size_t)scan_tc_subchunks(d);
   p.lb_bytes = 256 + (size_t)d.Bsz * d.H * nsub * 4;
-  p.lb = take(p.lb_bytes);  // directly after dcounts: run_front clears both with one memset
+  p.lb = take(p.lb_bytes);  // directly after dcounts: run_front clears both with one kernel
   p.dbase = take((size_t)dispatch_tiles(d) * d.E * 4);
   p.offsets = take((size_t)(d.E + 1) * 4);
   p.perm = take(Mk * 4);
@@ -193,10 +193,11 @@ static swimba_status run_proj(const Dims& d, const void* X, const void* w_exp, c
 static swimba_status run_front(const Dims& d, const void* X, const swimba_weights* w, char* ws, const WsPlan& p,
                                int32_t* idx, float* wts, int mode, unsigned* st, cudaStream_t s) {
   float* dt = (float*)(ws + p.dt);
-  // one memset clears the router's per-tile counts and the scan's hand-off flags (adjacent regions)
-  SW_CUDA(cudaMemsetAsync(ws + p.dcounts, 0, p.lb + p.lb_bytes - p.dcounts, s));
+  // one small kernel clears the router's per-tile counts and the scan's hand-off flags (adjacent regions);
+  // the router's prologue and loads overlap it
+  SW_CUDA(launch_zero_u32((unsigned*)(ws + p.dcounts), (p.lb + p.lb_bytes - p.dcounts) / 4, s));
   int32_t* counts = (int32_t*)(ws + p.dcounts);
-  SW_CUDA(launch_router(d, X, *w, idx, wts, dt, counts, st, s));
+  SW_CUDA(launch_router(d, X, *w, idx, wts, dt, counts, st, s, /*after_zero=*/true));
   prof_mark(s, "router");
   int32_t* offsets = (int32_t*)(ws + p.offsets);
   int32_t* perm = (int32_t*)(ws + p.perm);
