@@ -352,6 +352,74 @@ def layer_fwd(X, W_r, W_dt, b_dt, A, W_exp, H, P, N, G, k, init=None, forced_idx
     return dict(y=y, final=final, g=g, dt=dt, idx=idx, w=w, z=z, Bpi=Bpi, Xs=Xs, Ct=Ct, Cpi=Cpi, At=At)
 
 
+def mix_bwd(dBpi, dXs, dCt, w, Bz, Cz):
+    """Reverse of mix: the gradient of each slot's projection z = [x | B | C] and of its router weight, from the
+    gradients of the mixed streams (Bpi = pi B, Xs = x, C~ = sum_j pi_j C_j):
+        dz_j = [dXs_j | pi_j dBpi_j | pi_j dC~],    dpi_j = <B_j, dBpi_j> + <C_j, dC~>.
+    dBpi [M,k,G,N], dXs [M,k,H,P], dCt [M,G,N], w [M,k], Bz/Cz [M,k,G,N]; returns dz [M,k,W_e], dpi [M,k]."""
+    M, k = w.shape
+    dz = np.concatenate([dXs.reshape(M, k, -1), (w[:, :, None, None] * dBpi).reshape(M, k, -1),
+                         (w[:, :, None, None] * dCt[:, None]).reshape(M, k, -1)], axis=-1)
+    dw = np.einsum("mjgn,mjgn->mj", Bz, dBpi) + np.einsum("mjgn,mgn->mj", Cz, dCt)
+    return dz, dw
+
+
+def router_bwd(w, dw):
+    """Reverse of the renormalised softmax over the winners: with pi_j = e^{g_j} / sum_i e^{g_i} over K_t,
+    dg_j = pi_j (dpi_j - sum_i pi_i dpi_i)  (the losers get no gradient)."""
+    return w * (dw - (w * dw).sum(axis=1, keepdims=True))
+
+
+def layer_bwd(X, W_r, W_dt, b_dt, A, W_exp, H, P, N, G, k, dy, init=None, forced_idx=None,
+              decision_dtype=np.float32):
+    """Gradients of L = sum <dy, y> for the layer of layer_fwd, with respect to X, every weight and the
+    initial state, by reverse-mode differentiation of each stage in turn (the notes train the model: loss
+    function / training strategy).  The active set K_t is held fixed (a top-k choice has no gradient); the dt
+    clamp passes the gradient only strictly inside [1e-3, 0.1].
+        scan   -> scan_backward: dBpi, dXs, dC~, d dt, dA, d init
+        mix    -> dz = [dXs_j | pi_j dBpi_j | pi_j dC~] per slot;  dpi_j = <B_j, dBpi_j> + <C_j, dC~>
+        router -> dg_j = pi_j (dpi_j - sum_i pi_i dpi_i) on the winners (softmax renormalised over K_t);
+                  du = d dt * sigmoid(u) on the unclamped tokens, u = W_dt X + b
+        linear -> dW_exp[e] = sum over (t, j) routed to e of dz_tj (x) X_t;  dX_t = sum_j W_exp[K_tj]^T dz_tj
+                  + W_r^T dg_t + W_dt^T du_t;  dW_r = dg^T X;  dW_dt = du^T X;  db_dt = sum_t du_t.
+    dy [B,T,H,P]; returns a dict with dX [B,T,D], dW_r, dW_dt, db_dt, dA, dW_exp, dinit [B,H,N,P]."""
+    Bsz, T, D = X.shape
+    M = Bsz * T
+    Xf = X.reshape(M, D)
+    fidx = None if forced_idx is None else forced_idx.reshape(M, k)
+    g, dt, idx, w = router(Xf, W_r, W_dt, b_dt, k, decision_dtype, fidx)
+    z = expert_proj(Xf, W_exp, idx)
+    Bpi, Xs, Ct, Cpi = mix(z, w, H, P, G, N)
+    x, Bz, Cz = split_streams(z, H, P, G, N)
+    dyf = dy.reshape(M, H, P)
+    dBpi = np.zeros(Bpi.shape); dXs = np.zeros(Xs.shape); dCt = np.zeros(Ct.shape); ddt = np.zeros(dt.shape)
+    dA = np.zeros(np.shape(A)); dinit = np.zeros((Bsz, H, N, P))
+    for b in range(Bsz):
+        r = slice(b * T, (b + 1) * T)
+        o = scan_backward(Bpi[r], Xs[r], Ct[r], dt[r], A, dyf[r], None if init is None else init[b])
+        dBpi[r], dXs[r], dCt[r], ddt[r] = o["dBpi"], o["dXs"], o["dCt"], o["ddt"]
+        dA = dA + o["dA"]
+        dinit[b] = o["dinit"]
+    dz, dw = mix_bwd(dBpi, dXs, dCt, w, Bz, Cz)
+    dg_sel = router_bwd(w, dw)
+    dg = np.zeros(g.shape)
+    np.put_along_axis(dg, idx, dg_sel, axis=1)
+    u = Xf @ W_dt.T + b_dt
+    sp = softplus(u)
+    du = ddt * (1.0 / (1.0 + np.exp(-u))) * ((sp > 1e-3) & (sp < 0.1))
+    # linear maps
+    dW_exp = np.zeros(W_exp.shape)
+    dX = Xf * 0.0
+    for m in range(M):
+        for j in range(k):
+            e = idx[m, j]
+            dW_exp[e] += np.outer(dz[m, j], Xf[m])
+            dX[m] += W_exp[e].T @ dz[m, j]
+    dX += dg @ W_r + du @ W_dt
+    return dict(dX=dX.reshape(Bsz, T, D), dW_r=dg.T @ Xf, dW_dt=du.T @ Xf, db_dt=du.sum(axis=0), dA=dA,
+                dW_exp=dW_exp, dinit=dinit)
+
+
 def out_proj(y, W_out):
     """out_t = W_out y_t: the one output projection that follows the shared recurrence's readout
     ([gist] Architecture Details).  There is one recurrence, so one projection, shared by all experts.

@@ -7,8 +7,9 @@ split, C~ summed without the router weights, the injection added before the deca
 flipped, the chunked form's causal mask shifted by one, the chunk-state decay taken from the chunk
 start instead of its end, the separated-E design advancing only the active experts, the output
 projection applied with its matrix transposed, the expert-mixed transition summed without the router
-weights or taken from the first active expert alone, and the scan's adjoint recurrence without its decay or
-with the decay gradient taken one state late."""
+weights or taken from the first active expert alone, the scan's adjoint recurrence without its decay or
+with the decay gradient taken one state late, and the layer backward passing the Bpi gradient on without its
+router weight or the softmax gradient without its renormalisation term."""
 import numpy as np
 import pytest
 
@@ -197,6 +198,22 @@ def _backward_decay_gradient_off_by_one(Bpi, Xs, Ct, dt, A, dy, init=None):
     return _backward_mutant(Bpi, Xs, Ct, dt, A, dy, init, h_shift=1)
 
 
+def _mix_bwd_unweighted_B(dBpi, dXs, dCt, w, Bz, Cz):
+    # the Bpi gradient passed on to the projection without its router weight
+    dz, dw = ORIG["mix_bwd"](dBpi, dXs, dCt, w, Bz, Cz)
+    M, k = w.shape
+    HP = dXs.shape[2] * dXs.shape[3]
+    GN = dBpi.shape[2] * dBpi.shape[3]
+    dz = dz.copy()
+    dz[:, :, HP:HP + GN] = dBpi.reshape(M, k, GN)
+    return dz, dw
+
+
+def _router_bwd_not_renormalised(w, dw):
+    # the softmax gradient without the renormalisation term
+    return w * dw
+
+
 def _out_proj_transposed(y, W_out):
     # the projection matrix applied transposed (shapes permitting: D == H*P)
     return np.asarray(y) @ np.asarray(W_out)
@@ -204,7 +221,7 @@ def _out_proj_transposed(y, W_out):
 
 ORIG = {name: getattr(O, name) for name in
         ("topk_weights", "topk_select", "dt_proj", "expert_proj", "split_streams", "mix", "scan_sequential",
-         "scan_chunked", "scan_separated_dense", "out_proj", "mixed_A", "scan_backward")}
+         "scan_chunked", "scan_separated_dense", "out_proj", "mixed_A", "scan_backward", "mix_bwd", "router_bwd")}
 
 # every pin, called with the parameters its decorator gives
 ALL_PINS = [
@@ -222,6 +239,7 @@ ALL_PINS = [
     pins.test_mixed_A_with_equal_experts_is_the_shared_layer, pins.test_mixed_A_decay_closed_form,
     pins.test_mixed_A_steps_equal_layer_fwd, pins.test_chunked_with_per_token_A_equals_sequential,
     lambda: pins.test_scan_backward_matches_finite_differences(2), pins.test_scan_backward_per_token_transition,
+    pins.test_layer_backward_matches_finite_differences,
 ]
 
 MUTATIONS = {
@@ -241,6 +259,8 @@ MUTATIONS = {
     "mixed_A_first_slot_only": ("mixed_A", _mixed_A_first_slot),
     "adjoint_without_decay": ("scan_backward", _backward_no_adjoint_decay),
     "decay_gradient_off_by_one": ("scan_backward", _backward_decay_gradient_off_by_one),
+    "mix_gradient_without_router_weight": ("mix_bwd", _mix_bwd_unweighted_B),
+    "router_gradient_not_renormalised": ("router_bwd", _router_bwd_not_renormalised),
 }
 
 

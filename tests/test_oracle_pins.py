@@ -156,6 +156,38 @@ def test_scan_backward_matches_finite_differences(G):
         np.testing.assert_allclose(got[names[name]], num, rtol=1e-6, atol=1e-7, err_msg=name)
 
 
+def test_layer_backward_matches_finite_differences():
+    # every gradient of L = sum <dy, y> for a tiny layer against central differences of layer_fwd, entry by
+    # entry; the inputs keep every token's top-k gap and every dt well away from the clamp bounds, so small
+    # perturbations change neither the active set nor the clamp
+    rng = np.random.default_rng(21)
+    L = _small_layer(rng, B=2, T=5, D=6, H=2, P=3, N=2, G=1, E=3, k=2)
+    L["b_dt"] = np.log(np.expm1(rng.uniform(0.02, 0.08, size=2)))
+    H, P, N, G, k = L["H"], L["P"], L["N"], L["G"], L["k"]
+    init = rng.standard_normal((2, H, N, P))
+    dy = rng.standard_normal((2, 5, H, P))
+    g = L["X"].reshape(-1, 6) @ L["W_r"].T
+    srt = -np.sort(-g, axis=1)
+    assert (srt[:, k - 1] - srt[:, k]).min() > 1e-3
+    got = O.layer_bwd(L["X"], L["W_r"], L["W_dt"], L["b_dt"], L["A"], L["W_exp"], H, P, N, G, k, dy, init)
+
+    def loss(X=L["X"], W_r=L["W_r"], W_dt=L["W_dt"], b_dt=L["b_dt"], A=L["A"], W_exp=L["W_exp"], init=init):
+        y = O.layer_fwd(X, W_r, W_dt, b_dt, A, W_exp, H, P, N, G, k, init=init)["y"]
+        return float((dy * y).sum())
+
+    args = dict(X=L["X"], W_r=L["W_r"], W_dt=L["W_dt"], b_dt=L["b_dt"], A=L["A"], W_exp=L["W_exp"], init=init)
+    names = dict(X="dX", W_r="dW_r", W_dt="dW_dt", b_dt="db_dt", A="dA", W_exp="dW_exp", init="dinit")
+    eps = 1e-6
+    for name, arr in args.items():
+        num = np.zeros(arr.shape)
+        for ix in np.ndindex(arr.shape):
+            hi, lo = arr.copy(), arr.copy()
+            hi[ix] += eps
+            lo[ix] -= eps
+            num[ix] = (loss(**{name: hi}) - loss(**{name: lo})) / (2 * eps)
+        np.testing.assert_allclose(got[names[name]], num, rtol=1e-5, atol=1e-7, err_msg=name)
+
+
 def test_scan_backward_per_token_transition():
     # with a [T,H] transition the dA gradient is per token; central differences on each entry
     rng = np.random.default_rng(17)
