@@ -214,6 +214,27 @@ swimba_status swimba_separated_scan(const swimba_dims* dims, const void* B, cons
                                     const float* dt, const float* A, const float* init_states, void* y,
                                     float* final_states, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of workspace swimba_layer_bwd needs for these dims (0 if invalid or unsupported): the layer's own
+ * workspace followed by fp32 gradient buffers (about M*k*(2*W_e + G*N + H*P + D)*4 bytes more). */
+size_t swimba_layer_bwd_workspace_size(const swimba_dims* dims);
+
+/* Gradients of the whole layer (swimba_layer_fwd with the shared A) for L = sum_t <dy_t, y_t>: the
+ * vector-Jacobian product with the upstream gradient dy.  Paper: notes, Method flowchart differentiated
+ * stage by stage in reverse (the notes train the model: loss function / training strategy).  The router's
+ * active set is recomputed and held fixed (a top-k choice has no gradient); the dt clamp passes the gradient
+ * only strictly inside [1e-3, 0.1].
+ *   X [M][D] dtype, weights as for swimba_layer_fwd (A_exp must be NULL: SWIMBA_ERR_UNSUPPORTED otherwise),
+ *   init_state [B][H][N][P] fp32 or NULL; dy [M][H][P] fp32
+ *   dX [M][D], dW_router [E][D], dW_dt [H][D], db_dt [H], dA [H], dW_exp [E][W_e][D] fp32 out;
+ *   d_init [B][H][N][P] fp32 out or NULL
+ * Runs the forward's router, dispatch and projections again, the scan gradients, then CUDA-core fp32
+ * kernels for the mix, router and dt gradients and the weight and input products.  ws must hold
+ * swimba_layer_bwd_workspace_size(dims) bytes (SWIMBA_ERR_WORKSPACE otherwise). */
+swimba_status swimba_layer_bwd(const swimba_dims* dims, const void* X, const swimba_weights* w,
+                               const float* init_state, const float* dy, float* dX, float* dW_router, float* dW_dt,
+                               float* db_dt, float* dA, float* dW_exp, float* d_init, void* ws, size_t ws_bytes,
+                               void* stream);
+
 /* Gradients of the chunked scan (swimba_ssd_scan over all k key and read slots) for the loss
  * L = sum_t <dy_t, y_t>, i.e. the vector-Jacobian product with an upstream gradient dy.  Paper: notes,
  * key design 1, second display equation differentiated in reverse (the notes train the model: loss

@@ -144,6 +144,17 @@ cudaError_t launch_scan_bwd(const Dims& d, const void* bpi, const void* xs, cons
                             const float* A, const float* init, const float* dy, float* dbpi, float* dxs, float* dct,
                             float* ddt, float* dA, float* dinit, float* hstart, float* work, float* cse,
                             cudaStream_t s);
+// The layer gradients after the scan gradients (mix, router and dt, expert and router weight gradients, dX).
+struct LayerBwdPtrs {
+  const void* X; const void* w_exp; const void* w_r; const void* w_dt;
+  const int32_t* idx; const float* wts; const float* dt; const float* ddt;
+  const int32_t* perm; const int32_t* tiles; const int32_t* ntiles; const int32_t* offsets;
+  float* z;      // [M*k][W_e] raw projections in, their gradients dz out
+  const float* dbpi; const float* dxs; const float* dct;
+  float* dpi; float* dg; float* du; float* dxp;
+  float* dX; float* dW_r; float* dW_dt; float* db_dt; float* dW_exp;
+};
+cudaError_t launch_layer_bwd_tail(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s);
 cudaError_t launch_mixed_a(const Dims& d, const int32_t* idx, const float* wts, const float* A_exp, const float* dt,
                            float* dA, float* ones, unsigned* st, cudaStream_t s);
 cudaError_t launch_out_proj(const Dims& d, const void* y, const void* w_out, void* out, unsigned* st,

@@ -1,0 +1,281 @@
+// Gradients of the whole layer: the stages after the scan gradients, on CUDA cores in fp32.
+//
+// Paper: Swimba notes, Method flowchart (router -> expert projections -> parameter-space mixing -> one
+// recurrence) differentiated stage by stage in reverse; the notes train the model (loss function / training
+// strategy).  With the scan's gradients (dBpi, dXs, dC~, d dt) in hand:
+//   mix     dz_j = [dXs_j | pi_j dBpi_j | pi_j dC~]  per (token, slot);  dpi_j = <B_j, dBpi_j> + <C_j, dC~>
+//   router  dg_j = pi_j (dpi_j - sum_i pi_i dpi_i) on the active set (held fixed: a top-k choice has no
+//           gradient);  du = d dt * sigmoid(u) where the clamp of dt = clamp(softplus(u)) is not active,
+//           with sigmoid(u) = 1 - e^{-softplus(u)} = -expm1(-dt)
+//   linear  dW_exp[e] = sum over the (token, slot) rows of expert e of dz (x) X_token
+//           dX_t = sum_j W_exp[K_tj]^T dz_tj + W_r^T dg_t + W_dt^T du_t;  dW_r = dg^T X;  dW_dt = du^T X;
+//           db_dt = sum_t du_t.
+// The (token, slot) rows are visited in the dispatch's expert order (perm, offsets, row tiles), as in the
+// forward projection.
+#include "common.cuh"
+
+namespace swimba {
+
+namespace {
+constexpr int kT = 64;   // output tile edge of the CUDA-core GEMMs
+constexpr int kK = 16;   // contraction step
+
+// mix: one CTA per (token, slot) pair p; z (raw projection, fp32) is overwritten by dz
+__global__ void __launch_bounds__(256) mix_bwd_kernel(Dims d, float* __restrict__ z, const float* __restrict__ wts,
+                                                      const float* __restrict__ dbpi, const float* __restrict__ dxs,
+                                                      const float* __restrict__ dct, float* __restrict__ dpi) {
+  __shared__ float red[8];
+  const size_t p = blockIdx.x;
+  const size_t m = p / d.k;
+  const float pi = wts[p];
+  float* zr = z + p * d.We;
+  const float* gb = dbpi + p * d.GN;
+  const float* gc = dct + m * d.GN;
+  float part = 0.f;
+  for (int c = threadIdx.x; c < d.GN; c += blockDim.x)
+    part = fmaf(zr[d.HP + c], gb[c], fmaf(zr[d.HP + d.GN + c], gc[c], part));
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = part;
+  __syncthreads();  // every read of z is done before it is overwritten below
+  if (threadIdx.x == 0) {
+    float v = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) v += red[w];
+    dpi[p] = v;
+  }
+  const float* gx = dxs + p * d.HP;
+  for (int c = threadIdx.x; c < d.HP; c += blockDim.x) zr[c] = gx[c];
+  for (int c = threadIdx.x; c < d.GN; c += blockDim.x) {
+    zr[d.HP + c] = pi * gb[c];
+    zr[d.HP + d.GN + c] = pi * gc[c];
+  }
+}
+
+// router and dt: dg [M][E] (zero off the active set), du [M][H]
+__global__ void router_bwd_kernel(Dims d, const int32_t* __restrict__ idx, const float* __restrict__ wts,
+                                  const float* __restrict__ dpi, const float* __restrict__ dt,
+                                  const float* __restrict__ ddt, float* __restrict__ dg, float* __restrict__ du) {
+  const size_t m = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (m >= (size_t)d.M) return;
+  float s = 0.f;
+  for (int j = 0; j < d.k; ++j) s = fmaf(wts[m * d.k + j], dpi[m * d.k + j], s);
+  for (int e = 0; e < d.E; ++e) dg[m * d.E + e] = 0.f;
+  for (int j = 0; j < d.k; ++j) {
+    const int e = idx[m * d.k + j];
+    if (e >= 0 && e < d.E) dg[m * d.E + e] = wts[m * d.k + j] * (dpi[m * d.k + j] - s);
+  }
+  for (int h = 0; h < d.H; ++h) {
+    const float v = dt[m * d.H + h];
+    du[m * d.H + h] = (v > 1e-3f && v < 0.1f) ? ddt[m * d.H + h] * -expm1f(-v) : 0.f;
+  }
+}
+
+// dXp[p][n] = sum_c dz[p][c] W_exp[e][c][n] for the rows of one dispatch tile (expert e), 64 columns n
+template <class T>
+__global__ void __launch_bounds__(256)
+dx_experts_kernel(Dims d, const float* __restrict__ dz, const T* __restrict__ W, const int32_t* __restrict__ perm,
+                  const int32_t* __restrict__ tiles, const int32_t* __restrict__ ntiles,
+                  const int32_t* __restrict__ offsets, float* __restrict__ dxp) {
+  __shared__ float As[kK][kRowTile + 4];
+  __shared__ float Bs[kK][kT + 4];
+  __shared__ int pr[kRowTile];
+  if ((int)blockIdx.x >= *ntiles) return;
+  const int e = tiles[2 * blockIdx.x], row0 = tiles[2 * blockIdx.x + 1];
+  const int rows = min(kRowTile, offsets[e + 1] - row0);
+  const int n0 = blockIdx.y * kT;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  for (int r = tid; r < kRowTile; r += 256) pr[r] = r < rows ? perm[row0 + r] : -1;
+  __syncthreads();
+  const T* We = W + (size_t)e * d.We * d.D;
+  float acc[8][4] = {};
+  for (int c0 = 0; c0 < d.We; c0 += kK) {
+    for (int i = tid; i < kK * kRowTile; i += 256) {
+      const int r = i / kK, kk = i % kK, p = pr[r];
+      As[kk][r] = (p >= 0 && c0 + kk < d.We) ? dz[(size_t)p * d.We + c0 + kk] : 0.f;
+    }
+    for (int i = tid; i < kK * kT; i += 256) {
+      const int kk = i / kT, n = i % kT;
+      Bs[kk][n] = (c0 + kk < d.We && n0 + n < d.D) ? to_f32(We[(size_t)(c0 + kk) * d.D + n0 + n]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kK; ++kk) {
+      float av[8], bv[4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) av[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = ty + 16 * i;
+    if (r >= rows) continue;
+    const int p = pr[r];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx + 16 * j;
+      if (n < d.D) dxp[(size_t)p * d.D + n] = acc[i][j];
+    }
+  }
+}
+
+// dW_exp[e][c][n] += sum over a slice of expert e's rows of dz[p][c] X[token(p)][n]; grid (row slices, c tiles,
+// n tiles) over the dispatch tiles, accumulated with atomic adds into a zeroed output
+template <class T>
+__global__ void __launch_bounds__(256)
+dw_experts_kernel(Dims d, const float* __restrict__ dz, const T* __restrict__ X, const int32_t* __restrict__ perm,
+                  const int32_t* __restrict__ tiles, const int32_t* __restrict__ ntiles,
+                  const int32_t* __restrict__ offsets, float* __restrict__ dW) {
+  __shared__ float As[kK][kT + 4];
+  __shared__ float Bs[kK][kT + 4];
+  __shared__ int pr[kRowTile];
+  if ((int)blockIdx.x >= *ntiles) return;
+  const int e = tiles[2 * blockIdx.x], row0 = tiles[2 * blockIdx.x + 1];
+  const int rows = min(kRowTile, offsets[e + 1] - row0);
+  const int c0 = blockIdx.y * kT, n0 = blockIdx.z * kT;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  for (int r = tid; r < kRowTile; r += 256) pr[r] = r < rows ? perm[row0 + r] : -1;
+  __syncthreads();
+  float acc[4][4] = {};
+  for (int r0 = 0; r0 < rows; r0 += kK) {
+    for (int i = tid; i < kK * kT; i += 256) {
+      const int kk = i / kT, c = i % kT, r = r0 + kk;
+      const int p = r < rows ? pr[r] : -1;
+      As[kk][c] = (p >= 0 && c0 + c < d.We) ? dz[(size_t)p * d.We + c0 + c] : 0.f;
+      Bs[kk][c] = (p >= 0 && n0 + c < d.D) ? to_f32(X[(size_t)(p / d.k) * d.D + n0 + c]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kK; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* out = dW + (size_t)e * d.We * d.D;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = c0 + ty + 16 * i;
+    if (c >= d.We) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx + 16 * j;
+      if (n < d.D) atomicAdd(&out[(size_t)c * d.D + n], acc[i][j]);
+    }
+  }
+}
+
+// out[r][n] += sum over a 256-token slice of G[m][r] X[m][n] (dW_r from dg, dW_dt from du); 64-row tiles of r
+template <class T>
+__global__ void __launch_bounds__(256)
+dw_dense_kernel(int M, int R, int D, const float* __restrict__ G, const T* __restrict__ X, float* __restrict__ out) {
+  __shared__ float As[kK][kT + 4];
+  __shared__ float Bs[kK][kT + 4];
+  const int n0 = blockIdx.x * kT, m_begin = blockIdx.y * 256, m_end = min(M, m_begin + 256), r0 = blockIdx.z * kT;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float acc[4][4] = {};
+  for (int m0 = m_begin; m0 < m_end; m0 += kK) {
+    for (int i = tid; i < kK * kT; i += 256) {
+      const int kk = i / kT, c = i % kT, m = m0 + kk;
+      As[kk][c] = (m < m_end && r0 + c < R) ? G[(size_t)m * R + r0 + c] : 0.f;
+      Bs[kk][c] = (m < m_end && n0 + c < D) ? to_f32(X[(size_t)m * D + n0 + c]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kK; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + ty + 16 * i;
+    if (r >= R) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx + 16 * j;
+      if (n < D) atomicAdd(&out[(size_t)r * D + n], acc[i][j]);
+    }
+  }
+}
+
+// dX[m][n] = sum_j dXp[m k + j][n] + sum_e dg[m][e] W_r[e][n] + sum_h du[m][h] W_dt[h][n];  db_dt[h] += du
+template <class T>
+__global__ void dx_final_kernel(Dims d, const float* __restrict__ dxp, const float* __restrict__ dg,
+                                const float* __restrict__ du, const T* __restrict__ Wr, const T* __restrict__ Wdt,
+                                float* __restrict__ dX) {
+  const size_t total = (size_t)d.M * d.D;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t m = i / d.D;
+    const int n = (int)(i % d.D);
+    float v = 0.f;
+    for (int j = 0; j < d.k; ++j) v += dxp[(m * d.k + j) * d.D + n];
+    for (int e = 0; e < d.E; ++e) v = fmaf(dg[m * d.E + e], to_f32(Wr[(size_t)e * d.D + n]), v);
+    for (int h = 0; h < d.H; ++h) v = fmaf(du[m * d.H + h], to_f32(Wdt[(size_t)h * d.D + n]), v);
+    dX[i] = v;
+  }
+}
+
+__global__ void db_kernel(Dims d, const float* __restrict__ du, float* __restrict__ db) {
+  const int h = blockIdx.x;
+  float s = 0.f;
+  for (int m = threadIdx.x; m < d.M; m += blockDim.x) s += du[(size_t)m * d.H + h];
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) v += red[w];
+    db[h] = v;
+  }
+}
+
+template <class T>
+cudaError_t launch_tail_typed(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s) {
+  mix_bwd_kernel<<<d.M * d.k, 256, 0, s>>>(d, q.z, q.wts, q.dbpi, q.dxs, q.dct, q.dpi);
+  router_bwd_kernel<<<ceil_div(d.M, 128), 128, 0, s>>>(d, q.idx, q.wts, q.dpi, q.dt, q.ddt, q.dg, q.du);
+  const dim3 gx(max_row_tiles(d), ceil_div(d.D, kT));
+  dx_experts_kernel<T><<<gx, 256, 0, s>>>(d, q.z, (const T*)q.w_exp, q.perm, q.tiles, q.ntiles, q.offsets, q.dxp);
+  cudaError_t e = cudaMemsetAsync(q.dW_exp, 0, (size_t)d.E * d.We * d.D * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(q.dW_r, 0, (size_t)d.E * d.D * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(q.dW_dt, 0, (size_t)d.H * d.D * 4, s);
+  if (e != cudaSuccess) return e;
+  const dim3 gw(max_row_tiles(d), ceil_div(d.We, kT), ceil_div(d.D, kT));
+  dw_experts_kernel<T><<<gw, 256, 0, s>>>(d, q.z, (const T*)q.X, q.perm, q.tiles, q.ntiles, q.offsets, q.dW_exp);
+  dw_dense_kernel<T><<<dim3(ceil_div(d.D, kT), ceil_div(d.M, 256), ceil_div(d.E, kT)), 256, 0, s>>>(
+      d.M, d.E, d.D, q.dg, (const T*)q.X, q.dW_r);
+  dw_dense_kernel<T><<<dim3(ceil_div(d.D, kT), ceil_div(d.M, 256), ceil_div(d.H, kT)), 256, 0, s>>>(
+      d.M, d.H, d.D, q.du, (const T*)q.X, q.dW_dt);
+  db_kernel<<<d.H, 256, 0, s>>>(d, q.du, q.db_dt);
+  dx_final_kernel<T><<<148 * 8, 256, 0, s>>>(d, q.dxp, q.dg, q.du, (const T*)q.w_r, (const T*)q.w_dt, q.dX);
+  count_launches(9);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_layer_bwd_tail(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s) {
+  return d.dtype == SWIMBA_BF16 ? launch_tail_typed<__nv_bfloat16>(d, q, s) : launch_tail_typed<float>(d, q, s);
+}
+
+}  // namespace swimba

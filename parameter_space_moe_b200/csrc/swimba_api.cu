@@ -546,6 +546,75 @@ swimba_status swimba_out_proj(const swimba_dims* dims, const void* y, const void
   return cuda_status(launch_out_proj(d, y, w_out, out, st, (cudaStream_t)stream));
 }
 
+// Workspace of swimba_layer_bwd: the layer's own, then the gradient buffers (all fp32).
+struct BwdPlan {
+  size_t z, dbpi, dxs, dct, ddt, dpi, dg, du, dxp, total;
+};
+static BwdPlan plan_bwd(const Dims& d) {
+  BwdPlan q{};
+  size_t o = align_up(plan_workspace(d).total, 256);
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+  const size_t Mk = (size_t)d.M * d.k;
+  q.z = take(Mk * d.We * 4);
+  q.dbpi = take(Mk * d.GN * 4);
+  q.dxs = take(Mk * d.HP * 4);
+  q.dct = take((size_t)d.M * d.GN * 4);
+  q.ddt = take((size_t)d.M * d.H * 4);
+  q.dpi = take(Mk * 4);
+  q.dg = take((size_t)d.M * d.E * 4);
+  q.du = take((size_t)d.M * d.H * 4);
+  q.dxp = take(Mk * d.D * 4);
+  q.total = o;
+  return q;
+}
+
+size_t swimba_layer_bwd_workspace_size(const swimba_dims* dims) {
+  Dims d;
+  if (make_dims(dims, &d) != SWIMBA_OK) return 0;
+  return plan_bwd(d).total;
+}
+
+swimba_status swimba_layer_bwd(const swimba_dims* dims, const void* X, const swimba_weights* w,
+                               const float* init_state, const float* dy, float* dX, float* dW_router, float* dW_dt,
+                               float* db_dt, float* dA, float* dW_exp, float* d_init, void* ws, size_t ws_bytes,
+                               void* stream) {
+  Dims d;
+  SW_TRY(make_dims(dims, &d));
+  SW_TRY(check_weights(w, true, true));
+  if (w->A_exp || !w->A) return SWIMBA_ERR_UNSUPPORTED;
+  if (!ok_ptr(X) || !ok_ptr(dy) || !ok_ptr(dX) || !ok_ptr(dW_router) || !ok_ptr(dW_dt) || !db_dt || !dA ||
+      !ok_ptr(dW_exp) || !ok_opt(init_state) || !ok_opt(d_init))
+    return SWIMBA_ERR_INVALID_ARG;
+  if (scan_bwd_smem(d) > (size_t)227 * 1024) return SWIMBA_ERR_UNSUPPORTED;
+  const BwdPlan q = plan_bwd(d);
+  if (!ws || ((uintptr_t)ws & 15u) || ws_bytes < q.total) return SWIMBA_ERR_WORKSPACE;
+  WsPlan p = plan_workspace(d);
+  char* b = (char*)ws;
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned* st = device_status();
+  if (!st) return SWIMBA_ERR_CUDA;
+  int32_t* idx = (int32_t*)(b + p.topk_idx);
+  float* wts = (float*)(b + p.topk_w);
+  float* dt = (float*)(b + p.dt);
+  prof_begin(s);
+  // the forward's router, dispatch and mixed streams, then the raw projections z for the mix's gradient
+  SW_TRY(run_front(d, X, w, b, p, idx, wts, 0, st, s));
+  SW_TRY(run_proj(d, X, w->w_exp, b, p, wts, 2, nullptr, nullptr, nullptr, (float*)(b + q.z), st, s,
+                  /*gathered=*/d.dtype == SWIMBA_BF16));
+  SW_CUDA(launch_scan_bwd(d, b + p.bpi, b + p.xs, b + p.cpi, dt, w->A, init_state, dy, (float*)(b + q.dbpi),
+                          (float*)(b + q.dxs), (float*)(b + q.dct), (float*)(b + q.ddt), dA, d_init,
+                          (float*)(b + p.hstart), (float*)(b + p.schunk), (float*)(b + p.cslast), s));
+  prof_mark(s, "ssd_scan_bwd");
+  LayerBwdPtrs t{X, w->w_exp, w->w_router, w->w_dt, idx, wts, dt, (const float*)(b + q.ddt),
+                 (const int32_t*)(b + p.perm), (const int32_t*)(b + p.tiles), (const int32_t*)(b + p.ntiles),
+                 (const int32_t*)(b + p.offsets), (float*)(b + q.z), (const float*)(b + q.dbpi),
+                 (const float*)(b + q.dxs), (const float*)(b + q.dct), (float*)(b + q.dpi), (float*)(b + q.dg),
+                 (float*)(b + q.du), (float*)(b + q.dxp), dX, dW_router, dW_dt, db_dt, dW_exp};
+  SW_CUDA(launch_layer_bwd_tail(d, t, s));
+  prof_mark(s, "mix_router_linear_bwd");
+  return SWIMBA_OK;
+}
+
 swimba_status swimba_ssd_scan_bwd(const swimba_dims* dims, const void* Bpi, const void* Xs, const void* Cpi,
                                   const float* dt, const float* A, const float* init_state, const float* dy,
                                   float* dBpi, float* dXs, float* dCt, float* d_dt, float* dA, float* d_init,

@@ -23,7 +23,7 @@ EXPORTS = ("swimba_workspace_size", "swimba_stream_dtype", "swimba_router_topk",
            "swimba_separated_scan", "swimba_check_device_status", "swimba_status_string",
            "swimba_profile_enable", "swimba_profile_read", "swimba_launch_count", "swimba_dispatch_noalloc",
            "swimba_layer_fwd_host", "swimba_debug_scan_lost_first_chunk", "swimba_out_proj",
-           "swimba_ssd_scan_bwd")
+           "swimba_ssd_scan_bwd", "swimba_layer_bwd", "swimba_layer_bwd_workspace_size")
 
 
 class SwimbaError(RuntimeError):
@@ -58,6 +58,8 @@ def lib():
         L.swimba_workspace_size.argtypes = [P(Dims)]
         L.swimba_stream_dtype.restype = ctypes.c_int
         L.swimba_stream_dtype.argtypes = [P(Dims)]
+        L.swimba_layer_bwd_workspace_size.restype = sz
+        L.swimba_layer_bwd_workspace_size.argtypes = [P(Dims)]
         L.swimba_status_string.restype = ctypes.c_char_p
         L.swimba_status_string.argtypes = [ctypes.c_int]
         sig = {
@@ -74,6 +76,7 @@ def lib():
             "swimba_separated_scan": [P(Dims), vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_out_proj": [P(Dims), vp, vp, vp, vp],
             "swimba_ssd_scan_bwd": [P(Dims), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "swimba_layer_bwd": [P(Dims), vp, P(Weights), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "swimba_check_device_status": [vp],
         }
         L.swimba_profile_enable.restype = ctypes.c_int
@@ -194,6 +197,16 @@ def ssd_scan_bwd(d, Bpi, Xs, Cpi, dt, A, init_state, dy, dBpi, dXs, dCt, d_dt, d
     _check("swimba_ssd_scan_bwd", lib().swimba_ssd_scan_bwd(
         ctypes.byref(d), _p(Bpi), _p(Xs), _p(Cpi), _p(dt), _p(A), _p(init_state), _p(dy), _p(dBpi), _p(dXs),
         _p(dCt), _p(d_dt), _p(dA), _p(d_init), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def layer_bwd_workspace_size(d):
+    return lib().swimba_layer_bwd_workspace_size(ctypes.byref(d))
+
+
+def layer_bwd(d, X, W, init_state, dy, dX, dW_r, dW_dt, db_dt, dA, dW_exp, d_init, ws, stream=None):
+    _check("swimba_layer_bwd", lib().swimba_layer_bwd(
+        ctypes.byref(d), _p(X), ctypes.byref(W.c), _p(init_state), _p(dy), _p(dX), _p(dW_r), _p(dW_dt), _p(db_dt),
+        _p(dA), _p(dW_exp), _p(d_init), _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def out_proj(d, y, w_out, out, stream=None):

@@ -132,6 +132,15 @@ def test_null_misaligned_and_workspace_errors(L):
     assert bwd(None) == 1
     assert bwd(odd) == 1
     assert bwd(fake, n=need - 1) == 4
+    # layer gradients: null pointers, a workspace sized for the forward only, the mixed transition
+    nb = swimba.layer_bwd_workspace_size(d)
+    assert nb > need
+    lbwd = lambda wts, dy, n: L.swimba_layer_bwd(ctypes.byref(d), fake, ctypes.byref(wts), None, dy, fake, fake,
+                                                 fake, fake, fake, fake, None, fake, n, None)
+    assert lbwd(w, None, nb) == 1
+    assert lbwd(w, fake, need) == 4
+    wmix = swimba.Weights(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    assert lbwd(wmix, fake, nb) == 2
     # output projection: every pointer non-null and 16-byte aligned
     assert L.swimba_out_proj(ctypes.byref(d), None, fake, fake, None) == 1
     assert L.swimba_out_proj(ctypes.byref(d), fake, odd, fake, None) == 1
