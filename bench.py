@@ -14,8 +14,9 @@ by HBM), "esweep" (the base layer at E in {8, 16, 32, 64}: layer and scan-stage 
 method's cost statement says are flat in E, plus the separated-trajectory scan that runs k trajectories) and
 "out_proj" (the output projection y W_out^T on the base layer's y, bound by the tensor cores), "mixed_A"
 (the base layer with the expert-mixed transition A~ = sum_j pi_j A_exp[K_j]), "groups" (the base layer
-with B and C shared by G in {H, H/4, 1} groups of heads: layer and scan times) and "scan_bwd" (the scan
-gradients at the base sizes, bound by fp32 CUDA-core arithmetic).
+with B and C shared by G in {H, H/4, 1} groups of heads: layer and scan times), "scan_bwd" (the scan
+gradients at the base sizes, bound by fp32 CUDA-core arithmetic) and "layer_bwd" (the whole layer's gradients
+at the base workload).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launching stream,
 with a write of 2x the L2 size between steps (outside the events) so every step reads its inputs from
@@ -509,6 +510,52 @@ def scan_bwd_measure(args, dev, flush, stream, swimba):
                          "peak_source": f"148 SMs x 128 fp32 lanes x 2 FLOP x {mhz:.0f} MHz (max SM clock)"}}
 
 
+def layer_bwd_measure(args, sess, inp, flush, stream, swimba):
+    """The layer gradients (swimba_layer_bwd) at the base workload with a seeded dy, timed alone: one call
+    recomputes the forward's router, dispatch and projections, then runs the scan gradients and the CUDA-core
+    mix, router and weight-gradient kernels.  The roofline counts the gradient arithmetic (scan gradients,
+    the two expert products dz W and dz^T X, the router and dt products) against the fp32 ALU peak."""
+    w = sess.w
+    dev = sess.X.device
+    g = torch.Generator().manual_seed(151)
+    dy = torch.randn(w.M, w.nheads, w.headdim, generator=g).to(dev)
+    outs = [torch.empty(w.M, w.d_model, device=dev), torch.empty(w.n_experts, w.d_model, device=dev),
+            torch.empty(w.nheads, w.d_model, device=dev), torch.empty(w.nheads, device=dev),
+            torch.empty(w.nheads, device=dev), torch.empty(w.n_experts, w.W_e, w.d_model, device=dev)]
+    ws = torch.empty(swimba.layer_bwd_workspace_size(sess.d), dtype=torch.uint8, device=dev)
+    call = lambda: swimba.layer_bwd(sess.d, sess.X, sess.W, None, dy, *outs, None, ws)
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tot = 0.0
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e0.record(stream)
+        call()
+        e1.record(stream)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    stages = {}
+    swimba.profile_enable(True)
+    flush.fill_(1)
+    call()
+    for name, ms in swimba.profile_read():
+        stages[name] = stages.get(name, 0.0) + ms
+    swimba.profile_enable(False)
+    if swimba.check_device_status() != 0:
+        raise RuntimeError("swimba_layer_bwd raised a device status")
+    secs = tot / args.steps / 1e3
+    flops = (scan_bwd_flops(w) + 2 * 2.0 * w.M * w.top_k * w.W_e * w.d_model
+             + 2 * 2.0 * w.M * (w.n_experts + w.nheads) * w.d_model)
+    peak = 148 * 128 * 2 * 1965e6 / 1e12
+    return {"ms": secs * 1e3, "stages_ms": stages, "gradient_flops": flops,
+            "roofline": {"bound": "alu", "achieved": flops / secs / 1e12, "peak": peak, "unit": "TFLOP/s",
+                         "frac": flops / secs / 1e12 / peak,
+                         "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz; the time includes the "
+                                        "forward recompute"}}
+
+
 def out_proj_measure(args, sess, inp, flush, stream, swimba):
     """The output projection out = y W_out^T (swimba_out_proj) on the layer's own y, timed alone: K launches
     between L2 flushes, against the burst bf16 peak (a kernel timed alone)."""
@@ -590,6 +637,7 @@ def run_gpu(args, w):
     # one GPU, default workload: the decode step and the expert-count sweep in the same line
     if world == 1 and w.name == configs.BASE.name and not args.no_extras:
         out["out_proj"] = out_proj_measure(args, sess, inp, flush, stream, swimba)
+        out["layer_bwd"] = layer_bwd_measure(args, sess, inp, flush, stream, swimba)
         del sess
         torch.cuda.empty_cache()
         msess = LayerSession(w, dev, inp, swimba, mixed_A=True)
