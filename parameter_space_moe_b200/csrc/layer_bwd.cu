@@ -69,110 +69,142 @@ __global__ void router_bwd_kernel(Dims d, const int32_t* __restrict__ idx, const
   }
 }
 
-// dXp[p][n] = sum_c dz[p][c] W_exp[e][c][n] for the rows of one dispatch tile (expert e), 64 columns n
+// 128 x 128 output tiles, 8 x 8 per thread (rows ty * 8 .., columns tx * 8 ..), contraction staged 8 at a
+// time through two shared-memory buffers: each thread loads the next stage's four A and four B values into
+// registers (one 16-byte dz load, one 4-element operand load) while the current stage is multiplied, so one
+// barrier per stage suffices and the global latency hides behind 512 FMAs.  W_e % 16 == 0 and D % 8 == 0,
+// so a 4-wide group never straddles a matrix edge.
+constexpr int kBT2 = 128, kBK2 = 8, kLd2 = kBT2 + 4;
+struct Stage {
+  float A[kBK2][kLd2];
+  float B[kBK2][kLd2];
+};
+
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
+__device__ __forceinline__ void mac8x8(const Stage& S, int ty, int tx, float (&acc)[8][8]) {
+#pragma unroll
+  for (int kk = 0; kk < kBK2; ++kk) {
+    const float4 a0 = *reinterpret_cast<const float4*>(&S.A[kk][ty * 8]);
+    const float4 a1 = *reinterpret_cast<const float4*>(&S.A[kk][ty * 8 + 4]);
+    const float4 b0 = *reinterpret_cast<const float4*>(&S.B[kk][tx * 8]);
+    const float4 b1 = *reinterpret_cast<const float4*>(&S.B[kk][tx * 8 + 4]);
+    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+  }
+}
+
+// dXp[p][n] = sum_c dz[p][c] W_exp[e][c][n] for the rows of one 128-row dispatch tile (expert e), 128 columns n.
+// A stage: A = dz[rows][c0 .. c0+8) transposed (thread: row tid/2, columns 4 (tid&1) ..), B = W_e[c0 .. c0+8)[n]
+// (thread: row tid/32, columns 4 (tid&31) ..).
 template <class T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 dx_experts_kernel(Dims d, const float* __restrict__ dz, const T* __restrict__ W, const int32_t* __restrict__ perm,
                   const int32_t* __restrict__ tiles, const int32_t* __restrict__ ntiles,
                   const int32_t* __restrict__ offsets, float* __restrict__ dxp) {
-  __shared__ float As[kK][kRowTile + 4];
-  __shared__ float Bs[kK][kT + 4];
+  __shared__ __align__(16) Stage st[2];
   __shared__ int pr[kRowTile];
   if ((int)blockIdx.x >= *ntiles) return;
   const int e = tiles[2 * blockIdx.x], row0 = tiles[2 * blockIdx.x + 1];
   const int rows = min(kRowTile, offsets[e + 1] - row0);
-  const int n0 = blockIdx.y * kT;
+  const int n0 = blockIdx.y * kBT2;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   for (int r = tid; r < kRowTile; r += 256) pr[r] = r < rows ? perm[row0 + r] : -1;
   __syncthreads();
   const T* We = W + (size_t)e * d.We * d.D;
-  float acc[8][4] = {};
-  for (int c0 = 0; c0 < d.We; c0 += kK) {
-    for (int i = tid; i < kK * kRowTile; i += 256) {
-      const int r = i / kK, kk = i % kK, p = pr[r];
-      As[kk][r] = (p >= 0 && c0 + kk < d.We) ? dz[(size_t)p * d.We + c0 + kk] : 0.f;
-    }
-    for (int i = tid; i < kK * kT; i += 256) {
-      const int kk = i / kT, n = i % kT;
-      Bs[kk][n] = (c0 + kk < d.We && n0 + n < d.D) ? to_f32(We[(size_t)(c0 + kk) * d.D + n0 + n]) : 0.f;
-    }
+  const int ar = tid >> 1, ak = (tid & 1) * 4, bk = tid >> 5, bn = (tid & 31) * 4;
+  const int ap = pr[ar];
+  const float* arow = dz + (size_t)max(ap, 0) * d.We + ak;
+  const T* bptr = We + (size_t)bk * d.D + n0 + bn;
+  const bool aok = ap >= 0, bok = n0 + bn < d.D;
+  const size_t bstep = (size_t)kBK2 * d.D;
+  const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto fetch = [&](int c0, float4& a, float4& b) {
+    a = (aok && c0 + ak < d.We) ? load4(arow + c0) : z4;
+    b = (bok && c0 + bk < d.We) ? load4(bptr) : z4;
+    bptr += bstep;
+  };
+  float4 a, b;
+  fetch(0, a, b);
+  float acc[8][8] = {};
+  int buf = 0;
+  for (int c0 = 0; c0 < d.We; c0 += kBK2) {
+    Stage& S = st[buf];
+    S.A[ak][ar] = a.x; S.A[ak + 1][ar] = a.y; S.A[ak + 2][ar] = a.z; S.A[ak + 3][ar] = a.w;
+    *reinterpret_cast<float4*>(&S.B[bk][bn]) = b;
     __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kK; ++kk) {
-      float av[8], bv[4];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) av[i] = As[kk][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx + 16 * j];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
+    if (c0 + kBK2 < d.We) fetch(c0 + kBK2, a, b);
+    mac8x8(S, ty, tx, acc);
+    buf ^= 1;
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int r = ty + 16 * i;
+    const int r = ty * 8 + i;
     if (r >= rows) continue;
     const int p = pr[r];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx + 16 * j;
-      if (n < d.D) dxp[(size_t)p * d.D + n] = acc[i][j];
+    for (int j = 0; j < 8; j += 4) {
+      const int n = n0 + tx * 8 + j;
+      if (n < d.D)
+        *reinterpret_cast<float4*>(dxp + (size_t)p * d.D + n) =
+            make_float4(acc[i][j], acc[i][j + 1], acc[i][j + 2], acc[i][j + 3]);
     }
   }
 }
 
-// dW_exp[e][c][n] += sum over a slice of expert e's rows of dz[p][c] X[token(p)][n]; grid (row slices, c tiles,
-// n tiles) over the dispatch tiles, accumulated with atomic adds into a zeroed output
+// dW_exp[e][c][n] = sum over all of expert e's (token, slot) rows of dz[p][c] X[token(p)][n]: one CTA per
+// (expert, 128 W_e columns c, 128 D columns n) walks the expert's sorted rows 8 at a time (plain stores, no
+// atomics).  A stage: A = dz[row][c0 ..], B = X[token][n0 ..] (thread: row tid/32, columns 4 (tid&31) ..).
 template <class T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 dw_experts_kernel(Dims d, const float* __restrict__ dz, const T* __restrict__ X, const int32_t* __restrict__ perm,
-                  const int32_t* __restrict__ tiles, const int32_t* __restrict__ ntiles,
                   const int32_t* __restrict__ offsets, float* __restrict__ dW) {
-  __shared__ float As[kK][kT + 4];
-  __shared__ float Bs[kK][kT + 4];
-  __shared__ int pr[kRowTile];
-  if ((int)blockIdx.x >= *ntiles) return;
-  const int e = tiles[2 * blockIdx.x], row0 = tiles[2 * blockIdx.x + 1];
-  const int rows = min(kRowTile, offsets[e + 1] - row0);
-  const int c0 = blockIdx.y * kT, n0 = blockIdx.z * kT;
+  __shared__ __align__(16) Stage st[2];
+  const int e = blockIdx.x, c0 = blockIdx.y * kBT2, n0 = blockIdx.z * kBT2;
+  const int rb = offsets[e], re = offsets[e + 1];
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  for (int r = tid; r < kRowTile; r += 256) pr[r] = r < rows ? perm[row0 + r] : -1;
-  __syncthreads();
-  float acc[4][4] = {};
-  for (int r0 = 0; r0 < rows; r0 += kK) {
-    for (int i = tid; i < kK * kT; i += 256) {
-      const int kk = i / kT, c = i % kT, r = r0 + kk;
-      const int p = r < rows ? pr[r] : -1;
-      As[kk][c] = (p >= 0 && c0 + c < d.We) ? dz[(size_t)p * d.We + c0 + c] : 0.f;
-      Bs[kk][c] = (p >= 0 && n0 + c < d.D) ? to_f32(X[(size_t)(p / d.k) * d.D + n0 + c]) : 0.f;
-    }
+  const int kr = tid >> 5, kc = (tid & 31) * 4;
+  const bool aok = c0 + kc < d.We, bok = n0 + kc < d.D;
+  const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto fetch = [&](int r0, float4& a, float4& b) {
+    const int p = r0 + kr < re ? perm[r0 + kr] : -1;
+    a = (p >= 0 && aok) ? load4(dz + (size_t)p * d.We + c0 + kc) : z4;
+    b = (p >= 0 && bok) ? load4(X + (size_t)(p / d.k) * d.D + n0 + kc) : z4;
+  };
+  float4 a, b;
+  if (rb < re) fetch(rb, a, b);
+  float acc[8][8] = {};
+  int buf = 0;
+  for (int r0 = rb; r0 < re; r0 += kBK2) {
+    Stage& S = st[buf];
+    *reinterpret_cast<float4*>(&S.A[kr][kc]) = a;
+    *reinterpret_cast<float4*>(&S.B[kr][kc]) = b;
     __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kK; ++kk) {
-      float av[4], bv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx + 16 * j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
+    if (r0 + kBK2 < re) fetch(r0 + kBK2, a, b);
+    mac8x8(S, ty, tx, acc);
+    buf ^= 1;
   }
   float* out = dW + (size_t)e * d.We * d.D;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int c = c0 + ty + 16 * i;
+  for (int i = 0; i < 8; ++i) {
+    const int c = c0 + ty * 8 + i;
     if (c >= d.We) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx + 16 * j;
-      if (n < d.D) atomicAdd(&out[(size_t)c * d.D + n], acc[i][j]);
+    for (int j = 0; j < 8; j += 4) {
+      const int n = n0 + tx * 8 + j;
+      if (n < d.D)
+        *reinterpret_cast<float4*>(out + (size_t)c * d.D + n) =
+            make_float4(acc[i][j], acc[i][j + 1], acc[i][j + 2], acc[i][j + 3]);
     }
   }
 }
@@ -255,14 +287,13 @@ template <class T>
 cudaError_t launch_tail_typed(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s) {
   mix_bwd_kernel<<<d.M * d.k, 256, 0, s>>>(d, q.z, q.wts, q.dbpi, q.dxs, q.dct, q.dpi);
   router_bwd_kernel<<<ceil_div(d.M, 128), 128, 0, s>>>(d, q.idx, q.wts, q.dpi, q.dt, q.ddt, q.dg, q.du);
-  const dim3 gx(max_row_tiles(d), ceil_div(d.D, kT));
+  const dim3 gx(max_row_tiles(d), ceil_div(d.D, kBT2));
   dx_experts_kernel<T><<<gx, 256, 0, s>>>(d, q.z, (const T*)q.w_exp, q.perm, q.tiles, q.ntiles, q.offsets, q.dxp);
-  cudaError_t e = cudaMemsetAsync(q.dW_exp, 0, (size_t)d.E * d.We * d.D * 4, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(q.dW_r, 0, (size_t)d.E * d.D * 4, s);
+  cudaError_t e = cudaMemsetAsync(q.dW_r, 0, (size_t)d.E * d.D * 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(q.dW_dt, 0, (size_t)d.H * d.D * 4, s);
   if (e != cudaSuccess) return e;
-  const dim3 gw(max_row_tiles(d), ceil_div(d.We, kT), ceil_div(d.D, kT));
-  dw_experts_kernel<T><<<gw, 256, 0, s>>>(d, q.z, (const T*)q.X, q.perm, q.tiles, q.ntiles, q.offsets, q.dW_exp);
+  const dim3 gw(d.E, ceil_div(d.We, kBT2), ceil_div(d.D, kBT2));
+  dw_experts_kernel<T><<<gw, 256, 0, s>>>(d, q.z, (const T*)q.X, q.perm, q.offsets, q.dW_exp);
   dw_dense_kernel<T><<<dim3(ceil_div(d.D, kT), ceil_div(d.M, 256), ceil_div(d.E, kT)), 256, 0, s>>>(
       d.M, d.E, d.D, q.dg, (const T*)q.X, q.dW_r);
   dw_dense_kernel<T><<<dim3(ceil_div(d.D, kT), ceil_div(d.M, 256), ceil_div(d.H, kT)), 256, 0, s>>>(
