@@ -1,4 +1,4 @@
-// Gradients of the whole layer: the stages after the scan gradients, on CUDA cores in fp32.
+// Gradients of the whole layer: the stages after the scan gradients, in fp32.
 //
 // Paper: Swimba notes, Method flowchart (router -> expert projections -> parameter-space mixing -> one
 // recurrence) differentiated stage by stage in reverse; the notes train the model (loss function / training
@@ -11,7 +11,8 @@
 //           dX_t = sum_j W_exp[K_tj]^T dz_tj + W_r^T dg_t + W_dt^T du_t;  dW_r = dg^T X;  dW_dt = du^T X;
 //           db_dt = sum_t du_t.
 // The (token, slot) rows are visited in the dispatch's expert order (perm, offsets, row tiles), as in the
-// forward projection.
+// forward projection.  The two expert products run on the tensor cores for bf16 layers (grad_tc.cu, on a
+// bf16 hi/lo split of dz) and on the CUDA-core kernels below for fp32 layers.
 #include "common.cuh"
 
 namespace swimba {
@@ -81,12 +82,6 @@ struct Stage {
 };
 
 __device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
-__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
-  const uint2 u = *reinterpret_cast<const uint2*>(p);
-  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-  return make_float4(a.x, a.y, b.x, b.y);
-}
 
 __device__ __forceinline__ void mac8x8(const Stage& S, int ty, int tx, float (&acc)[8][8]) {
 #pragma unroll
@@ -287,20 +282,29 @@ template <class T>
 cudaError_t launch_tail_typed(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s) {
   mix_bwd_kernel<<<d.M * d.k, 256, 0, s>>>(d, q.z, q.wts, q.dbpi, q.dxs, q.dct, q.dpi);
   router_bwd_kernel<<<ceil_div(d.M, 128), 128, 0, s>>>(d, q.idx, q.wts, q.dpi, q.dt, q.ddt, q.dg, q.du);
-  const dim3 gx(max_row_tiles(d), ceil_div(d.D, kBT2));
-  dx_experts_kernel<T><<<gx, 256, 0, s>>>(d, q.z, (const T*)q.w_exp, q.perm, q.tiles, q.ntiles, q.offsets, q.dxp);
-  cudaError_t e = cudaMemsetAsync(q.dW_r, 0, (size_t)d.E * d.D * 4, s);
+  cudaError_t e;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    // tensor cores on the bf16 hi/lo split of dz
+    e = launch_grad_tc(d, q.z, q.xsorted, q.w_exp, q.perm, q.offsets, q.poff, q.prow, q.dzs, q.xsp, q.dxp, q.dW_exp,
+                       q.st, s);
+    if (e != cudaSuccess) return e;
+  } else {
+    const dim3 gx(max_row_tiles(d), ceil_div(d.D, kBT2));
+    dx_experts_kernel<T><<<gx, 256, 0, s>>>(d, q.z, (const T*)q.w_exp, q.perm, q.tiles, q.ntiles, q.offsets, q.dxp);
+    const dim3 gw(d.E, ceil_div(d.We, kBT2), ceil_div(d.D, kBT2));
+    dw_experts_kernel<T><<<gw, 256, 0, s>>>(d, q.z, (const T*)q.X, q.perm, q.offsets, q.dW_exp);
+    count_launches(2);
+  }
+  e = cudaMemsetAsync(q.dW_r, 0, (size_t)d.E * d.D * 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(q.dW_dt, 0, (size_t)d.H * d.D * 4, s);
   if (e != cudaSuccess) return e;
-  const dim3 gw(d.E, ceil_div(d.We, kBT2), ceil_div(d.D, kBT2));
-  dw_experts_kernel<T><<<gw, 256, 0, s>>>(d, q.z, (const T*)q.X, q.perm, q.offsets, q.dW_exp);
   dw_dense_kernel<T><<<dim3(ceil_div(d.D, kT), ceil_div(d.M, 256), ceil_div(d.E, kT)), 256, 0, s>>>(
       d.M, d.E, d.D, q.dg, (const T*)q.X, q.dW_r);
   dw_dense_kernel<T><<<dim3(ceil_div(d.D, kT), ceil_div(d.M, 256), ceil_div(d.H, kT)), 256, 0, s>>>(
       d.M, d.H, d.D, q.du, (const T*)q.X, q.dW_dt);
   db_kernel<<<d.H, 256, 0, s>>>(d, q.du, q.db_dt);
   dx_final_kernel<T><<<148 * 8, 256, 0, s>>>(d, q.dxp, q.dg, q.du, (const T*)q.w_r, (const T*)q.w_dt, q.dX);
-  count_launches(9);
+  count_launches(6);
   return cudaGetLastError();
 }
 }  // namespace

@@ -548,7 +548,7 @@ swimba_status swimba_out_proj(const swimba_dims* dims, const void* y, const void
 
 // Workspace of swimba_layer_bwd: the layer's own, then the gradient buffers (all fp32).
 struct BwdPlan {
-  size_t z, dbpi, dxs, dct, ddt, dpi, dg, du, dxp, total;
+  size_t z, dbpi, dxs, dct, ddt, dpi, dg, du, dxp, poff, prow, dzs, xsp, total;
 };
 static BwdPlan plan_bwd(const Dims& d) {
   BwdPlan q{};
@@ -564,6 +564,13 @@ static BwdPlan plan_bwd(const Dims& d) {
   q.dg = take((size_t)d.M * d.E * 4);
   q.du = take((size_t)d.M * d.H * 4);
   q.dxp = take(Mk * d.D * 4);
+  if (d.dtype == SWIMBA_BF16) {  // the tensor-core expert gradients' operands
+    const size_t Rp = grad_tc_rows(d), Wp = (size_t)grad_tc_wp(d);
+    q.poff = take((size_t)(d.E + 1) * 4);
+    q.prow = take(Rp * 4);
+    q.dzs = take(Rp * 2 * Wp * 2);
+    q.xsp = take(Rp * d.D * 2);
+  }
   q.total = o;
   return q;
 }
@@ -609,7 +616,8 @@ swimba_status swimba_layer_bwd(const swimba_dims* dims, const void* X, const swi
                  (const int32_t*)(b + p.perm), (const int32_t*)(b + p.tiles), (const int32_t*)(b + p.ntiles),
                  (const int32_t*)(b + p.offsets), (float*)(b + q.z), (const float*)(b + q.dbpi),
                  (const float*)(b + q.dxs), (const float*)(b + q.dct), (float*)(b + q.dpi), (float*)(b + q.dg),
-                 (float*)(b + q.du), (float*)(b + q.dxp), dX, dW_router, dW_dt, db_dt, dW_exp};
+                 (float*)(b + q.du), (float*)(b + q.dxp), dX, dW_router, dW_dt, db_dt, dW_exp,
+                 b + p.xsorted, (int32_t*)(b + q.poff), (int32_t*)(b + q.prow), b + q.dzs, b + q.xsp, st};
   SW_CUDA(launch_layer_bwd_tail(d, t, s));
   prof_mark(s, "mix_router_linear_bwd");
   return SWIMBA_OK;

@@ -1,7 +1,8 @@
 """Gradients of the whole layer (swimba_layer_bwd) against the oracle's stage-by-stage reverse mode, through
 the C ABI.  The active set the GPU's router chose is replayed in the oracle on near-tied tokens (as in the
 forward tests); the upstream gradient dy is seeded.  Shapes: the tiny fp32 layer (CUDA-core forward), bf16
-tensor-core layers (N = 128) with G = H and G < H, k = 3 with a ragged tail, and an initial state."""
+tensor-core layers (N = 128) with G = H and G < H, k = 3 with a ragged tail, W_e not a multiple of 64, experts
+that receive no rows, and an initial state."""
 import numpy as np
 import pytest
 import torch
@@ -19,6 +20,12 @@ CASES = [
                        seed=142),
     configs.BASE.with_(name="lbwd_bf16_G1_k3_ragged", batch=1, seqlen=333, d_model=192, nheads=4, ngroups=1,
                        n_experts=6, top_k=3, chunk=128, seed=143),
+    # W_e = 3*16 + 2*3*32 = 240, not a multiple of the tensor-core products' 64-wide K blocks
+    configs.BASE.with_(name="lbwd_bf16_We240", batch=1, seqlen=300, d_model=128, nheads=3, headdim=16, dstate=32,
+                       n_experts=5, chunk=64, seed=144),
+    # 40 (token, slot) rows over 64 experts: most experts receive no rows and their weight gradient is 0
+    configs.BASE.with_(name="lbwd_bf16_empty_experts", batch=1, seqlen=40, d_model=64, nheads=2, headdim=16,
+                       dstate=16, n_experts=64, top_k=1, chunk=64, seed=145),
 ]
 NAMES = ("dX", "dW_r", "dW_dt", "db_dt", "dA", "dW_exp", "dinit")
 
@@ -56,6 +63,8 @@ def test_layer_gradients_match_oracle(w, with_init):
     swimba.layer_bwd(d, X, W, None if init is None else init.cuda(), dy.cuda(), out["dX"], out["dW_r"],
                      out["dW_dt"], out["db_dt"], out["dA"], out["dW_exp"], out["dinit"], ws)
     assert swimba.check_device_status() == 0
+    if w.name.endswith("empty_experts"):
+        assert len(np.unique(idx.cpu().numpy())) < w.n_experts
     Xf = f64(inp["X"])
     g = O.router_logits(Xf.reshape(w.M, -1), f64(inp["W_r"]))
     fl, forced = check_topk(idx.cpu().numpy(), g, w.top_k)
