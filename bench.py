@@ -16,7 +16,7 @@ method's cost statement says are flat in E, plus the separated-trajectory scan t
 (the base layer with the expert-mixed transition A~ = sum_j pi_j A_exp[K_j]), "groups" (the base layer
 with B and C shared by G in {H, H/4, 1} groups of heads: layer and scan times), "scan_bwd" (the scan
 gradients at the base sizes, bound by fp32 CUDA-core arithmetic) and "layer_bwd" (the whole layer's gradients
-at the base workload).
+at the base workload, tensor-core expert products plus CUDA-core scan gradients).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the launching stream,
 with a write of 2x the L2 size between steps (outside the events) so every step reads its inputs from
@@ -512,9 +512,12 @@ def scan_bwd_measure(args, dev, flush, stream, swimba):
 
 def layer_bwd_measure(args, sess, inp, flush, stream, swimba):
     """The layer gradients (swimba_layer_bwd) at the base workload with a seeded dy, timed alone: one call
-    recomputes the forward's router, dispatch and projections, then runs the scan gradients and the CUDA-core
-    mix, router and weight-gradient kernels.  The roofline counts the gradient arithmetic (scan gradients,
-    the two expert products dz W and dz^T X, the router and dt products) against the fp32 ALU peak."""
+    recomputes the forward's router, dispatch and projections, runs the scan gradients (CUDA cores), the mix and
+    router gradients, the two expert products dz W_e and dz^T X (tensor cores, on a bf16 hi/lo split of dz) and
+    the router and dt weight gradients.  The roofline is the sum of two floors: the tensor-core FLOPs (forward
+    recompute GEMM and router, the two expert products; algorithmic counts, the split's second MMA not counted)
+    at the bf16 burst peak plus the CUDA-core FLOPs (scan gradients, router and dt products) at the fp32 ALU
+    peak.  The expert products also get their own roofline from their stage time (pack of dz included)."""
     w = sess.w
     dev = sess.X.device
     g = torch.Generator().manual_seed(151)
@@ -538,22 +541,32 @@ def layer_bwd_measure(args, sess, inp, flush, stream, swimba):
         tot += e0.elapsed_time(e1)
     stages = {}
     swimba.profile_enable(True)
-    flush.fill_(1)
-    call()
-    for name, ms in swimba.profile_read():
-        stages[name] = stages.get(name, 0.0) + ms
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        call()
+        for name, ms in swimba.profile_read():
+            stages[name] = stages.get(name, 0.0) + ms / args.steps
     swimba.profile_enable(False)
     if swimba.check_device_status() != 0:
         raise RuntimeError("swimba_layer_bwd raised a device status")
     secs = tot / args.steps / 1e3
-    flops = (scan_bwd_flops(w) + 2 * 2.0 * w.M * w.top_k * w.W_e * w.d_model
-             + 2 * 2.0 * w.M * (w.n_experts + w.nheads) * w.d_model)
-    peak = 148 * 128 * 2 * 1965e6 / 1e12
-    return {"ms": secs * 1e3, "stages_ms": stages, "gradient_flops": flops,
-            "roofline": {"bound": "alu", "achieved": flops / secs / 1e12, "peak": peak, "unit": "TFLOP/s",
-                         "frac": flops / secs / 1e12 / peak,
-                         "peak_source": "148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz; the time includes the "
-                                        "forward recompute"}}
+    peaks, psrc = load_peaks()
+    gemm = 2.0 * w.M * w.top_k * w.W_e * w.d_model          # one expert product over all (token, slot) rows
+    small = 2.0 * w.M * (w.n_experts + w.nheads) * w.d_model  # one router + dt product over all tokens
+    t_flops = 3 * gemm + small                               # recompute GEMM and router, dz W_e, dz^T X
+    a_flops = scan_bwd_flops(w) + 2 * small                  # scan gradients, dg^T X / du^T X and their dX terms
+    tpk = peaks["bf16_tflops"]
+    apk = 148 * 128 * 2 * 1965e6 / 1e12
+    floor = t_flops / (tpk * 1e12) + a_flops / (apk * 1e12)
+    eg = stages.get("expert_grad", 0.0) / 1e3
+    res = {"ms": secs * 1e3, "stages_ms": stages, "tensor_flops": t_flops, "alu_flops": a_flops,
+           "roofline": {"bound": "tensor+alu", "floor_ms": floor * 1e3, "frac": floor / secs,
+                        "tensor_peak_tflops": tpk, "alu_peak_tflops": apk,
+                        "peak_source": f"bf16 burst ({psrc}); fp32 ALU = 148 SMs x 128 lanes x 2 FLOP x 1965 MHz"}}
+    if eg > 0:
+        res["expert_grad"] = {"ms": eg * 1e3, "flops": 2 * gemm, "achieved": 2 * gemm / eg / 1e12, "peak": tpk,
+                              "unit": "TFLOP/s", "frac": 2 * gemm / eg / 1e12 / tpk, "peak_source": psrc}
+    return res
 
 
 def out_proj_measure(args, sess, inp, flush, stream, swimba):

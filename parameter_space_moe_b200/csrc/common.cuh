@@ -154,16 +154,20 @@ struct LayerBwdPtrs {
   float* dpi; float* dg; float* du; float* dxp;
   float* dX; float* dW_r; float* dW_dt; float* db_dt; float* dW_exp;
   // bf16 layers: the tensor-core expert gradients' operands (gathered X rows, padded offsets, pair per
-  // padded row, dz split into bf16 hi/lo, padded X rows) and the device status word
-  const void* xsorted; int32_t* poff; int32_t* prow; void* dzs; void* xsp; unsigned* st;
+  // padded row and padded row per pair, dz split into bf16 hi/lo, padded X rows) and the device status word
+  const void* xsorted; int32_t* poff; int32_t* prow; int32_t* rp_of_p; void* dzs; void* xsp; unsigned* st;
 };
-cudaError_t launch_layer_bwd_tail(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s);
+// The layer gradients after the scan's, in three parts: 0 mix and router, 1 expert products, 2 the router
+// and dt weight gradients, db_dt and dX.
+cudaError_t launch_layer_bwd_tail(const Dims& d, const LayerBwdPtrs& q, int part, cudaStream_t s);
 // Rows of the padded sorted order (each expert's rows rounded up to 64) and W_e rounded up to 64.
 size_t grad_tc_rows(const Dims& d);
 int grad_tc_wp(const Dims& d);
-cudaError_t launch_grad_tc(const Dims& d, const float* dz, const void* xsorted, const void* w_exp,
-                           const int32_t* perm, const int32_t* offsets, int32_t* poff, int32_t* prow, void* dzs,
-                           void* xsp, float* dxp, float* dW_exp, unsigned* st, cudaStream_t s);
+cudaError_t launch_grad_tc_pack(const Dims& d, const void* xsorted, const int32_t* perm, const int32_t* offsets,
+                                int32_t* poff, int32_t* prow, int32_t* rp_of_p, void* dzs, void* xsp, cudaStream_t s);
+cudaError_t launch_grad_tc(const Dims& d, const void* w_exp, const int32_t* offsets, const int32_t* poff,
+                           const int32_t* prow, const void* dzs, const void* xsp, float* dxp, float* dW_exp,
+                           unsigned* st, cudaStream_t s);
 cudaError_t launch_mixed_a(const Dims& d, const int32_t* idx, const float* wts, const float* A_exp, const float* dt,
                            float* dA, float* ones, unsigned* st, cudaStream_t s);
 cudaError_t launch_out_proj(const Dims& d, const void* y, const void* w_out, void* out, unsigned* st,

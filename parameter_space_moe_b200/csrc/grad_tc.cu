@@ -11,8 +11,9 @@
 // bf16 MMAs into one fp32 TMEM accumulator, so the operand rounding stays near 2^-17 relative -- the same
 // accuracy class as fp32 CUDA-core arithmetic -- while X and W_e are exact in bf16.
 //
-// Operands (built by the pack kernel below, in "padded sorted" row order rp: expert e's sorted rows start
-// at poff[e], a multiple of 64, and its segment is padded with zero rows up to the next multiple of 64):
+// Operands, in "padded sorted" row order rp (expert e's sorted rows start at poff[e], a multiple of 64, and
+// its segment is padded with zero rows up to the next multiple of 64); the pack kernel below lays out the rows
+// and the mix gradient writes each pair's dz split into its padded row:
 //   dzs [Rp][2 Wp] bf16   row rp = [hi(dz) | 0 | lo(dz) | 0] of the pair there (Wp = W_e rounded up to 64)
 //   xsp [Rp][D]    bf16   X row of that pair's token, zero on pad rows
 //   prow[Rp]       int32  the pair index, -1 on pad rows
@@ -46,12 +47,11 @@ struct GArgs {
   unsigned* st;
 };
 
-// Where tile t reads and writes.  K block kb reads A at (ax0 + 64 kb', ay0) and B at (bx0, by0 + 64 kb')
-// for the MN-major operands / (bx0 + 64 kb', by0) for K-major ones, with kb' = kb mod half and the lo
-// part (kb >= half) shifted by (ax_lo, ay_lo).
+// Tile t: its expert, its K blocks (half of them on the hi part of dz, then as many on the lo part), and its
+// first output row (padded sorted row, or W_e column) and column.
 struct Tile {
   int e, nkb, half;
-  int m0, n0;  // first output row (padded sorted row, or W_e column) and column
+  int m0, n0;
 };
 
 __device__ __forceinline__ bool resolve(const GArgs& g, const int* poff_s, const int* tpre_s, int t, Tile& T) {
@@ -259,12 +259,13 @@ __global__ void pad_offsets_kernel(int E, const int32_t* __restrict__ offsets, i
   poff[E] = acc;
 }
 
-// One CTA per padded row rp: the row's pair (or none), dz split into bf16 hi and lo, and the token's X row.
+// One CTA per padded row rp: the row's pair (or -1), the pair's padded row (for the mix gradient, which writes
+// the pair's dz split there), and the token's X row; a pad row's dz split is zeroed here.
 template <class T>
 __global__ void __launch_bounds__(256)
-pack_kernel(int E, int We, int Wp, int D, int k, const int32_t* __restrict__ poff, const int32_t* __restrict__ offsets,
-            const int32_t* __restrict__ perm, const float* __restrict__ dz, const T* __restrict__ xsorted,
-            __nv_bfloat16* __restrict__ dzs, __nv_bfloat16* __restrict__ xsp, int32_t* __restrict__ prow) {
+pack_rows_kernel(int E, int Wp, int D, const int32_t* __restrict__ poff, const int32_t* __restrict__ offsets,
+                 const int32_t* __restrict__ perm, const T* __restrict__ xsorted, __nv_bfloat16* __restrict__ dzs,
+                 __nv_bfloat16* __restrict__ xsp, int32_t* __restrict__ prow, int32_t* __restrict__ rp_of_p) {
   __shared__ int s_r;
   const int rp = blockIdx.x;
   if (threadIdx.x == 0) {
@@ -276,25 +277,15 @@ pack_kernel(int E, int We, int Wp, int D, int k, const int32_t* __restrict__ pof
       if (rr < offsets[e + 1]) r = rr;
     }
     s_r = r;
-    prow[rp] = r >= 0 ? perm[r] : -1;
+    const int p = r >= 0 ? perm[r] : -1;
+    prow[rp] = p;
+    if (p >= 0) rp_of_p[p] = rp;
   }
   __syncthreads();
   const int r = s_r;
-  __nv_bfloat16* hi = dzs + (size_t)rp * 2 * Wp;
-  __nv_bfloat16* lo = hi + Wp;
-  const float* src = r >= 0 ? dz + (size_t)perm[r] * We : nullptr;
-  for (int c = 4 * threadIdx.x; c < Wp; c += 4 * blockDim.x) {
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (src && c < We) v = *reinterpret_cast<const float4*>(src + c);
-    const __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y), h1 = __floats2bfloat162_rn(v.z, v.w);
-    const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
-    const __nv_bfloat162 l0 = __floats2bfloat162_rn(v.x - f0.x, v.y - f0.y);
-    const __nv_bfloat162 l1 = __floats2bfloat162_rn(v.z - f1.x, v.w - f1.y);
-    uint2 uh, ul;
-    uh.x = *reinterpret_cast<const uint32_t*>(&h0); uh.y = *reinterpret_cast<const uint32_t*>(&h1);
-    ul.x = *reinterpret_cast<const uint32_t*>(&l0); ul.y = *reinterpret_cast<const uint32_t*>(&l1);
-    *reinterpret_cast<uint2*>(hi + c) = uh;
-    *reinterpret_cast<uint2*>(lo + c) = ul;
+  if (r < 0) {
+    uint2* z = reinterpret_cast<uint2*>(dzs + (size_t)rp * 2 * Wp);
+    for (int c = threadIdx.x; c < Wp / 2; c += blockDim.x) z[c] = make_uint2(0u, 0u);
   }
   const T* xr = r >= 0 ? xsorted + (size_t)r * D : nullptr;
   for (int c = 4 * threadIdx.x; c < D; c += 4 * blockDim.x) {
@@ -314,16 +305,26 @@ int sm_count() {
 size_t grad_tc_rows(const Dims& d) { return align_up((size_t)d.M * d.k + (size_t)64 * d.E, 128); }
 int grad_tc_wp(const Dims& d) { return ceil_div(d.We, BK) * BK; }
 
-// dXp (per pair) and dW_exp from the fp32 dz (pair-indexed [M*k][W_e]); bf16 layers only.
-cudaError_t launch_grad_tc(const Dims& d, const float* dz, const void* xsorted, const void* w_exp,
-                           const int32_t* perm, const int32_t* offsets, int32_t* poff, int32_t* prow, void* dzs,
-                           void* xsp, float* dxp, float* dW_exp, unsigned* st, cudaStream_t s) {
+// The operand layout of the expert products: padded offsets, pair per padded row and padded row per pair,
+// padded X rows, zeroed pad rows of the dz split (the mix gradient fills the others).  bf16 layers only.
+cudaError_t launch_grad_tc_pack(const Dims& d, const void* xsorted, const int32_t* perm, const int32_t* offsets,
+                                int32_t* poff, int32_t* prow, int32_t* rp_of_p, void* dzs, void* xsp, cudaStream_t s) {
   if (d.dtype != SWIMBA_BF16 || d.E > kMaxE) return cudaErrorInvalidValue;
   const int Rp = (int)grad_tc_rows(d), Wp = grad_tc_wp(d);
   pad_offsets_kernel<<<1, 32, 0, s>>>(d.E, offsets, poff);
-  pack_kernel<__nv_bfloat16><<<Rp, 256, 0, s>>>(d.E, d.We, Wp, d.D, d.k, poff, offsets, perm, dz,
-                                                 (const __nv_bfloat16*)xsorted, (__nv_bfloat16*)dzs,
-                                                 (__nv_bfloat16*)xsp, prow);
+  pack_rows_kernel<__nv_bfloat16><<<Rp, 256, 0, s>>>(d.E, Wp, d.D, poff, offsets, perm,
+                                                      (const __nv_bfloat16*)xsorted, (__nv_bfloat16*)dzs,
+                                                      (__nv_bfloat16*)xsp, prow, rp_of_p);
+  count_launches(2);
+  return cudaGetLastError();
+}
+
+// dXp (per pair) and dW_exp from the packed operands.
+cudaError_t launch_grad_tc(const Dims& d, const void* w_exp, const int32_t* offsets, const int32_t* poff,
+                           const int32_t* prow, const void* dzs, const void* xsp, float* dxp, float* dW_exp,
+                           unsigned* st, cudaStream_t s) {
+  if (d.dtype != SWIMBA_BF16 || d.E > kMaxE) return cudaErrorInvalidValue;
+  const int Rp = (int)grad_tc_rows(d), Wp = grad_tc_wp(d);
   CUtensorMap ta_dx, ta_dw, tb_dx, tb_dw;
   if (!encode_tmap_2d(&ta_dx, dzs, SWIMBA_BF16, (uint64_t)2 * Wp, (uint64_t)Rp, (uint64_t)2 * Wp * 2, BK, BM) ||
       !encode_tmap_2d(&ta_dw, dzs, SWIMBA_BF16, (uint64_t)2 * Wp, (uint64_t)Rp, (uint64_t)2 * Wp * 2, 64, BK) ||
@@ -340,7 +341,7 @@ cudaError_t launch_grad_tc(const Dims& d, const float* dz, const void* xsorted, 
   g.out = dW_exp;
   const int dw_tiles = d.E * ceil_div(d.We, BM) * ceil_div(d.D, BN);
   grad_tc_kernel<<<dw_tiles < sms ? dw_tiles : sms, kThreads, kSmemBytes, s>>>(ta_dw, tb_dw, g);
-  count_launches(4);
+  count_launches(2);
   return cudaGetLastError();
 }
 

@@ -21,10 +21,15 @@ namespace {
 constexpr int kT = 64;   // output tile edge of the CUDA-core GEMMs
 constexpr int kK = 16;   // contraction step
 
-// mix: one CTA per (token, slot) pair p; z (raw projection, fp32) is overwritten by dz
+// mix: one CTA per (token, slot) pair p.  fp32 layers: z (raw projection) is overwritten by dz.  bf16 layers
+// (kSplit): dz goes straight into the pair's padded row of the tensor-core products' operand as a bf16 split,
+// hi = bf16(dz) in columns [0, W_e), lo = bf16(dz - hi) in [Wp, Wp + W_e), zeros up to each half's end.
+template <bool kSplit>
 __global__ void __launch_bounds__(256) mix_bwd_kernel(Dims d, float* __restrict__ z, const float* __restrict__ wts,
                                                       const float* __restrict__ dbpi, const float* __restrict__ dxs,
-                                                      const float* __restrict__ dct, float* __restrict__ dpi) {
+                                                      const float* __restrict__ dct, float* __restrict__ dpi,
+                                                      const int32_t* __restrict__ rp_of_p,
+                                                      __nv_bfloat16* __restrict__ dzs, int Wp) {
   __shared__ float red[8];
   const size_t p = blockIdx.x;
   const size_t m = p / d.k;
@@ -44,10 +49,27 @@ __global__ void __launch_bounds__(256) mix_bwd_kernel(Dims d, float* __restrict_
     dpi[p] = v;
   }
   const float* gx = dxs + p * d.HP;
-  for (int c = threadIdx.x; c < d.HP; c += blockDim.x) zr[c] = gx[c];
-  for (int c = threadIdx.x; c < d.GN; c += blockDim.x) {
-    zr[d.HP + c] = pi * gb[c];
-    zr[d.HP + d.GN + c] = pi * gc[c];
+  if constexpr (kSplit) {
+    // pairs of columns (H*P and G*N are even, so a pair never straddles two streams)
+    __nv_bfloat162* hi = reinterpret_cast<__nv_bfloat162*>(dzs + (size_t)rp_of_p[p] * 2 * Wp);
+    __nv_bfloat162* lo = hi + Wp / 2;
+    for (int c2 = threadIdx.x; c2 < Wp / 2; c2 += blockDim.x) {
+      const int c = 2 * c2;
+      float2 v = make_float2(0.f, 0.f);
+      if (c < d.HP) v = make_float2(gx[c], gx[c + 1]);
+      else if (c < d.HP + d.GN) v = make_float2(pi * gb[c - d.HP], pi * gb[c - d.HP + 1]);
+      else if (c < d.We) v = make_float2(pi * gc[c - d.HP - d.GN], pi * gc[c - d.HP - d.GN + 1]);
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+      const float2 hf = __bfloat1622float2(h);
+      hi[c2] = h;
+      lo[c2] = __floats2bfloat162_rn(v.x - hf.x, v.y - hf.y);
+    }
+  } else {
+    for (int c = threadIdx.x; c < d.HP; c += blockDim.x) zr[c] = gx[c];
+    for (int c = threadIdx.x; c < d.GN; c += blockDim.x) {
+      zr[d.HP + c] = pi * gb[c];
+      zr[d.HP + d.GN + c] = pi * gc[c];
+    }
   }
 }
 
@@ -278,24 +300,42 @@ __global__ void db_kernel(Dims d, const float* __restrict__ du, float* __restric
   }
 }
 
-template <class T>
-cudaError_t launch_tail_typed(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s) {
-  mix_bwd_kernel<<<d.M * d.k, 256, 0, s>>>(d, q.z, q.wts, q.dbpi, q.dxs, q.dct, q.dpi);
-  router_bwd_kernel<<<ceil_div(d.M, 128), 128, 0, s>>>(d, q.idx, q.wts, q.dpi, q.dt, q.ddt, q.dg, q.du);
-  cudaError_t e;
-  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-    // tensor cores on the bf16 hi/lo split of dz
-    e = launch_grad_tc(d, q.z, q.xsorted, q.w_exp, q.perm, q.offsets, q.poff, q.prow, q.dzs, q.xsp, q.dxp, q.dW_exp,
-                       q.st, s);
+// 1. the mix and router gradients: dz (over z, or as the bf16 split of the tensor-core products), dpi, dg, du
+cudaError_t launch_mix_router(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s) {
+  if (d.dtype == SWIMBA_BF16) {
+    const cudaError_t e = launch_grad_tc_pack(d, q.xsorted, q.perm, q.offsets, q.poff, q.prow, q.rp_of_p, q.dzs,
+                                              q.xsp, s);
     if (e != cudaSuccess) return e;
+    mix_bwd_kernel<true><<<d.M * d.k, 256, 0, s>>>(d, q.z, q.wts, q.dbpi, q.dxs, q.dct, q.dpi, q.rp_of_p,
+                                                   (__nv_bfloat16*)q.dzs, grad_tc_wp(d));
+  } else {
+    mix_bwd_kernel<false><<<d.M * d.k, 256, 0, s>>>(d, q.z, q.wts, q.dbpi, q.dxs, q.dct, q.dpi, nullptr, nullptr, 0);
+  }
+  router_bwd_kernel<<<ceil_div(d.M, 128), 128, 0, s>>>(d, q.idx, q.wts, q.dpi, q.dt, q.ddt, q.dg, q.du);
+  count_launches(2);
+  return cudaGetLastError();
+}
+
+// 2. the expert products dXp = dz W_e and dW_exp = dz^T X
+template <class T>
+cudaError_t launch_experts_typed(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    // tensor cores on the bf16 hi/lo split of dz (laid out by the mix gradient)
+    return launch_grad_tc(d, q.w_exp, q.offsets, q.poff, q.prow, q.dzs, q.xsp, q.dxp, q.dW_exp, q.st, s);
   } else {
     const dim3 gx(max_row_tiles(d), ceil_div(d.D, kBT2));
     dx_experts_kernel<T><<<gx, 256, 0, s>>>(d, q.z, (const T*)q.w_exp, q.perm, q.tiles, q.ntiles, q.offsets, q.dxp);
     const dim3 gw(d.E, ceil_div(d.We, kBT2), ceil_div(d.D, kBT2));
     dw_experts_kernel<T><<<gw, 256, 0, s>>>(d, q.z, (const T*)q.X, q.perm, q.offsets, q.dW_exp);
     count_launches(2);
+    return cudaGetLastError();
   }
-  e = cudaMemsetAsync(q.dW_r, 0, (size_t)d.E * d.D * 4, s);
+}
+
+// 3. the router and dt weight gradients, db_dt, and dX summed over the slots with the router and dt terms
+template <class T>
+cudaError_t launch_linear_typed(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(q.dW_r, 0, (size_t)d.E * d.D * 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(q.dW_dt, 0, (size_t)d.H * d.D * 4, s);
   if (e != cudaSuccess) return e;
   dw_dense_kernel<T><<<dim3(ceil_div(d.D, kT), ceil_div(d.M, 256), ceil_div(d.E, kT)), 256, 0, s>>>(
@@ -304,13 +344,19 @@ cudaError_t launch_tail_typed(const Dims& d, const LayerBwdPtrs& q, cudaStream_t
       d.M, d.H, d.D, q.du, (const T*)q.X, q.dW_dt);
   db_kernel<<<d.H, 256, 0, s>>>(d, q.du, q.db_dt);
   dx_final_kernel<T><<<148 * 8, 256, 0, s>>>(d, q.dxp, q.dg, q.du, (const T*)q.w_r, (const T*)q.w_dt, q.dX);
-  count_launches(6);
+  count_launches(4);
   return cudaGetLastError();
 }
 }  // namespace
 
-cudaError_t launch_layer_bwd_tail(const Dims& d, const LayerBwdPtrs& q, cudaStream_t s) {
-  return d.dtype == SWIMBA_BF16 ? launch_tail_typed<__nv_bfloat16>(d, q, s) : launch_tail_typed<float>(d, q, s);
+cudaError_t launch_layer_bwd_tail(const Dims& d, const LayerBwdPtrs& q, int part, cudaStream_t s) {
+  const bool bf = d.dtype == SWIMBA_BF16;
+  switch (part) {
+    case 0: return launch_mix_router(d, q, s);
+    case 1: return bf ? launch_experts_typed<__nv_bfloat16>(d, q, s) : launch_experts_typed<float>(d, q, s);
+    case 2: return bf ? launch_linear_typed<__nv_bfloat16>(d, q, s) : launch_linear_typed<float>(d, q, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace swimba

@@ -548,7 +548,7 @@ swimba_status swimba_out_proj(const swimba_dims* dims, const void* y, const void
 
 // Workspace of swimba_layer_bwd: the layer's own, then the gradient buffers (all fp32).
 struct BwdPlan {
-  size_t z, dbpi, dxs, dct, ddt, dpi, dg, du, dxp, poff, prow, dzs, xsp, total;
+  size_t z, dbpi, dxs, dct, ddt, dpi, dg, du, dxp, poff, prow, rp_of_p, dzs, xsp, total;
 };
 static BwdPlan plan_bwd(const Dims& d) {
   BwdPlan q{};
@@ -568,6 +568,7 @@ static BwdPlan plan_bwd(const Dims& d) {
     const size_t Rp = grad_tc_rows(d), Wp = (size_t)grad_tc_wp(d);
     q.poff = take((size_t)(d.E + 1) * 4);
     q.prow = take(Rp * 4);
+    q.rp_of_p = take(Mk * 4);
     q.dzs = take(Rp * 2 * Wp * 2);
     q.xsp = take(Rp * d.D * 2);
   }
@@ -617,9 +618,14 @@ swimba_status swimba_layer_bwd(const swimba_dims* dims, const void* X, const swi
                  (const int32_t*)(b + p.offsets), (float*)(b + q.z), (const float*)(b + q.dbpi),
                  (const float*)(b + q.dxs), (const float*)(b + q.dct), (float*)(b + q.dpi), (float*)(b + q.dg),
                  (float*)(b + q.du), (float*)(b + q.dxp), dX, dW_router, dW_dt, db_dt, dW_exp,
-                 b + p.xsorted, (int32_t*)(b + q.poff), (int32_t*)(b + q.prow), b + q.dzs, b + q.xsp, st};
-  SW_CUDA(launch_layer_bwd_tail(d, t, s));
-  prof_mark(s, "mix_router_linear_bwd");
+                 b + p.xsorted, (int32_t*)(b + q.poff), (int32_t*)(b + q.prow), (int32_t*)(b + q.rp_of_p),
+                 b + q.dzs, b + q.xsp, st};
+  SW_CUDA(launch_layer_bwd_tail(d, t, 0, s));
+  prof_mark(s, "mix_router_bwd");
+  SW_CUDA(launch_layer_bwd_tail(d, t, 1, s));
+  prof_mark(s, "expert_grad");
+  SW_CUDA(launch_layer_bwd_tail(d, t, 2, s));
+  prof_mark(s, "linear_bwd");
   return SWIMBA_OK;
 }
 
