@@ -618,6 +618,28 @@ def groups_measure(args, dev, flush, stream, swimba, base_out):
     return res
 
 
+def run_measure(args):
+    """One nested measurement alone (layer gradients, scan gradients or output projection) on the base workload,
+    one GPU: the same timing as inside the default line, printed as its own JSON object."""
+    from parameter_space_moe_b200 import swimba
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    swimba.lib()
+    w = configs.BASE
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    if args.measure == "scan_bwd":
+        res = scan_bwd_measure(args, dev, flush, stream, swimba)
+    else:
+        inp = inputs.make_inputs(w)
+        sess = LayerSession(w, dev, inp, swimba)
+        fn = layer_bwd_measure if args.measure == "layer_bwd" else out_proj_measure
+        res = fn(args, sess, inp, flush, stream, swimba)
+    print(json.dumps({"measure": args.measure, "workload": w.name, "steps": args.steps, "warmup": args.warmup,
+                      **res}))
+
+
 def run_gpu(args, w):
     from parameter_space_moe_b200 import swimba
     rank, world, local = rank_env()
@@ -758,11 +780,15 @@ def main():
                     help="also time the separated-trajectory scan (k scans) on the layer's streams")
     ap.add_argument("--no-extras", action="store_true",
                     help="default workload on one GPU: skip the nested decode and expert-count sweep measurements")
+    ap.add_argument("--measure", choices=["layer_bwd", "scan_bwd", "out_proj"],
+                    help="one GPU, base workload: run only this nested measurement and print its JSON")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = configs.ALL[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
+    elif args.measure:
+        run_measure(args)
     else:
         run_gpu(args, w)
 

@@ -37,9 +37,22 @@ def _tol(w, name):
     return 1e-5 if w.dtype == "f32" else 2e-3
 
 
+# the base layer's widths (D 768, H24 P64 N128, W_e 7680, E8 k2) over 512 tokens: the tensor-core expert
+# products at their full K and N extents (the oracle needs about 25 s; the full base workload takes minutes)
+BASE_WIDTH = configs.BASE.with_(name="lbwd_bf16_base_width", batch=1, seqlen=512, seed=146)
+
+
 @pytest.mark.parametrize("with_init", [False, True], ids=["zero_init", "init"])
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
 def test_layer_gradients_match_oracle(w, with_init):
+    _check(w, with_init)
+
+
+def test_layer_gradients_base_width():
+    _check(BASE_WIDTH, False)
+
+
+def _check(w, with_init):
     inp = inputs.make_inputs(w)
     d = swimba.dims_of(w)
     W = device_weights(inp)
