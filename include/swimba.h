@@ -215,7 +215,8 @@ swimba_status swimba_separated_scan(const swimba_dims* dims, const void* B, cons
                                     float* final_states, void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of workspace swimba_layer_bwd needs for these dims (0 if invalid or unsupported): the layer's own
- * workspace followed by fp32 gradient buffers (about M*k*(2*W_e + G*N + H*P + D)*4 bytes more). */
+ * workspace followed by fp32 gradient buffers (about M*k*(W_e + G*N + H*P + D)*4 bytes more) and, for bf16
+ * layers, the tensor-core products' operands (about (M*k + 64*E)*(2*W_e + D)*2 bytes). */
 size_t swimba_layer_bwd_workspace_size(const swimba_dims* dims);
 
 /* Gradients of the whole layer (swimba_layer_fwd with the shared A) for L = sum_t <dy_t, y_t>: the
@@ -227,9 +228,12 @@ size_t swimba_layer_bwd_workspace_size(const swimba_dims* dims);
  *   init_state [B][H][N][P] fp32 or NULL; dy [M][H][P] fp32
  *   dX [M][D], dW_router [E][D], dW_dt [H][D], db_dt [H], dA [H], dW_exp [E][W_e][D] fp32 out;
  *   d_init [B][H][N][P] fp32 out or NULL
- * Runs the forward's router, dispatch and projections again, the scan gradients, then CUDA-core fp32
- * kernels for the mix, router and dt gradients and the weight and input products.  ws must hold
- * swimba_layer_bwd_workspace_size(dims) bytes (SWIMBA_ERR_WORKSPACE otherwise). */
+ * Runs the forward's router, dispatch and projections again, the scan gradients, then fp32 kernels for the
+ * mix, router and dt gradients.  The expert products dz W_e and dz^T X run on the tensor cores for bf16
+ * layers (dz split into bf16 hi + lo, two MMAs into one fp32 accumulator: fp32-class accuracy) and on CUDA
+ * cores in fp32 for fp32 layers; the router and dt products on CUDA cores.  ws must hold
+ * swimba_layer_bwd_workspace_size(dims) bytes (SWIMBA_ERR_WORKSPACE otherwise); a device status of
+ * SWIMBA_ERR_TIMEOUT means a bounded wait of the tensor-core kernel gave up (outputs invalid). */
 swimba_status swimba_layer_bwd(const swimba_dims* dims, const void* X, const swimba_weights* w,
                                const float* init_state, const float* dy, float* dX, float* dW_router, float* dW_dt,
                                float* db_dt, float* dA, float* dW_exp, float* d_init, void* ws, size_t ws_bytes,
