@@ -134,8 +134,9 @@ __device__ __forceinline__ void load_rows_sum(const S* src, size_t m0, int k, in
   }
 }
 
-// 1. sub-chunk end states S_c (keys of every slot) and cs at the last token
-template <class S>
+// 1. sub-chunk end states S_c (keys of every slot) and cs at the last token.  PJ = P / 16 column groups per
+// thread (a compile-time count, so no FMA runs on a padding column).
+template <class S, int PJ>
 __global__ void __launch_bounds__(kBT) bwd_fwd_chunk_kernel(BwdArgs a) {
   extern __shared__ float sm[];
   const Dims& d = a.d;
@@ -149,12 +150,12 @@ __global__ void __launch_bounds__(kBT) bwd_fwd_chunk_kernel(BwdArgs a) {
   const size_t m0 = (size_t)b * d.T + t0;
   const int NP = d.N * d.P;
   // thread (ty, tx) of a 16 x 16 grid holds S_c[n][p] for n = ty + 16 i, p = tx + 16 jj
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4, ni = d.N / 16, nj = d.P / 16;
-  float acc[8][8];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4, ni = d.N / 16;
+  float acc[8][PJ];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
+    for (int jj = 0; jj < PJ; ++jj) acc[i][jj] = 0.f;
   for (int j = 0; j < d.k; ++j) {
     load_rows<S>((const S*)a.bpi, m0, d.k, j, d.N, d.GN, (size_t)g * d.N, L, Bs, d.N);
     load_rows<S>((const S*)a.xs, m0, d.k, j, d.P, d.HP, (size_t)h * d.P, L, Xv, d.P);
@@ -164,15 +165,15 @@ __global__ void __launch_bounds__(kBT) bwd_fwd_chunk_kernel(BwdArgs a) {
       if (i < L) Xv[x] *= expf(cs[L - 1] - cs[i]);
     }
     __syncthreads();
-    tile_mac<8, 8>(acc, nj, L, Bs, d.N, 1, Xv, d.P, 1, ty, tx, ni);
+    tile_mac<PJ, 8>(acc, PJ, L, Bs, d.N, 1, Xv, d.P, 1, ty, tx, ni);
     __syncthreads();
   }
   const size_t base = (((size_t)b * d.H + h) * a.nc + c) * NP;
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj)
-      if (i < ni && jj < nj) a.work[base + (size_t)(ty + 16 * i) * d.P + tx + 16 * jj] = acc[i][jj];
+    for (int jj = 0; jj < PJ; ++jj)
+      if (i < ni) a.work[base + (size_t)(ty + 16 * i) * d.P + tx + 16 * jj] = acc[i][jj];
   if (threadIdx.x == 0) a.cse[((size_t)b * d.H + h) * a.nc + c] = cs[L - 1];
 }
 
@@ -193,7 +194,7 @@ __global__ void bwd_fwd_pass_kernel(BwdArgs a) {
 }
 
 // 3. D_c = sum_t e^{cs_t} C~_t (x) dy_t  (overwrites S_c)
-template <class S>
+template <class S, int PJ>
 __global__ void __launch_bounds__(kBT) bwd_d_kernel(BwdArgs a) {
   extern __shared__ float sm[];
   const Dims& d = a.d;
@@ -214,18 +215,18 @@ __global__ void __launch_bounds__(kBT) bwd_d_kernel(BwdArgs a) {
   __syncthreads();
   const int NP = d.N * d.P;
   const size_t base = (((size_t)b * d.H + h) * a.nc + c) * NP;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4, ni = d.N / 16, nj = d.P / 16;
-  float acc[8][8];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4, ni = d.N / 16;
+  float acc[8][PJ];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
-  tile_mac<8, 8>(acc, nj, L, Cs, d.N, 1, Dy, d.P, 1, ty, tx, ni);
+    for (int jj = 0; jj < PJ; ++jj) acc[i][jj] = 0.f;
+  tile_mac<PJ, 8>(acc, PJ, L, Cs, d.N, 1, Dy, d.P, 1, ty, tx, ni);
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj)
-      if (i < ni && jj < nj) a.work[base + (size_t)(ty + 16 * i) * d.P + tx + 16 * jj] = acc[i][jj];
+    for (int jj = 0; jj < PJ; ++jj)
+      if (i < ni) a.work[base + (size_t)(ty + 16 * i) * d.P + tx + 16 * jj] = acc[i][jj];
 }
 
 // 4. Lam_{c+1} for every sub-chunk (into work, replacing D_c), and d init = Lam_0
@@ -272,8 +273,8 @@ struct GradSmem {
   }
 };
 
-// 5. the per-sub-chunk gradients
-template <class S>
+// 5. the per-sub-chunk gradients (PJ = P / 16 column groups of the dXs tile, compile-time)
+template <class S, int PJ>
 __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
   extern __shared__ float sm[];
   const Dims& d = a.d;
@@ -320,7 +321,7 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
   // carried-state terms: dC~_t = e^{cs_t} H_c dy_t, kept per thread over the slots as a 4 x N/16 tile of
   // (t = ty + 16 i, n = tx + 16 jj); q_t = C~_t . that (the 16 lanes of a half-warp share t)
   const int tx = tid & 15, ty = tid >> 4;
-  const int nN = N / 16, nP = P / 16;
+  const int nN = N / 16;
   float dC[4][8];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
@@ -407,26 +408,28 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
       }
     }
     __syncthreads();
-    float acc[4][8];
     // dXs_s = e^{cs_end - cs_s} Lam^T B_s + sum_t K1[t][s] dy_t   (tile of s = ty + 16 i, p = tx + 16 jj)
+    {
+      float ax[4][PJ];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
-    tile_mac<8>(acc, nP, N, Bs, 1, ldN, Lam, ldP, 1, ty, tx);
+        for (int jj = 0; jj < PJ; ++jj) ax[i][jj] = 0.f;
+      tile_mac<PJ>(ax, PJ, N, Bs, 1, ldN, Lam, ldP, 1, ty, tx);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) acc[i][jj] *= eend[ty + 16 * i];
-    tile_mac<8>(acc, nP, L, S1, BL, 1, Dy, ldP, 1, ty, tx);
+        for (int jj = 0; jj < PJ; ++jj) ax[i][jj] *= eend[ty + 16 * i];
+      tile_mac<PJ>(ax, PJ, L, S1, BL, 1, Dy, ldP, 1, ty, tx);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int s = ty + 16 * i;
-      if (s >= L) continue;
+      for (int i = 0; i < 4; ++i) {
+        const int s = ty + 16 * i;
+        if (s >= L) continue;
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj)
-        if (jj < nP) a.dxs[((m0 + s) * d.k + j) * d.HP + (size_t)h * P + tx + 16 * jj] = acc[i][jj];
+        for (int jj = 0; jj < PJ; ++jj) a.dxs[((m0 + s) * d.k + j) * d.HP + (size_t)h * P + tx + 16 * jj] = ax[i][jj];
+      }
     }
+    float acc[4][8];
     // dBpi_s = e^{cs_end - cs_s} Lam x_s + sum_t K2[t][s] C~_t   (tile of s, n = tx + 16 jj); bv_s += B_s . Lam x_s
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -498,26 +501,38 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
   }
 }
 
-template <class S>
+template <class S, int PJ>
 cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s) {
   const Dims& d = a.d;
   const dim3 grid(a.nc, d.H, d.Bsz);
   const size_t sm1 = (BL + (size_t)BL * d.N + (size_t)BL * d.P) * 4;
-  cudaError_t e = set_max_dynamic_smem((const void*)bwd_fwd_chunk_kernel<S>, sm1);
+  cudaError_t e = set_max_dynamic_smem((const void*)bwd_fwd_chunk_kernel<S, PJ>, sm1);
   if (e != cudaSuccess) return e;
-  bwd_fwd_chunk_kernel<S><<<grid, kBT, sm1, s>>>(a);
+  bwd_fwd_chunk_kernel<S, PJ><<<grid, kBT, sm1, s>>>(a);
   const dim3 pgrid(ceil_div(d.N * d.P, kBT), d.H, d.Bsz);
   bwd_fwd_pass_kernel<<<pgrid, kBT, 0, s>>>(a);
-  e = set_max_dynamic_smem((const void*)bwd_d_kernel<S>, sm1);
+  e = set_max_dynamic_smem((const void*)bwd_d_kernel<S, PJ>, sm1);
   if (e != cudaSuccess) return e;
-  bwd_d_kernel<S><<<grid, kBT, sm1, s>>>(a);
+  bwd_d_kernel<S, PJ><<<grid, kBT, sm1, s>>>(a);
   bwd_adj_pass_kernel<<<pgrid, kBT, 0, s>>>(a);
   const size_t sm5 = GradSmem(d.N, d.P).total * 4;
-  e = set_max_dynamic_smem((const void*)bwd_grad_kernel<S>, sm5);
+  e = set_max_dynamic_smem((const void*)bwd_grad_kernel<S, PJ>, sm5);
   if (e != cudaSuccess) return e;
-  bwd_grad_kernel<S><<<grid, kBT, sm5, s>>>(a);
+  bwd_grad_kernel<S, PJ><<<grid, kBT, sm5, s>>>(a);
   count_launches(5);
   return cudaGetLastError();
+}
+
+// P in {16, 32, 64, 128}: the column-group count of the register tiles as a template argument
+template <class S>
+cudaError_t launch_bwd_p(const BwdArgs& a, cudaStream_t s) {
+  switch (a.d.P) {
+    case 16: return launch_bwd_typed<S, 1>(a, s);
+    case 32: return launch_bwd_typed<S, 2>(a, s);
+    case 64: return launch_bwd_typed<S, 4>(a, s);
+    case 128: return launch_bwd_typed<S, 8>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 }  // namespace
 
@@ -538,7 +553,7 @@ cudaError_t launch_scan_bwd(const Dims& d, const void* bpi, const void* xs, cons
   if (e == cudaSuccess && d.hpg > 1) e = cudaMemsetAsync(dbpi, 0, (size_t)d.M * d.k * d.GN * 4, s);
   if (e == cudaSuccess && d.hpg > 1) e = cudaMemsetAsync(dct, 0, (size_t)d.M * d.GN * 4, s);
   if (e != cudaSuccess) return e;
-  return d.dtype == SWIMBA_BF16 ? launch_bwd_typed<__half>(a, s) : launch_bwd_typed<float>(a, s);
+  return d.dtype == SWIMBA_BF16 ? launch_bwd_p<__half>(a, s) : launch_bwd_p<float>(a, s);
 }
 
 }  // namespace swimba
