@@ -42,7 +42,8 @@ struct TcArgs {
   const int32_t* tiles;
   const int32_t* ntiles;
   const int32_t* offsets;
-  int mode;  // 0 mix, 1 mix with unscaled B, 2 raw fp32 Z, 3 plain bf16 product (the output projection)
+  int mode;  // 0 mix, 1 mix with unscaled B, 2 raw fp32 Z, 3 plain bf16 product (the output projection),
+             // 4 mix plus the raw fp32 B and C columns of Z (the layer gradients' forward recompute)
   int dense;  // 1: one operand group over rows 0 .. M-1 in order (no dispatch schedule, offsets or row metadata)
   __half* bpi;
   __half* xs;
@@ -105,6 +106,22 @@ __device__ __forceinline__ void store_chunk(const TcArgs& a, int p, float pi, in
     else { o = pi * v; dst = a.cpi + (size_t)p * GN + (c - HP - GN); }
     range_bad |= !(fabsf(o) <= kF16Max);
     *dst = __float2half_rn(o);
+  }
+}
+
+// Mode 4: the raw B and C columns (W_e columns from H*P on) of one row's 32-column group, fp32 into row p of
+// Z [M*k][W_e]; the x columns are not stored (the mix's gradient does not read them).
+__device__ __forceinline__ void store_raw_bc(const TcArgs& a, int p, int c0, const uint32_t (&r)[32]) {
+  const Dims& d = a.d;
+  float* dst = a.Z + (size_t)p * d.We + c0;
+  if (c0 >= d.HP && c0 + 32 <= d.We) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 4)
+      *reinterpret_cast<float4*>(dst + i) = make_float4(u2f(r[i]), u2f(r[i + 1]), u2f(r[i + 2]), u2f(r[i + 3]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)  // constant indices keep r in registers
+      if (c0 + i >= d.HP && c0 + i < d.We) dst[i] = u2f(r[i]);
   }
 }
 
@@ -188,6 +205,8 @@ __device__ __forceinline__ void store_dense32(const TcArgs& a, uint8_t* stage, i
 
 // One epilogue warp drains its 32 accumulator rows x nch 32-column chunks (starting at output column col0)
 // of a tile: the TMEM load of the next chunk is in flight while the current one is converted and stored.
+// kRaw: mode 4, whose raw B/C stores are compiled only into the kernels that run it.
+template <bool kRaw>
 __device__ __forceinline__ void drain_tile(const TcArgs& a, uint32_t taddr, int col0, int nch, bool valid, int2 meta,
                                            uint8_t* stage, int lane, bool& range_bad) {
   const Dims& d = a.d;
@@ -206,6 +225,7 @@ __device__ __forceinline__ void drain_tile(const TcArgs& a, uint32_t taddr, int 
       store_dense32(a, stage, lane, valid, meta.x, c0, cur);
       continue;
     }
+    if (kRaw && valid && c0 + 32 > d.HP && c0 < d.We) store_raw_bc(a, meta.x, c0, cur);
     float sc_probe;
     // fast path: the warp's 32-column group lies in one fp16 stream for every valid row
     const bool fast = a.mode != 2 && c0 + 32 <= d.We &&
@@ -215,6 +235,7 @@ __device__ __forceinline__ void drain_tile(const TcArgs& a, uint32_t taddr, int 
   }
 }
 
+template <bool kRaw>
 __global__ void __launch_bounds__(kThreads, 1)
 proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -345,7 +366,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
       }
       tc::fence_after_sync();
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 32 * ch0);
-      drain_tile(a, taddr, ct * BN + 32 * ch0, nch, valid, meta, epi_stage, lane, range_bad);
+      drain_tile<kRaw>(a, taddr, ct * BN + 32 * ch0, nch, valid, meta, epi_stage, lane, range_bad);
       tc::fence_before_sync();
       tc::mbar_arrive(&acc_empty[buf]);
       if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
@@ -384,6 +405,7 @@ __device__ __forceinline__ int2 pair_tile(const int* off_s, const int* pt_s, int
   return make_int2(e, off_s[e] + (rt - pt_s[e]) * kPairRows);
 }
 
+template <bool kRaw>
 __global__ void __launch_bounds__(kThreads, 1)
 proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -524,7 +546,7 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
       }
       tc::fence_after_sync();
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 32 * ch0);
-      drain_tile(a, taddr, ct * BN + 32 * ch0, nch, valid, meta, epi_stage, lane, range_bad);
+      drain_tile<kRaw>(a, taddr, ct * BN + 32 * ch0, nch, valid, meta, epi_stage, lane, range_bad);
       // the accumulator's TMEM reads are complete (tcgen05.wait::ld) and ordered by the tcgen05 fence; the
       // tile's global stores need not be visible to the even CTA, so the arrival is relaxed
       tc::fence_before_sync();
@@ -546,9 +568,10 @@ proj_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
 
 // Host side --------------------------------------------------------------------------------------
 // The CTA-pair kernel, persistent: as many pairs as can be resident at once, at most one per pair tile.
+template <bool kRaw>
 static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb2, const TcArgs& a, int max_pairs, int sms,
                                cudaStream_t s) {
-  cudaError_t e = set_max_dynamic_smem((const void*)proj_tc_pair_kernel, kPairSmemBytes);
+  cudaError_t e = set_max_dynamic_smem((const void*)proj_tc_pair_kernel<kRaw>, kPairSmemBytes);
   if (e != cudaSuccess) return e;
   static int resident = 0;
   if (resident == 0) {
@@ -565,16 +588,17 @@ static cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb2, co
     cfg.numAttrs = 1;
     cfg.gridDim = dim3((unsigned)sms);
     int n = 0;
-    resident = cudaOccupancyMaxActiveClusters(&n, proj_tc_pair_kernel, &cfg) == cudaSuccess && n > 0 ? n : sms / 2;
+    resident = cudaOccupancyMaxActiveClusters(&n, proj_tc_pair_kernel<kRaw>, &cfg) == cudaSuccess && n > 0 ? n : sms / 2;
   }
   const int pairs = resident < max_pairs ? resident : max_pairs;
-  return launch_dependent(proj_tc_pair_kernel, dim3((unsigned)(2 * pairs)), dim3(kThreads), kPairSmemBytes, s, 2, ta,
+  return launch_dependent(proj_tc_pair_kernel<kRaw>, dim3((unsigned)(2 * pairs)), dim3(kThreads), kPairSmemBytes, s, 2, ta,
                           tb2, a);
 }
 
-cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int2* rowmeta,
-                           const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, int mode, void* bpi,
-                           void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s) {
+template <bool kRaw>
+static cudaError_t launch_proj_tc_t(const Dims& d, const void* xsorted, const void* w_exp, const int2* rowmeta,
+                                   const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, int mode,
+                                   void* bpi, void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s) {
   CUtensorMap ta, tb;
   if (!encode_tmap_2d(&ta, xsorted, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.M * d.k, (uint64_t)d.D * 2, BK, BM))
     return cudaErrorInvalidValue;
@@ -593,20 +617,29 @@ cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp
     CUtensorMap tb2;
     if (!encode_tmap_2d(&tb2, w_exp, SWIMBA_BF16, (uint64_t)d.D, (uint64_t)d.E * d.We, (uint64_t)d.D * 2, BK, 128))
       return cudaErrorInvalidValue;
-    e = launch_pair(ta, tb2, a, (ceil_div(d.M * d.k, kPairRows) + d.E) * ceil_div(d.We, BN), sms, s);
+    e = launch_pair<kRaw>(ta, tb2, a, (ceil_div(d.M * d.k, kPairRows) + d.E) * ceil_div(d.We, BN), sms, s);
     if (e == cudaSuccess) {
       count_launches(1);
       return cudaGetLastError();
     }
     (void)cudaGetLastError();  // pairs could not be launched: the one-CTA kernel below does the work
   }
-  e = set_max_dynamic_smem((const void*)proj_tc_kernel, kSmemBytes);
+  e = set_max_dynamic_smem((const void*)proj_tc_kernel<kRaw>, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int max_tiles = max_row_tiles(d) * ceil_div(d.We, BN);
   const int grid = max_tiles < sms ? max_tiles : sms;
-  e = launch_dependent(proj_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, s, 1, ta, tb, a);
+  e = launch_dependent(proj_tc_kernel<kRaw>, dim3(grid), dim3(kThreads), kSmemBytes, s, 1, ta, tb, a);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_proj_tc(const Dims& d, const void* xsorted, const void* w_exp, const int2* rowmeta,
+                           const int32_t* tiles, const int32_t* ntiles, const int32_t* offsets, int mode, void* bpi,
+                           void* xs, void* cpi, float* Z, unsigned* st, cudaStream_t s) {
+  return mode == 4 ? launch_proj_tc_t<true>(d, xsorted, w_exp, rowmeta, tiles, ntiles, offsets, mode, bpi, xs, cpi, Z,
+                                            st, s)
+                   : launch_proj_tc_t<false>(d, xsorted, w_exp, rowmeta, tiles, ntiles, offsets, mode, bpi, xs, cpi,
+                                             Z, st, s);
 }
 
 // The output projection out = y W_out^T as one dense product on the one-CTA kernel: A = y [M][K] (K = H*P),
@@ -630,17 +663,17 @@ cudaError_t launch_out_proj_tc(int M, int K, int N, const void* y, const void* w
     CUtensorMap tb2;
     if (!encode_tmap_2d(&tb2, w_out, SWIMBA_BF16, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, BK, 128))
       return cudaErrorInvalidValue;
-    e = launch_pair(ta, tb2, a, ceil_div(M, kPairRows) * ceil_div(N, BN), sms, s);
+    e = launch_pair<false>(ta, tb2, a, ceil_div(M, kPairRows) * ceil_div(N, BN), sms, s);
     if (e == cudaSuccess) {
       count_launches(1);
       return cudaGetLastError();
     }
     (void)cudaGetLastError();  // pairs could not be launched: the one-CTA kernel below does the work
   }
-  e = set_max_dynamic_smem((const void*)proj_tc_kernel, kSmemBytes);
+  e = set_max_dynamic_smem((const void*)proj_tc_kernel<false>, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int tiles = ceil_div(M, BM) * ceil_div(N, BN);
-  e = launch_dependent(proj_tc_kernel, dim3(tiles < sms ? tiles : sms), dim3(kThreads), kSmemBytes, s, 1, ta, tb, a);
+  e = launch_dependent(proj_tc_kernel<false>, dim3(tiles < sms ? tiles : sms), dim3(kThreads), kSmemBytes, s, 1, ta, tb, a);
   count_launches(1);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

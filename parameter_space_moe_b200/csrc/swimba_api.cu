@@ -189,9 +189,11 @@ static swimba_status run_proj(const Dims& d, const void* X, const void* w_exp, c
   return SWIMBA_OK;
 }
 
-// Router + dispatch + projection with the fused mix, into the workspace's streams.
+// Router + dispatch + projection with the fused mix, into the workspace's streams (mode 4: also the raw B
+// and C columns of z into Z).
 static swimba_status run_front(const Dims& d, const void* X, const swimba_weights* w, char* ws, const WsPlan& p,
-                               int32_t* idx, float* wts, int mode, unsigned* st, cudaStream_t s) {
+                               int32_t* idx, float* wts, int mode, unsigned* st, cudaStream_t s,
+                               float* Z = nullptr) {
   float* dt = (float*)(ws + p.dt);
   // one small kernel clears the router's per-tile counts and the scan's hand-off flags (adjacent regions);
   // the router's prologue and loads overlap it
@@ -209,7 +211,7 @@ static swimba_status run_front(const Dims& d, const void* X, const swimba_weight
     SW_CUDA(launch_dispatch_fused(d, idx, counts, p, ws, offsets, perm, wts, s));
     prof_mark(s, "dispatch");
   }
-  SW_TRY(run_proj(d, X, w->w_exp, ws, p, wts, mode, ws + p.bpi, ws + p.xs, ws + p.cpi, nullptr, st, s, fused_gather));
+  SW_TRY(run_proj(d, X, w->w_exp, ws, p, wts, mode, ws + p.bpi, ws + p.xs, ws + p.cpi, Z, st, s, fused_gather));
   return SWIMBA_OK;
 }
 
@@ -605,10 +607,14 @@ swimba_status swimba_layer_bwd(const swimba_dims* dims, const void* X, const swi
   float* wts = (float*)(b + p.topk_w);
   float* dt = (float*)(b + p.dt);
   prof_begin(s);
-  // the forward's router, dispatch and mixed streams, then the raw projections z for the mix's gradient
-  SW_TRY(run_front(d, X, w, b, p, idx, wts, 0, st, s));
-  SW_TRY(run_proj(d, X, w->w_exp, b, p, wts, 2, nullptr, nullptr, nullptr, (float*)(b + q.z), st, s,
-                  /*gathered=*/d.dtype == SWIMBA_BF16));
+  // the forward's router, dispatch and mixed streams, and the raw projections z the mix's gradient reads:
+  // one tensor-core GEMM writes both for bf16 layers; fp32 layers run the CUDA-core projection twice
+  if (d.dtype == SWIMBA_BF16) {
+    SW_TRY(run_front(d, X, w, b, p, idx, wts, 4, st, s, (float*)(b + q.z)));
+  } else {
+    SW_TRY(run_front(d, X, w, b, p, idx, wts, 0, st, s));
+    SW_TRY(run_proj(d, X, w->w_exp, b, p, wts, 2, nullptr, nullptr, nullptr, (float*)(b + q.z), st, s));
+  }
   SW_CUDA(launch_scan_bwd(d, b + p.bpi, b + p.xs, b + p.cpi, dt, w->A, init_state, dy, (float*)(b + q.dbpi),
                           (float*)(b + q.dxs), (float*)(b + q.dct), (float*)(b + q.ddt), dA, d_init,
                           (float*)(b + p.hstart), (float*)(b + p.schunk), (float*)(b + p.cslast), s));
