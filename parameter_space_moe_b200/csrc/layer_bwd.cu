@@ -18,8 +18,6 @@
 namespace swimba {
 
 namespace {
-constexpr int kT = 64;   // output tile edge of the CUDA-core GEMMs
-constexpr int kK = 16;   // contraction step
 
 // mix: one CTA per (token, slot) pair p.  fp32 layers: z (raw projection) is overwritten by dz.  bf16 layers
 // (kSplit): dz goes straight into the pair's padded row of the tensor-core products' operand as a bf16 split,
@@ -226,62 +224,135 @@ dw_experts_kernel(Dims d, const float* __restrict__ dz, const T* __restrict__ X,
   }
 }
 
-// out[r][n] += sum over a 256-token slice of G[m][r] X[m][n] (dW_r from dg, dW_dt from du); 64-row tiles of r
-template <class T>
-__global__ void __launch_bounds__(256)
-dw_dense_kernel(int M, int R, int D, const float* __restrict__ G, const T* __restrict__ X, float* __restrict__ out) {
-  __shared__ float As[kK][kT + 4];
-  __shared__ float Bs[kK][kT + 4];
-  const int n0 = blockIdx.x * kT, m_begin = blockIdx.y * 256, m_end = min(M, m_begin + 256), r0 = blockIdx.z * kT;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  float acc[4][4] = {};
-  for (int m0 = m_begin; m0 < m_end; m0 += kK) {
-    for (int i = tid; i < kK * kT; i += 256) {
-      const int kk = i / kT, c = i % kT, m = m0 + kk;
-      As[kk][c] = (m < m_end && r0 + c < R) ? G[(size_t)m * R + r0 + c] : 0.f;
-      Bs[kk][c] = (m < m_end && n0 + c < D) ? to_f32(X[(size_t)m * D + n0 + c]) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kK; ++kk) {
-      float av[4], bv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bv[j] = Bs[kk][tx + 16 * j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
+// The gate rows r < E + H of a token: dg[m][r] for r < E, then du[m][r - E].
+__device__ __forceinline__ float gate_at(const Dims& d, const float* __restrict__ dg, const float* __restrict__ du,
+                                         int m, int r) {
+  return r < d.E ? dg[(size_t)m * d.E + r] : du[(size_t)m * d.H + (r - d.E)];
+}
+
+// dW_r[e][n] = sum_m dg[m][e] X[m][n] and dW_dt[h][n] = sum_m du[m][h] X[m][n] as one product over the gate
+// rows: a CTA takes 32 gate rows x 128 columns over a 128-token slice, 16 tokens per stage through two
+// shared-memory buffers (each thread fetches the next stage's 8 X values in one 16-byte load and 2 gate values
+// while the current stage is multiplied); thread (column c, row half) keeps 16 accumulators; atomic adds into
+// the zeroed outputs.  D % 8 == 0, so an 8-column group never straddles the matrix edge.
+constexpr int kGR = 32, kGC = 128, kGM = 128, kGK = 16;
+__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int r = r0 + ty + 16 * i;
-    if (r >= R) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx + 16 * j;
-      if (n < D) atomicAdd(&out[(size_t)r * D + n], acc[i][j]);
-    }
+    const float2 v = __bfloat1622float2(h[i]);
+    f[2 * i] = v.x;
+    f[2 * i + 1] = v.y;
   }
 }
 
-// dX[m][n] = sum_j dXp[m k + j][n] + sum_e dg[m][e] W_r[e][n] + sum_h du[m][h] W_dt[h][n];  db_dt[h] += du
 template <class T>
-__global__ void dx_final_kernel(Dims d, const float* __restrict__ dxp, const float* __restrict__ dg,
-                                const float* __restrict__ du, const T* __restrict__ Wr, const T* __restrict__ Wdt,
-                                float* __restrict__ dX) {
-  const size_t total = (size_t)d.M * d.D;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-    const size_t m = i / d.D;
-    const int n = (int)(i % d.D);
-    float v = 0.f;
-    for (int j = 0; j < d.k; ++j) v += dxp[(m * d.k + j) * d.D + n];
-    for (int e = 0; e < d.E; ++e) v = fmaf(dg[m * d.E + e], to_f32(Wr[(size_t)e * d.D + n]), v);
-    for (int h = 0; h < d.H; ++h) v = fmaf(du[m * d.H + h], to_f32(Wdt[(size_t)h * d.D + n]), v);
-    dX[i] = v;
+__global__ void __launch_bounds__(256)
+dw_gate_kernel(Dims d, const float* __restrict__ dg, const float* __restrict__ du, const T* __restrict__ X,
+               float* __restrict__ dWr, float* __restrict__ dWdt) {
+  __shared__ __align__(16) float Gs[2][kGK][kGR];
+  __shared__ __align__(16) float Xs[2][kGK][kGC];
+  const int R = d.E + d.H;
+  const int n0 = blockIdx.x * kGC, m_begin = blockIdx.y * kGM, m_end = min(d.M, m_begin + kGM);
+  const int r0 = blockIdx.z * kGR;
+  const int tid = threadIdx.x, c = tid & (kGC - 1), rh = tid >> 7;  // a warp shares its row half
+  const int xr = tid >> 4, xc = (tid & 15) * 8;                      // X stage: token xr, columns xc ..
+  float xv[8], gv[2];
+  auto fetch = [&](int m0) {
+    const int m = m0 + xr;
+    if (m < m_end && n0 + xc < d.D) {
+      load8(X + (size_t)m * d.D + n0 + xc, xv);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) xv[u] = 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = 2 * tid + u, mm = m0 + i / kGR, r = r0 + i % kGR;
+      gv[u] = (mm < m_end && r < R) ? gate_at(d, dg, du, mm, r) : 0.f;
+    }
+  };
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  fetch(m_begin);
+  int buf = 0;
+  for (int m0 = m_begin; m0 < m_end; m0 += kGK) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) Xs[buf][xr][xc + u] = xv[u];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) (&Gs[buf][0][0])[2 * tid + u] = gv[u];
+    __syncthreads();
+    if (m0 + kGK < m_end) fetch(m0 + kGK);
+#pragma unroll
+    for (int kk = 0; kk < kGK; ++kk) {
+      const float x = Xs[buf][kk][c];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] = fmaf(Gs[buf][kk][rh * 16 + i], x, acc[i]);
+    }
+    buf ^= 1;
+  }
+  const int n = n0 + c;
+  if (n >= d.D) return;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = r0 + rh * 16 + i;
+    if (r < d.E) atomicAdd(&dWr[(size_t)r * d.D + n], acc[i]);
+    else if (r < R) atomicAdd(&dWdt[(size_t)(r - d.E) * d.D + n], acc[i]);
+  }
+}
+
+// dX[m][n] = sum_j dXp[m k + j][n] + sum_{r < E + H} gate[m][r] Wg[r][n]  (Wg = W_r rows, then W_dt rows):
+// a CTA takes 128 columns and a 64-token slice; 16 tokens at a time, thread c starts from its column's slot
+// sum, the tokens' gate rows are staged in shared memory (256 rows per pass) and each weight is loaded once
+// for the 16 tokens.
+constexpr int kXC = 128, kXM = 64, kXT = 16, kXR = 256;
+template <class T>
+__global__ void __launch_bounds__(kXC)
+dx_final_kernel(Dims d, const float* __restrict__ dxp, const float* __restrict__ dg, const float* __restrict__ du,
+                const T* __restrict__ Wr, const T* __restrict__ Wdt, float* __restrict__ dX) {
+  __shared__ float Gs[kXT][kXR];
+  const int R = d.E + d.H;
+  const int n0 = blockIdx.x * kXC, m_begin = blockIdx.y * kXM, m_end = min(d.M, m_begin + kXM);
+  const int n = n0 + threadIdx.x;
+  for (int m0 = m_begin; m0 < m_end; m0 += kXT) {
+    // the slot sum of dXp first: all its loads are in flight while the gate rows are staged and multiplied
+    float acc[kXT];
+#pragma unroll
+    for (int t = 0; t < kXT; ++t) {
+      const int m = m0 + t;
+      float v = 0.f;
+      if (n < d.D && m < m_end)
+        for (int j = 0; j < d.k; ++j) v += dxp[((size_t)m * d.k + j) * d.D + n];
+      acc[t] = v;
+    }
+    for (int rb = 0; rb < R; rb += kXR) {
+      const int nr = min(kXR, R - rb);
+      __syncthreads();  // the previous pass's rows are consumed
+      for (int i = threadIdx.x; i < kXT * nr; i += blockDim.x) {
+        const int t = i / nr, r = i % nr, m = m0 + t;
+        Gs[t][r] = m < m_end ? gate_at(d, dg, du, m, rb + r) : 0.f;
+      }
+      __syncthreads();
+      if (n < d.D) {
+        for (int r = 0; r < nr; ++r) {
+          const int rr = rb + r;
+          const float w = rr < d.E ? to_f32(Wr[(size_t)rr * d.D + n]) : to_f32(Wdt[(size_t)(rr - d.E) * d.D + n]);
+#pragma unroll
+          for (int t = 0; t < kXT; ++t) acc[t] = fmaf(Gs[t][r], w, acc[t]);
+        }
+      }
+    }
+    if (n < d.D) {
+#pragma unroll
+      for (int t = 0; t < kXT; ++t)
+        if (m0 + t < m_end) dX[(size_t)(m0 + t) * d.D + n] = acc[t];
+    }
   }
 }
 
@@ -338,13 +409,13 @@ cudaError_t launch_linear_typed(const Dims& d, const LayerBwdPtrs& q, cudaStream
   cudaError_t e = cudaMemsetAsync(q.dW_r, 0, (size_t)d.E * d.D * 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(q.dW_dt, 0, (size_t)d.H * d.D * 4, s);
   if (e != cudaSuccess) return e;
-  dw_dense_kernel<T><<<dim3(ceil_div(d.D, kT), ceil_div(d.M, 256), ceil_div(d.E, kT)), 256, 0, s>>>(
-      d.M, d.E, d.D, q.dg, (const T*)q.X, q.dW_r);
-  dw_dense_kernel<T><<<dim3(ceil_div(d.D, kT), ceil_div(d.M, 256), ceil_div(d.H, kT)), 256, 0, s>>>(
-      d.M, d.H, d.D, q.du, (const T*)q.X, q.dW_dt);
+  dw_gate_kernel<T><<<dim3(ceil_div(d.D, kGC), ceil_div(d.M, kGM), ceil_div(d.E + d.H, kGR)), 256, 0, s>>>(
+      d, q.dg, q.du, (const T*)q.X, q.dW_r, q.dW_dt);
   db_kernel<<<d.H, 256, 0, s>>>(d, q.du, q.db_dt);
-  dx_final_kernel<T><<<148 * 8, 256, 0, s>>>(d, q.dxp, q.dg, q.du, (const T*)q.w_r, (const T*)q.w_dt, q.dX);
-  count_launches(4);
+  dx_final_kernel<T><<<dim3(ceil_div(d.D, kXC), ceil_div(d.M, kXM)), kXC, 0, s>>>(d, q.dxp, q.dg, q.du,
+                                                                                  (const T*)q.w_r,
+                                                                                  (const T*)q.w_dt, q.dX);
+  count_launches(3);
   return cudaGetLastError();
 }
 }  // namespace
