@@ -308,50 +308,61 @@ dw_gate_kernel(Dims d, const float* __restrict__ dg, const float* __restrict__ d
 }
 
 // dX[m][n] = sum_j dXp[m k + j][n] + sum_{r < E + H} gate[m][r] Wg[r][n]  (Wg = W_r rows, then W_dt rows):
-// a CTA takes 128 columns and a 64-token slice; 16 tokens at a time, thread c starts from its column's slot
-// sum, the tokens' gate rows are staged in shared memory (256 rows per pass) and each weight is loaded once
-// for the 16 tokens.
-constexpr int kXC = 128, kXM = 64, kXT = 16, kXR = 256;
+// 128 x 128 output tiles on the 8 x 8-per-thread tile code of the expert products, K = E + H staged 8 at a
+// time; each thread starts from its outputs' slot sums (16-byte loads, all issued before the first stage).
 template <class T>
-__global__ void __launch_bounds__(kXC)
+__global__ void __launch_bounds__(256, 2)
 dx_final_kernel(Dims d, const float* __restrict__ dxp, const float* __restrict__ dg, const float* __restrict__ du,
                 const T* __restrict__ Wr, const T* __restrict__ Wdt, float* __restrict__ dX) {
-  __shared__ float Gs[kXT][kXR];
+  __shared__ __align__(16) Stage st;
   const int R = d.E + d.H;
-  const int n0 = blockIdx.x * kXC, m_begin = blockIdx.y * kXM, m_end = min(d.M, m_begin + kXM);
-  const int n = n0 + threadIdx.x;
-  for (int m0 = m_begin; m0 < m_end; m0 += kXT) {
-    // the slot sum of dXp first: all its loads are in flight while the gate rows are staged and multiplied
-    float acc[kXT];
+  const int n0 = blockIdx.x * kBT2, m0 = blockIdx.y * kBT2;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float acc[8][8];
 #pragma unroll
-    for (int t = 0; t < kXT; ++t) {
-      const int m = m0 + t;
-      float v = 0.f;
-      if (n < d.D && m < m_end)
-        for (int j = 0; j < d.k; ++j) v += dxp[((size_t)m * d.k + j) * d.D + n];
-      acc[t] = v;
-    }
-    for (int rb = 0; rb < R; rb += kXR) {
-      const int nr = min(kXR, R - rb);
-      __syncthreads();  // the previous pass's rows are consumed
-      for (int i = threadIdx.x; i < kXT * nr; i += blockDim.x) {
-        const int t = i / nr, r = i % nr, m = m0 + t;
-        Gs[t][r] = m < m_end ? gate_at(d, dg, du, m, rb + r) : 0.f;
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + ty * 8 + i;
+#pragma unroll
+    for (int jv = 0; jv < 8; jv += 4) {
+      const int n = n0 + tx * 8 + jv;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (m < d.M && n < d.D) {
+        const float* row = dxp + (size_t)m * d.k * d.D + n;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)  // k <= 8: a fixed trip count keeps the loads independent
+          if (j < d.k) {
+            const float4 u = *reinterpret_cast<const float4*>(row + (size_t)j * d.D);
+            v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+          }
       }
-      __syncthreads();
-      if (n < d.D) {
-        for (int r = 0; r < nr; ++r) {
-          const int rr = rb + r;
-          const float w = rr < d.E ? to_f32(Wr[(size_t)rr * d.D + n]) : to_f32(Wdt[(size_t)(rr - d.E) * d.D + n]);
-#pragma unroll
-          for (int t = 0; t < kXT; ++t) acc[t] = fmaf(Gs[t][r], w, acc[t]);
-        }
-      }
+      acc[i][jv] = v.x; acc[i][jv + 1] = v.y; acc[i][jv + 2] = v.z; acc[i][jv + 3] = v.w;
     }
-    if (n < d.D) {
+  }
+  for (int r0 = 0; r0 < R; r0 += kBK2) {
+    __syncthreads();  // the previous stage is consumed
 #pragma unroll
-      for (int t = 0; t < kXT; ++t)
-        if (m0 + t < m_end) dX[(size_t)(m0 + t) * d.D + n] = acc[t];
+    for (int u = 0; u < kBK2 * kBT2 / 256; ++u) {
+      const int i = tid + 256 * u;
+      const int row = i >> 3, kk = i & 7, m = m0 + row, r = r0 + kk;
+      st.A[kk][row] = (m < d.M && r < R) ? gate_at(d, dg, du, m, r) : 0.f;
+      const int kb = i >> 7, col = i & 127, n = n0 + col, rb = r0 + kb;
+      float w = 0.f;
+      if (rb < R && n < d.D) w = rb < d.E ? to_f32(Wr[(size_t)rb * d.D + n]) : to_f32(Wdt[(size_t)(rb - d.E) * d.D + n]);
+      st.B[kb][col] = w;
+    }
+    __syncthreads();
+    mac8x8(st, ty, tx, acc);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + ty * 8 + i;
+    if (m >= d.M) continue;
+#pragma unroll
+    for (int jv = 0; jv < 8; jv += 4) {
+      const int n = n0 + tx * 8 + jv;
+      if (n < d.D)
+        *reinterpret_cast<float4*>(dX + (size_t)m * d.D + n) =
+            make_float4(acc[i][jv], acc[i][jv + 1], acc[i][jv + 2], acc[i][jv + 3]);
     }
   }
 }
@@ -412,9 +423,9 @@ cudaError_t launch_linear_typed(const Dims& d, const LayerBwdPtrs& q, cudaStream
   dw_gate_kernel<T><<<dim3(ceil_div(d.D, kGC), ceil_div(d.M, kGM), ceil_div(d.E + d.H, kGR)), 256, 0, s>>>(
       d, q.dg, q.du, (const T*)q.X, q.dW_r, q.dW_dt);
   db_kernel<<<d.H, 256, 0, s>>>(d, q.du, q.db_dt);
-  dx_final_kernel<T><<<dim3(ceil_div(d.D, kXC), ceil_div(d.M, kXM)), kXC, 0, s>>>(d, q.dxp, q.dg, q.du,
-                                                                                  (const T*)q.w_r,
-                                                                                  (const T*)q.w_dt, q.dX);
+  dx_final_kernel<T><<<dim3(ceil_div(d.D, kBT2), ceil_div(d.M, kBT2)), 256, 0, s>>>(d, q.dxp, q.dg, q.du,
+                                                                                   (const T*)q.w_r,
+                                                                                   (const T*)q.w_dt, q.dX);
   count_launches(3);
   return cudaGetLastError();
 }
