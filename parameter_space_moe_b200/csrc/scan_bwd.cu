@@ -486,18 +486,35 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
       else atomicAdd(o, dC[i][jj]);
     }
   }
-  if (tid == 0) {
-    q[L - 1] += expf(cs_end) * red[0] + red[1];
-    // dA_r = sum_{t >= r} q_t;  d dt_r = dA_r A_h;  dA_h += sum_r dA_r dt_r
-    float run = 0.f, dAh = 0.f;
-    const float Ah = a.A[h];
-    for (int r = L - 1; r >= 0; --r) {
-      run += q[r];
-      const size_t o = (m0 + r) * d.H + h;
-      a.ddt[o] = run * Ah;
-      dAh = fmaf(run, a.dt[o], dAh);
+  if (tid < 32) {
+    // dA_r = sum_{t >= r} q_t (a shuffle scan over the tokens in reverse order, two per lane);
+    // d dt_r = dA_r A_h;  dA_h += sum_r dA_r dt_r
+    const int lane = tid;
+    if (lane == 0) q[L - 1] += expf(cs_end) * red[0] + red[1];
+    __syncwarp();
+    const int r0 = L - 1 - lane, r1 = L - 33 - lane;
+    float v0 = r0 >= 0 ? q[r0] : 0.f, v1 = r1 >= 0 ? q[r1] : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float u0 = __shfl_up_sync(0xffffffffu, v0, o), u1 = __shfl_up_sync(0xffffffffu, v1, o);
+      if (lane >= o) { v0 += u0; v1 += u1; }
     }
-    atomicAdd(&a.dA[h], dAh);
+    v1 += __shfl_sync(0xffffffffu, v0, 31);
+    const float Ah = a.A[h];
+    float part = 0.f;
+    if (r0 >= 0) {
+      const size_t o = (m0 + r0) * d.H + h;
+      a.ddt[o] = v0 * Ah;
+      part = v0 * a.dt[o];
+    }
+    if (r1 >= 0) {
+      const size_t o = (m0 + r1) * d.H + h;
+      a.ddt[o] = v1 * Ah;
+      part = fmaf(v1, a.dt[o], part);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) atomicAdd(&a.dA[h], part);
   }
 }
 
