@@ -60,7 +60,7 @@ __device__ __forceinline__ void sub_cumsum(const BwdArgs& a, int b, int h, int t
 template <int MJ, int MI = 4>
 __device__ __forceinline__ void tile_mac(float (&acc)[MI][MJ], int nj, int K, const float* X, int xk, int xr,
                                          const float* Y, int yk, int yc, int ty, int tx, int ni = MI) {
-#pragma unroll 4
+#pragma unroll 8
   for (int k = 0; k < K; ++k) {
     float xv[MI], yv[MJ];
 #pragma unroll
@@ -364,6 +364,7 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) { s1[i][jj] = 0.f; s2[i][jj] = 0.f; }
+#pragma unroll 8
       for (int n = 0; n < N; ++n) {
         float cv[4], bw[4];
 #pragma unroll
@@ -373,6 +374,7 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) s1[i][jj] = fmaf(cv[i], bw[jj], s1[i][jj]);
       }
+#pragma unroll 8
       for (int p = 0; p < P; ++p) {
         float dv[4], xv[4];
 #pragma unroll
