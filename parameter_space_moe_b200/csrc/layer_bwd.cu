@@ -28,16 +28,24 @@ __global__ void __launch_bounds__(256) mix_bwd_kernel(Dims d, float* __restrict_
                                                       const float* __restrict__ dct, float* __restrict__ dpi,
                                                       const int32_t* __restrict__ rp_of_p,
                                                       __nv_bfloat16* __restrict__ dzs, int Wp) {
+  // 16-byte vectors throughout: H*P and G*N are multiples of 16, so a 4-column group never straddles streams
   __shared__ float red[8];
   const size_t p = blockIdx.x;
   const size_t m = p / d.k;
   const float pi = wts[p];
   float* zr = z + p * d.We;
-  const float* gb = dbpi + p * d.GN;
-  const float* gc = dct + m * d.GN;
+  const float4* zb = reinterpret_cast<const float4*>(zr + d.HP);
+  const float4* zc = reinterpret_cast<const float4*>(zr + d.HP + d.GN);
+  const float4* gb = reinterpret_cast<const float4*>(dbpi + p * d.GN);
+  const float4* gc = reinterpret_cast<const float4*>(dct + m * d.GN);
+  const int GN4 = d.GN / 4;
   float part = 0.f;
-  for (int c = threadIdx.x; c < d.GN; c += blockDim.x)
-    part = fmaf(zr[d.HP + c], gb[c], fmaf(zr[d.HP + d.GN + c], gc[c], part));
+#pragma unroll 4
+  for (int c = threadIdx.x; c < GN4; c += blockDim.x) {
+    const float4 b = zb[c], g = gb[c], cc = zc[c], h = gc[c];
+    part = fmaf(b.x, g.x, fmaf(b.y, g.y, fmaf(b.z, g.z, fmaf(b.w, g.w, part))));
+    part = fmaf(cc.x, h.x, fmaf(cc.y, h.y, fmaf(cc.z, h.z, fmaf(cc.w, h.w, part))));
+  }
   for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = part;
   __syncthreads();  // every read of z is done before it is overwritten below
@@ -46,28 +54,32 @@ __global__ void __launch_bounds__(256) mix_bwd_kernel(Dims d, float* __restrict_
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) v += red[w];
     dpi[p] = v;
   }
-  const float* gx = dxs + p * d.HP;
+  const float4* gx = reinterpret_cast<const float4*>(dxs + p * d.HP);
+  const int HP4 = d.HP / 4, We4 = d.We / 4;
+  // column group c4 of dz = [dXs | pi dBpi | pi dC~]
+  auto dz4 = [&](int c4) {
+    if (c4 < HP4) return gx[c4];
+    float4 v = c4 < HP4 + GN4 ? gb[c4 - HP4] : gc[c4 - HP4 - GN4];
+    v.x *= pi; v.y *= pi; v.z *= pi; v.w *= pi;
+    return v;
+  };
   if constexpr (kSplit) {
-    // pairs of columns (H*P and G*N are even, so a pair never straddles two streams)
-    __nv_bfloat162* hi = reinterpret_cast<__nv_bfloat162*>(dzs + (size_t)rp_of_p[p] * 2 * Wp);
-    __nv_bfloat162* lo = hi + Wp / 2;
-    for (int c2 = threadIdx.x; c2 < Wp / 2; c2 += blockDim.x) {
-      const int c = 2 * c2;
-      float2 v = make_float2(0.f, 0.f);
-      if (c < d.HP) v = make_float2(gx[c], gx[c + 1]);
-      else if (c < d.HP + d.GN) v = make_float2(pi * gb[c - d.HP], pi * gb[c - d.HP + 1]);
-      else if (c < d.We) v = make_float2(pi * gc[c - d.HP - d.GN], pi * gc[c - d.HP - d.GN + 1]);
-      const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
-      const float2 hf = __bfloat1622float2(h);
-      hi[c2] = h;
-      lo[c2] = __floats2bfloat162_rn(v.x - hf.x, v.y - hf.y);
+    uint2* hi = reinterpret_cast<uint2*>(dzs + (size_t)rp_of_p[p] * 2 * Wp);
+    uint2* lo = hi + Wp / 4;
+#pragma unroll 4
+    for (int c4 = threadIdx.x; c4 < Wp / 4; c4 += blockDim.x) {
+      const float4 v = c4 < We4 ? dz4(c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y), h1 = __floats2bfloat162_rn(v.z, v.w);
+      const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+      const __nv_bfloat162 l0 = __floats2bfloat162_rn(v.x - f0.x, v.y - f0.y);
+      const __nv_bfloat162 l1 = __floats2bfloat162_rn(v.z - f1.x, v.w - f1.y);
+      hi[c4] = make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+      lo[c4] = make_uint2(*reinterpret_cast<const uint32_t*>(&l0), *reinterpret_cast<const uint32_t*>(&l1));
     }
   } else {
-    for (int c = threadIdx.x; c < d.HP; c += blockDim.x) zr[c] = gx[c];
-    for (int c = threadIdx.x; c < d.GN; c += blockDim.x) {
-      zr[d.HP + c] = pi * gb[c];
-      zr[d.HP + d.GN + c] = pi * gc[c];
-    }
+    float4* zw = reinterpret_cast<float4*>(zr);
+#pragma unroll 4
+    for (int c4 = threadIdx.x; c4 < We4; c4 += blockDim.x) zw[c4] = dz4(c4);
   }
 }
 
