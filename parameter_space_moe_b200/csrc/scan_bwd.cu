@@ -16,7 +16,7 @@
 //     dA_r    = sum_{t >= r} q_t,   d dt_r = dA_r A_h,   dA_h = sum_r dA_r dt_r,   d init = Lam_0.
 // With G < H the Bpi and C~ gradients of a group's heads are summed (atomic adds into zeroed outputs); with
 // G = H every output element is written by exactly one CTA.
-#include "common.cuh"
+#include "tc_common.cuh"
 
 namespace swimba {
 
@@ -33,6 +33,7 @@ struct BwdArgs {
   float* hstart;           // [B][H][nc][N][P]  H_c
   float* work;             // [B][H][nc][N][P]  S_c, then D_c, then Lam_{c+1}
   float* cse;              // [B][H][nc]        cs at each sub-chunk's last token
+  unsigned* st;            // device status word (bounded waits of the tensor-core state kernels)
 };
 
 // cs[i] = sum_{r <= i} dt_r A_h over the sub-chunk (warp 0: two tokens per lane, shuffle scans; L <= 64)
@@ -247,6 +248,187 @@ __global__ void bwd_adj_pass_kernel(BwdArgs a) {
     lam = fmaf(expf(a.cse[bh * a.nc + c]), lam, Dc);
   }
   if (a.dinit) a.dinit[bh * NP + e] = lam;
+}
+
+// 1'/3'. The end states S_c and the adjoint sources D_c on the tensor cores (fp16 streams, N = 128,
+// P in {64, 128}).  Both are [N x P] = A^T B over the sub-chunk's tokens:
+//   S_c = sum_j Bpi_j^T (e^{cs_end - cs} * Xs_j),   D_c = sum_j Cpi_j^T (e^{cs} * dy)
+// A (the fp16 stream rows, exact) is M = n by K = token, read MN-major; B is formed in fp32 and split into two
+// fp16 halves hi + lo (two MMAs into one fp32 accumulator: about 2^-22 relative); dy first takes a
+// power-of-two scale that puts the tile's largest value near 2^15 (exact, undone on the result), so the
+// split stays inside fp16's range.  One CTA of 4 warps per (sequence, head, 64-token sub-chunk); operands
+// are staged slot by slot in 128-byte-swizzled shared memory by plain 16-byte loads; the accumulator sits in
+// P TMEM columns.
+constexpr uint32_t kTcBlk = BL * 128;  // one 64-wide MN block of 64 K rows of 128 bytes
+// dynamic shared memory of the tensor-core state kernels: alignment slack, A, B hi and lo, cs, scale
+// partials, mbarrier, TMEM slot and abort flag
+inline size_t states_tc_smem(int P) { return 1024 + 2 * kTcBlk + 2 * (size_t)(P / 64) * kTcBlk + (BL + 4) * 4 + 24; }
+template <bool kD>
+__global__ void __launch_bounds__(128) bwd_states_tc_kernel(BwdArgs a) {
+  extern __shared__ uint8_t smraw[];
+  const uint32_t raw = tc::smem_u32(smraw);
+  uint8_t* sm = smraw + (((raw + 1023u) & ~1023u) - raw);
+  const Dims& d = a.d;
+  const int N = d.N, P = d.P, PB = P / 64;
+  uint8_t* As = sm;                          // 2 MN blocks (n 0..63, 64..127)
+  uint8_t* Bhi = As + 2 * kTcBlk;            // PB MN blocks
+  uint8_t* Blo = Bhi + PB * kTcBlk;
+  float* cs = reinterpret_cast<float*>(Blo + PB * kTcBlk);  // [BL]
+  float* red = cs + BL;                                     // [4]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(red + 4);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, g = h / d.hpg;
+  const int t0 = c * BL, L = min(BL, d.T - t0);
+  const size_t m0 = (size_t)b * d.T + t0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  sub_cumsum(a, b, h, t0, L, cs);
+  if (tid == 0) {
+    tc::mbar_init(bar, 1);
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) { tc::tmem_alloc(tslot, (uint32_t)P); tc::tmem_relinquish(); }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tslot;
+  const float cs_end = cs[L - 1];
+  // B: row s (token), column p; 8 columns (one 16-byte fp16 chunk) per step
+  auto put_b = [&](int s, int p0, const float (&v)[8]) {
+    uint4 uh, ul;
+    __half2* hh = reinterpret_cast<__half2*>(&uh);
+    __half2* hl = reinterpret_cast<__half2*>(&ul);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      hh[e] = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
+      const float2 f = __half22float2(hh[e]);
+      hl[e] = __floats2half2_rn(v[2 * e] - f.x, v[2 * e + 1] - f.y);
+    }
+    const uint32_t off = (p0 >> 6) * kTcBlk + tc::sw128_chunk(s, (p0 & 63) >> 3);
+    *reinterpret_cast<uint4*>(Bhi + off) = uh;
+    *reinterpret_cast<uint4*>(Blo + off) = ul;
+  };
+  int sc = 0;  // D_c: power-of-two scale of e^{cs} dy
+  if constexpr (kD) {
+    float mx = 0.f;
+    for (int x = tid; x < BL * (P / 8); x += blockDim.x) {
+      const int s = x / (P / 8), p0 = (x % (P / 8)) * 8;
+      if (s < L) {
+        const float e = expf(cs[s]);
+        const float* src = a.dy + (m0 + s) * d.HP + (size_t)h * P + p0;
+        const float4 u0 = *reinterpret_cast<const float4*>(src), u1 = *reinterpret_cast<const float4*>(src + 4);
+        mx = fmaxf(mx, e * fmaxf(fmaxf(fmaxf(fabsf(u0.x), fabsf(u0.y)), fmaxf(fabsf(u0.z), fabsf(u0.w))),
+                                 fmaxf(fmaxf(fabsf(u1.x), fabsf(u1.y)), fmaxf(fabsf(u1.z), fabsf(u1.w)))));
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    if (mx > 0.f && mx < 3.0e38f) {
+      int ex;
+      frexpf(mx, &ex);
+      sc = 15 - ex;
+    }
+    // B = e^{cs_t} dy_t 2^sc, the same for every slot
+    for (int x = tid; x < BL * (P / 8); x += blockDim.x) {
+      const int s = x / (P / 8), p0 = (x % (P / 8)) * 8;
+      float v[8];
+      if (s < L) {
+        // the scale applies to the product (bounded by the tile's maximum), never to e^{cs} alone
+        const float e = expf(cs[s]);
+        const float* src = a.dy + (m0 + s) * d.HP + (size_t)h * P + p0;
+        const float4 u0 = *reinterpret_cast<const float4*>(src), u1 = *reinterpret_cast<const float4*>(src + 4);
+        v[0] = ldexpf(e * u0.x, sc); v[1] = ldexpf(e * u0.y, sc); v[2] = ldexpf(e * u0.z, sc);
+        v[3] = ldexpf(e * u0.w, sc); v[4] = ldexpf(e * u1.x, sc); v[5] = ldexpf(e * u1.y, sc);
+        v[6] = ldexpf(e * u1.z, sc); v[7] = ldexpf(e * u1.w, sc);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = 0.f;
+      }
+      put_b(s, p0, v);
+    }
+  }
+  constexpr uint32_t kIdescS = tc::idesc_f16(128, 64, /*bf16=*/false, /*a_mn=*/true, /*b_mn=*/true);
+  constexpr uint32_t kIdescS2 = tc::idesc_f16(128, 128, /*bf16=*/false, /*a_mn=*/true, /*b_mn=*/true);
+  const uint32_t idesc = P == 64 ? kIdescS : kIdescS2;
+  const __half* Asrc = reinterpret_cast<const __half*>(kD ? a.cpi : a.bpi);
+  uint32_t phase = 0;
+  bool ok = true;
+  for (int j = 0; j < d.k && ok; ++j) {
+    // A_j: the slot's N-wide stream rows, 16 chunks of 8 per row
+    for (int x = tid; x < BL * 16; x += blockDim.x) {
+      const int s = x >> 4, ch = x & 15;
+      uint4 u = make_uint4(0u, 0u, 0u, 0u);
+      if (s < L) u = *reinterpret_cast<const uint4*>(Asrc + ((m0 + s) * d.k + j) * d.GN + (size_t)g * N + ch * 8);
+      *reinterpret_cast<uint4*>(As + (ch >> 3) * kTcBlk + tc::sw128_chunk(s, ch & 7)) = u;
+    }
+    if constexpr (!kD) {
+      // B_j = e^{cs_end - cs_s} Xs_j
+      for (int x = tid; x < BL * (P / 8); x += blockDim.x) {
+        const int s = x / (P / 8), p0 = (x % (P / 8)) * 8;
+        float v[8];
+        if (s < L) {
+          const float e = expf(cs_end - cs[s]);
+          const uint4 q = *reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(a.xs) +
+                                                          ((m0 + s) * d.k + j) * d.HP + (size_t)h * P + p0);
+          const __half2* hq = reinterpret_cast<const __half2*>(&q);
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 f = __half22float2(hq[e2]);
+            v[2 * e2] = e * f.x;
+            v[2 * e2 + 1] = e * f.y;
+          }
+        } else {
+#pragma unroll
+          for (int q2 = 0; q2 < 8; ++q2) v[q2] = 0.f;
+        }
+        put_b(s, p0, v);
+      }
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (tid == 0) {
+      const uint32_t sa = tc::smem_u32(As), sh = tc::smem_u32(Bhi), sl = tc::smem_u32(Blo);
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+#pragma unroll
+        for (int kk = 0; kk < BL / 16; ++kk)
+          tc::mma_f16(tmem, tc::sdesc_mnmajor_sw128(sa + kk * 2048, kTcBlk),
+                      tc::sdesc_mnmajor_sw128((part ? sl : sh) + kk * 2048, kTcBlk), idesc,
+                      (j | part | kk) != 0);
+      tc::mma_commit(bar);
+    }
+    // the slot's MMAs read the staged operands: wait before the next slot overwrites them
+    ok = tc::mbar_wait(bar, phase, abort_flag);
+    phase ^= 1u;
+    tc::fence_after_sync();
+  }
+  if (!ok && lane == 0) atomicOr(a.st, ST_TIMEOUT);
+  // TMEM lane n (warp w: lanes 32w ..) holds row n of the [N x P] result
+  const size_t base = (((size_t)b * d.H + h) * a.nc + c) * (size_t)N * P;
+  const int n = 32 * warp + lane;
+  for (int c0 = 0; c0 < P && ok; c0 += 32) {
+    uint32_t r[32];
+    tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0, r);
+    tc::tmem_ld_wait(r);
+    float* dst = a.work + base + (size_t)n * P + c0;
+#pragma unroll
+    for (int i = 0; i < 32; i += 4)
+      *reinterpret_cast<float4*>(dst + i) =
+          make_float4(ldexpf(__uint_as_float(r[i]), -sc), ldexpf(__uint_as_float(r[i + 1]), -sc),
+                      ldexpf(__uint_as_float(r[i + 2]), -sc), ldexpf(__uint_as_float(r[i + 3]), -sc));
+  }
+  if (!kD && tid == 0) a.cse[((size_t)b * d.H + h) * a.nc + c] = cs_end;
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, (uint32_t)P);
+  }
 }
 
 // Shared-memory plan of the gradient kernel (floats): per sub-chunk C~, dy, then per slot keys, values,
@@ -524,15 +706,31 @@ template <class S, int PJ>
 cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s) {
   const Dims& d = a.d;
   const dim3 grid(a.nc, d.H, d.Bsz);
+  // fp16 streams with N = 128 and P in {64, 128}: the end states and adjoint sources on the tensor cores
+  const bool tc_states = std::is_same<S, __half>::value && d.N == 128 && (d.P == 64 || d.P == 128);
   const size_t sm1 = (BL + (size_t)BL * d.N + (size_t)BL * d.P) * 4;
-  cudaError_t e = set_max_dynamic_smem((const void*)bwd_fwd_chunk_kernel<S, PJ>, sm1);
-  if (e != cudaSuccess) return e;
-  bwd_fwd_chunk_kernel<S, PJ><<<grid, kBT, sm1, s>>>(a);
+  const size_t smt = states_tc_smem(d.P);
+  cudaError_t e;
+  if (tc_states) {
+    e = set_max_dynamic_smem((const void*)bwd_states_tc_kernel<false>, smt);
+    if (e != cudaSuccess) return e;
+    bwd_states_tc_kernel<false><<<grid, 128, smt, s>>>(a);
+  } else {
+    e = set_max_dynamic_smem((const void*)bwd_fwd_chunk_kernel<S, PJ>, sm1);
+    if (e != cudaSuccess) return e;
+    bwd_fwd_chunk_kernel<S, PJ><<<grid, kBT, sm1, s>>>(a);
+  }
   const dim3 pgrid(ceil_div(d.N * d.P, kBT), d.H, d.Bsz);
   bwd_fwd_pass_kernel<<<pgrid, kBT, 0, s>>>(a);
-  e = set_max_dynamic_smem((const void*)bwd_d_kernel<S, PJ>, sm1);
-  if (e != cudaSuccess) return e;
-  bwd_d_kernel<S, PJ><<<grid, kBT, sm1, s>>>(a);
+  if (tc_states) {
+    e = set_max_dynamic_smem((const void*)bwd_states_tc_kernel<true>, smt);
+    if (e != cudaSuccess) return e;
+    bwd_states_tc_kernel<true><<<grid, 128, smt, s>>>(a);
+  } else {
+    e = set_max_dynamic_smem((const void*)bwd_d_kernel<S, PJ>, sm1);
+    if (e != cudaSuccess) return e;
+    bwd_d_kernel<S, PJ><<<grid, kBT, sm1, s>>>(a);
+  }
   bwd_adj_pass_kernel<<<pgrid, kBT, 0, s>>>(a);
   const size_t sm5 = GradSmem(d.N, d.P).total * 4;
   e = set_max_dynamic_smem((const void*)bwd_grad_kernel<S, PJ>, sm5);
@@ -566,7 +764,8 @@ cudaError_t launch_scan_bwd(const Dims& d, const void* bpi, const void* xs, cons
                             float* ddt, float* dA, float* dinit, float* hstart, float* work, float* cse,
                             cudaStream_t s) {
   BwdArgs a{d, scan_bwd_subchunks(d), bpi, xs, cpi, dt, A, init, dy, dbpi, dxs, dct, ddt, dA, dinit,
-            hstart, work, cse};
+            hstart, work, cse, device_status()};
+  if (!a.st) return cudaErrorInvalidValue;
   // the A gradient, and with G < H the Bpi and C~ gradients (summed over a group's heads), are accumulated
   cudaError_t e = cudaMemsetAsync(dA, 0, (size_t)d.H * 4, s);
   if (e == cudaSuccess && d.hpg > 1) e = cudaMemsetAsync(dbpi, 0, (size_t)d.M * d.k * d.GN * 4, s);

@@ -1,7 +1,8 @@
 """Gradients of the chunked scan (swimba_ssd_scan_bwd) against the oracle's adjoint recurrence, through the
 C ABI.  The streams are the oracle layer's own, rounded to the stream dtype the GPU reads; the oracle then
 differentiates exactly those values.  Shapes: the tiny fp32 layer, bf16 layers with N = 128 (one head per
-group, two groups of two, G = 1 with k = 3), ragged sequence tails (64-token sub-chunks), an initial state."""
+group, two groups of two, G = 1 with k = 3, P = 128), ragged sequence tails (64-token sub-chunks), an initial
+state, and upstream gradients scaled by 2^-110 and 2^100."""
 import numpy as np
 import pytest
 import torch
@@ -22,6 +23,8 @@ CASES = [
                        chunk=128, seed=123),
     configs.BASE.with_(name="bwd_bf16_G1_k3", batch=1, seqlen=190, d_model=128, nheads=3, ngroups=1, n_experts=5,
                        top_k=3, chunk=64, seed=124),
+    configs.BASE.with_(name="bwd_bf16_P128", batch=1, seqlen=200, d_model=128, nheads=2, headdim=128, n_experts=4,
+                       chunk=128, seed=125),
 ]
 # fp32 arithmetic on the same inputs: norm-wise bounds (measured 2e-7 .. 4e-7 for the stream and state
 # gradients).  d dt and dA sum many terms of both signs (the log-decay gradient is a difference of score-tile
@@ -32,6 +35,17 @@ TOL = dict(dBpi=1e-5, dXs=1e-5, dCt=1e-5, dinit=1e-5, ddt=2e-5, dA=2e-5)
 @pytest.mark.parametrize("with_init", [False, True], ids=["zero_init", "init"])
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
 def test_scan_gradients_match_oracle(w, with_init):
+    _check(w, with_init)
+
+
+@pytest.mark.parametrize("scale", [2.0 ** -110, 2.0 ** 100], ids=["dy_2^-110", "dy_2^100"])
+def test_scan_gradients_extreme_dy_scale(scale):
+    """Every gradient is linear in dy; the tensor-core adjoint sources scale dy by a power of two before
+    splitting it into fp16 halves, which must hold for upstream gradients far outside fp16's range."""
+    _check(CASES[2], True, scale)
+
+
+def _check(w, with_init, dy_scale=1.0):
     inp = inputs.make_inputs(w)
     ref = O.layer_fwd(f64(inp["X"]), f64(inp["W_r"]), f64(inp["W_dt"]), f64(inp["b_dt"]), f64(inp["A"]),
                       f64(inp["W_exp"]), w.nheads, w.headdim, w.dstate, w.G, w.top_k)
@@ -40,7 +54,7 @@ def test_scan_gradients_match_oracle(w, with_init):
     dt = torch.from_numpy(ref["dt"]).float()
     A = inp["A"]
     rng = np.random.default_rng(w.seed)
-    dy = torch.from_numpy(rng.standard_normal((w.M, w.nheads, w.headdim)).astype(np.float32))
+    dy = torch.from_numpy((rng.standard_normal((w.M, w.nheads, w.headdim)) * dy_scale).astype(np.float32))
     init = (torch.from_numpy(rng.standard_normal((w.batch, w.nheads, w.dstate, w.headdim)).astype(np.float32))
             if with_init else None)
     d = swimba.dims_of(w)
