@@ -462,9 +462,21 @@ def scan_bwd_flops(w):
     return 2.0 * total * w.batch * w.nheads
 
 
+def scan_bwd_tensor_flops(w):
+    """The part of scan_bwd_flops the tensor cores run for fp16 streams with N = 128 and P in {64, 128}: the
+    sub-chunk end states (k L N P FMAs) and adjoint sources (L N P), algorithmic counts (the hi/lo split's
+    second MMA not counted); 0 where the CUDA-core kernels run them."""
+    if w.dtype != "bf16" or w.dstate != 128 or w.headdim not in (64, 128):
+        return 0.0
+    return 2.0 * (w.top_k + 1) * w.seqlen * w.dstate * w.headdim * w.batch * w.nheads
+
+
 def scan_bwd_measure(args, dev, flush, stream, swimba):
-    """The scan gradients (swimba_ssd_scan_bwd) at the base layer's sizes on seeded streams, timed alone; bound by
-    the fp32 CUDA-core arithmetic, against 148 SMs x 128 fp32 lanes x 2 FLOP x the maximum SM clock."""
+    """The scan gradients (swimba_ssd_scan_bwd) at the base layer's sizes on seeded streams, timed alone.  The
+    end states and adjoint sources run on the tensor cores, the rest on CUDA cores: the floor is the sum of
+    their FLOPs at the bf16 burst peak and at the fp32 ALU peak (148 SMs x 128 lanes x 2 FLOP x the maximum SM
+    clock); achieved counts all of the work against the ALU peak as well, for comparison with the CUDA-core
+    kernels alone."""
     w = configs.BASE
     g = torch.Generator().manual_seed(131)
     M, k, H, P, N = w.M, w.top_k, w.nheads, w.headdim, w.dstate
@@ -504,20 +516,26 @@ def scan_bwd_measure(args, dev, flush, stream, swimba):
     except Exception:
         pass
     peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
-    return {"ms": secs * 1e3, "flops": flops,
+    tflops = scan_bwd_tensor_flops(w)
+    peaks, psrc = load_peaks()
+    floor = tflops / (peaks["bf16_tflops"] * 1e12) + (flops - tflops) / (peak * 1e12)
+    return {"ms": secs * 1e3, "flops": flops, "tensor_flops": tflops,
             "roofline": {"bound": "alu", "achieved": flops / secs / 1e12, "peak": peak, "unit": "TFLOP/s",
                          "frac": flops / secs / 1e12 / peak,
-                         "peak_source": f"148 SMs x 128 fp32 lanes x 2 FLOP x {mhz:.0f} MHz (max SM clock)"}}
+                         "peak_source": f"148 SMs x 128 fp32 lanes x 2 FLOP x {mhz:.0f} MHz (max SM clock)"},
+            "floor": {"bound": "tensor+alu", "floor_ms": floor * 1e3, "frac": floor / secs,
+                      "tensor_peak_tflops": peaks["bf16_tflops"], "peak_source": f"bf16 burst ({psrc})"}}
 
 
 def layer_bwd_measure(args, sess, inp, flush, stream, swimba):
     """The layer gradients (swimba_layer_bwd) at the base workload with a seeded dy, timed alone: one call
-    recomputes the forward's router, dispatch and projections, runs the scan gradients (CUDA cores), the mix and
-    router gradients, the two expert products dz W_e and dz^T X (tensor cores, on a bf16 hi/lo split of dz) and
-    the router and dt weight gradients.  The roofline is the sum of two floors: the tensor-core FLOPs (forward
-    recompute GEMM and router, the two expert products; algorithmic counts, the split's second MMA not counted)
-    at the bf16 burst peak plus the CUDA-core FLOPs (scan gradients, router and dt products) at the fp32 ALU
-    peak.  The expert products also get their own roofline from their stage time (pack of dz included)."""
+    recomputes the forward's router, dispatch and projections, runs the scan gradients (end states and adjoint
+    sources on the tensor cores, the rest on CUDA cores), the mix and router gradients, the two expert products
+    dz W_e and dz^T X (tensor cores, on a bf16 hi/lo split of dz) and the router and dt weight gradients.  The
+    roofline is the sum of two floors: the tensor-core FLOPs (forward recompute GEMM and router, the scan's
+    end states and adjoint sources, the two expert products; algorithmic counts, the split's second MMA not
+    counted) at the bf16 burst peak plus the CUDA-core FLOPs (the rest of the scan gradients, the router and
+    dt products) at the fp32 ALU peak.  The expert products also get their own roofline from their stage time (pack of dz included)."""
     w = sess.w
     dev = sess.X.device
     g = torch.Generator().manual_seed(151)
@@ -553,8 +571,9 @@ def layer_bwd_measure(args, sess, inp, flush, stream, swimba):
     peaks, psrc = load_peaks()
     gemm = 2.0 * w.M * w.top_k * w.W_e * w.d_model          # one expert product over all (token, slot) rows
     small = 2.0 * w.M * (w.n_experts + w.nheads) * w.d_model  # one router + dt product over all tokens
-    t_flops = 3 * gemm + small                               # recompute GEMM and router, dz W_e, dz^T X
-    a_flops = scan_bwd_flops(w) + 2 * small                  # scan gradients, dg^T X / du^T X and their dX terms
+    st = scan_bwd_tensor_flops(w)                            # scan end states and adjoint sources
+    t_flops = 3 * gemm + small + st                          # recompute GEMM and router, dz W_e, dz^T X
+    a_flops = scan_bwd_flops(w) - st + 2 * small             # rest of the scan gradients, dg^T X / du^T X, dX terms
     tpk = peaks["bf16_tflops"]
     apk = 148 * 128 * 2 * 1965e6 / 1e12
     floor = t_flops / (tpk * 1e12) + a_flops / (apk * 1e12)
