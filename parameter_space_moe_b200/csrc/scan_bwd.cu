@@ -263,13 +263,15 @@ constexpr uint32_t kTcBlk = BL * 128;  // one 64-wide MN block of 64 K rows of 1
 // dynamic shared memory of the tensor-core state kernels: alignment slack, A, B hi and lo, cs, scale
 // partials, mbarrier, TMEM slot and abort flag
 inline size_t states_tc_smem(int P) { return 1024 + 2 * kTcBlk + 2 * (size_t)(P / 64) * kTcBlk + (BL + 4) * 4 + 24; }
-template <bool kD>
+template <bool kD, int kP>
 __global__ void __launch_bounds__(128) bwd_states_tc_kernel(BwdArgs a) {
   extern __shared__ uint8_t smraw[];
   const uint32_t raw = tc::smem_u32(smraw);
   uint8_t* sm = smraw + (((raw + 1023u) & ~1023u) - raw);
   const Dims& d = a.d;
-  const int N = d.N, P = d.P, PB = P / 64;
+  constexpr int N = 128, PB = kP / 64;
+  constexpr int kAU = BL * 16 / 128;        // 16-byte A chunks per thread (8)
+  constexpr int kBU = BL * (kP / 8) / 128;  // 8-column B groups per thread (4 or 8)
   uint8_t* As = sm;                          // 2 MN blocks (n 0..63, 64..127)
   uint8_t* Bhi = As + 2 * kTcBlk;            // PB MN blocks
   uint8_t* Blo = Bhi + PB * kTcBlk;
@@ -288,13 +290,13 @@ __global__ void __launch_bounds__(128) bwd_states_tc_kernel(BwdArgs a) {
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
-  if (warp == 1) { tc::tmem_alloc(tslot, (uint32_t)P); tc::tmem_relinquish(); }
+  if (warp == 1) { tc::tmem_alloc(tslot, (uint32_t)kP); tc::tmem_relinquish(); }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tslot;
   const float cs_end = cs[L - 1];
-  // B: row s (token), column p; 8 columns (one 16-byte fp16 chunk) per step
+  // B: row s (token), columns p0 .. p0+7 as one 16-byte fp16 chunk of each half
   auto put_b = [&](int s, int p0, const float (&v)[8]) {
     uint4 uh, ul;
     __half2* hh = reinterpret_cast<__half2*>(&uh);
@@ -311,15 +313,30 @@ __global__ void __launch_bounds__(128) bwd_states_tc_kernel(BwdArgs a) {
   };
   int sc = 0;  // D_c: power-of-two scale of e^{cs} dy
   if constexpr (kD) {
-    float mx = 0.f;
-    for (int x = tid; x < BL * (P / 8); x += blockDim.x) {
-      const int s = x / (P / 8), p0 = (x % (P / 8)) * 8;
+    // e^{cs_t} dy_t for this thread's groups, all loads issued before any use
+    float v[kBU][8];
+#pragma unroll
+    for (int u = 0; u < kBU; ++u) {
+      const int x = tid + 128 * u, s = x / (kP / 8), p0 = (x % (kP / 8)) * 8;
       if (s < L) {
-        const float e = expf(cs[s]);
-        const float* src = a.dy + (m0 + s) * d.HP + (size_t)h * P + p0;
+        const float* src = a.dy + (m0 + s) * d.HP + (size_t)h * kP + p0;
         const float4 u0 = *reinterpret_cast<const float4*>(src), u1 = *reinterpret_cast<const float4*>(src + 4);
-        mx = fmaxf(mx, e * fmaxf(fmaxf(fmaxf(fabsf(u0.x), fabsf(u0.y)), fmaxf(fabsf(u0.z), fabsf(u0.w))),
-                                 fmaxf(fmaxf(fabsf(u1.x), fabsf(u1.y)), fmaxf(fabsf(u1.z), fabsf(u1.w)))));
+        v[u][0] = u0.x; v[u][1] = u0.y; v[u][2] = u0.z; v[u][3] = u0.w;
+        v[u][4] = u1.x; v[u][5] = u1.y; v[u][6] = u1.z; v[u][7] = u1.w;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[u][q] = 0.f;
+      }
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int u = 0; u < kBU; ++u) {
+      const int s = (tid + 128 * u) / (kP / 8);
+      const float e = s < L ? expf(cs[s]) : 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        v[u][q] *= e;
+        mx = fmaxf(mx, fabsf(v[u][q]));
       }
     }
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -331,58 +348,56 @@ __global__ void __launch_bounds__(128) bwd_states_tc_kernel(BwdArgs a) {
       frexpf(mx, &ex);
       sc = 15 - ex;
     }
-    // B = e^{cs_t} dy_t 2^sc, the same for every slot
-    for (int x = tid; x < BL * (P / 8); x += blockDim.x) {
-      const int s = x / (P / 8), p0 = (x % (P / 8)) * 8;
-      float v[8];
-      if (s < L) {
-        // the scale applies to the product (bounded by the tile's maximum), never to e^{cs} alone
-        const float e = expf(cs[s]);
-        const float* src = a.dy + (m0 + s) * d.HP + (size_t)h * P + p0;
-        const float4 u0 = *reinterpret_cast<const float4*>(src), u1 = *reinterpret_cast<const float4*>(src + 4);
-        v[0] = ldexpf(e * u0.x, sc); v[1] = ldexpf(e * u0.y, sc); v[2] = ldexpf(e * u0.z, sc);
-        v[3] = ldexpf(e * u0.w, sc); v[4] = ldexpf(e * u1.x, sc); v[5] = ldexpf(e * u1.y, sc);
-        v[6] = ldexpf(e * u1.z, sc); v[7] = ldexpf(e * u1.w, sc);
-      } else {
+    // B = e^{cs_t} dy_t 2^sc (the scale applies to the product, bounded by the tile's maximum), every slot
 #pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = 0.f;
-      }
-      put_b(s, p0, v);
+    for (int u = 0; u < kBU; ++u) {
+      const int x = tid + 128 * u, s = x / (kP / 8), p0 = (x % (kP / 8)) * 8;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[u][q] = ldexpf(v[u][q], sc);
+      put_b(s, p0, v[u]);
     }
   }
-  constexpr uint32_t kIdescS = tc::idesc_f16(128, 64, /*bf16=*/false, /*a_mn=*/true, /*b_mn=*/true);
-  constexpr uint32_t kIdescS2 = tc::idesc_f16(128, 128, /*bf16=*/false, /*a_mn=*/true, /*b_mn=*/true);
-  const uint32_t idesc = P == 64 ? kIdescS : kIdescS2;
+  constexpr uint32_t idesc = tc::idesc_f16(128, kP, /*bf16=*/false, /*a_mn=*/true, /*b_mn=*/true);
   const __half* Asrc = reinterpret_cast<const __half*>(kD ? a.cpi : a.bpi);
   uint32_t phase = 0;
   bool ok = true;
   for (int j = 0; j < d.k && ok; ++j) {
-    // A_j: the slot's N-wide stream rows, 16 chunks of 8 per row
-    for (int x = tid; x < BL * 16; x += blockDim.x) {
-      const int s = x >> 4, ch = x & 15;
-      uint4 u = make_uint4(0u, 0u, 0u, 0u);
-      if (s < L) u = *reinterpret_cast<const uint4*>(Asrc + ((m0 + s) * d.k + j) * d.GN + (size_t)g * N + ch * 8);
-      *reinterpret_cast<uint4*>(As + (ch >> 3) * kTcBlk + tc::sw128_chunk(s, ch & 7)) = u;
+    // A_j: the slot's N-wide stream rows (16 chunks of 8 per row); B_j (end states): e^{cs_end - cs_s} Xs_j.
+    // All of this thread's loads are issued before the first store.
+    uint4 av[kAU];
+#pragma unroll
+    for (int u = 0; u < kAU; ++u) {
+      const int x = tid + 128 * u, s = x >> 4, ch = x & 15;
+      av[u] = s < L ? *reinterpret_cast<const uint4*>(Asrc + ((m0 + s) * d.k + j) * d.GN + (size_t)g * N + ch * 8)
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+    uint4 xv[kD ? 1 : kBU];
+    if constexpr (!kD) {
+#pragma unroll
+      for (int u = 0; u < kBU; ++u) {
+        const int x = tid + 128 * u, s = x / (kP / 8), p0 = (x % (kP / 8)) * 8;
+        xv[u] = s < L ? *reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(a.xs) +
+                                                        ((m0 + s) * d.k + j) * d.HP + (size_t)h * kP + p0)
+                      : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kAU; ++u) {
+      const int x = tid + 128 * u, s = x >> 4, ch = x & 15;
+      *reinterpret_cast<uint4*>(As + (ch >> 3) * kTcBlk + tc::sw128_chunk(s, ch & 7)) = av[u];
     }
     if constexpr (!kD) {
-      // B_j = e^{cs_end - cs_s} Xs_j
-      for (int x = tid; x < BL * (P / 8); x += blockDim.x) {
-        const int s = x / (P / 8), p0 = (x % (P / 8)) * 8;
+#pragma unroll
+      for (int u = 0; u < kBU; ++u) {
+        const int x = tid + 128 * u, s = x / (kP / 8), p0 = (x % (kP / 8)) * 8;
+        const float e = s < L ? expf(cs_end - cs[s]) : 0.f;
+        const __half2* hq = reinterpret_cast<const __half2*>(&xv[u]);
         float v[8];
-        if (s < L) {
-          const float e = expf(cs_end - cs[s]);
-          const uint4 q = *reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(a.xs) +
-                                                          ((m0 + s) * d.k + j) * d.HP + (size_t)h * P + p0);
-          const __half2* hq = reinterpret_cast<const __half2*>(&q);
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const float2 f = __half22float2(hq[e2]);
-            v[2 * e2] = e * f.x;
-            v[2 * e2 + 1] = e * f.y;
-          }
-        } else {
-#pragma unroll
-          for (int q2 = 0; q2 < 8; ++q2) v[q2] = 0.f;
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const float2 f = __half22float2(hq[e2]);
+          v[2 * e2] = e * f.x;
+          v[2 * e2 + 1] = e * f.y;
         }
         put_b(s, p0, v);
       }
@@ -409,13 +424,15 @@ __global__ void __launch_bounds__(128) bwd_states_tc_kernel(BwdArgs a) {
   }
   if (!ok && lane == 0) atomicOr(a.st, ST_TIMEOUT);
   // TMEM lane n (warp w: lanes 32w ..) holds row n of the [N x P] result
-  const size_t base = (((size_t)b * d.H + h) * a.nc + c) * (size_t)N * P;
+  const size_t base = (((size_t)b * d.H + h) * a.nc + c) * (size_t)N * kP;
   const int n = 32 * warp + lane;
-  for (int c0 = 0; c0 < P && ok; c0 += 32) {
+#pragma unroll
+  for (int c0 = 0; c0 < kP; c0 += 32) {
+    if (!ok) break;
     uint32_t r[32];
     tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0, r);
     tc::tmem_ld_wait(r);
-    float* dst = a.work + base + (size_t)n * P + c0;
+    float* dst = a.work + base + (size_t)n * kP + c0;
 #pragma unroll
     for (int i = 0; i < 32; i += 4)
       *reinterpret_cast<float4*>(dst + i) =
@@ -427,7 +444,7 @@ __global__ void __launch_bounds__(128) bwd_states_tc_kernel(BwdArgs a) {
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, (uint32_t)P);
+    tc::tmem_dealloc(tmem, (uint32_t)kP);
   }
 }
 
@@ -702,6 +719,16 @@ __global__ void __launch_bounds__(kBT) bwd_grad_kernel(BwdArgs a) {
   }
 }
 
+template <bool kD>
+cudaError_t launch_states_tc(const BwdArgs& a, dim3 grid, size_t smt, cudaStream_t s) {
+  const void* k = a.d.P == 64 ? (const void*)bwd_states_tc_kernel<kD, 64> : (const void*)bwd_states_tc_kernel<kD, 128>;
+  const cudaError_t e = set_max_dynamic_smem(k, smt);
+  if (e != cudaSuccess) return e;
+  if (a.d.P == 64) bwd_states_tc_kernel<kD, 64><<<grid, 128, smt, s>>>(a);
+  else bwd_states_tc_kernel<kD, 128><<<grid, 128, smt, s>>>(a);
+  return cudaSuccess;
+}
+
 template <class S, int PJ>
 cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s) {
   const Dims& d = a.d;
@@ -712,9 +739,8 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s) {
   const size_t smt = states_tc_smem(d.P);
   cudaError_t e;
   if (tc_states) {
-    e = set_max_dynamic_smem((const void*)bwd_states_tc_kernel<false>, smt);
+    e = launch_states_tc<false>(a, grid, smt, s);
     if (e != cudaSuccess) return e;
-    bwd_states_tc_kernel<false><<<grid, 128, smt, s>>>(a);
   } else {
     e = set_max_dynamic_smem((const void*)bwd_fwd_chunk_kernel<S, PJ>, sm1);
     if (e != cudaSuccess) return e;
@@ -723,9 +749,8 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, cudaStream_t s) {
   const dim3 pgrid(ceil_div(d.N * d.P, kBT), d.H, d.Bsz);
   bwd_fwd_pass_kernel<<<pgrid, kBT, 0, s>>>(a);
   if (tc_states) {
-    e = set_max_dynamic_smem((const void*)bwd_states_tc_kernel<true>, smt);
+    e = launch_states_tc<true>(a, grid, smt, s);
     if (e != cudaSuccess) return e;
-    bwd_states_tc_kernel<true><<<grid, 128, smt, s>>>(a);
   } else {
     e = set_max_dynamic_smem((const void*)bwd_d_kernel<S, PJ>, sm1);
     if (e != cudaSuccess) return e;
