@@ -1,4 +1,4 @@
-// Gradients of the whole layer: the stages after the scan gradients, in fp32.
+// Gradients of the whole layer: the stages after the scan gradients, fp32 values and accumulation.
 //
 // Paper: Swimba notes, Method flowchart (router -> expert projections -> parameter-space mixing -> one
 // recurrence) differentiated stage by stage in reverse; the notes train the model (loss function / training

@@ -1,4 +1,6 @@
-// Gradients of the chunked scan: reverse-mode of the single shared-transition recurrence, CUDA cores, fp32.
+// Gradients of the chunked scan: reverse-mode of the single shared-transition recurrence, fp32 values and
+// accumulation (the sub-chunk end states and adjoint sources on the tensor cores for fp16 streams with
+// N = 128, everything else on CUDA cores).
 //
 // Paper: Swimba notes, key design 1, second display equation (h_t = a_t h_{t-1} + U~_t, y_t = C~_t^T h_t);
 // the notes train the model (loss function / training strategy), which needs these gradients.  For
