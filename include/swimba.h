@@ -249,8 +249,12 @@ swimba_status swimba_layer_bwd(const swimba_dims* dims, const void* X, const swi
  *   dCt     [M][G][N] fp32 out: gradient of C~ = sum_j Cpi_j (every slot's Cpi receives it)
  *   d_dt    [M][H] fp32 out           dA [H] fp32 out (summed over tokens and sequences)
  *   d_init  [B][H][N][P] fp32 out or NULL
- * CUDA cores in fp32 over 64-token sub-chunks (the gradient kernel takes up to 226 KB of shared memory at
- * N = P = 128); needs the layer workspace (the same dims' swimba_workspace_size). */
+ * fp32 values and accumulation over 64-token sub-chunks: for fp16 streams with N = 128 and P in {64, 128} the
+ * sub-chunk end states and adjoint sources run on the tensor cores (fp16 stream operands, the other operand as
+ * an fp16 hi + lo pair under a power-of-two scale), everything else on CUDA cores (the gradient kernel takes
+ * up to 226 KB of shared memory at N = P = 128); needs the layer workspace (the same dims'
+ * swimba_workspace_size).  A device status of SWIMBA_ERR_TIMEOUT means a bounded wait of the tensor-core
+ * kernels gave up (outputs invalid). */
 swimba_status swimba_ssd_scan_bwd(const swimba_dims* dims, const void* Bpi, const void* Xs, const void* Cpi,
                                   const float* dt, const float* A, const float* init_state, const float* dy,
                                   float* dBpi, float* dXs, float* dCt, float* d_dt, float* dA, float* d_init,
