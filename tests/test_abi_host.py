@@ -148,6 +148,22 @@ def test_null_misaligned_and_workspace_errors(L):
     assert L.swimba_out_proj(None, fake, fake, fake, None) == 1
 
 
+@pytest.mark.parametrize("w", [configs.BASE, configs.BASE.with_(name="ws_We240", nheads=3, headdim=16, dstate=32,
+                                                                n_experts=5)], ids=lambda w: w.name)
+def test_layer_bwd_workspace_holds_the_tensor_core_operands(w):
+    """A bf16 layer's gradient workspace holds, besides the forward's workspace and the fp32 gradient buffers,
+    the tensor-core expert products' operands: dz as bf16 hi and lo over expert-padded rows
+    (Rp = M*k + 64 E rows rounded up to 128, 2 Wp columns with Wp = W_e rounded up to 64) and the X rows in
+    the same padded order."""
+    d = swimba.dims_of(w)
+    Mk = w.M * w.top_k
+    Rp = -(-(Mk + 64 * w.n_experts) // 128) * 128
+    Wp = -(-w.W_e // 64) * 64
+    fp32_bufs = Mk * (w.W_e + w.G * w.dstate + w.nheads * w.headdim + w.d_model) * 4
+    operands = Rp * 2 * Wp * 2 + Rp * w.d_model * 2 + Rp * 4 + Mk * 4
+    assert swimba.layer_bwd_workspace_size(d) >= swimba.workspace_size(d) + fp32_bufs + operands
+
+
 def test_host_pipeline_and_debug_hook_validation(L):
     """swimba_layer_fwd_host and the failure-detection hook reject bad arguments before any CUDA call."""
     d = swimba.dims_of(configs.BASE.with_(batch=2, seqlen=512, d_model=128, nheads=2))
