@@ -209,6 +209,23 @@ def _mix_bwd_unweighted_B(dBpi, dXs, dCt, w, Bz, Cz):
     return dz, dw
 
 
+def _mix_bwd_no_readout_term(dBpi, dXs, dCt, w, Bz, Cz):
+    # the router weight's gradient without the readout's term <C_j, dC~>
+    dz, _ = ORIG["mix_bwd"](dBpi, dXs, dCt, w, Bz, Cz)
+    return dz, np.einsum("mjgn,mjgn->mj", Bz, dBpi)
+
+
+def _mix_bwd_unweighted_C(dBpi, dXs, dCt, w, Bz, Cz):
+    # the C~ gradient passed on to every slot's C without its router weight
+    dz, dw = ORIG["mix_bwd"](dBpi, dXs, dCt, w, Bz, Cz)
+    M, k = w.shape
+    HP = dXs.shape[2] * dXs.shape[3]
+    GN = dBpi.shape[2] * dBpi.shape[3]
+    dz = dz.copy()
+    dz[:, :, HP + GN:] = np.broadcast_to(dCt.reshape(M, 1, GN), (M, k, GN))
+    return dz, dw
+
+
 def _router_bwd_not_renormalised(w, dw):
     # the softmax gradient without the renormalisation term
     return w * dw
@@ -260,6 +277,8 @@ MUTATIONS = {
     "adjoint_without_decay": ("scan_backward", _backward_no_adjoint_decay),
     "decay_gradient_off_by_one": ("scan_backward", _backward_decay_gradient_off_by_one),
     "mix_gradient_without_router_weight": ("mix_bwd", _mix_bwd_unweighted_B),
+    "router_weight_gradient_without_readout_term": ("mix_bwd", _mix_bwd_no_readout_term),
+    "readout_gradient_without_router_weight": ("mix_bwd", _mix_bwd_unweighted_C),
     "router_gradient_not_renormalised": ("router_bwd", _router_bwd_not_renormalised),
 }
 
